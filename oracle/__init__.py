@@ -1,0 +1,154 @@
+"""fp64 CPU oracle of the Mamba-1 selective scan (S6) and its decode update.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The product path (the CUDA library and its Python binding) never
+imports, loads or calls anything here, and this package never imports the
+product package.
+
+The arithmetic lives in ``oracle_ssm.c`` (plain C, double precision, evaluated
+in the order the definition states).  This module only compiles it with gcc,
+widens inputs to float64 and splits the independent channels across host
+threads (ctypes releases the GIL during the call), which does not change the
+order of any floating-point operation inside a channel.
+
+Sources: "Jamba: A Hybrid Transformer-Mamba Language Model" (obsidian-dorae222
+notes), section "Mamba 레이어" -- the S6 recurrence h_t = Abar_t h_{t-1} +
+Bbar_t x_t, y_t = C_t h_t with input-dependent Bbar, C, Delta; and "Jamba --
+Hybrid SSM-Transformer" (factory.pai-world.com), section "한 페이지로 보는 SSM"
+-- the O(1)-per-token decode step.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle_ssm.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle_ssm.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_i64 = ctypes.c_int64
+
+
+def build(src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile the oracle with gcc (strict IEEE: no fast-math, no FMA contraction)."""
+    cmd = ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fPIC", "-shared",
+           "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _declare(lib):
+    lib.oracle_softplus.restype = ctypes.c_double
+    lib.oracle_softplus.argtypes = [ctypes.c_double]
+    lib.oracle_silu.restype = ctypes.c_double
+    lib.oracle_silu.argtypes = [ctypes.c_double]
+    lib.oracle_scan_f64.restype = ctypes.c_int
+    lib.oracle_scan_f64.argtypes = [_i64] * 6 + [_dp] * 8 + [ctypes.c_int, _dp, _dp, _dp]
+    lib.oracle_state_update_f64.restype = ctypes.c_int
+    lib.oracle_state_update_f64.argtypes = ([_i64] * 3 + [_dp] * 9
+                                            + [ctypes.c_int, _dp])
+    return lib
+
+
+def load(path: str | None = None):
+    """Load (building first if needed) the oracle shared library."""
+    global _lib
+    with _lock:
+        if path is not None:
+            return _declare(ctypes.CDLL(path))
+        if _lib is None:
+            if (not os.path.exists(_LIB_PATH)
+                    or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+                build()
+            _lib = _declare(ctypes.CDLL(_LIB_PATH))
+        return _lib
+
+
+def _f64(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor -> numpy, exact widening
+        a = a.detach().to("cpu")
+        import torch
+        a = a.to(torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_dp)
+
+
+def softplus(v: float, lib=None) -> float:
+    return (lib or load()).oracle_softplus(float(v))
+
+
+def silu(v: float, lib=None) -> float:
+    return (lib or load()).oracle_silu(float(v))
+
+
+def scan(x, delta, z, B, C, A, D=None, delta_bias=None, delta_softplus=True,
+         h0=None, threads: int = 1, lib=None):
+    """Sequential fp64 scan.
+
+    Shapes: x, delta, z [batch, seqlen, d_inner]; B, C [batch, seqlen, d_state];
+    A [d_inner, d_state]; D, delta_bias [d_inner]; h0 [batch, d_inner, d_state].
+    Returns (out [batch, seqlen, d_inner], h_final [batch, d_inner, d_state]) as
+    float64 numpy arrays.  Inputs are widened exactly to float64 first.
+    """
+    lib = lib or load()
+    x, delta, z, B, C, A = map(_f64, (x, delta, z, B, C, A))
+    D, delta_bias, h0 = _f64(D), _f64(delta_bias), _f64(h0)
+    batch, seqlen, d_inner = x.shape
+    d_state = A.shape[1]
+    assert delta.shape == x.shape and z.shape == x.shape
+    assert B.shape == (batch, seqlen, d_state) and C.shape == B.shape
+    assert A.shape == (d_inner, d_state)
+    out = np.empty_like(x)
+    h_final = np.empty((batch, d_inner, d_state), dtype=np.float64)
+
+    def run(lo, hi):
+        rc = lib.oracle_scan_f64(batch, seqlen, d_inner, d_state, lo, hi,
+                                 _ptr(x), _ptr(delta), _ptr(z), _ptr(B), _ptr(C),
+                                 _ptr(A), _ptr(D), _ptr(delta_bias),
+                                 int(bool(delta_softplus)), _ptr(h0), _ptr(out),
+                                 _ptr(h_final))
+        if rc != 0:
+            raise ValueError("oracle_scan_f64 rejected its arguments")
+
+    threads = max(1, min(int(threads), d_inner))
+    if threads == 1:
+        run(0, d_inner)
+    else:
+        bounds = np.linspace(0, d_inner, threads + 1).astype(np.int64)
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(lambda i: run(int(bounds[i]), int(bounds[i + 1])), range(threads)))
+    return out, h_final
+
+
+def state_update(state, x, delta, z, B, C, A, D=None, delta_bias=None,
+                 delta_softplus=True, lib=None):
+    """One fp64 decode step.  Returns (out [batch, d_inner], new_state)."""
+    lib = lib or load()
+    st = _f64(state).copy()
+    x, delta, z, B, C, A = map(_f64, (x, delta, z, B, C, A))
+    D, delta_bias = _f64(D), _f64(delta_bias)
+    batch, d_inner = x.shape
+    d_state = A.shape[1]
+    assert st.shape == (batch, d_inner, d_state)
+    out = np.empty_like(x)
+    rc = lib.oracle_state_update_f64(batch, d_inner, d_state, _ptr(st), _ptr(x),
+                                     _ptr(delta), _ptr(z), _ptr(B), _ptr(C), _ptr(A),
+                                     _ptr(D), _ptr(delta_bias),
+                                     int(bool(delta_softplus)), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_state_update_f64 rejected its arguments")
+    return out, st

@@ -1,0 +1,141 @@
+/*
+ * oracle_ssm.c -- plain, slow, sequential fp64 oracle of the Mamba-1 selective
+ * scan (S6) and of its one-token decode state update.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file; it is used by the tests, by the smoke check and by the CPU
+ * baseline leg of the benchmark.  It shares no code, header, table or constant
+ * with the CUDA library.
+ *
+ * What it computes (sources):
+ *   - "Jamba: A Hybrid Transformer-Mamba Language Model" (obsidian-dorae222
+ *     notes), section "Mamba 레이어" (Mamba layer): the selective SSM
+ *         h_t = Abar_t h_{t-1} + Bbar_t x_t ,   y_t = C_t h_t ,
+ *     with Bbar_t, C_t, Delta_t produced from the input (selectivity), state
+ *     size d_state = 16, expansion factor 2.
+ *   - "Jamba -- Hybrid SSM-Transformer" (factory.pai-world.com lesson), section
+ *     "한 페이지로 보는 SSM" (SSM on one page): y_t needs only h_{t-1} and x_t,
+ *     constant memory, O(1) work per token -- the decode update below.
+ *   - same lesson, "Mamba-3" item 2: Mamba's state matrix is real diagonal, so
+ *     every (channel d, state n) pair is an independent scalar recurrence.
+ * The pages print only the symbols Abar, Bbar.  Readings taken where they are
+ * silent (all listed in the design doc):
+ *   - discretisation: Abar = exp(Delta * A[d,n]),  Bbar x = Delta * B[t,n] * x;
+ *   - Delta = softplus(delta + delta_bias[d]) when delta_softplus != 0, else
+ *     Delta = delta + delta_bias[d];
+ *   - output: out = (sum_n C[t,n] h[n] + D[d] x) * silu(z), silu(z) = z/(1+e^-z).
+ *
+ * Everything is evaluated in the order the definition states: channel by
+ * channel, step by step, state by state, in double precision.
+ *
+ * Parity: this file is pinned by tests/test_oracle_pins.py (brute-force
+ * unrolled sums, the geometric-series closed form, the Delta->0 and large-Delta
+ * limits, libm softplus/silu, split-scan and decode==scan identities).
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+
+/* softplus(v) = log(1 + e^v), written in the form that does not overflow. */
+double oracle_softplus(double v) {
+    if (v > 0.0) return v + log1p(exp(-v));
+    return log1p(exp(v));
+}
+
+/* silu(z) = z * sigmoid(z) = z / (1 + e^-z). */
+double oracle_silu(double z) {
+    return z / (1.0 + exp(-z));
+}
+
+/* Delta for one (t, d): the raw input plus the per-channel bias, through
+ * softplus when requested. */
+static double oracle_delta(double raw, const double *delta_bias, int64_t d,
+                           int delta_softplus) {
+    double v = raw + (delta_bias ? delta_bias[d] : 0.0);
+    return delta_softplus ? oracle_softplus(v) : v;
+}
+
+/*
+ * Prefill scan over channels [d_lo, d_hi) of every sequence.
+ *   x, delta, z : [batch, seqlen, d_inner]
+ *   B, C        : [batch, seqlen, d_state]
+ *   A           : [d_inner, d_state]
+ *   D, delta_bias : [d_inner] or NULL (zero)
+ *   h0          : [batch, d_inner, d_state] or NULL (zero initial state)
+ *   out         : [batch, seqlen, d_inner]             (written for d in range)
+ *   h_final     : [batch, d_inner, d_state] or NULL    (written for d in range)
+ * The channel range only selects which independent recurrences to run, so a
+ * caller may split [0, d_inner) across threads.  Returns 0, or -1 on a bad
+ * argument.
+ */
+int oracle_scan_f64(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
+                    int64_t d_lo, int64_t d_hi,
+                    const double *x, const double *delta, const double *z,
+                    const double *B, const double *C, const double *A,
+                    const double *D, const double *delta_bias, int delta_softplus,
+                    const double *h0, double *out, double *h_final) {
+    if (batch < 0 || seqlen < 0 || d_inner < 0 || d_state < 1 || d_state > 64)
+        return -1;
+    if (d_lo < 0 || d_hi > d_inner || d_lo > d_hi) return -1;
+    double h[64];
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = d_lo; d < d_hi; ++d) {
+            for (int64_t n = 0; n < d_state; ++n)
+                h[n] = h0 ? h0[(b * d_inner + d) * d_state + n] : 0.0;
+            for (int64_t t = 0; t < seqlen; ++t) {
+                int64_t i = (b * seqlen + t) * d_inner + d;
+                const double *Bt = B + (b * seqlen + t) * d_state;
+                const double *Ct = C + (b * seqlen + t) * d_state;
+                double xv = x[i];
+                double dv = oracle_delta(delta[i], delta_bias, d, delta_softplus);
+                double y = 0.0;
+                for (int64_t n = 0; n < d_state; ++n) {
+                    double abar = exp(dv * A[d * d_state + n]);
+                    double bbar_x = dv * Bt[n] * xv;
+                    h[n] = abar * h[n] + bbar_x;
+                    y += Ct[n] * h[n];
+                }
+                double skip = D ? D[d] * xv : 0.0;
+                out[i] = (y + skip) * oracle_silu(z[i]);
+            }
+            if (h_final)
+                for (int64_t n = 0; n < d_state; ++n)
+                    h_final[(b * d_inner + d) * d_state + n] = h[n];
+        }
+    }
+    return 0;
+}
+
+/*
+ * One decode step for every request: the same recurrence for a single token,
+ * reading the cached state and writing the new state in place.
+ *   state : [batch, d_inner, d_state]  (in/out)
+ *   x, delta, z, out : [batch, d_inner]
+ *   B, C  : [batch, d_state]
+ */
+int oracle_state_update_f64(int64_t batch, int64_t d_inner, int64_t d_state,
+                            double *state,
+                            const double *x, const double *delta, const double *z,
+                            const double *B, const double *C, const double *A,
+                            const double *D, const double *delta_bias,
+                            int delta_softplus, double *out) {
+    if (batch < 0 || d_inner < 0 || d_state < 1) return -1;
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < d_inner; ++d) {
+            int64_t i = b * d_inner + d;
+            double *h = state + i * d_state;
+            double xv = x[i];
+            double dv = oracle_delta(delta[i], delta_bias, d, delta_softplus);
+            double y = 0.0;
+            for (int64_t n = 0; n < d_state; ++n) {
+                double abar = exp(dv * A[d * d_state + n]);
+                double bbar_x = dv * B[b * d_state + n] * xv;
+                h[n] = abar * h[n] + bbar_x;
+                y += C[b * d_state + n] * h[n];
+            }
+            double skip = D ? D[d] * xv : 0.0;
+            out[i] = (y + skip) * oracle_silu(z[i]);
+        }
+    }
+    return 0;
+}
