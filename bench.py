@@ -1,0 +1,491 @@
+"""Benchmark of the S6 hot path on B200: prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of the workload: the
+prefill scan (jamba_ssm_scan: Delta, discretisation, recurrence, readout, skip,
+gate, final state) followed by one decode state update (jamba_ssm_state_update)
+of the next token from that final state.  Default workload: Jamba-Mini's Mamba
+layer prefill, batch 1, L = 4096, d_inner = 8192, d_state = 16, bf16 I/O, fp32
+state.  Inputs are seeded synthetic tensors of that shape resident in HBM; L2 is
+flushed (a 256 MiB write) before every timed step, outside the timed events.
+
+Timing: CUDA events on the launching stream around every step (and around the
+scan alone, for the roofline), summed over the K timed steps after W warm-up
+steps; barrier + synchronize on both sides; the max over ranks.  N > 1 runs one
+independent replica per GPU (each its own sequence: weak scaling; the scan has
+no exchange step).  `e2e` repeats the step through the public API with the
+inputs copied from pinned host memory and the results copied back inside the
+timed region.  `--impl reference` times the fp64 CPU oracle instead, on a
+bounded channel sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+MUFU_OPS_PER_CLK_PER_SM = 16   # exp2 / rcp throughput per SM per clock (sm_100)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_SM_MHZ = 1965.0
+
+
+# ----------------------------------------------------------------- helpers
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", FALLBACK_SM_MHZ)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_SM_MHZ, "fallback"
+
+
+def kernel_source_hash():
+    d = os.path.join(ROOT, "selective_state_space_26_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        r = rec[kernel][workload]
+        if r.get("source_hash") == kernel_source_hash():
+            return float(r["bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def prefill_bytes(batch, seqlen, d_inner, d_state, io_bytes):
+    """Minimum bytes of one prefill scan: x, delta, z, B, C read once, out
+    written once, A / D / delta_bias read once, fp32 final state written."""
+    tok = batch * seqlen
+    return (tok * (4 * d_inner + 2 * d_state) * io_bytes + (d_inner * d_state + 2 * d_inner) * 4
+            + batch * d_inner * d_state * 4)
+
+
+def decode_bytes(batch, d_inner, d_state, io_bytes):
+    """Minimum bytes of one decode step: fp32 state read + written, x / delta /
+    z read, out written, B / C read, parameters read."""
+    return (2 * batch * d_inner * d_state * 4 + 4 * batch * d_inner * io_bytes
+            + 2 * batch * d_state * io_bytes + (d_inner * d_state + 2 * d_inner) * 4)
+
+
+def exp_ops(tokens, d_inner, d_state):
+    """Transcendental ops the method needs per (token, channel): d_state exps
+    for Abar, exp + log for softplus, exp + reciprocal for the gate."""
+    return tokens * d_inner * (d_state + 4)
+
+
+class ClockSampler:
+    """NVML sampling of SM clock and clock-event reasons during the timed region."""
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+             0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+             0x100: "display_clock_setting"}
+
+    def __init__(self, props, period=0.002):
+        self.period = period
+        self.samples, self.reasons, self.ok = [], 0, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            try:  # the CUDA device's own NVML handle (indices can differ)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_reasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for bit, n in self.NAMES.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "reasons": names}
+
+
+# ------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import selective_state_space_26_b200 as jssm
+    from selective_state_space_26_b200 import build, synth
+
+    build.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[args.workload]
+    io_bytes = 2 if w.dtype == torch.bfloat16 else 4
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    props = torch.cuda.get_device_properties(dev)
+    sms = props.multi_processor_count
+
+    if w.kind == "prefill":
+        inp = synth.workload_inputs(w, device=dev, seq_offset=rank * w.batch)
+        nxt = synth.decode_step(w.batch, w.d_inner, w.d_state, 0, w.seed, w.dtype, dev)
+        out = torch.empty_like(inp.x)
+        hf = torch.empty(w.batch, w.d_inner, w.d_state, dtype=torch.float32, device=dev)
+        dec_out = torch.empty_like(nxt.x)
+        tokens = w.batch * (w.seqlen + 1)
+
+        def step():
+            jssm.jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, D=inp.D,
+                                delta_bias=inp.delta_bias, out=out, h_final=hf)
+            ev_mid.record(stream)
+            jssm.jamba_ssm_state_update(hf, nxt.x, nxt.delta, nxt.z, nxt.B, nxt.C, inp.A,
+                                        D=inp.D, delta_bias=inp.delta_bias, out=dec_out)
+        launches_per_step = 2
+        dom_name = "s6_scan_fwd_kernel"
+        dom_bytes = prefill_bytes(w.batch, w.seqlen, w.d_inner, w.d_state, io_bytes)
+        plan = jssm.scan_plan(inp.x, inp.A)
+    else:
+        A = synth.make_A(w.d_inner, w.d_state).to(dev)
+        Dv = torch.ones(w.d_inner, device=dev)
+        bias = synth.dt_bias_for(w.d_inner, w.seed).to(dev)
+        st = synth.decode_state(w.batch, w.d_inner, w.d_state, w.seed + 1000 * rank, device=dev)
+        steps_in = [synth.decode_step(w.batch, w.d_inner, w.d_state, k, w.seed, w.dtype, dev)
+                    for k in range(w.seqlen)]
+        dec_out = torch.empty(w.batch, w.d_inner, dtype=w.dtype, device=dev)
+        tokens = w.batch
+        counter = [0]
+
+        def step():
+            s = steps_in[counter[0] % len(steps_in)]
+            counter[0] += 1
+            jssm.jamba_ssm_state_update(st, s.x, s.delta, s.z, s.B, s.C, A, D=Dv,
+                                        delta_bias=bias, out=dec_out)
+            ev_mid.record(stream)
+        launches_per_step = 1
+        dom_name = "s6_state_update_kernel"
+        dom_bytes = decode_bytes(w.batch, w.d_inner, w.d_state, io_bytes)
+        plan = None
+
+    ev_mid = torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(props) as clk:
+        for k in range(args.steps):
+            flush.zero_()
+            e0, e1, e2 = evs[k]
+            e0.record(stream)
+            ev_mid = e1
+            step()
+            e2.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    step_ms = sum(e0.elapsed_time(e2) for e0, _, e2 in evs)
+    dom_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in evs)
+    if w.kind == "decode":
+        dom_ms = step_ms
+    times = torch.tensor([step_ms, dom_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    step_ms, dom_ms = float(times[0]), float(times[1])
+    ms_per_step = step_ms / args.steps
+    dom_launch_s = dom_ms / args.steps / 1e3
+
+    # ---- e2e: inputs from pinned host memory, results back, inside the timed region
+    e2e = None
+    if w.kind == "prefill":
+        host = {k: getattr(inp, k).cpu().pin_memory() for k in ("x", "delta", "z", "B", "C")}
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h_hf = torch.empty(hf.shape, dtype=hf.dtype).pin_memory()
+        h_dec = torch.empty(dec_out.shape, dtype=dec_out.dtype).pin_memory()
+        dbuf = {k: torch.empty_like(getattr(inp, k)) for k in host}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in (h_out, h_hf, h_dec))
+
+        def e2e_step():
+            for k, t in host.items():
+                dbuf[k].copy_(t, non_blocking=True)
+            jssm.jamba_ssm_scan(dbuf["x"], dbuf["delta"], dbuf["z"], dbuf["B"], dbuf["C"], inp.A,
+                                D=inp.D, delta_bias=inp.delta_bias, out=out, h_final=hf)
+            jssm.jamba_ssm_state_update(hf, nxt.x, nxt.delta, nxt.z, nxt.B, nxt.C, inp.A,
+                                        D=inp.D, delta_bias=inp.delta_bias, out=dec_out)
+            h_out.copy_(out, non_blocking=True)
+            h_hf.copy_(hf, non_blocking=True)
+            h_dec.copy_(dec_out, non_blocking=True)
+    else:
+        h_steps = [{k: getattr(s, k).cpu().pin_memory() for k in ("x", "delta", "z", "B", "C")}
+                   for s in steps_in[:8]]
+        dbuf = {k: torch.empty_like(getattr(steps_in[0], k)) for k in h_steps[0]}
+        h_dec = torch.empty(dec_out.shape, dtype=dec_out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in h_steps[0].values())
+        d2h = h_dec.numel() * h_dec.element_size()
+        ctr = [0]
+
+        def e2e_step():
+            hs = h_steps[ctr[0] % len(h_steps)]
+            ctr[0] += 1
+            for k, t in hs.items():
+                dbuf[k].copy_(t, non_blocking=True)
+            jssm.jamba_ssm_state_update(st, dbuf["x"], dbuf["delta"], dbuf["z"], dbuf["B"],
+                                        dbuf["C"], A, D=Dv, delta_bias=bias, out=dec_out)
+            h_dec.copy_(dec_out, non_blocking=True)
+    k_e2e = max(3, min(args.steps, 20))
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(k_e2e):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    t_e2e = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t_e2e, op=torch.distributed.ReduceOp.MAX)
+    e2e = {"value": tokens * world * k_e2e / (float(t_e2e[0]) / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": k_e2e}
+
+    # ---- roofline of the dominant kernel
+    hbm_gbs, sm_mhz_peak, peak_kind = peaks()
+    clocks = clk.summary()
+    traffic = recorded_traffic(dom_name, w.name)
+    if w.kind == "prefill":
+        ops = exp_ops(w.batch * w.seqlen, w.d_inner, w.d_state)
+        peak = sms * MUFU_OPS_PER_CLK_PER_SM * sm_mhz_peak * 1e6 / 1e12
+        achieved = ops / dom_launch_s / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak,
+                "unit": "Top/s (exp-class, MUFU)", "frac": achieved / peak, "traffic": traffic,
+                "kernel": dom_name,
+                "peak_basis": f"{sms} SMs x {MUFU_OPS_PER_CLK_PER_SM}/clk x {sm_mhz_peak:.0f} MHz "
+                              f"({peak_kind} max clock)",
+                "algorithmic_ops_per_launch": ops,
+                "algorithmic_bytes_per_launch": dom_bytes,
+                "hbm_gbs": dom_bytes / dom_launch_s / 1e9,
+                "hbm_frac": dom_bytes / dom_launch_s / 1e9 / hbm_gbs,
+                "launch_us": dom_launch_s * 1e6}
+        if clocks.get("sm_mhz"):
+            roof["frac_at_observed_clock"] = achieved / (peak * clocks["sm_mhz"] / sm_mhz_peak)
+    else:
+        achieved = dom_bytes / dom_launch_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                "frac": achieved / hbm_gbs, "traffic": traffic, "kernel": dom_name,
+                "peak_basis": f"{peak_kind} copy bandwidth",
+                "algorithmic_bytes_per_launch": dom_bytes, "launch_us": dom_launch_s * 1e6}
+
+    line = {
+        "metric": "selective-scan tokens/s & HBM GB/s (fraction of roofline) at d_inner=8192, N=16",
+        "value": tokens * world / (ms_per_step / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded N(0,1) activations, log-uniform dt0, A=-(n+1), D=1)",
+        "config": {"workload": w.name, "global_batch": w.batch * world, "seq_len": w.seqlen,
+                   "d_inner": w.d_inner, "d_state": w.d_state,
+                   "step": ("prefill scan + 1 decode update" if w.kind == "prefill"
+                            else "1 decode update of every request"),
+                   "tokens_per_step_per_gpu": tokens,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed (256 MiB write) before every timed step",
+                   "scan_plan": plan},
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp if w.kind == "prefill" else None,
+                                            target_s=args.cpu_seconds)
+    return line
+
+
+# ------------------------------------------------------- the oracle on the host
+def _oracle_sample_prefill(w, inp_host, channels):
+    import oracle
+    sel = slice(0, channels)
+    threads = os.cpu_count() or 1
+    t = time.perf_counter()
+    oracle.scan(inp_host["x"][:, :, sel], inp_host["delta"][:, :, sel], inp_host["z"][:, :, sel],
+                inp_host["B"], inp_host["C"], inp_host["A"][sel], D=inp_host["D"][sel],
+                delta_bias=inp_host["delta_bias"][sel], threads=threads)
+    return time.perf_counter() - t, threads
+
+
+def _host_inputs(w, inp=None, channels=None):
+    import numpy as np
+    from selective_state_space_26_b200 import synth
+    if inp is None:
+        inp = synth.workload_inputs(w, device="cpu")
+    ch = slice(None) if channels is None else slice(0, channels)
+    f = lambda t: np.ascontiguousarray(t.detach().to("cpu", torch.float64).numpy())  # noqa: E731
+    return {"x": f(inp.x[:, :, ch]), "delta": f(inp.delta[:, :, ch]), "z": f(inp.z[:, :, ch]),
+            "B": f(inp.B), "C": f(inp.C), "A": f(inp.A[ch]), "D": f(inp.D[ch]),
+            "delta_bias": f(inp.delta_bias[ch])}
+
+
+def _decode_sample(w, requests, steps):
+    import oracle
+    from selective_state_space_26_b200 import synth
+    A = synth.make_A(w.d_inner, w.d_state)
+    bias = synth.dt_bias_for(w.d_inner, w.seed)
+    st = synth.decode_state(requests, w.d_inner, w.d_state, w.seed)
+    ins = [synth.decode_step(requests, w.d_inner, w.d_state, k, w.seed, w.dtype) for k in range(steps)]
+    t = time.perf_counter()
+    for s in ins:
+        _, st = oracle.state_update(st, s.x, s.delta, s.z, s.B, s.C, A, D=torch.ones(w.d_inner),
+                                    delta_bias=bias)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(w, inp=None, target_s=10.0):
+    """The oracle as it stands on the host cores, on a bounded sample."""
+    if w.kind == "prefill":
+        probe = min(w.d_inner, 64)
+        host = _host_inputs(w, inp, channels=w.d_inner)
+        t, threads = _oracle_sample_prefill(w, host, probe)
+        rate = probe / max(t, 1e-6)
+        ch = int(min(w.d_inner, max(probe, rate * target_s)))
+        t, threads = _oracle_sample_prefill(w, host, ch)
+        tok_equiv = w.batch * w.seqlen * ch / w.d_inner
+        return {"value": tok_equiv / t, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                "sample": f"channels 0..{ch - 1} of {w.d_inner}, all {w.batch}x{w.seqlen} steps; "
+                          f"value = token-equivalents (tokens x sampled/total channels) / wall",
+                "wall_s": t}
+    req, steps = 4, 4
+    t = _decode_sample(w, req, steps)
+    return {"value": req * steps / t, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{req} requests x {steps} steps of {w.d_inner} channels", "wall_s": t}
+
+
+def run_reference(args):
+    from selective_state_space_26_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    budget = args.ref_seconds
+    if w.kind == "prefill":
+        host = _host_inputs(w, None)
+        probe = 32
+        t, threads = _oracle_sample_prefill(w, host, probe)
+        per_step = budget / (args.steps + args.warmup)
+        ch = int(max(8, min(w.d_inner, probe * per_step / max(t, 1e-6))))
+        for _ in range(args.warmup):
+            _oracle_sample_prefill(w, host, ch)
+        tot = 0.0
+        for _ in range(args.steps):
+            dt, threads = _oracle_sample_prefill(w, host, ch)
+            tot += dt
+        tok_equiv = w.batch * w.seqlen * ch / w.d_inner
+        value = tok_equiv * args.steps / tot
+        sample = (f"each step: channels 0..{ch - 1} of {w.d_inner} over all {w.batch}x{w.seqlen} "
+                  f"steps (token-equivalents)")
+        cores = threads
+    else:
+        t1 = _decode_sample(w, 2, 1)
+        tot = 0.0
+        for _ in range(args.steps):
+            tot += _decode_sample(w, 2, 1)
+        value = 2 * args.steps / tot
+        sample = f"each step: 2 requests x 1 decode step of {w.d_inner} channels"
+        cores = 1
+        del t1
+    ms = tot / args.steps * 1e3
+    return {
+        "impl": "reference",
+        "metric": "selective-scan tokens/s & HBM GB/s (fraction of roofline) at d_inner=8192, N=16",
+        "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (same recipe as our arm)",
+        "config": {"workload": w.name, "global_batch": w.batch, "seq_len": w.seqlen,
+                   "d_inner": w.d_inner, "d_state": w.d_state},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="s6_prefill_bf16_b1_l4096_d8192_n16")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+/*
+ * jamba_ssm.h -- C ABI of the B200 (sm_100a) Mamba-1 selective-scan (S6)
+ * library: the prefill scan and the one-token decode state update of the S6
+ * mixer that makes up seven of every eight Jamba layers.
+ *
+ * The operation (sources):
+ *   - "Jamba: A Hybrid Transformer-Mamba Language Model" (obsidian-dorae222
+ *     notes), section "Mamba 레이어" (Mamba layer): the selective SSM
+ *         h_t = Abar_t h_{t-1} + Bbar_t x_t,   y_t = C_t h_t,
+ *     with Bbar_t, C_t, Delta_t functions of the input; d_state = 16 and
+ *     expansion factor 2 (d_model 4096 -> d_inner 8192).
+ *   - the same notes, section "KV 캐시 효율 분석": the Mamba state is a fixed
+ *     D x N array per layer and sequence, independent of the length L.
+ *   - "Jamba -- Hybrid SSM-Transformer" (factory.pai-world.com), section
+ *     "한 페이지로 보는 SSM": y_t needs only h_{t-1} and x_t (O(1) decode);
+ *     item 2 of its Mamba-3 list: Mamba's state matrix A is real diagonal.
+ *   Readings where the pages are silent: Abar = exp(Delta * A[d,n]),
+ *   Bbar x = Delta * B[t,n] * x, Delta = softplus(delta + delta_bias[d]) (or
+ *   delta + delta_bias[d] without softplus), and the layer output
+ *   out = (sum_n C[t,n] h[n] + D[d] x) * silu(z), silu(z) = z / (1 + e^-z).
+ *
+ * Conventions shared by every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates nothing, frees nothing and keeps no per-call state (it caches
+ *     only per-device attributes).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously on it.
+ *   - Activations are row-major with the channel index innermost:
+ *     x/delta/z/out [batch, seqlen, d_inner], B/C [batch, seqlen, d_state];
+ *     the state is fp32 [batch, d_inner, d_state]; A is fp32
+ *     [d_inner, d_state]; D and delta_bias are fp32 [d_inner].
+ *   - Argument errors are detected on the host before anything is enqueued and
+ *     returned as a status; nothing is launched then.  A failed launch returns
+ *     JAMBA_SSM_ERR_CUDA (the CUDA error code is kept per host thread, see
+ *     jamba_ssm_last_cuda_error).  A device-side condition (a bounded wait that
+ *     ran out) is recorded in a per-device status word read by
+ *     jamba_ssm_get_status.  No C++ exception crosses this interface.
+ */
+#ifndef JAMBA_SSM_H
+#define JAMBA_SSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define JAMBA_SSM_ABI_VERSION 1
+
+typedef enum {
+    JAMBA_SSM_OK = 0,
+    JAMBA_SSM_ERR_INVALID_ARG = 1,  /* NULL pointer, negative size, aliasing, bad struct_size */
+    JAMBA_SSM_ERR_UNSUPPORTED = 2,  /* d_state / dtype / d_inner combination not built        */
+    JAMBA_SSM_ERR_MISALIGNED = 3,   /* a pointer is not aligned as documented below            */
+    JAMBA_SSM_ERR_CUDA = 4,         /* a CUDA runtime/driver call or the launch failed         */
+    JAMBA_SSM_ERR_TIMEOUT = 5,      /* device side: a bounded wait ran out (get_status only)   */
+    JAMBA_SSM_ERR_NO_DEVICE = 6     /* no usable sm_100 device is current                      */
+} jamba_ssm_status;
+
+typedef enum {
+    JAMBA_SSM_BF16 = 0,  /* x, delta, z, B, C, out are bfloat16 */
+    JAMBA_SSM_F32 = 1    /* x, delta, z, B, C, out are float32  */
+} jamba_ssm_dtype;
+
+/*
+ * Prefill scan over whole sequences (the S6 recurrence of "Mamba 레이어",
+ * evaluated for t = 0 .. seqlen-1 from the initial state h0).
+ *
+ * Sizes: batch >= 0, seqlen >= 0, d_inner >= 1, d_state in the supported set:
+ *   bf16 I/O: d_state in {8, 16} and d_inner % 8 == 0;
+ *   f32  I/O: d_state in {4, 8, 16} and d_inner % 4 == 0.
+ * (Each activation row must be a multiple of 16 bytes.)  Jamba's layer is
+ * d_inner = 8192, d_state = 16.
+ * Pointers (device):
+ *   x, delta, z   [batch, seqlen, d_inner] io_dtype, 16-byte aligned, required.
+ *                 delta is the raw step input; Delta is formed in the kernel.
+ *   B, C          [batch, seqlen, d_state] io_dtype, 16-byte aligned, required.
+ *   A             [d_inner, d_state] fp32, 16-byte aligned, required (A < 0
+ *                 in a trained layer; any finite value is accepted).
+ *   D             [d_inner] fp32 or NULL (no skip term).
+ *   delta_bias    [d_inner] fp32 or NULL (zero bias).
+ *   h0            [batch, d_inner, d_state] fp32, 16-byte aligned, or NULL
+ *                 (zero initial state).  Resuming a sequence = passing the
+ *                 h_final of the previous chunk here (chunked prefill).
+ *   out           [batch, seqlen, d_inner] io_dtype, 16-byte aligned, required;
+ *                 must not overlap any input.
+ *   h_final       [batch, d_inner, d_state] fp32, 16-byte aligned, or NULL.
+ *                 The state after the last step: the decode cache entry.
+ *                 h_final == h0 (resume in place) is allowed.
+ * delta_softplus: nonzero -> Delta = softplus(delta + delta_bias), else
+ *                 Delta = delta + delta_bias.
+ * kernel_variant: 0 = let the library choose the launch shape; k > 0 forces
+ *                 built variant k (see jamba_ssm_scan_variant_info); an
+ *                 unknown or inapplicable k returns JAMBA_SSM_ERR_UNSUPPORTED.
+ * debug_flags / timeout_cycles: 0 in production.  Bit 0 of debug_flags
+ *                 withholds the first input tile of every CTA so its bounded
+ *                 wait runs out (test of the timeout path); timeout_cycles
+ *                 overrides the wait limit (SM clock cycles, 0 = ~1 s).
+ * Empty input: batch == 0 does nothing; seqlen == 0 copies h0 (or zeros)
+ * into h_final.
+ */
+typedef struct jamba_ssm_scan_params {
+    size_t struct_size;          /* = sizeof(jamba_ssm_scan_params)            */
+    int64_t batch, seqlen, d_inner, d_state;
+    int32_t io_dtype;            /* jamba_ssm_dtype                            */
+    int32_t delta_softplus;
+    const void *x, *delta, *z;
+    const void *B, *C;
+    const float *A;
+    const float *D;
+    const float *delta_bias;
+    const float *h0;
+    void *out;
+    float *h_final;
+    int32_t kernel_variant;
+    uint32_t debug_flags;
+    uint64_t timeout_cycles;
+} jamba_ssm_scan_params;
+
+jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream);
+
+/*
+ * One decode step for `batch` requests (the O(1) update of "한 페이지로 보는
+ * SSM"): for every request b and channel d,
+ *   h'[n] = exp(Delta A[d,n]) h[n] + Delta B[b,n] x,
+ *   out   = (sum_n C[b,n] h'[n] + D[d] x) * silu(z),
+ * and the state is overwritten with h' IN PLACE.
+ * Sizes: as jamba_ssm_scan with seqlen = 1, except d_inner only needs
+ * d_inner >= 1 and d_state in {4, 8, 16} for both dtypes.
+ * Pointers (device):
+ *   state      [batch, d_inner, d_state] fp32, 16-byte aligned, read + written.
+ *   x, delta, z, out [batch, d_inner] io_dtype (naturally aligned); out must
+ *              not overlap an input.
+ *   B, C       [batch, d_state] io_dtype (naturally aligned).
+ *   A          [d_inner, d_state] fp32, 16-byte aligned; D, delta_bias as above.
+ */
+typedef struct jamba_ssm_state_update_params {
+    size_t struct_size;          /* = sizeof(jamba_ssm_state_update_params)    */
+    int64_t batch, d_inner, d_state;
+    int32_t io_dtype;
+    int32_t delta_softplus;
+    float *state;
+    const void *x, *delta, *z;
+    const void *B, *C;
+    const float *A;
+    const float *D;
+    const float *delta_bias;
+    void *out;
+} jamba_ssm_state_update_params;
+
+jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, void *stream);
+
+/* Launch shape the scan would use for these parameters (no launch).  Any of
+ * the out pointers may be NULL.  variant: the built variant chosen;
+ * lanes_per_channel: lanes sharing one channel's states; channels_per_cta;
+ * grid: CTAs launched; tasks: (sequence, channel-group) units. */
+jamba_ssm_status jamba_ssm_scan_plan(const jamba_ssm_scan_params *p, int32_t *variant,
+                                     int32_t *lanes_per_channel, int32_t *channels_per_cta,
+                                     int32_t *grid, int64_t *tasks);
+
+/* Description of built scan variant k (1-based); returns
+ * JAMBA_SSM_ERR_UNSUPPORTED past the last one.  Out pointers may be NULL. */
+jamba_ssm_status jamba_ssm_scan_variant_info(int32_t k, int32_t *io_dtype, int32_t *d_state,
+                                             int32_t *lanes_per_channel, int32_t *warps_per_cta,
+                                             int32_t *time_tile);
+
+/* Synchronizes `stream`, then reads and clears the current device's sticky
+ * status word: JAMBA_SSM_OK, or the first device-side error recorded since the
+ * last call (JAMBA_SSM_ERR_TIMEOUT).  Returns JAMBA_SSM_ERR_CUDA if the
+ * synchronization itself failed. */
+jamba_ssm_status jamba_ssm_get_status(void *stream);
+
+/* CUDA error code (cudaError_t as int) behind the last JAMBA_SSM_ERR_CUDA
+ * returned on this host thread, 0 if none. */
+int jamba_ssm_last_cuda_error(void);
+
+/* Static, NUL-terminated description of a status code. */
+const char *jamba_ssm_status_string(jamba_ssm_status s);
+
+/* JAMBA_SSM_ABI_VERSION the library was built with. */
+int jamba_ssm_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JAMBA_SSM_H */

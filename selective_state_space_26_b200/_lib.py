@@ -1,0 +1,157 @@
+"""ctypes view of the C ABI in include/jamba_ssm.h (argument marshalling only).
+
+The structures below mirror the header field by field.  Loading fails loudly
+when libjamba_ssm.so has not been built: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libjamba_ssm.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_NO_DEVICE = range(7)
+BF16, F32 = 0, 1
+
+# Every symbol the header declares.
+EXPORTS = (
+    "jamba_ssm_scan",
+    "jamba_ssm_state_update",
+    "jamba_ssm_scan_plan",
+    "jamba_ssm_scan_variant_info",
+    "jamba_ssm_get_status",
+    "jamba_ssm_last_cuda_error",
+    "jamba_ssm_status_string",
+    "jamba_ssm_abi_version",
+)
+
+_vp = ctypes.c_void_p
+_fp = ctypes.c_void_p  # float* passed as raw address
+
+
+class ScanParams(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t),
+        ("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+        ("d_inner", ctypes.c_int64), ("d_state", ctypes.c_int64),
+        ("io_dtype", ctypes.c_int32), ("delta_softplus", ctypes.c_int32),
+        ("x", _vp), ("delta", _vp), ("z", _vp),
+        ("B", _vp), ("C", _vp),
+        ("A", _fp), ("D", _fp), ("delta_bias", _fp), ("h0", _fp),
+        ("out", _vp), ("h_final", _fp),
+        ("kernel_variant", ctypes.c_int32), ("debug_flags", ctypes.c_uint32),
+        ("timeout_cycles", ctypes.c_uint64),
+    ]
+
+
+class StateUpdateParams(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t),
+        ("batch", ctypes.c_int64), ("d_inner", ctypes.c_int64), ("d_state", ctypes.c_int64),
+        ("io_dtype", ctypes.c_int32), ("delta_softplus", ctypes.c_int32),
+        ("state", _fp),
+        ("x", _vp), ("delta", _vp), ("z", _vp),
+        ("B", _vp), ("C", _vp),
+        ("A", _fp), ("D", _fp), ("delta_bias", _fp),
+        ("out", _vp),
+    ]
+
+
+class JambaSSMError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = status_string(status)
+        if status == ERR_CUDA:
+            msg += f" (cudaError {lib().jamba_ssm_last_cuda_error()})"
+        super().__init__(f"{what}: {msg}")
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib():
+    """Load libjamba_ssm.so (raises if it is missing: build it first)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(
+                        f"{LIB_PATH} is not built; run selective_state_space_26_b200.build.build()"
+                        " (nvcc, sm_100a). There is no CPU fallback.")
+                L = ctypes.CDLL(LIB_PATH)
+                L.jamba_ssm_scan.restype = ctypes.c_int
+                L.jamba_ssm_scan.argtypes = [ctypes.POINTER(ScanParams), _vp]
+                L.jamba_ssm_state_update.restype = ctypes.c_int
+                L.jamba_ssm_state_update.argtypes = [ctypes.POINTER(StateUpdateParams), _vp]
+                i32p, i64p = ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64)
+                L.jamba_ssm_scan_plan.restype = ctypes.c_int
+                L.jamba_ssm_scan_plan.argtypes = [ctypes.POINTER(ScanParams), i32p, i32p, i32p,
+                                                  i32p, i64p]
+                L.jamba_ssm_scan_variant_info.restype = ctypes.c_int
+                L.jamba_ssm_scan_variant_info.argtypes = [ctypes.c_int32] + [i32p] * 5
+                L.jamba_ssm_get_status.restype = ctypes.c_int
+                L.jamba_ssm_get_status.argtypes = [_vp]
+                L.jamba_ssm_last_cuda_error.restype = ctypes.c_int
+                L.jamba_ssm_last_cuda_error.argtypes = []
+                L.jamba_ssm_status_string.restype = ctypes.c_char_p
+                L.jamba_ssm_status_string.argtypes = [ctypes.c_int]
+                L.jamba_ssm_abi_version.restype = ctypes.c_int
+                L.jamba_ssm_abi_version.argtypes = []
+                _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().jamba_ssm_status_string(int(status)).decode()
+
+
+def new_scan_params(**kw) -> ScanParams:
+    p = ScanParams()
+    p.struct_size = ctypes.sizeof(ScanParams)
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def new_state_update_params(**kw) -> StateUpdateParams:
+    p = StateUpdateParams()
+    p.struct_size = ctypes.sizeof(StateUpdateParams)
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def call_scan(p: ScanParams, stream: int) -> int:
+    return lib().jamba_ssm_scan(ctypes.byref(p), _vp(stream or None))
+
+
+def call_state_update(p: StateUpdateParams, stream: int) -> int:
+    return lib().jamba_ssm_state_update(ctypes.byref(p), _vp(stream or None))
+
+
+def scan_plan(p: ScanParams):
+    v, g, cc, grid = (ctypes.c_int32() for _ in range(4))
+    tasks = ctypes.c_int64()
+    st = lib().jamba_ssm_scan_plan(ctypes.byref(p), ctypes.byref(v), ctypes.byref(g),
+                                   ctypes.byref(cc), ctypes.byref(grid), ctypes.byref(tasks))
+    if st != OK:
+        raise JambaSSMError(st, "jamba_ssm_scan_plan")
+    return dict(variant=v.value, lanes_per_channel=g.value, channels_per_cta=cc.value,
+                grid=grid.value, tasks=tasks.value)
+
+
+def variant_info(k: int):
+    vals = [ctypes.c_int32() for _ in range(5)]
+    st = lib().jamba_ssm_scan_variant_info(int(k), *[ctypes.byref(v) for v in vals])
+    if st != OK:
+        return None
+    keys = ("io_dtype", "d_state", "lanes_per_channel", "warps_per_cta", "time_tile")
+    return dict(zip(keys, (v.value for v in vals)))
+
+
+def get_status(stream: int) -> int:
+    return lib().jamba_ssm_get_status(_vp(stream or None))

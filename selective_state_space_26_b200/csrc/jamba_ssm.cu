@@ -1,0 +1,445 @@
+// jamba_ssm.cu -- host side of the C ABI declared in include/jamba_ssm.h:
+// argument validation, variant selection, TMA tensor-map encoding and the
+// launches of the S6 kernels.  Nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "jamba_ssm.h"
+#include "s6_scan.cuh"
+#include "s6_state_update.cuh"
+
+using jssm::ScanArgs;
+using jssm::UpdateArgs;
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+jamba_ssm_status cuda_fail(cudaError_t e) {
+    t_last_cuda_error = static_cast<int>(e);
+    return JAMBA_SSM_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ devices
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+    bool ready = false;
+    bool usable = false;
+    int sms = 0;
+};
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+// Returns the current device's info, or sets *st on failure.
+const DeviceInfo *current_device(jamba_ssm_status *st) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        *st = e == cudaSuccess ? JAMBA_SSM_ERR_NO_DEVICE : cuda_fail(e);
+        if (e != cudaSuccess && (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver))
+            *st = JAMBA_SSM_ERR_NO_DEVICE;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo &info = g_devices[dev];
+    if (!info.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) {
+            *st = cuda_fail(e);
+            return nullptr;
+        }
+        info.usable = (major == 10 && minor == 0);  // built for sm_100a only
+        info.sms = sms;
+        info.ready = true;
+    }
+    if (!info.usable) {
+        *st = JAMBA_SSM_ERR_NO_DEVICE;
+        return nullptr;
+    }
+    return &info;
+}
+
+// ---------------------------------------------------------- tensor maps (TMA)
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn(jamba_ssm_status *st) {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else if (err == cudaSuccess)
+            err = cudaErrorSymbolNotFound;
+    });
+    if (!fn) *st = cuda_fail(err);
+    return fn;
+}
+
+// 3-D map over [dim2][dim1][dim0] (dim0 innermost), box {box0, box1, 1}.
+bool encode_3d(EncodeTiledFn fn, CUtensorMap *map, const void *ptr, CUtensorMapDataType dt,
+               int elem_bytes, int64_t dim0, int64_t dim1, int64_t dim2, int box0, int box1) {
+    cuuint64_t dims[3] = {(cuuint64_t)dim0, (cuuint64_t)dim1, (cuuint64_t)dim2};
+    cuuint64_t strides[2] = {(cuuint64_t)(dim0 * elem_bytes), (cuuint64_t)(dim0 * dim1 * elem_bytes)};
+    cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ----------------------------------------------------------- scan variants
+struct ScanVariant {
+    int io_dtype, n, g, nw, tt;
+    int smem;
+    const void *kernel;
+    bool attr_set[kMaxDevices];
+};
+
+template <typename IoT, int N, int G, int NW, int TT, int S>
+ScanVariant make_variant() {
+    using Cfg = jssm::ScanCfg<IoT, N, G, NW, TT, S>;
+    ScanVariant v{};
+    v.io_dtype = std::is_same<IoT, float>::value ? JAMBA_SSM_F32 : JAMBA_SSM_BF16;
+    v.n = N;
+    v.g = G;
+    v.nw = NW;
+    v.tt = TT;
+    v.smem = Cfg::kSmemBytes;
+    v.kernel = reinterpret_cast<const void *>(&jssm::s6_scan_fwd_kernel<IoT, N, G, NW, TT, S>);
+    return v;
+}
+
+ScanVariant g_variants[] = {
+    make_variant<__nv_bfloat16, 16, 1, 4, 64, 3>(),   // 1: 128 channels / CTA, 1 lane each
+    make_variant<__nv_bfloat16, 16, 2, 4, 64, 3>(),   // 2:  64 channels, 2 lanes each
+    make_variant<__nv_bfloat16, 16, 2, 8, 64, 3>(),   // 3: 128 channels, 2 lanes each
+    make_variant<__nv_bfloat16, 16, 4, 8, 64, 3>(),   // 4:  64 channels, 4 lanes each
+    make_variant<__nv_bfloat16, 8, 1, 4, 64, 3>(),    // 5
+    make_variant<__nv_bfloat16, 8, 2, 4, 64, 3>(),    // 6
+    make_variant<float, 16, 1, 2, 32, 3>(),           // 7
+    make_variant<float, 8, 1, 2, 32, 3>(),            // 8
+    make_variant<float, 4, 1, 2, 32, 3>(),            // 9
+};
+constexpr int kNumVariants = sizeof(g_variants) / sizeof(g_variants[0]);
+
+int channels_per_cta(const ScanVariant &v) { return v.nw * (32 / v.g); }
+
+bool variant_applies(const ScanVariant &v, const jamba_ssm_scan_params *p) {
+    return v.io_dtype == p->io_dtype && v.n == p->d_state;
+}
+
+// Estimated relative time of a variant on `sms` SMs.  One CTA runs per SM and
+// loops over its share of the (sequence, channel-group) tasks; the busiest SM
+// decides, and its work is the channel-steps it owns divided over the warp
+// schedulers its warps occupy.
+double variant_cost(const ScanVariant &v, const jamba_ssm_scan_params *p, int sms) {
+    const int cc = channels_per_cta(v);
+    const int64_t tasks = p->batch * ((p->d_inner + cc - 1) / cc);
+    const int64_t per_cta = (tasks + sms - 1) / sms;
+    const int schedulers = v.nw < 4 ? v.nw : 4;
+    double cost = double(per_cta) * cc / schedulers;
+    // mild preference for fewer lanes per channel (less exchange work)
+    return cost * (1.0 + 0.04 * (v.g - 1));
+}
+
+int choose_variant(const jamba_ssm_scan_params *p, int sms) {
+    int best = -1;
+    double best_cost = 0;
+    for (int i = 0; i < kNumVariants; ++i) {
+        if (!variant_applies(g_variants[i], p)) continue;
+        const double c = variant_cost(g_variants[i], p, sms);
+        if (best < 0 || c < best_cost) {
+            best = i;
+            best_cost = c;
+        }
+    }
+    return best;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void *a, size_t an, const void *b, size_t bn) {
+    if (!a || !b || !an || !bn) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + bn && b0 < a0 + an;
+}
+
+constexpr int64_t kMaxElems = int64_t(1) << 40;
+
+jamba_ssm_status validate_scan(const jamba_ssm_scan_params *p) {
+    if (!p || p->struct_size < sizeof(jamba_ssm_scan_params)) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->batch < 0 || p->seqlen < 0 || p->d_inner < 1 || p->d_state < 1)
+        return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->io_dtype != JAMBA_SSM_BF16 && p->io_dtype != JAMBA_SSM_F32)
+        return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->batch > (int64_t(1) << 31) - 1 || p->seqlen > (int64_t(1) << 31) - 1 ||
+        p->d_inner > (int64_t(1) << 30))
+        return JAMBA_SSM_ERR_UNSUPPORTED;
+    if (p->batch && p->seqlen && p->batch * p->seqlen > kMaxElems / p->d_inner)
+        return JAMBA_SSM_ERR_UNSUPPORTED;
+    const int es = p->io_dtype == JAMBA_SSM_BF16 ? 2 : 4;
+    const bool n_ok = p->io_dtype == JAMBA_SSM_BF16 ? (p->d_state == 8 || p->d_state == 16)
+                                                    : (p->d_state == 4 || p->d_state == 8 ||
+                                                       p->d_state == 16);
+    if (!n_ok || (p->d_inner * es) % 16 != 0) return JAMBA_SSM_ERR_UNSUPPORTED;
+    if (p->kernel_variant < 0 || p->kernel_variant > kNumVariants) return JAMBA_SSM_ERR_UNSUPPORTED;
+    if (p->kernel_variant > 0 && !variant_applies(g_variants[p->kernel_variant - 1], p))
+        return JAMBA_SSM_ERR_UNSUPPORTED;
+    const int64_t tok = p->batch * p->seqlen;
+    const size_t state_bytes = size_t(p->batch) * p->d_inner * p->d_state * 4;
+    if (tok > 0) {
+        if (!p->x || !p->delta || !p->z || !p->B || !p->C || !p->A || !p->out)
+            return JAMBA_SSM_ERR_INVALID_ARG;
+        if (!aligned(p->x, 16) || !aligned(p->delta, 16) || !aligned(p->z, 16) ||
+            !aligned(p->B, 16) || !aligned(p->C, 16) || !aligned(p->out, 16) ||
+            !aligned(p->A, 16) || !aligned(p->D, 4) || !aligned(p->delta_bias, 4) ||
+            !aligned(p->h0, 16) || !aligned(p->h_final, 16))
+            return JAMBA_SSM_ERR_MISALIGNED;
+        const size_t act = size_t(tok) * p->d_inner * es, bc = size_t(tok) * p->d_state * es;
+        const void *ins[] = {p->x, p->delta, p->z, p->B, p->C};
+        const size_t insz[] = {act, act, act, bc, bc};
+        for (int i = 0; i < 5; ++i)
+            if (overlaps(p->out, act, ins[i], insz[i])) return JAMBA_SSM_ERR_INVALID_ARG;
+        if (overlaps(p->h_final, state_bytes, p->out, act)) return JAMBA_SSM_ERR_INVALID_ARG;
+    } else if (p->batch > 0 && p->seqlen == 0) {
+        if (!aligned(p->h0, 16) || !aligned(p->h_final, 16)) return JAMBA_SSM_ERR_MISALIGNED;
+    }
+    if (p->h0 && p->h_final && p->h0 != p->h_final &&
+        overlaps(p->h0, state_bytes, p->h_final, state_bytes))
+        return JAMBA_SSM_ERR_INVALID_ARG;
+    return JAMBA_SSM_OK;
+}
+
+struct ScanPlan {
+    int variant;  // index into g_variants
+    int grid;
+    int64_t tasks;
+};
+
+jamba_ssm_status plan_scan(const jamba_ssm_scan_params *p, const DeviceInfo *dev, ScanPlan *plan) {
+    const int vi = p->kernel_variant > 0 ? p->kernel_variant - 1 : choose_variant(p, dev->sms);
+    if (vi < 0) return JAMBA_SSM_ERR_UNSUPPORTED;
+    const ScanVariant &v = g_variants[vi];
+    const int cc = channels_per_cta(v);
+    plan->variant = vi;
+    plan->tasks = p->batch * ((p->d_inner + cc - 1) / cc);
+    const int64_t g = plan->tasks < dev->sms ? plan->tasks : dev->sms;
+    plan->grid = static_cast<int>(g < 1 ? 1 : g);
+    return JAMBA_SSM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *jamba_ssm_status_string(jamba_ssm_status s) {
+    switch (s) {
+        case JAMBA_SSM_OK: return "ok";
+        case JAMBA_SSM_ERR_INVALID_ARG: return "invalid argument";
+        case JAMBA_SSM_ERR_UNSUPPORTED: return "unsupported size, dtype or variant";
+        case JAMBA_SSM_ERR_MISALIGNED: return "misaligned pointer";
+        case JAMBA_SSM_ERR_CUDA: return "CUDA call failed";
+        case JAMBA_SSM_ERR_TIMEOUT: return "device-side bounded wait ran out";
+        case JAMBA_SSM_ERR_NO_DEVICE: return "no usable sm_100 device";
+    }
+    return "unknown status";
+}
+
+int jamba_ssm_last_cuda_error(void) { return t_last_cuda_error; }
+
+int jamba_ssm_abi_version(void) { return JAMBA_SSM_ABI_VERSION; }
+
+jamba_ssm_status jamba_ssm_scan_variant_info(int32_t k, int32_t *io_dtype, int32_t *d_state,
+                                             int32_t *lanes_per_channel, int32_t *warps_per_cta,
+                                             int32_t *time_tile) {
+    if (k < 1 || k > kNumVariants) return JAMBA_SSM_ERR_UNSUPPORTED;
+    const ScanVariant &v = g_variants[k - 1];
+    if (io_dtype) *io_dtype = v.io_dtype;
+    if (d_state) *d_state = v.n;
+    if (lanes_per_channel) *lanes_per_channel = v.g;
+    if (warps_per_cta) *warps_per_cta = v.nw;
+    if (time_tile) *time_tile = v.tt;
+    return JAMBA_SSM_OK;
+}
+
+jamba_ssm_status jamba_ssm_scan_plan(const jamba_ssm_scan_params *p, int32_t *variant,
+                                     int32_t *lanes_per_channel, int32_t *channels_per_cta_out,
+                                     int32_t *grid, int64_t *tasks) {
+    jamba_ssm_status st = validate_scan(p);
+    if (st != JAMBA_SSM_OK) return st;
+    const DeviceInfo *dev = current_device(&st);
+    if (!dev) return st;
+    ScanPlan plan;
+    if ((st = plan_scan(p, dev, &plan)) != JAMBA_SSM_OK) return st;
+    const ScanVariant &v = g_variants[plan.variant];
+    if (variant) *variant = plan.variant + 1;
+    if (lanes_per_channel) *lanes_per_channel = v.g;
+    if (channels_per_cta_out) *channels_per_cta_out = channels_per_cta(v);
+    if (grid) *grid = plan.grid;
+    if (tasks) *tasks = plan.tasks;
+    return JAMBA_SSM_OK;
+}
+
+jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream) {
+    jamba_ssm_status st = validate_scan(p);
+    if (st != JAMBA_SSM_OK) return st;
+    const DeviceInfo *dev = current_device(&st);
+    if (!dev) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t state_bytes = size_t(p->batch) * p->d_inner * p->d_state * 4;
+    if (p->batch == 0) return JAMBA_SSM_OK;
+    if (p->seqlen == 0) {  // no steps: the final state is the initial state
+        if (!p->h_final) return JAMBA_SSM_OK;
+        cudaError_t e = p->h0 ? (p->h0 == p->h_final
+                                     ? cudaSuccess
+                                     : cudaMemcpyAsync(p->h_final, p->h0, state_bytes,
+                                                       cudaMemcpyDeviceToDevice, s))
+                              : cudaMemsetAsync(p->h_final, 0, state_bytes, s);
+        return e == cudaSuccess ? JAMBA_SSM_OK : cuda_fail(e);
+    }
+
+    ScanPlan plan;
+    if ((st = plan_scan(p, dev, &plan)) != JAMBA_SSM_OK) return st;
+    ScanVariant &v = g_variants[plan.variant];
+    EncodeTiledFn fn = encode_fn(&st);
+    if (!fn) return st;
+
+    const int cc = channels_per_cta(v);
+    const int es = p->io_dtype == JAMBA_SSM_BF16 ? 2 : 4;
+    const CUtensorMapDataType dt =
+        p->io_dtype == JAMBA_SSM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    CUtensorMap maps[6];
+    const void *act_ptrs[4] = {p->x, p->delta, p->z, p->out};
+    const int act_idx[4] = {0, 1, 2, 5};
+    for (int i = 0; i < 4; ++i)
+        if (!encode_3d(fn, &maps[act_idx[i]], act_ptrs[i], dt, es, p->d_inner, p->seqlen, p->batch,
+                       cc, v.tt))
+            return JAMBA_SSM_ERR_UNSUPPORTED;
+    if (!encode_3d(fn, &maps[3], p->B, dt, es, p->d_state, p->seqlen, p->batch, (int)p->d_state, v.tt) ||
+        !encode_3d(fn, &maps[4], p->C, dt, es, p->d_state, p->seqlen, p->batch, (int)p->d_state, v.tt))
+        return JAMBA_SSM_ERR_UNSUPPORTED;
+
+    int devid = 0;
+    cudaGetDevice(&devid);
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!v.attr_set[devid]) {
+            cudaError_t e = cudaFuncSetAttribute(v.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 v.smem);
+            if (e != cudaSuccess) return cuda_fail(e);
+            v.attr_set[devid] = true;
+        }
+    }
+
+    ScanArgs args{};
+    args.batch = p->batch;
+    args.seqlen = p->seqlen;
+    args.d_inner = p->d_inner;
+    args.A = p->A;
+    args.D = p->D;
+    args.delta_bias = p->delta_bias;
+    args.h0 = p->h0;
+    args.h_final = p->h_final;
+    args.delta_softplus = p->delta_softplus != 0;
+    args.debug_flags = p->debug_flags;
+    args.timeout_cycles = p->timeout_cycles ? p->timeout_cycles : (uint64_t(1) << 31);
+
+    void *kargs[] = {&maps[0], &maps[1], &maps[2], &maps[3], &maps[4], &maps[5], &args};
+    cudaError_t e = cudaLaunchKernel(v.kernel, dim3(plan.grid), dim3(v.nw * 32), kargs,
+                                     static_cast<size_t>(v.smem), s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return JAMBA_SSM_OK;
+}
+
+jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, void *stream) {
+    if (!p || p->struct_size < sizeof(jamba_ssm_state_update_params)) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->batch < 0 || p->d_inner < 1 || p->d_state < 1) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->io_dtype != JAMBA_SSM_BF16 && p->io_dtype != JAMBA_SSM_F32) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->d_state != 4 && p->d_state != 8 && p->d_state != 16) return JAMBA_SSM_ERR_UNSUPPORTED;
+    if (p->batch > (int64_t(1) << 31) || p->d_inner > (int64_t(1) << 30)) return JAMBA_SSM_ERR_UNSUPPORTED;
+    if (p->batch == 0) return JAMBA_SSM_OK;
+    if (!p->state || !p->x || !p->delta || !p->z || !p->B || !p->C || !p->A || !p->out)
+        return JAMBA_SSM_ERR_INVALID_ARG;
+    const int es = p->io_dtype == JAMBA_SSM_BF16 ? 2 : 4;
+    if (!aligned(p->state, 16) || !aligned(p->A, 16) || !aligned(p->B, 16) || !aligned(p->C, 16) ||
+        !aligned(p->x, es) || !aligned(p->delta, es) || !aligned(p->z, es) || !aligned(p->out, es) ||
+        !aligned(p->D, 4) || !aligned(p->delta_bias, 4))
+        return JAMBA_SSM_ERR_MISALIGNED;
+    const size_t act = size_t(p->batch) * p->d_inner * es, bc = size_t(p->batch) * p->d_state * es;
+    const size_t sb = size_t(p->batch) * p->d_inner * p->d_state * 4;
+    const void *ins[] = {p->x, p->delta, p->z, p->B, p->C, p->state};
+    const size_t insz[] = {act, act, act, bc, bc, sb};
+    for (int i = 0; i < 6; ++i)
+        if (overlaps(p->out, act, ins[i], insz[i])) return JAMBA_SSM_ERR_INVALID_ARG;
+    for (int i = 0; i < 5; ++i)
+        if (overlaps(p->state, sb, ins[i], insz[i])) return JAMBA_SSM_ERR_INVALID_ARG;
+
+    jamba_ssm_status st;
+    const DeviceInfo *dev = current_device(&st);
+    if (!dev) return st;
+
+    UpdateArgs a{};
+    a.batch = p->batch;
+    a.d_inner = p->d_inner;
+    a.state = p->state;
+    a.x = p->x;
+    a.delta = p->delta;
+    a.z = p->z;
+    a.B = p->B;
+    a.C = p->C;
+    a.A = p->A;
+    a.D = p->D;
+    a.delta_bias = p->delta_bias;
+    a.out = p->out;
+    a.delta_softplus = p->delta_softplus != 0;
+    const int64_t threads = p->batch * p->d_inner * (p->d_state / 4);
+    const int64_t blocks = (threads + 255) / 256;
+    if (blocks > 0x7fffffff) return JAMBA_SSM_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool bf = p->io_dtype == JAMBA_SSM_BF16;
+    const void *k = nullptr;
+    switch (p->d_state) {
+        case 4: k = bf ? (const void *)&jssm::s6_state_update_kernel<__nv_bfloat16, 4>
+                       : (const void *)&jssm::s6_state_update_kernel<float, 4>; break;
+        case 8: k = bf ? (const void *)&jssm::s6_state_update_kernel<__nv_bfloat16, 8>
+                       : (const void *)&jssm::s6_state_update_kernel<float, 8>; break;
+        default: k = bf ? (const void *)&jssm::s6_state_update_kernel<__nv_bfloat16, 16>
+                        : (const void *)&jssm::s6_state_update_kernel<float, 16>; break;
+    }
+    void *kargs[] = {&a};
+    cudaError_t e = cudaLaunchKernel(k, dim3(static_cast<unsigned>(blocks)), dim3(256), kargs, 0, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return JAMBA_SSM_OK;
+}
+
+jamba_ssm_status jamba_ssm_get_status(void *stream) {
+    jamba_ssm_status st;
+    if (!current_device(&st)) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    int word = 0;
+    e = cudaMemcpyFromSymbol(&word, jssm::g_status_word, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (word != 0) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(jssm::g_status_word, &zero, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return static_cast<jamba_ssm_status>(word);
+}
+
+}  // extern "C"

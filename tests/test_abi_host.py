@@ -1,0 +1,168 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/jamba_ssm.h declares, its structures have the layout
+the binding assumes, and argument validation rejects bad calls before any CUDA
+work is enqueued (fake, never-dereferenced pointer values are enough)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from selective_state_space_26_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "jamba_ssm.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(jamba_ssm_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert set(names) == set(_lib.EXPORTS), names
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    for n in names:
+        assert n in exported, f"{n} declared in the header but not exported"
+        assert hasattr(L, n)
+
+
+def test_struct_layout_matches_header(tmp_path):
+    fields = {
+        "jamba_ssm_scan_params": _lib.ScanParams,
+        "jamba_ssm_state_update_params": _lib.StateUpdateParams,
+    }
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "jamba_ssm.h"',
+             "int main(void) {"]
+    for cname, cls in fields.items():
+        lines.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
+        for f, _ in cls._fields_:
+            lines.append(f'printf("{cname} {f} %zu\\n", offsetof({cname}, {f}));')
+    lines.append("return 0; }")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.dirname(HEADER), "-o", str(exe), str(src)], check=True)
+    got = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    for row in filter(None, got):
+        cname, f, v = row.split()
+        cls = fields[cname]
+        if f == "size":
+            assert ctypes.sizeof(cls) == int(v), cname
+        else:
+            assert getattr(cls, f).offset == int(v), (cname, f)
+
+
+def test_status_strings_and_version(L):
+    assert L.jamba_ssm_abi_version() == 1
+    for s in range(7):
+        assert _lib.status_string(s)
+    assert _lib.status_string(99) == "unknown status"
+
+
+def test_variant_table(L):
+    infos = []
+    k = 1
+    while (info := _lib.variant_info(k)) is not None:
+        infos.append(info)
+        k += 1
+    assert len(infos) >= 9
+    for i in infos:
+        assert i["d_state"] % (4 * i["lanes_per_channel"]) == 0
+        assert 32 % i["lanes_per_channel"] == 0
+        assert i["time_tile"] % i["lanes_per_channel"] == 0
+    assert _lib.variant_info(0) is None
+
+
+def _valid_scan(**kw):
+    base = dict(batch=2, seqlen=100, d_inner=256, d_state=16, io_dtype=_lib.BF16,
+                delta_softplus=1, x=0x10000000, delta=0x20000000, z=0x30000000,
+                B=0x40000000, C=0x50000000, A=0x60000000, D=0x70000000,
+                delta_bias=0x80000000, h0=None, out=0x90000000, h_final=0xA0000000)
+    base.update(kw)
+    return _lib.new_scan_params(**base)
+
+
+def _scan(p):
+    return _lib.call_scan(p, 0)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(batch=-1), _lib.ERR_INVALID_ARG),
+    (dict(seqlen=-5), _lib.ERR_INVALID_ARG),
+    (dict(d_inner=0), _lib.ERR_INVALID_ARG),
+    (dict(io_dtype=7), _lib.ERR_INVALID_ARG),
+    (dict(d_state=5), _lib.ERR_UNSUPPORTED),
+    (dict(d_state=4), _lib.ERR_UNSUPPORTED),          # bf16 rows of 8 bytes: not TMA-able
+    (dict(d_state=32), _lib.ERR_UNSUPPORTED),
+    (dict(d_inner=12), _lib.ERR_UNSUPPORTED),         # bf16 row not a multiple of 16 bytes
+    (dict(kernel_variant=99), _lib.ERR_UNSUPPORTED),
+    (dict(kernel_variant=7), _lib.ERR_UNSUPPORTED),   # an fp32 variant for bf16 data
+    (dict(x=None), _lib.ERR_INVALID_ARG),
+    (dict(A=None), _lib.ERR_INVALID_ARG),
+    (dict(out=None), _lib.ERR_INVALID_ARG),
+    (dict(x=0x10000002), _lib.ERR_MISALIGNED),
+    (dict(B=0x40000008), _lib.ERR_MISALIGNED),
+    (dict(h0=0xB0000004), _lib.ERR_MISALIGNED),
+    (dict(D=0x70000002), _lib.ERR_MISALIGNED),
+    (dict(out=0x10000000 + 64), _lib.ERR_INVALID_ARG),  # out overlaps x
+    (dict(h_final=0x90000000 + 1024), _lib.ERR_INVALID_ARG),  # h_final inside out
+    (dict(h0=0xA0000000 + 16), _lib.ERR_INVALID_ARG),  # h0 partially overlaps h_final
+    (dict(batch=1 << 20, seqlen=1 << 20, d_inner=1 << 12), _lib.ERR_UNSUPPORTED),
+    (dict(io_dtype=_lib.F32, d_state=2), _lib.ERR_UNSUPPORTED),
+    (dict(io_dtype=_lib.F32, d_inner=10), _lib.ERR_UNSUPPORTED),
+])
+def test_scan_argument_errors(L, kw, expect):
+    assert _scan(_valid_scan(**kw)) == expect
+
+
+def test_scan_struct_size_and_null(L):
+    p = _valid_scan()
+    p.struct_size = 8
+    assert _scan(p) == _lib.ERR_INVALID_ARG
+    assert L.jamba_ssm_scan(None, None) == _lib.ERR_INVALID_ARG
+    assert L.jamba_ssm_state_update(None, None) == _lib.ERR_INVALID_ARG
+
+
+def _valid_update(**kw):
+    base = dict(batch=4, d_inner=64, d_state=16, io_dtype=_lib.BF16, delta_softplus=1,
+                state=0x10000000, x=0x20000000, delta=0x30000000, z=0x40000000,
+                B=0x50000000, C=0x60000000, A=0x70000000, D=None, delta_bias=None,
+                out=0x80000000)
+    base.update(kw)
+    return _lib.new_state_update_params(**base)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(batch=-1), _lib.ERR_INVALID_ARG),
+    (dict(d_state=2), _lib.ERR_UNSUPPORTED),
+    (dict(d_state=12), _lib.ERR_UNSUPPORTED),
+    (dict(state=None), _lib.ERR_INVALID_ARG),
+    (dict(state=0x10000008), _lib.ERR_MISALIGNED),
+    (dict(x=0x20000001), _lib.ERR_MISALIGNED),
+    (dict(io_dtype=_lib.F32, x=0x20000002), _lib.ERR_MISALIGNED),
+    (dict(out=0x20000000), _lib.ERR_INVALID_ARG),     # out aliases x
+    (dict(out=0x10000000 + 256), _lib.ERR_INVALID_ARG),  # out inside the state
+])
+def test_state_update_argument_errors(L, kw, expect):
+    assert _lib.call_state_update(_valid_update(**kw), 0) == expect
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_device_reports_no_device(L):
+    assert _scan(_valid_scan()) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
+    assert _lib.call_state_update(_valid_update(), 0) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
+    p = _valid_scan(batch=0)
+    assert _scan(p) == _lib.OK or _scan(p) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)

@@ -1,0 +1,212 @@
+"""Parity of the CUDA prefill scan with the fp64 oracle (needs a B200).
+
+Every case runs through the C ABI (the Python binding only marshals pointers)
+on seeded synthetic inputs, copies the very same input tensors to the host for
+the oracle, and applies the comparison rules of tests/parity.py.
+"""
+import os
+
+import pytest
+import torch
+
+import oracle
+from selective_state_space_26_b200 import (JambaSSMError, jamba_ssm_get_status, jamba_ssm_scan,
+                                           synth)
+from selective_state_space_26_b200 import _lib
+from tests.parity import assert_out, assert_state
+
+pytestmark = pytest.mark.gpu
+THREADS = max(1, min(32, os.cpu_count() or 1))
+
+
+def _dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda", 0)
+
+
+def run_gpu(inp, variant=0, h0=None, out=None, h_final=None):
+    out, hf = jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, D=inp.D,
+                             delta_bias=inp.delta_bias, delta_softplus=inp.delta_softplus,
+                             h0=inp.h0 if h0 is None else h0, out=out, h_final=h_final,
+                             variant=variant)
+    torch.cuda.synchronize()
+    return out, hf
+
+
+def run_oracle(inp, channels=None):
+    sel = slice(None) if channels is None else channels
+    h0 = None if inp.h0 is None else inp.h0[:, sel]
+    return oracle.scan(inp.x[:, :, sel], inp.delta[:, :, sel], inp.z[:, :, sel], inp.B, inp.C,
+                       inp.A[sel], D=inp.D[sel], delta_bias=inp.delta_bias[sel],
+                       delta_softplus=inp.delta_softplus, h0=h0, threads=THREADS)
+
+
+def variants_for(dtype, n):
+    out = []
+    k = 1
+    while True:
+        info = _lib.variant_info(k)
+        if info is None:
+            return out
+        if info["io_dtype"] == (_lib.BF16 if dtype == torch.bfloat16 else _lib.F32) and \
+                info["d_state"] == n:
+            out.append(k)
+        k += 1
+
+
+def test_tiny_fp32_workload_matches_oracle():
+    dev = _dev()
+    w = synth.WORKLOADS["s6_tiny_fp32_b1_l64_d16_n4"]
+    inp = synth.workload_inputs(w, device=dev)
+    out, hf = run_gpu(inp)
+    ref, ref_h = run_oracle(inp)
+    assert_out(out, ref, torch.float32, "tiny fp32")
+    assert_state(hf, ref_h, torch.float32, "tiny fp32")
+
+
+@pytest.mark.parametrize("dtype,n", [(torch.bfloat16, 16), (torch.bfloat16, 8),
+                                     (torch.float32, 16), (torch.float32, 8),
+                                     (torch.float32, 4)])
+def test_every_variant_ragged_tiles(dtype, n):
+    """Several time tiles plus a ragged tail, a ragged channel group, two
+    sequences, a random (unstructured) A and a nonzero initial state."""
+    dev = _dev()
+    inp = synth.scan_inputs(2, 203, 200 if dtype == torch.bfloat16 else 196, n, dtype,
+                            seed=101, device=dev, h0_std=0.5, A_kind="random")
+    ref, ref_h = run_oracle(inp)
+    vs = variants_for(dtype, n)
+    assert vs, "no variant built for this dtype / d_state"
+    for v in [0] + vs:
+        out, hf = run_gpu(inp, variant=v)
+        assert_out(out, ref, dtype, f"variant {v}")
+        assert_state(hf, ref_h, dtype, f"variant {v}")
+
+
+@pytest.mark.parametrize("seqlen", [1, 2, 63, 64, 65, 129])
+def test_short_and_boundary_lengths(seqlen):
+    dev = _dev()
+    inp = synth.scan_inputs(3, seqlen, 136, 16, torch.bfloat16, seed=7, device=dev, h0_std=0.2)
+    ref, ref_h = run_oracle(inp)
+    for v in [0] + variants_for(torch.bfloat16, 16):
+        out, hf = run_gpu(inp, variant=v)
+        assert_out(out, ref, torch.bfloat16, f"L={seqlen} variant {v}")
+        assert_state(hf, ref_h, torch.bfloat16, f"L={seqlen} variant {v}")
+
+
+def test_empty_inputs():
+    dev = _dev()
+    inp = synth.scan_inputs(2, 0, 64, 16, torch.bfloat16, seed=3, device=dev, h0_std=1.0)
+    hf = torch.full((2, 64, 16), float("nan"), device=dev)
+    run_gpu(inp, h_final=hf)
+    assert torch.equal(hf, inp.h0)
+    inp0 = synth.scan_inputs(2, 0, 64, 16, torch.bfloat16, seed=3, device=dev)
+    run_gpu(inp0, h_final=hf)
+    assert not torch.any(hf)
+    inpb = synth.scan_inputs(0, 16, 64, 16, torch.bfloat16, seed=3, device=dev)
+    out, hfb = run_gpu(inpb)
+    assert out.numel() == 0 and hfb.numel() == 0
+
+
+def test_smaller_than_one_channel_tile():
+    dev = _dev()
+    inp = synth.scan_inputs(1, 70, 8, 16, torch.bfloat16, seed=5, device=dev)
+    ref, ref_h = run_oracle(inp)
+    for v in [0] + variants_for(torch.bfloat16, 16):
+        out, hf = run_gpu(inp, variant=v)
+        assert_out(out, ref, torch.bfloat16, f"d_inner=8 variant {v}")
+        assert_state(hf, ref_h, torch.bfloat16, f"d_inner=8 variant {v}")
+
+
+def test_delta_zero_limit_and_no_softplus():
+    dev = _dev()
+    inp = synth.scan_inputs(2, 77, 64, 16, torch.bfloat16, seed=9, device=dev, h0_std=1.0)
+    inp.delta.zero_()
+    inp.delta_bias.zero_()
+    inp.delta_softplus = False
+    out, hf = run_gpu(inp)
+    assert torch.equal(hf, inp.h0)  # Abar = 1, Bbar x = 0: state untouched, bit for bit
+    ref, _ = run_oracle(inp)
+    assert_out(out, ref, torch.bfloat16, "Delta=0")
+
+
+def test_split_scan_is_bitwise_whole_scan():
+    """Chunked prefill: scan(L1) then scan(L2, h0 = h_final) == scan(L1 + L2)."""
+    dev = _dev()
+    inp = synth.scan_inputs(2, 300, 256, 16, torch.bfloat16, seed=11, device=dev, h0_std=0.3)
+    whole, hw = run_gpu(inp)
+    for cut in (1, 64, 100):
+        a = synth.ScanInputs(inp.x[:, :cut].contiguous(), inp.delta[:, :cut].contiguous(),
+                             inp.z[:, :cut].contiguous(), inp.B[:, :cut].contiguous(),
+                             inp.C[:, :cut].contiguous(), inp.A, inp.D, inp.delta_bias, inp.h0)
+        b = synth.ScanInputs(inp.x[:, cut:].contiguous(), inp.delta[:, cut:].contiguous(),
+                             inp.z[:, cut:].contiguous(), inp.B[:, cut:].contiguous(),
+                             inp.C[:, cut:].contiguous(), inp.A, inp.D, inp.delta_bias, None)
+        o1, h1 = run_gpu(a)
+        o2, h2 = run_gpu(b, h0=h1)
+        assert torch.equal(torch.cat([o1, o2], dim=1), whole), cut
+        assert torch.equal(h2, hw), cut
+
+
+def test_resume_in_place():
+    dev = _dev()
+    inp = synth.scan_inputs(1, 50, 64, 16, torch.bfloat16, seed=12, device=dev, h0_std=0.3)
+    _, expect = run_gpu(inp)
+    st = inp.h0.clone()
+    run_gpu(inp, h0=st, h_final=st)
+    assert torch.equal(st, expect)
+
+
+def test_deterministic():
+    dev = _dev()
+    inp = synth.scan_inputs(2, 150, 256, 16, torch.bfloat16, seed=13, device=dev)
+    o1, h1 = run_gpu(inp)
+    o2, h2 = run_gpu(inp)
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
+
+def test_large_activation_range():
+    """Activations 1e3-1e4 (the pages report layer outputs up to ~4e6 before
+    the activation penalty): nothing overflows in the fp32 path."""
+    dev = _dev()
+    inp = synth.scan_inputs(1, 130, 64, 16, torch.bfloat16, seed=14, device=dev)
+    inp.x.mul_(2048.0)
+    ref, ref_h = run_oracle(inp)
+    out, hf = run_gpu(inp)
+    assert torch.isfinite(out.float()).all()
+    assert_out(out / 2048.0, ref / 2048.0, torch.bfloat16, "x scaled by 2048")
+    assert_state(hf, ref_h, torch.bfloat16, "x scaled by 2048")
+
+
+def test_argument_errors_do_not_launch():
+    dev = _dev()
+    inp = synth.scan_inputs(1, 16, 64, 16, torch.bfloat16, seed=15, device=dev)
+    with pytest.raises(JambaSSMError) as e:  # out overlaps x
+        jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, out=inp.x)
+    assert e.value.status == _lib.ERR_INVALID_ARG
+    with pytest.raises(JambaSSMError) as e:  # variant built for another d_state
+        jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A,
+                       variant=variants_for(torch.bfloat16, 8)[0])
+    assert e.value.status == _lib.ERR_UNSUPPORTED
+    buf = torch.zeros(16 * 64 + 8, dtype=torch.bfloat16, device=dev)
+    x8 = buf[1:1 + 16 * 64].view(1, 16, 64)  # 2-byte offset: not 16-byte aligned
+    with pytest.raises(JambaSSMError) as e:
+        jamba_ssm_scan(x8, inp.delta, inp.z, inp.B, inp.C, inp.A)
+    assert e.value.status == _lib.ERR_MISALIGNED
+    assert jamba_ssm_get_status() == _lib.OK
+
+
+def test_bounded_wait_times_out_and_reports():
+    """A tile load that never arrives (withheld on purpose) makes the bounded
+    mbarrier wait run out: the kernel records TIMEOUT and returns; the context
+    stays usable and the next call is correct."""
+    dev = _dev()
+    inp = synth.scan_inputs(1, 200, 128, 16, torch.bfloat16, seed=16, device=dev)
+    assert jamba_ssm_get_status() == _lib.OK
+    jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, D=inp.D,
+                   delta_bias=inp.delta_bias, debug_flags=1, timeout_cycles=2_000_000)
+    assert jamba_ssm_get_status() == _lib.ERR_TIMEOUT
+    assert jamba_ssm_get_status() == _lib.OK  # read-and-clear
+    ref, _ = run_oracle(inp)
+    out, _ = run_gpu(inp)
+    assert_out(out, ref, torch.bfloat16, "after timeout")
