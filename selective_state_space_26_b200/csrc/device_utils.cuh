@@ -65,6 +65,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Bounded wait on an mbarrier phase that also gives up as soon as *abort is
+// set by another thread of the CTA.  Returns false on either.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, uint64_t limit,
+                                                   const volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long start = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (static_cast<uint64_t>(clock64() - start) > limit) return false;
+    }
+}
+
 // Bounded wait on an mbarrier phase.  Returns false if `limit` SM clock cycles
 // pass without the phase completing (the caller records the timeout and winds
 // the CTA down without touching the barrier again).
