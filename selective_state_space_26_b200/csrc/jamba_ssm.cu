@@ -9,6 +9,7 @@
 
 #include "jamba_ssm.h"
 #include "s6_scan.cuh"
+#include "s6_scan_fused.cuh"
 #include "s6_state_update.cuh"
 
 using jssm::ScanArgs;
@@ -102,47 +103,49 @@ bool encode_3d(EncodeTiledFn fn, CUtensorMap *map, const void *ptr, CUtensorMapD
 
 // ----------------------------------------------------------- scan variants
 struct ScanVariant {
-    int io_dtype, n, g, nwb, nws, tt;
+    int io_dtype, n, g, nw, tt;
+    int threads;
     double step_cost;  // measured time per channel-step, relative (multi-task steady state)
     int smem;
     const void *kernel;
     bool attr_set[kMaxDevices];
 };
 
-template <typename IoT, int N, int G, int NWB, int NWS, int TT, int S>
-ScanVariant make_variant(double step_cost) {
-    using Cfg = jssm::ScanCfg<IoT, N, G, NWB, NWS, TT, S>;
+// NW compute warps (each does its channels' recurrence, softplus and gate) and
+// one producer warp (TMA, B/C widening).
+template <typename IoT, int N, int G, int NW, int TT, int S>
+ScanVariant make_fused(double step_cost) {
+    using Cfg = jssm::FusedCfg<IoT, N, G, NW, TT, S>;
     ScanVariant v{};
     v.io_dtype = std::is_same<IoT, float>::value ? JAMBA_SSM_F32 : JAMBA_SSM_BF16;
     v.n = N;
     v.g = G;
-    v.nwb = NWB;
-    v.nws = NWS;
+    v.nw = NW;
     v.tt = TT;
+    v.threads = (NW + 1) * 32;
     v.step_cost = step_cost;
     v.smem = Cfg::kSmemBytes;
-    v.kernel = reinterpret_cast<const void *>(&jssm::s6_scan_fwd_kernel<IoT, N, G, NWB, NWS, TT, S>);
+    v.kernel = reinterpret_cast<const void *>(&jssm::s6_scan_fused_kernel<IoT, N, G, NW, TT, S>);
     return v;
 }
 
-// <io type, d_state, lanes per channel, recurrence warps, scalar warps, time tile,
-//  TMA stages>(relative time per channel-step, measured on B200 at Jamba's sizes)
+// <io type, d_state, lanes per channel, compute warps, time tile, TMA stages>
+// (relative time per channel-step in the multi-task steady state, measured on
+// B200 at Jamba's sizes; used by the launch-shape choice below)
 ScanVariant g_variants[] = {
-    make_variant<__nv_bfloat16, 16, 2, 4, 4, 32, 4>(1.50),   // 1:  64 channels / CTA
-    make_variant<__nv_bfloat16, 16, 4, 8, 4, 32, 4>(1.60),   // 2:  64 channels / CTA
-    make_variant<__nv_bfloat16, 16, 4, 8, 8, 32, 4>(1.15),   // 3:  64 channels / CTA
-    make_variant<__nv_bfloat16, 16, 2, 8, 4, 32, 3>(1.10),   // 4: 128 channels / CTA
-    make_variant<__nv_bfloat16, 16, 2, 8, 8, 32, 3>(1.00),   // 5: 128 channels / CTA
-    make_variant<__nv_bfloat16, 16, 1, 4, 4, 32, 3>(1.25),   // 6: 128 channels / CTA
-    make_variant<__nv_bfloat16, 8, 2, 4, 4, 32, 4>(1.00),    // 7:  64 channels / CTA
-    make_variant<__nv_bfloat16, 8, 1, 4, 4, 32, 3>(1.00),    // 8: 128 channels / CTA
-    make_variant<float, 16, 1, 2, 2, 32, 3>(1.00),           // 9:  64 channels / CTA
-    make_variant<float, 8, 1, 2, 2, 32, 3>(1.00),            // 10
-    make_variant<float, 4, 1, 2, 2, 32, 3>(1.00),            // 11
+    make_fused<__nv_bfloat16, 16, 2, 8, 32, 4>(1.00),   // 1: 128 channels / CTA
+    make_fused<__nv_bfloat16, 16, 4, 8, 32, 4>(1.37),   // 2:  64 channels / CTA
+    make_fused<__nv_bfloat16, 16, 2, 4, 32, 4>(1.78),   // 3:  64 channels / CTA
+    make_fused<__nv_bfloat16, 16, 1, 4, 32, 4>(1.70),   // 4: 128 channels / CTA
+    make_fused<__nv_bfloat16, 8, 2, 8, 32, 4>(1.00),    // 5: 128 channels / CTA
+    make_fused<__nv_bfloat16, 8, 1, 4, 32, 4>(1.00),    // 6: 128 channels / CTA
+    make_fused<float, 16, 1, 2, 32, 3>(1.00),           // 7:  64 channels / CTA
+    make_fused<float, 8, 1, 2, 32, 3>(1.00),            // 8:  64 channels / CTA
+    make_fused<float, 4, 1, 2, 32, 3>(1.00),            // 9:  64 channels / CTA
 };
 constexpr int kNumVariants = sizeof(g_variants) / sizeof(g_variants[0]);
 
-int channels_per_cta(const ScanVariant &v) { return v.nwb * (32 / v.g); }
+int channels_per_cta(const ScanVariant &v) { return v.nw * (32 / v.g); }
 
 bool variant_applies(const ScanVariant &v, const jamba_ssm_scan_params *p) {
     return v.io_dtype == p->io_dtype && v.n == p->d_state;
@@ -274,7 +277,7 @@ jamba_ssm_status jamba_ssm_scan_variant_info(int32_t k, int32_t *io_dtype, int32
     if (io_dtype) *io_dtype = v.io_dtype;
     if (d_state) *d_state = v.n;
     if (lanes_per_channel) *lanes_per_channel = v.g;
-    if (warps_per_cta) *warps_per_cta = v.nwb + v.nws + 1;
+    if (warps_per_cta) *warps_per_cta = v.threads / 32;
     if (time_tile) *time_tile = v.tt;
     return JAMBA_SSM_OK;
 }
@@ -362,7 +365,7 @@ jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream) {
     args.timeout_cycles = p->timeout_cycles ? p->timeout_cycles : (uint64_t(1) << 31);
 
     void *kargs[] = {&maps[0], &maps[1], &maps[2], &maps[3], &maps[4], &maps[5], &args};
-    cudaError_t e = cudaLaunchKernel(v.kernel, dim3(plan.grid), dim3((v.nwb + v.nws + 1) * 32), kargs,
+    cudaError_t e = cudaLaunchKernel(v.kernel, dim3(plan.grid), dim3(v.threads), kargs,
                                      static_cast<size_t>(v.smem), s);
     if (e != cudaSuccess) return cuda_fail(e);
     return JAMBA_SSM_OK;

@@ -109,7 +109,7 @@ def _scan(p):
     (dict(d_state=32), _lib.ERR_UNSUPPORTED),
     (dict(d_inner=12), _lib.ERR_UNSUPPORTED),         # bf16 row not a multiple of 16 bytes
     (dict(kernel_variant=99), _lib.ERR_UNSUPPORTED),
-    (dict(kernel_variant=9), _lib.ERR_UNSUPPORTED),   # an fp32 variant for bf16 data
+    (dict(kernel_variant=7), _lib.ERR_UNSUPPORTED),   # an fp32 variant for bf16 data
     (dict(x=None), _lib.ERR_INVALID_ARG),
     (dict(A=None), _lib.ERR_INVALID_ARG),
     (dict(out=None), _lib.ERR_INVALID_ARG),
