@@ -412,22 +412,52 @@ jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, 
     a.delta_bias = p->delta_bias;
     a.out = p->out;
     a.delta_softplus = p->delta_softplus != 0;
-    const int64_t threads = p->batch * p->d_inner * (p->d_state / 4);
-    const int64_t blocks = (threads + 255) / 256;
-    if (blocks > 0x7fffffff) return JAMBA_SSM_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool bf = p->io_dtype == JAMBA_SSM_BF16;
+    // Streaming kernel when every slice is a whole number of 16-byte chunks.
+    const bool stream_ok = (p->d_inner * es) % 16 == 0 && (p->d_state * es) % 16 == 0 &&
+                           aligned(p->x, 16) && aligned(p->delta, 16) && aligned(p->z, 16);
+    if (stream_ok) {
+        constexpr int kCPB = 64, kBPC = 16, kS = 4;
+        const int64_t gx = (p->d_inner + kCPB - 1) / kCPB, gy = (p->batch + kBPC - 1) / kBPC;
+        if (gx > 0x7fffffff || gy > 65535) return JAMBA_SSM_ERR_UNSUPPORTED;
+        const void *k = nullptr;
+        int threads = 0, smem = 0;
+#define JSSM_STREAM(T, NN)                                                                    \
+    do {                                                                                      \
+        k = (const void *)&jssm::s6_state_update_stream_kernel<T, NN, kCPB, kBPC, kS>;        \
+        threads = kCPB * (NN / 4);                                                            \
+        smem = jssm::UpdateCfg<T, NN, kCPB, kS>::kSmemBytes;                                  \
+    } while (0)
+        switch (p->d_state) {
+            case 4: JSSM_STREAM(float, 4); break;  // bf16 rows of 4 states are not 16 bytes
+            case 8: if (bf) JSSM_STREAM(__nv_bfloat16, 8); else JSSM_STREAM(float, 8); break;
+            default: if (bf) JSSM_STREAM(__nv_bfloat16, 16); else JSSM_STREAM(float, 16); break;
+        }
+#undef JSSM_STREAM
+        uint64_t limit = uint64_t(1) << 31;
+        void *kargs[] = {&a, &limit};
+        cudaError_t e = cudaLaunchKernel(k, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
+                                         dim3(threads), kargs, static_cast<size_t>(smem), s);
+        if (e != cudaSuccess) return cuda_fail(e);
+        return JAMBA_SSM_OK;
+    }
+    constexpr int kBPC = 2;  // requests per block (parameters reused across them)
+    const int64_t cpb = 256 / (p->d_state / 4);
+    const int64_t gx = (p->d_inner + cpb - 1) / cpb, gy = (p->batch + kBPC - 1) / kBPC;
+    if (gx > 0x7fffffff || gy > 65535) return JAMBA_SSM_ERR_UNSUPPORTED;
     const void *k = nullptr;
     switch (p->d_state) {
-        case 4: k = bf ? (const void *)&jssm::s6_state_update_kernel<__nv_bfloat16, 4>
-                       : (const void *)&jssm::s6_state_update_kernel<float, 4>; break;
-        case 8: k = bf ? (const void *)&jssm::s6_state_update_kernel<__nv_bfloat16, 8>
-                       : (const void *)&jssm::s6_state_update_kernel<float, 8>; break;
-        default: k = bf ? (const void *)&jssm::s6_state_update_kernel<__nv_bfloat16, 16>
-                        : (const void *)&jssm::s6_state_update_kernel<float, 16>; break;
+        case 4: k = bf ? (const void *)&jssm::s6_state_update_kernel<__nv_bfloat16, 4, kBPC>
+                       : (const void *)&jssm::s6_state_update_kernel<float, 4, kBPC>; break;
+        case 8: k = bf ? (const void *)&jssm::s6_state_update_kernel<__nv_bfloat16, 8, kBPC>
+                       : (const void *)&jssm::s6_state_update_kernel<float, 8, kBPC>; break;
+        default: k = bf ? (const void *)&jssm::s6_state_update_kernel<__nv_bfloat16, 16, kBPC>
+                        : (const void *)&jssm::s6_state_update_kernel<float, 16, kBPC>; break;
     }
     void *kargs[] = {&a};
-    cudaError_t e = cudaLaunchKernel(k, dim3(static_cast<unsigned>(blocks)), dim3(256), kargs, 0, s);
+    cudaError_t e = cudaLaunchKernel(k, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
+                                     dim3(256), kargs, 0, s);
     if (e != cudaSuccess) return cuda_fail(e);
     return JAMBA_SSM_OK;
 }

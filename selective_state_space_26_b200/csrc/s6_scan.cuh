@@ -14,7 +14,6 @@
 
 namespace jssm {
 
-__device__ int g_status_word;  // sticky device-side status (0 = ok)
 
 struct ScanArgs {
     int64_t batch, seqlen, d_inner;
