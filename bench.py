@@ -150,6 +150,27 @@ class ClockSampler:
                 "samples": len(self.samples), "reasons": names}
 
 
+# ------------------------------------------------------------- ranks
+def max_over_ranks(vals, world, device):
+    """Element-wise max of per-rank timings (the job ends when its slowest
+    rank ends); a plain copy at world size 1."""
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_tokens_per_s(tokens_per_rank, world, seconds):
+    """Whole-job throughput of N independent replicas (weak scaling)."""
+    return tokens_per_rank * world / seconds
+
+
+def replica_seq_offset(rank, batch):
+    """First sequence index of this rank's replica: rank r scans sequences
+    r*batch .. r*batch+batch-1 of the workload's seeded stream."""
+    return rank * batch
+
+
 # ------------------------------------------------------------- our arm
 def time_e2e(e2e_step, tokens, world, k_e2e, h2d, d2h, dev, stream):
     """Whole-step time through the public API with host<->device copies of
@@ -165,10 +186,8 @@ def time_e2e(e2e_step, tokens, world, k_e2e, h2d, d2h, dev, stream):
         e2e_step()
     b.record(stream)
     torch.cuda.synchronize(dev)
-    t_e2e = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t_e2e, op=torch.distributed.ReduceOp.MAX)
-    return {"value": tokens * world * k_e2e / (float(t_e2e[0]) / 1e3), "unit": "tokens/s",
+    (t_e2e,) = max_over_ranks([a.elapsed_time(b)], world, dev)
+    return {"value": job_tokens_per_s(tokens * k_e2e, world, t_e2e / 1e3), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": k_e2e}
 
 
@@ -187,7 +206,7 @@ def run_ours(args, rank, world, local_rank):
     sms = props.multi_processor_count
 
     if w.kind == "prefill":
-        inp = synth.workload_inputs(w, device=dev, seq_offset=rank * w.batch)
+        inp = synth.workload_inputs(w, device=dev, seq_offset=replica_seq_offset(rank, w.batch))
         nxt = synth.decode_step(w.batch, w.d_inner, w.d_state, 0, w.seed, w.dtype, dev)
         out = torch.empty_like(inp.x)
         hf = torch.empty(w.batch, w.d_inner, w.d_state, dtype=torch.float32, device=dev)
@@ -201,7 +220,7 @@ def run_ours(args, rank, world, local_rank):
             jssm.jamba_ssm_state_update(hf, nxt.x, nxt.delta, nxt.z, nxt.B, nxt.C, inp.A,
                                         D=inp.D, delta_bias=inp.delta_bias, out=dec_out)
         launches_per_step = 2
-        dom_name = "s6_scan_fwd_kernel"
+        dom_name = "s6_scan_fused_kernel"
         dom_bytes = prefill_bytes(w.batch, w.seqlen, w.d_inner, w.d_state, io_bytes)
         plan = jssm.scan_plan(inp.x, inp.A)
     else:
@@ -253,10 +272,7 @@ def run_ours(args, rank, world, local_rank):
     dom_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in evs)
     if w.kind == "decode":
         dom_ms = step_ms
-    times = torch.tensor([step_ms, dom_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    step_ms, dom_ms = float(times[0]), float(times[1])
+    step_ms, dom_ms = max_over_ranks([step_ms, dom_ms], world, dev)
     ms_per_step = step_ms / args.steps
     dom_launch_s = dom_ms / args.steps / 1e3
 
@@ -331,7 +347,7 @@ def run_ours(args, rank, world, local_rank):
 
     line = {
         "metric": "selective-scan tokens/s & HBM GB/s (fraction of roofline) at d_inner=8192, N=16",
-        "value": tokens * world / (ms_per_step / 1e3),
+        "value": job_tokens_per_s(tokens, world, ms_per_step / 1e3),
         "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",

@@ -130,10 +130,13 @@ jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream);
  * d_inner >= 1 and d_state in {4, 8, 16} for both dtypes.
  * Pointers (device):
  *   state      [batch, d_inner, d_state] fp32, 16-byte aligned, read + written.
- *   x, delta, z, out [batch, d_inner] io_dtype (naturally aligned); out must
- *              not overlap an input.
- *   B, C       [batch, d_state] io_dtype (naturally aligned).
- *   A          [d_inner, d_state] fp32, 16-byte aligned; D, delta_bias as above.
+ *   x, delta, z, out [batch, d_inner] io_dtype, aligned to the element size;
+ *              out must not overlap an input.  (When x, delta and z are
+ *              16-byte aligned and the rows are multiples of 16 bytes, a
+ *              bulk-copy kernel is used; otherwise a plain-load kernel.)
+ *   B, C       [batch, d_state] io_dtype, 16-byte aligned.
+ *   A          [d_inner, d_state] fp32, 16-byte aligned; D, delta_bias as above
+ *              (4-byte aligned or NULL).
  */
 typedef struct jamba_ssm_state_update_params {
     size_t struct_size;          /* = sizeof(jamba_ssm_state_update_params)    */

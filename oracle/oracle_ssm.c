@@ -19,7 +19,7 @@
  *   - same lesson, "Mamba-3" item 2: Mamba's state matrix is real diagonal, so
  *     every (channel d, state n) pair is an independent scalar recurrence.
  * The pages print only the symbols Abar, Bbar.  Readings taken where they are
- * silent (all listed in the design doc):
+ * silent:
  *   - discretisation: Abar = exp(Delta * A[d,n]),  Bbar x = Delta * B[t,n] * x;
  *   - Delta = softplus(delta + delta_bias[d]) when delta_softplus != 0, else
  *     Delta = delta + delta_bias[d];
