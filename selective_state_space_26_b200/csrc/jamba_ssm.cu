@@ -103,7 +103,7 @@ bool encode_3d(EncodeTiledFn fn, CUtensorMap *map, const void *ptr, CUtensorMapD
 
 // ----------------------------------------------------------- scan variants
 struct ScanVariant {
-    int io_dtype, n, g, nw, tt;
+    int io_dtype, n, g, nw, tt, cw;
     int threads;
     double step_cost;  // measured time per channel-step, relative (multi-task steady state)
     int smem;
@@ -122,6 +122,7 @@ ScanVariant make_fused(double step_cost) {
     v.g = G;
     v.nw = NW;
     v.tt = TT;
+    v.cw = Cfg::CW;
     v.threads = (NW + 1) * 32;
     v.step_cost = step_cost;
     v.smem = Cfg::kSmemBytes;
@@ -130,22 +131,26 @@ ScanVariant make_fused(double step_cost) {
 }
 
 // <io type, d_state, lanes per channel, compute warps, time tile, TMA stages>
-// (relative time per channel-step in the multi-task steady state, measured on
-// B200 at Jamba's sizes; used by the launch-shape choice below)
+// with the relative time per channel-step each variant sustains when every SM
+// is busy (measured on B200 at Jamba's sizes, bf16 I/O; the fp32 ones serve
+// small and test shapes).  Fewer lanes per channel cost less per step; more
+// lanes give narrower CTAs, so a single sequence's 8192 channels still cover
+// the 148 SMs (56 channels per CTA -> 147 CTAs).
 ScanVariant g_variants[] = {
-    make_fused<__nv_bfloat16, 16, 2, 8, 32, 4>(1.00),   // 1: 128 channels / CTA
-    make_fused<__nv_bfloat16, 16, 4, 8, 32, 4>(1.37),   // 2:  64 channels / CTA
-    make_fused<__nv_bfloat16, 16, 2, 4, 32, 4>(1.78),   // 3:  64 channels / CTA
-    make_fused<__nv_bfloat16, 16, 1, 4, 32, 4>(1.70),   // 4: 128 channels / CTA
+    make_fused<__nv_bfloat16, 16, 2, 8, 64, 2>(1.00),   // 1: 128 channels / CTA
+    make_fused<__nv_bfloat16, 16, 4, 7, 64, 3>(1.29),   // 2:  56 channels / CTA
+    make_fused<__nv_bfloat16, 16, 4, 8, 64, 3>(1.31),   // 3:  64 channels / CTA
+    make_fused<__nv_bfloat16, 16, 4, 7, 32, 4>(1.43),   // 4:  56 channels / CTA
     make_fused<__nv_bfloat16, 8, 2, 8, 32, 4>(1.00),    // 5: 128 channels / CTA
-    make_fused<__nv_bfloat16, 8, 1, 4, 32, 4>(1.00),    // 6: 128 channels / CTA
-    make_fused<float, 16, 1, 2, 32, 3>(1.00),           // 7:  64 channels / CTA
-    make_fused<float, 8, 1, 2, 32, 3>(1.00),            // 8:  64 channels / CTA
-    make_fused<float, 4, 1, 2, 32, 3>(1.00),            // 9:  64 channels / CTA
+    make_fused<__nv_bfloat16, 8, 1, 4, 32, 4>(1.70),    // 6: 128 channels / CTA
+    make_fused<__nv_bfloat16, 8, 4, 7, 64, 3>(1.29),    // 7:  56 channels / CTA
+    make_fused<float, 16, 1, 2, 32, 3>(1.00),           // 8:  64 channels / CTA
+    make_fused<float, 8, 1, 2, 32, 3>(1.00),            // 9:  64 channels / CTA
+    make_fused<float, 4, 1, 2, 32, 3>(1.00),            // 10: 64 channels / CTA
 };
 constexpr int kNumVariants = sizeof(g_variants) / sizeof(g_variants[0]);
 
-int channels_per_cta(const ScanVariant &v) { return v.nw * (32 / v.g); }
+int channels_per_cta(const ScanVariant &v) { return v.nw * v.cw; }
 
 bool variant_applies(const ScanVariant &v, const jamba_ssm_scan_params *p) {
     return v.io_dtype == p->io_dtype && v.n == p->d_state;

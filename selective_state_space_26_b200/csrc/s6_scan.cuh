@@ -24,20 +24,83 @@ struct ScanArgs {
     uint64_t timeout_cycles;
 };
 
-// Widen 16 bytes of B or C to floats.
-__device__ __forceinline__ void widen16(const uint4 v, const __nv_bfloat16 *, float (&f)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// Staged B / C of one step.  The producer lays each step out in fp32 as G
+// slots, one per lane of a channel: slot s holds the NS values of B and then
+// the NS values of C that lane s's states use ([G][2][NS] floats), so a lane
+// reads its slot with NS / 2 16-byte loads and gets B and C already paired
+// for the packed fp32x2 math.
+template <int NS>
+struct BCPairs {
+    float2 b[NS / 2], c[NS / 2];
+};
+
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+template <int NS>
+__device__ __forceinline__ BCPairs<NS> load_bc(const float *row, int sub) {
+    const float4 *p = reinterpret_cast<const float4 *>(row + sub * 2 * NS);
+    float f[2 * NS];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    for (int q = 0; q < NS / 2; ++q) {
+        const float4 v = p[q];
+        f[4 * q] = v.x;
+        f[4 * q + 1] = v.y;
+        f[4 * q + 2] = v.z;
+        f[4 * q + 3] = v.w;
+    }
+    BCPairs<NS> r;
+#pragma unroll
+    for (int i = 0; i < NS / 2; ++i) {
+        r.b[i] = make_float2(f[2 * i], f[2 * i + 1]);
+        r.c[i] = make_float2(f[NS + 2 * i], f[NS + 2 * i + 1]);
+    }
+    return r;
+}
+
+// One B or C slice of NS values from the TMA tile into its staged slot: a
+// copy when both have the same type, else bf16 widened to fp32.
+template <int NS>
+__device__ __forceinline__ void stage_slice(float *dst, const __nv_bfloat16 *src) {
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(src);
+    float f[NS];
+#pragma unroll
+    for (int i = 0; i < NS / 2; ++i) {
+        const float2 v = bf16x2_to_f2(w[i]);
+        f[2 * i] = v.x;
+        f[2 * i + 1] = v.y;
+    }
+    if constexpr (NS % 4 == 0) {
+#pragma unroll
+        for (int q = 0; q < NS / 4; ++q)
+            reinterpret_cast<float4 *>(dst)[q] =
+                make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
+    } else {
+        static_assert(NS == 2, "slices of 2 or 4k values");
+        *reinterpret_cast<float2 *>(dst) = make_float2(f[0], f[1]);
     }
 }
-__device__ __forceinline__ void widen16(const uint4 v, const float *, float (&f)[4]) {
-    f[0] = __uint_as_float(v.x);
-    f[1] = __uint_as_float(v.y);
-    f[2] = __uint_as_float(v.z);
-    f[3] = __uint_as_float(v.w);
+
+// Copy of W 32-bit words with the widest aligned vector accesses.
+template <int W>
+__device__ __forceinline__ void copy_words(uint32_t *dst, const uint32_t *src) {
+    if constexpr (W % 4 == 0) {
+#pragma unroll
+        for (int q = 0; q < W / 4; ++q)
+            reinterpret_cast<uint4 *>(dst)[q] = reinterpret_cast<const uint4 *>(src)[q];
+    } else if constexpr (W == 2) {
+        *reinterpret_cast<uint2 *>(dst) = *reinterpret_cast<const uint2 *>(src);
+    } else {
+        static_assert(W == 1, "slice of 1, 2 or 4k words");
+        *dst = *src;
+    }
+}
+
+template <int NS, typename T>
+__device__ __forceinline__ void stage_slice(T *dst, const T *src) {
+    copy_words<NS * (int)sizeof(T) / 4>(reinterpret_cast<uint32_t *>(dst),
+                                        reinterpret_cast<const uint32_t *>(src));
 }
 
 // Sum of v over the G lanes of a channel.  Partners are taken in the order
@@ -74,31 +137,33 @@ __device__ __forceinline__ float reduce_transpose(const float *v, int sub) {
 // One step of a lane's recurrence: its NS states advance by one token and its
 // partial sum of C.h is returned.  States are processed in pairs with packed
 // fp32x2 multiplies / FMAs (one issue slot per two states); Abar comes from the
-// MUFU ex2.
-template <int N, int NS>
-__device__ __forceinline__ float recurrence_step(float2 (&h)[NS / 2], const float2 (&a2)[NS / 2],
-                                                 float2 dlx, const float *bcrow, int sub) {
-    const float4 *row = reinterpret_cast<const float4 *>(bcrow);
-    const float2 dl = make_float2(dlx.x, dlx.x), dx = make_float2(dlx.y, dlx.y);
-    float2 y0 = make_float2(0.0f, 0.0f), y1 = make_float2(0.0f, 0.0f);
+// MUFU ex2.  dl = (Delta, Delta) and dx = (Delta x, Delta x) are duplicated
+// into both halves of a register pair for the packed math.
+template <int NS>
+__device__ __forceinline__ float recurrence_step2(float2 (&h)[NS / 2], const float2 (&a2)[NS / 2],
+                                                  const float2 dl, const float2 dx,
+                                                  const BCPairs<NS> &bc) {
+    static_assert(NS == 2 || NS % 4 == 0, "states per lane: 2 or a multiple of 4");
+    float2 y0, y1;
 #pragma unroll
-    for (int q = 0; q < NS / 4; ++q) {
-        const float4 bq = row[(sub * NS) / 4 + q];
-        const float4 cq = row[(N + sub * NS) / 4 + q];
-        const float2 bv[2] = {make_float2(bq.x, bq.y), make_float2(bq.z, bq.w)};
-        const float2 cv[2] = {make_float2(cq.x, cq.y), make_float2(cq.z, cq.w)};
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int i = 2 * q + e;
-            const float2 arg = mul2(dl, a2[i]);
-            const float2 abar = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
-            h[i] = fma2(abar, h[i], mul2(dx, bv[e]));
-            if (e) y1 = fma2(cv[e], h[i], y1);
-            else y0 = fma2(cv[e], h[i], y0);
-        }
+    for (int i = 0; i < NS / 2; ++i) {
+        const float2 arg = mul2(dl, a2[i]);
+        const float2 abar = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+        h[i] = fma2(abar, h[i], mul2(dx, bc.b[i]));
+        if (i == 0) y0 = mul2(bc.c[i], h[i]);
+        else if (i == 1) y1 = mul2(bc.c[i], h[i]);
+        else if (i & 1) y1 = fma2(bc.c[i], h[i], y1);
+        else y0 = fma2(bc.c[i], h[i], y0);
     }
-    const float2 y = add2(y0, y1);
-    return y.x + y.y;
+    if constexpr (NS > 2) y0 = add2(y0, y1);
+    return y0.x + y0.y;
+}
+
+template <int NS, typename T>
+__device__ __forceinline__ float recurrence_step(float2 (&h)[NS / 2], const float2 (&a2)[NS / 2],
+                                                 float2 dlx, const T *row, int sub) {
+    return recurrence_step2<NS>(h, a2, make_float2(dlx.x, dlx.x), make_float2(dlx.y, dlx.y),
+                                load_bc<NS>(row, sub));
 }
 
 }  // namespace jssm

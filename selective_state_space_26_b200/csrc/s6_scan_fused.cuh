@@ -16,8 +16,8 @@
 //    the owner, which applies the skip and the gate and writes the output tile.
 //  * One producer warp: lane 0 issues the TMA loads (no multicast) of the x,
 //    delta, z tiles [TT x CC] and of B, C [TT x N] into a STAGES-deep ring and
-//    the TMA stores of the output tiles; all 32 lanes widen each tile's B and C
-//    to fp32 once (shared by every channel of the CTA).
+//    the TMA stores of the output tiles; all 32 lanes regroup each tile's B
+//    and C into per-lane slots (load_bc) once for every channel of the CTA.
 //  * Persistent CTAs over (sequence, channel-group) tasks; the tiles of a CTA's
 //    tasks form one stream.
 //  * Every wait is a bounded mbarrier wait that also watches a CTA abort flag;
@@ -33,26 +33,31 @@
 
 namespace jssm {
 
+// IoT: I/O element type; N: d_state; G: lanes per channel; NW: compute warps;
+// TT: time tile; STAGES: TMA ring depth.
 template <typename IoT, int N_, int G_, int NW_, int TT_, int STAGES_>
 struct FusedCfg {
     static constexpr int N = N_, G = G_, NW = NW_, TT = TT_, STAGES = STAGES_;
     static constexpr int NS = N / G;    // states per lane
     static constexpr int CW = 32 / G;   // channels per warp
     static constexpr int CC = NW * CW;  // channels per CTA tile
+    static_assert((CC * (int)sizeof(IoT)) % 16 == 0, "TMA boxes and offsets of 16-byte multiples");
     static constexpr int kThreads = (NW + 1) * 32;
     static constexpr int VEC = 16 / (int)sizeof(IoT);
-    static_assert(NS % 4 == 0 && NS >= 4, "a lane reads its B/C slice as float4");
+    static_assert(NS == 2 || (NS % 4 == 0 && NS >= 4), "a lane reads its B/C slice as float2/float4");
     static_assert(32 % G == 0 && TT % G == 0, "step groups of G");
-    static_assert(N % VEC == 0, "B/C widened 16 bytes at a time");
+    static_assert(N % VEC == 0, "B / C rows are whole 16-byte TMA units");
     static constexpr int kActTile = TT * CC * (int)sizeof(IoT);
     static constexpr int kBCTile = TT * N * (int)sizeof(IoT);
     static constexpr int kStageBytes = 3 * kActTile + 2 * kBCTile;
     static_assert(kActTile % 128 == 0 && kBCTile % 128 == 0, "TMA destinations 128B aligned");
-    static constexpr int kBCRow = 2 * N + 4;
-    static constexpr int kBCf = TT * kBCRow;  // floats per stage
-    static constexpr int kOffBCf = STAGES * kStageBytes;
+    // staged fp32 B / C rows ([G][2][NS] floats per step, see load_bc)
+    static constexpr int kBCRow = 2 * N;
+    static constexpr int kBCe = TT * kBCRow;  // floats per stage
+    static constexpr int kOffBCs = STAGES * kStageBytes;
     static constexpr int NOUT = 3;  // output tiles in flight (compute, TMA store, spare)
-    static constexpr int kOffOut = kOffBCf + STAGES * kBCf * 4;
+    static constexpr int kOffOut = kOffBCs + STAGES * kBCe * 4;
+    static_assert(kOffOut % 128 == 0, "TMA store source 128B aligned");
     // full[S], bc_ready[S], out_full[NOUT], out_free[NOUT]
     static constexpr int kOffBar = kOffOut + NOUT * kActTile;
     static constexpr int kNumBars = 2 * STAGES + 2 * NOUT;
@@ -77,33 +82,92 @@ __device__ __forceinline__ OwnedStep owned_step(const IoT *xs, const IoT *dts, c
     return OwnedStep{dl, dl * xo, gate, dskip * xo * gate};
 }
 
-// One full tile (TT steps) of a compute lane: lane `sub` of each channel owns
-// steps sub, sub + G, ...; the owner's scalars for the next group of G steps
-// are computed while the current group's states advance (software pipelining
-// over groups), so the softplus / gate latency hides behind the recurrence.
+// Delta and Delta x of the G steps owned in `o` gathered from the channel's
+// lanes, and the group's Abar = exp(Delta A) (NS / 2 packed multiplies and NS
+// MUFU ex2 per step).
+template <int G, int NS>
+__device__ __forceinline__ void group_exps(const OwnedStep &o, const float2 (&a2)[NS / 2], int gbase,
+                                           float2 (&dxp)[G], float2 (&ab)[G][NS / 2]) {
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+        const float dl = G == 1 ? o.dl : __shfl_sync(0xffffffffu, o.dl, gbase | j);
+        const float dx = G == 1 ? o.dx : __shfl_sync(0xffffffffu, o.dx, gbase | j);
+        dxp[j] = make_float2(dx, dx);
+#pragma unroll
+        for (int i = 0; i < NS / 2; ++i) {
+            const float2 arg = mul2(make_float2(dl, dl), a2[i]);
+            ab[j][i] = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+        }
+    }
+}
+
+// One full tile (TT steps) of a compute lane.  Lane `sub` of each channel
+// owns steps sub, sub + G, ... of the tile: it computes their Delta, Delta x,
+// gate and skip (owned_step) and hands Delta and Delta x to the channel's
+// other lanes by shuffles.  The loop is software-pipelined over groups of G
+// steps because a sub-partition holds only a few of these warps and issue is
+// in order (a warp whose next instruction waits on a dependency issues
+// nothing): while the states of group g advance, the exps of group g+1 are
+// issued and the owners' softplus / gate of group g+2 are computed.
+// SOFTPLUS is a template parameter: a runtime test inside the unrolled body
+// would split it into basic blocks that the scheduler cannot interleave.
 template <bool SOFTPLUS, typename IoT, int N, int G, int NS, int TT, int CC, int BCROW>
 __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float2 (&a2)[NS / 2],
                                                 float bias, float dskip,
                                                 const IoT *xs, const IoT *dts, const IoT *zs,
-                                                const float *bcf, IoT *outs, int c_local, int sub,
+                                                const float *bcs, IoT *outs, int c_local, int sub,
                                                 int gbase) {
-    OwnedStep cur = owned_step<SOFTPLUS>(xs, dts, zs, sub * CC + c_local, bias, dskip);
+    constexpr int NG = TT / G;
+    static_assert(NG >= 2, "a tile holds at least two groups");
+    OwnedStep o0 = owned_step<SOFTPLUS>(xs, dts, zs, sub * CC + c_local, bias, dskip);
+    OwnedStep o1 = owned_step<SOFTPLUS>(xs, dts, zs, (G + sub) * CC + c_local, bias, dskip);
+    float2 dxp[G], ab[G][NS / 2];
+    group_exps<G, NS>(o0, a2, gbase, dxp, ab);
 #pragma unroll
-    for (int t0 = 0; t0 < TT; t0 += G) {
-        OwnedStep nxt = cur;
-        if (t0 + G < TT)
-            nxt = owned_step<SOFTPLUS>(xs, dts, zs, (t0 + G + sub) * CC + c_local, bias, dskip);
+    for (int g = 0; g < NG; ++g) {
+        const int t0 = g * G;
+        OwnedStep o2 = o1;
+        if (g + 2 < NG)
+            o2 = owned_step<SOFTPLUS>(xs, dts, zs, (t0 + 2 * G + sub) * CC + c_local, bias, dskip);
+        float2 dxn[G], abn[G][NS / 2];
         float yp[G];
 #pragma unroll
         for (int j = 0; j < G; ++j) {
-            const float dlj = G == 1 ? cur.dl : __shfl_sync(0xffffffffu, cur.dl, gbase | j);
-            const float dxj = G == 1 ? cur.dx : __shfl_sync(0xffffffffu, cur.dx, gbase | j);
-            yp[j] = recurrence_step<N, NS>(h, a2, make_float2(dlj, dxj),
-                                              bcf + (t0 + j) * BCROW, sub);
+            if (g + 1 < NG) {
+                const float dl = G == 1 ? o1.dl : __shfl_sync(0xffffffffu, o1.dl, gbase | j);
+                const float dx = G == 1 ? o1.dx : __shfl_sync(0xffffffffu, o1.dx, gbase | j);
+                dxn[j] = make_float2(dx, dx);
+#pragma unroll
+                for (int i = 0; i < NS / 2; ++i) {
+                    const float2 arg = mul2(make_float2(dl, dl), a2[i]);
+                    abn[j][i] = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+                }
+            }
+            const BCPairs<NS> bc = load_bc<NS>(bcs + (t0 + j) * BCROW, sub);
+            float2 y0, y1;
+#pragma unroll
+            for (int i = 0; i < NS / 2; ++i) {
+                h[i] = fma2(ab[j][i], h[i], mul2(dxp[j], bc.b[i]));
+                if (i == 0) y0 = mul2(bc.c[i], h[i]);
+                else if (i == 1) y1 = mul2(bc.c[i], h[i]);
+                else if (i & 1) y1 = fma2(bc.c[i], h[i], y1);
+                else y0 = fma2(bc.c[i], h[i], y0);
+            }
+            if constexpr (NS > 2) y0 = add2(y0, y1);
+            yp[j] = y0.x + y0.y;
         }
         const float y = reduce_transpose<G>(yp, sub);
-        outs[(t0 + sub) * CC + c_local] = from_f32<IoT>(fmaf(y, cur.gate, cur.skg));
-        cur = nxt;
+        outs[(t0 + sub) * CC + c_local] = from_f32<IoT>(fmaf(y, o0.gate, o0.skg));
+        if (g + 1 < NG) {
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+                dxp[j] = dxn[j];
+#pragma unroll
+                for (int i = 0; i < NS / 2; ++i) ab[j][i] = abn[j][i];
+            }
+        }
+        o0 = o1;
+        o1 = o2;
     }
 }
 
@@ -116,14 +180,14 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
                          const __grid_constant__ CUtensorMap tm_C,
                          const __grid_constant__ CUtensorMap tm_out, const ScanArgs args) {
     using Cfg = FusedCfg<IoT, N, G, NW, TT, STAGES>;
-    constexpr int NS = Cfg::NS, CW = Cfg::CW, CC = Cfg::CC, VEC = Cfg::VEC, NOUT = Cfg::NOUT;
+    constexpr int NS = Cfg::NS, CW = Cfg::CW, CC = Cfg::CC, NOUT = Cfg::NOUT;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
     uint64_t *bc_ready = full + STAGES;
     uint64_t *out_full = bc_ready + STAGES;
     uint64_t *out_free = out_full + NOUT;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffFlag);
-    float *bcf_all = reinterpret_cast<float *>(smem + Cfg::kOffBCf);
+    float *bcs_all = reinterpret_cast<float *>(smem + Cfg::kOffBCs);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t d_inner = args.d_inner, seqlen = args.seqlen;
@@ -244,7 +308,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
         }
         __syncwarp();
         int64_t consumed = 0;
-        // fp32 copy of tile g's B and C (after its TMA load landed)
+        // tile g's B and C regrouped into per-lane slots (after its TMA load landed)
         auto widen = [&](int64_t g) -> bool {
             int64_t b;
             int c0, k;
@@ -259,19 +323,12 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             const uint8_t *base = smem + s * Cfg::kStageBytes;
             const IoT *Bs = reinterpret_cast<const IoT *>(base + 3 * Cfg::kActTile);
             const IoT *Cs = reinterpret_cast<const IoT *>(base + 3 * Cfg::kActTile + Cfg::kBCTile);
-            float *bcf = bcf_all + s * Cfg::kBCf;
-            for (int v = lane; v < nsteps * N / VEC; v += 32) {
-                const int t = (v * VEC) / N, n = (v * VEC) % N;
-                float fb[VEC], fc[VEC];
-                widen16(*reinterpret_cast<const uint4 *>(Bs + v * VEC), Bs, fb);
-                widen16(*reinterpret_cast<const uint4 *>(Cs + v * VEC), Cs, fc);
-#pragma unroll
-                for (int q = 0; q < VEC / 4; ++q) {
-                    *reinterpret_cast<float4 *>(bcf + t * Cfg::kBCRow + n + 4 * q) =
-                        make_float4(fb[4 * q], fb[4 * q + 1], fb[4 * q + 2], fb[4 * q + 3]);
-                    *reinterpret_cast<float4 *>(bcf + t * Cfg::kBCRow + N + n + 4 * q) =
-                        make_float4(fc[4 * q], fc[4 * q + 1], fc[4 * q + 2], fc[4 * q + 3]);
-                }
+            float *dst = bcs_all + s * Cfg::kBCe;
+            // unit u = (step t, slot j, half: 0 = B, 1 = C): one slice of NS values
+            for (int u = lane; u < nsteps * 2 * G; u += 32) {
+                const int t = u / (2 * G), j = (u / 2) % G, half = u & 1;
+                stage_slice<NS>(dst + t * Cfg::kBCRow + (2 * j + half) * NS,
+                                (half ? Cs : Bs) + t * N + j * NS);
             }
             mbar_arrive(&bc_ready[s]);
             return true;
@@ -348,7 +405,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
         const IoT *xs = reinterpret_cast<const IoT *>(base);
         const IoT *dts = reinterpret_cast<const IoT *>(base + Cfg::kActTile);
         const IoT *zs = reinterpret_cast<const IoT *>(base + 2 * Cfg::kActTile);
-        const float *bcf = bcf_all + s * Cfg::kBCf;
+        const float *bcs = bcs_all + s * Cfg::kBCe;
         IoT *outs = reinterpret_cast<IoT *>(smem + Cfg::kOffOut + slot * Cfg::kActTile);
 
         // One group of G steps starting at t0: the owner lane's scalars, the
@@ -368,20 +425,18 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
                 const float dxj = G == 1 ? dx : __shfl_sync(0xffffffffu, dx, gbase | j);
                 yp[j] = 0.0f;
                 if (j < valid)
-                    yp[j] = recurrence_step<N, NS>(h, a2, make_float2(dlj, dxj),
-                                                      bcf + (t0 + j) * Cfg::kBCRow, sub);
+                    yp[j] = recurrence_step<NS>(h, a2, make_float2(dlj, dxj),
+                                                bcs + (t0 + j) * Cfg::kBCRow, sub);
             }
             const float y = reduce_transpose<G>(yp, sub);
             if (sub < valid) outs[idx] = from_f32<IoT>((y + dskip * xo) * gate);
         };
-        // use_softplus picks between two straight-line bodies outside the tile
-        // (a per-element select would split the unrolled code into blocks)
         if (nsteps == TT && use_softplus) {
             fused_tile_full<true, IoT, N, G, NS, TT, CC, Cfg::kBCRow>(h, a2, bias, dskip, xs, dts, zs,
-                                                                     bcf, outs, c_local, sub, gbase);
+                                                                     bcs, outs, c_local, sub, gbase);
         } else if (nsteps == TT) {
             fused_tile_full<false, IoT, N, G, NS, TT, CC, Cfg::kBCRow>(h, a2, bias, dskip, xs, dts,
-                                                                      zs, bcf, outs, c_local, sub,
+                                                                      zs, bcs, outs, c_local, sub,
                                                                       gbase);
         } else {
             for (int t0 = 0; t0 < nsteps; t0 += G) group(t0, nsteps - t0 < G ? nsteps - t0 : G);

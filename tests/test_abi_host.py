@@ -80,7 +80,9 @@ def test_variant_table(L):
         k += 1
     assert len(infos) >= 9
     for i in infos:
-        assert i["d_state"] % (4 * i["lanes_per_channel"]) == 0
+        ns = i["d_state"] // i["lanes_per_channel"]
+        assert ns * i["lanes_per_channel"] == i["d_state"]
+        assert ns == 2 or ns % 4 == 0
         assert 32 % i["lanes_per_channel"] == 0
         assert i["time_tile"] % i["lanes_per_channel"] == 0
     assert _lib.variant_info(0) is None
@@ -109,7 +111,8 @@ def _scan(p):
     (dict(d_state=32), _lib.ERR_UNSUPPORTED),
     (dict(d_inner=12), _lib.ERR_UNSUPPORTED),         # bf16 row not a multiple of 16 bytes
     (dict(kernel_variant=99), _lib.ERR_UNSUPPORTED),
-    (dict(kernel_variant=7), _lib.ERR_UNSUPPORTED),   # an fp32 variant for bf16 data
+    (dict(kernel_variant=8), _lib.ERR_UNSUPPORTED),   # an fp32 variant for bf16 data
+    (dict(kernel_variant=5), _lib.ERR_UNSUPPORTED),   # a d_state=8 variant for d_state=16
     (dict(x=None), _lib.ERR_INVALID_ARG),
     (dict(A=None), _lib.ERR_INVALID_ARG),
     (dict(out=None), _lib.ERR_INVALID_ARG),
