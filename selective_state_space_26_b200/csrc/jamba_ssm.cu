@@ -423,7 +423,7 @@ jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, 
     const bool stream_ok = (p->d_inner * es) % 16 == 0 && (p->d_state * es) % 16 == 0 &&
                            aligned(p->x, 16) && aligned(p->delta, 16) && aligned(p->z, 16);
     if (stream_ok) {
-        constexpr int kCPB = 64, kBPC = 16, kS = 4;
+        constexpr int kCPB = 32, kBPC = 16, kS = 8;
         const int64_t gx = (p->d_inner + kCPB - 1) / kCPB, gy = (p->batch + kBPC - 1) / kBPC;
         if (gx > 0x7fffffff || gy > 65535) return JAMBA_SSM_ERR_UNSUPPORTED;
         const void *k = nullptr;
@@ -431,7 +431,7 @@ jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, 
 #define JSSM_STREAM(T, NN)                                                                    \
     do {                                                                                      \
         k = (const void *)&jssm::s6_state_update_stream_kernel<T, NN, kCPB, kBPC, kS>;        \
-        threads = kCPB * (NN / 4);                                                            \
+        threads = jssm::UpdateCfg<T, NN, kCPB, kS>::kThreads;                                 \
         smem = jssm::UpdateCfg<T, NN, kCPB, kS>::kSmemBytes;                                  \
     } while (0)
         switch (p->d_state) {

@@ -144,19 +144,15 @@ __device__ __forceinline__ float recurrence_step2(float2 (&h)[NS / 2], const flo
                                                   const float2 dl, const float2 dx,
                                                   const BCPairs<NS> &bc) {
     static_assert(NS == 2 || NS % 4 == 0, "states per lane: 2 or a multiple of 4");
-    float2 y0, y1;
+    float2 y2;
 #pragma unroll
     for (int i = 0; i < NS / 2; ++i) {
         const float2 arg = mul2(dl, a2[i]);
         const float2 abar = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
         h[i] = fma2(abar, h[i], mul2(dx, bc.b[i]));
-        if (i == 0) y0 = mul2(bc.c[i], h[i]);
-        else if (i == 1) y1 = mul2(bc.c[i], h[i]);
-        else if (i & 1) y1 = fma2(bc.c[i], h[i], y1);
-        else y0 = fma2(bc.c[i], h[i], y0);
+        y2 = i == 0 ? mul2(bc.c[i], h[i]) : fma2(bc.c[i], h[i], y2);
     }
-    if constexpr (NS > 2) y0 = add2(y0, y1);
-    return y0.x + y0.y;
+    return y2.x + y2.y;
 }
 
 template <int NS, typename T>

@@ -144,17 +144,13 @@ __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float
                 }
             }
             const BCPairs<NS> bc = load_bc<NS>(bcs + (t0 + j) * BCROW, sub);
-            float2 y0, y1;
+            float2 y2;
 #pragma unroll
             for (int i = 0; i < NS / 2; ++i) {
                 h[i] = fma2(ab[j][i], h[i], mul2(dxp[j], bc.b[i]));
-                if (i == 0) y0 = mul2(bc.c[i], h[i]);
-                else if (i == 1) y1 = mul2(bc.c[i], h[i]);
-                else if (i & 1) y1 = fma2(bc.c[i], h[i], y1);
-                else y0 = fma2(bc.c[i], h[i], y0);
+                y2 = i == 0 ? mul2(bc.c[i], h[i]) : fma2(bc.c[i], h[i], y2);
             }
-            if constexpr (NS > 2) y0 = add2(y0, y1);
-            yp[j] = y0.x + y0.y;
+            yp[j] = y2.x + y2.y;
         }
         const float y = reduce_transpose<G>(yp, sub);
         outs[(t0 + sub) * CC + c_local] = from_f32<IoT>(fmaf(y, o0.gate, o0.skg));

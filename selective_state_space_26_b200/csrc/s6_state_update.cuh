@@ -19,6 +19,7 @@
 
 #include "device_utils.cuh"
 #include "s6_math.cuh"
+#include "s6_scan.cuh"  // reduce_transpose
 
 namespace jssm {
 
@@ -120,153 +121,179 @@ __global__ void __launch_bounds__(256) s6_state_update_kernel(const UpdateArgs a
     }
 }
 
-// Streaming form for the usual shapes (d_inner a multiple of 16 bytes of I/O):
-// a CTA owns one block of CPB channels and walks BPC requests; thread 0 keeps a
-// STAGES-deep
-// ring of 1-D bulk copies (no multicast) in flight -- the request's CPB x N fp32
-// state slab (contiguous), its x / delta / z slices and its B / C rows -- so
-// the bytes in flight per SM are set by shared memory, not by registers.  The
-// threads read their float4 of state from shared memory, update it and write
-// it back to HBM with coalesced 128-bit stores.  Waits are bounded; on a
-// timeout the CTA records JAMBA_SSM_ERR_TIMEOUT and stops after the barrier.
+// Streaming form for the usual shapes (rows of whole 16-byte chunks).  A CTA
+// owns one block of CPB channels and walks BPC requests.  One producer warp
+// keeps a STAGES-deep ring of 1-D bulk copies (no multicast) in flight -- per
+// request the CPB x N fp32 state slab (contiguous) and the x / delta / z
+// slices and B / C rows -- so the bytes in flight per SM are set by shared
+// memory, not registers; full / empty mbarriers per stage let it refill a
+// stage as soon as the compute warps have read it (no CTA-wide barrier).
+// Q = N/4 lanes own a channel, 4 states each.  Requests are taken in groups of
+// Q: lane q computes the per-(request, channel) scalars of request q of the
+// group (softplus, Delta x, gate, skip) and hands Delta, Delta x to the other
+// lanes by shuffles, so no lane repeats another's transcendental work; the Q
+// partial sums of C.h of the group's requests are reduced with the
+// transposing butterfly, which leaves request q's sum on lane q, who writes
+// its output.  The new state goes straight back to HBM (128-bit stores).
+// Every wait is bounded; on a timeout the CTA records JAMBA_SSM_ERR_TIMEOUT
+// and leaves, the producer first waiting (bounded) for its copies in flight.
 template <typename IoT, int N, int CPB, int STAGES>
 struct UpdateCfg {
     static constexpr int Q = N / 4;
-    static constexpr int kThreads = CPB * Q;
+    static constexpr int kComputeThreads = CPB * Q;
+    static constexpr int kComputeWarps = kComputeThreads / 32;
+    static constexpr int kThreads = kComputeThreads + 32;
     static constexpr int kStateBytes = CPB * N * 4;
     static constexpr int kActBytes = CPB * (int)sizeof(IoT);
     static constexpr int kBCBytes = N * (int)sizeof(IoT);
     static constexpr int kStage = kStateBytes + 3 * kActBytes + 2 * kBCBytes;
+    static_assert(kComputeThreads % 32 == 0, "whole compute warps");
+    static_assert(STAGES % Q == 0 && STAGES >= 2 * Q, "two request groups in flight");
     static_assert(kActBytes % 16 == 0 && kBCBytes % 16 == 0 && kStage % 16 == 0, "bulk sizes");
-    static constexpr int kOffBar = STAGES * kStage;
-    static constexpr int kSmemBytes = kOffBar + STAGES * 8 + 16;
+    static constexpr int kOffBar = STAGES * kStage;  // full[STAGES], empty[STAGES]
+    static constexpr int kSmemBytes = kOffBar + 2 * STAGES * 8 + 16;
 };
 
 template <typename IoT, int N, int CPB, int BPC, int STAGES>
-__global__ void __launch_bounds__(CPB *(N / 4), 6) s6_state_update_stream_kernel(const UpdateArgs a,
-                                                                            uint64_t limit) {
+__global__ void __launch_bounds__(UpdateCfg<IoT, N, CPB, STAGES>::kThreads, 4)
+    s6_state_update_stream_kernel(const UpdateArgs a, uint64_t limit) {
     using Cfg = UpdateCfg<IoT, N, CPB, STAGES>;
-    constexpr int Q = Cfg::Q;
+    constexpr int Q = Cfg::Q, NW = Cfg::kComputeWarps;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffBar + STAGES * 8);
-    const int tid = threadIdx.x, q = tid % Q, cl = tid / Q;
-    // This CTA: channel block blockIdx.x, requests [blockIdx.y * BPC, +BPC).
+    uint64_t *empty = full + STAGES;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + STAGES);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // This CTA: channels [blockIdx.x * CPB, +nd), requests [blockIdx.y * BPC, +nu).
+    const int64_t d0 = static_cast<int64_t>(blockIdx.x) * CPB;
+    const int nd = static_cast<int>(a.d_inner - d0 < CPB ? a.d_inner - d0 : CPB);
     const int64_t breq0 = static_cast<int64_t>(blockIdx.y) * BPC;
     const int nu = static_cast<int>(a.batch - breq0 < BPC ? a.batch - breq0 : BPC);
-    const IoT *xg = static_cast<const IoT *>(a.x);
-    const IoT *dtg = static_cast<const IoT *>(a.delta);
-    const IoT *zg = static_cast<const IoT *>(a.z);
-    const IoT *Bg = static_cast<const IoT *>(a.B);
-    const IoT *Cg = static_cast<const IoT *>(a.C);
 
     if (tid == 0) {
-        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NW);
+        }
         *abort_flag = 0;
         fence_mbarrier_init();
     }
     __syncthreads();
-    // (channel block, request) cursors advance by one unit without divisions
-    struct Unit {
-        int64_t blk, b;
-        __device__ void next(int64_t batch) {
-            if (++b == batch) {
-                b = 0;
-                ++blk;
-            }
-        }
-    };
-    const Unit first{static_cast<int64_t>(blockIdx.x), breq0};
-    Unit icur = first;  // thread 0: next unit to load
-    auto issue = [&](int j) {  // thread 0, called for j = 0, 1, 2, ... in order
-        const int64_t blk = icur.blk, b = icur.b;
-        icur.next(a.batch);
-        const int64_t d0 = blk * CPB;
-        const int nd = static_cast<int>(a.d_inner - d0 < CPB ? a.d_inner - d0 : CPB);
-        const uint32_t state_bytes = static_cast<uint32_t>(nd) * N * 4;
-        const uint32_t act_bytes = static_cast<uint32_t>(nd) * sizeof(IoT);
-        const int s = j % STAGES;
-        uint8_t *st = smem + s * Cfg::kStage;
-        const int64_t row = b * a.d_inner + d0;
-        mbar_arrive_expect_tx(&full[s], state_bytes + 3 * act_bytes + 2 * Cfg::kBCBytes);
-        bulk_load_1d(st, a.state + row * N, state_bytes, &full[s]);
-        bulk_load_1d(st + Cfg::kStateBytes, xg + row, act_bytes, &full[s]);
-        bulk_load_1d(st + Cfg::kStateBytes + Cfg::kActBytes, dtg + row, act_bytes, &full[s]);
-        bulk_load_1d(st + Cfg::kStateBytes + 2 * Cfg::kActBytes, zg + row, act_bytes, &full[s]);
-        bulk_load_1d(st + Cfg::kStateBytes + 3 * Cfg::kActBytes, Bg + b * N, Cfg::kBCBytes, &full[s]);
-        bulk_load_1d(st + Cfg::kStateBytes + 3 * Cfg::kActBytes + Cfg::kBCBytes, Cg + b * N,
-                     Cfg::kBCBytes, &full[s]);
-    };
-    int issued = nu < STAGES ? nu : STAGES;
-    if (tid == 0)
-        for (int j = 0; j < issued; ++j) issue(j);
 
-    const bool use_softplus = a.delta_softplus != 0;
-    int64_t cur_blk = -1;
-    float Av[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    float bias = 0.0f, dskip = 0.0f;
-    Unit cur = first;
-    for (int j = 0; j < nu; ++j, cur.next(a.batch)) {
-        const int64_t blk = cur.blk, b = cur.b;
-        const int64_t d0 = blk * CPB;
-        const int nd = static_cast<int>(a.d_inner - d0 < CPB ? a.d_inner - d0 : CPB);
-        const bool dvalid = cl < nd;
-        const int c = dvalid ? cl : nd - 1;
-        const int64_t d = d0 + c;
-        if (blk != cur_blk) {  // parameters of this channel block
-            cur_blk = blk;
-            load4<float>(a.A + d * N + 4 * q, Av);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) Av[i] *= kLog2e;
-            bias = a.delta_bias ? __ldg(a.delta_bias + d) : 0.0f;
-            dskip = a.D ? __ldg(a.D + d) : 0.0f;
+    if (warp == NW) {
+        // ================= producer warp: the bulk-copy ring =================
+        if (lane == 0) {
+            const IoT *xg = static_cast<const IoT *>(a.x);
+            const IoT *dtg = static_cast<const IoT *>(a.delta);
+            const IoT *zg = static_cast<const IoT *>(a.z);
+            const IoT *Bg = static_cast<const IoT *>(a.B);
+            const IoT *Cg = static_cast<const IoT *>(a.C);
+            const uint32_t state_bytes = static_cast<uint32_t>(nd) * N * 4;
+            const uint32_t act_bytes = static_cast<uint32_t>(nd) * sizeof(IoT);
+            int issued = 0;
+            bool ok = true;
+            for (int u = 0; u < nu; ++u) {
+                const int s = u % STAGES;
+                if (u >= STAGES &&
+                    !mbar_wait_or_abort(&empty[s], static_cast<uint32_t>(u / STAGES - 1) & 1u, limit,
+                                        abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *st = smem + s * Cfg::kStage;
+                const int64_t b = breq0 + u, row = b * a.d_inner + d0;
+                mbar_arrive_expect_tx(&full[s], state_bytes + 3 * act_bytes + 2 * Cfg::kBCBytes);
+                bulk_load_1d(st, a.state + row * N, state_bytes, &full[s]);
+                bulk_load_1d(st + Cfg::kStateBytes, xg + row, act_bytes, &full[s]);
+                bulk_load_1d(st + Cfg::kStateBytes + Cfg::kActBytes, dtg + row, act_bytes, &full[s]);
+                bulk_load_1d(st + Cfg::kStateBytes + 2 * Cfg::kActBytes, zg + row, act_bytes, &full[s]);
+                bulk_load_1d(st + Cfg::kStateBytes + 3 * Cfg::kActBytes, Bg + b * N, Cfg::kBCBytes,
+                             &full[s]);
+                bulk_load_1d(st + Cfg::kStateBytes + 3 * Cfg::kActBytes + Cfg::kBCBytes, Cg + b * N,
+                             Cfg::kBCBytes, &full[s]);
+                issued = u + 1;
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+            }
+            // copies still in flight when the compute warps may have left:
+            // wait (bounded) for each stage's last fill before the CTA exits
+            for (int u = issued - STAGES > 0 ? issued - STAGES : 0; u < issued; ++u)
+                mbar_wait_bounded(&full[u % STAGES], static_cast<uint32_t>(u / STAGES) & 1u, limit);
         }
-        const int s = j % STAGES;
-        const uint8_t *st = smem + s * Cfg::kStage;
-        if (mbar_wait_bounded(&full[s], static_cast<uint32_t>(j / STAGES) & 1u, limit)) {
-            const float4 h4 = reinterpret_cast<const float4 *>(st)[c * Q + q];
-            const IoT *xs = reinterpret_cast<const IoT *>(st + Cfg::kStateBytes);
-            const IoT *dts = xs + CPB, *zs = dts + CPB;
-            const IoT *Bs = zs + CPB, *Cs = Bs + N;
-            float Bv[4], Cv[4];
-            load4<IoT>(Bs + 4 * q, Bv);
-            load4<IoT>(Cs + 4 * q, Cv);
-            const float xv = to_f32(xs[c]);
-            const float dl = delta_f32(to_f32(dts[c]), bias, use_softplus);
-            const float dx = dl * xv;
-            float h[4] = {h4.x, h4.y, h4.z, h4.w};
-            float y = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float abar = ex2_mufu(dl * Av[i]);
-                h[i] = fmaf(abar, h[i], dx * Bv[i]);
-                y = fmaf(Cv[i], h[i], y);
-            }
-#pragma unroll
-            for (int off = 1; off < Q; off <<= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
-            if (dvalid) {
-                const int64_t bd = b * a.d_inner + d;
-                reinterpret_cast<float4 *>(a.state)[bd * Q + q] = make_float4(h[0], h[1], h[2], h[3]);
-                if (q == 0)
-                    static_cast<IoT *>(a.out)[bd] =
-                        from_f32<IoT>((y + dskip * xv) * silu_f32(to_f32(zs[c])));
-            }
-        } else {
+        return;
+    }
+
+    // =========================== compute warps ===========================
+    const int q = tid % Q, cl = tid / Q;
+    const int gbase = lane & ~(Q - 1);
+    const bool dvalid = cl < nd;
+    const int c = dvalid ? cl : nd - 1;  // idle lanes shadow a valid channel
+    const int64_t d = d0 + c;
+    float2 a2[2];
+    {
+        float Av[4];
+        load4<float>(a.A + d * N + 4 * q, Av);
+        a2[0] = make_float2(Av[0] * kLog2e, Av[1] * kLog2e);
+        a2[1] = make_float2(Av[2] * kLog2e, Av[3] * kLog2e);
+    }
+    const float bias = a.delta_bias ? __ldg(a.delta_bias + d) : 0.0f;
+    const float dskip = a.D ? __ldg(a.D + d) : 0.0f;
+    const bool use_softplus = a.delta_softplus != 0;
+    float4 *stg = reinterpret_cast<float4 *>(a.state);
+    IoT *outg = static_cast<IoT *>(a.out);
+
+    for (int r0 = 0; r0 < nu; r0 += Q) {
+        const int nr = nu - r0 < Q ? nu - r0 : Q;
+        bool ok = true;
+        for (int r = 0; r < nr && ok; ++r)
+            ok = mbar_wait_or_abort(&full[(r0 + r) % STAGES], static_cast<uint32_t>((r0 + r) / STAGES) & 1u,
+                                    limit, abort_flag);
+        if (!ok) {
             *abort_flag = 1;
             atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+            break;
         }
-        __syncthreads();  // stage s has been read by every thread
+        // this lane's owned request r0 + q (a copy of request r0 when q >= nr)
+        const uint8_t *so = smem + ((r0 + (q < nr ? q : 0)) % STAGES) * Cfg::kStage;
+        const IoT *xs = reinterpret_cast<const IoT *>(so + Cfg::kStateBytes);
+        const float xv = to_f32(xs[c]);
+        const float dl = delta_f32(to_f32(xs[CPB + c]), bias, use_softplus);
+        const float gate = silu_f32(to_f32(xs[2 * CPB + c]));
+        const float dxo = dl * xv, skg = dskip * xv * gate;
+        float yp[Q];
+#pragma unroll
+        for (int r = 0; r < Q; ++r) {
+            const float dlr = Q == 1 ? dl : __shfl_sync(0xffffffffu, dl, gbase | r);
+            const float dxr = Q == 1 ? dxo : __shfl_sync(0xffffffffu, dxo, gbase | r);
+            yp[r] = 0.0f;
+            if (r < nr) {
+                const uint8_t *st = smem + ((r0 + r) % STAGES) * Cfg::kStage;
+                const float4 h4 = reinterpret_cast<const float4 *>(st)[c * Q + q];
+                const IoT *Bs = reinterpret_cast<const IoT *>(st + Cfg::kStateBytes + 3 * Cfg::kActBytes);
+                float Bv[4], Cv[4];
+                load4<IoT>(Bs + 4 * q, Bv);
+                load4<IoT>(Bs + N + 4 * q, Cv);
+                const float2 dlp = make_float2(dlr, dlr), dxp = make_float2(dxr, dxr);
+                const float2 arg0 = mul2(dlp, a2[0]), arg1 = mul2(dlp, a2[1]);
+                float2 h0 = fma2(make_float2(ex2_mufu(arg0.x), ex2_mufu(arg0.y)), make_float2(h4.x, h4.y),
+                                 mul2(dxp, make_float2(Bv[0], Bv[1])));
+                float2 h1 = fma2(make_float2(ex2_mufu(arg1.x), ex2_mufu(arg1.y)), make_float2(h4.z, h4.w),
+                                 mul2(dxp, make_float2(Bv[2], Bv[3])));
+                float2 y2 = mul2(make_float2(Cv[0], Cv[1]), h0);
+                y2 = fma2(make_float2(Cv[2], Cv[3]), h1, y2);
+                yp[r] = y2.x + y2.y;
+                if (dvalid) stg[((breq0 + r0 + r) * a.d_inner + d) * Q + q] = make_float4(h0.x, h0.y, h1.x, h1.y);
+            }
+        }
+        // every lane of the warp has read the group's stages
+        __syncwarp();
+        if (lane == 0)
+            for (int r = 0; r < nr; ++r) mbar_arrive(&empty[(r0 + r) % STAGES]);
+        const float y = reduce_transpose<Q>(yp, q);
+        if (dvalid && q < nr) outg[(breq0 + r0 + q) * a.d_inner + d] = from_f32<IoT>(fmaf(y, gate, skg));
         if (*abort_flag) break;
-        if (tid == 0 && issued < nu) {
-            fence_proxy_async_smem();
-            issue(issued);
-            ++issued;
-        }
-    }
-    if (tid == 0 && *abort_flag) {
-        // loads still in flight on the ring: wait (bounded) before the CTA exits
-        for (int j = 0; j < issued; ++j)
-            mbar_wait_bounded(&full[j % STAGES], static_cast<uint32_t>(j / STAGES) & 1u, limit);
     }
 }
 
