@@ -138,9 +138,9 @@ ScanVariant make_fused(double step_cost) {
 // the 148 SMs (56 channels per CTA -> 147 CTAs).
 ScanVariant g_variants[] = {
     make_fused<__nv_bfloat16, 16, 2, 8, 64, 2>(1.00),   // 1: 128 channels / CTA
-    make_fused<__nv_bfloat16, 16, 4, 7, 64, 3>(1.29),   // 2:  56 channels / CTA
-    make_fused<__nv_bfloat16, 16, 4, 8, 64, 3>(1.31),   // 3:  64 channels / CTA
-    make_fused<__nv_bfloat16, 16, 4, 7, 32, 4>(1.43),   // 4:  56 channels / CTA
+    make_fused<__nv_bfloat16, 16, 4, 7, 64, 3>(1.33),   // 2:  56 channels / CTA
+    make_fused<__nv_bfloat16, 16, 4, 8, 64, 3>(1.35),   // 3:  64 channels / CTA
+    make_fused<__nv_bfloat16, 16, 4, 7, 32, 4>(1.47),   // 4:  56 channels / CTA
     make_fused<__nv_bfloat16, 8, 2, 8, 32, 4>(1.00),    // 5: 128 channels / CTA
     make_fused<__nv_bfloat16, 8, 1, 4, 32, 4>(1.70),    // 6: 128 channels / CTA
     make_fused<__nv_bfloat16, 8, 4, 7, 64, 3>(1.29),    // 7:  56 channels / CTA
