@@ -107,10 +107,12 @@ __device__ __forceinline__ void group_exps(const OwnedStep &o, const float2 (&a2
 // other lanes by shuffles.  The loop is software-pipelined over groups of G
 // steps because a sub-partition holds only a few of these warps and issue is
 // in order (a warp whose next instruction waits on a dependency issues
-// nothing): while the states of group g advance, the exps of group g+1 are
-// issued and the owners' softplus / gate of group g+2 are computed.
-// SOFTPLUS is a template parameter: a runtime test inside the unrolled body
-// would split it into basic blocks that the scheduler cannot interleave.
+// nothing): while the states of group g advance, the exps of group g+2 are
+// issued and the owners' softplus / gate of group g+3 are computed, so an
+// exp's result is consumed about 2G steps after issue even when the MUFU
+// queue is long.  SOFTPLUS is a template parameter: a runtime test inside the
+// unrolled body would split it into basic blocks that the scheduler cannot
+// interleave.
 template <bool SOFTPLUS, typename IoT, int N, int G, int NS, int TT, int CC, int BCROW>
 __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float2 (&a2)[NS / 2],
                                                 float bias, float dskip,
@@ -118,52 +120,57 @@ __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float
                                                 const float *bcs, IoT *outs, int c_local, int sub,
                                                 int gbase) {
     constexpr int NG = TT / G;
-    static_assert(NG >= 2, "a tile holds at least two groups");
+    static_assert(NG >= 3, "a tile holds at least three groups");
     OwnedStep o0 = owned_step<SOFTPLUS>(xs, dts, zs, sub * CC + c_local, bias, dskip);
     OwnedStep o1 = owned_step<SOFTPLUS>(xs, dts, zs, (G + sub) * CC + c_local, bias, dskip);
-    float2 dxp[G], ab[G][NS / 2];
-    group_exps<G, NS>(o0, a2, gbase, dxp, ab);
+    OwnedStep o2 = owned_step<SOFTPLUS>(xs, dts, zs, (2 * G + sub) * CC + c_local, bias, dskip);
+    float2 dxa[G], aba[G][NS / 2], dxb[G], abb[G][NS / 2];
+    group_exps<G, NS>(o0, a2, gbase, dxa, aba);
+    group_exps<G, NS>(o1, a2, gbase, dxb, abb);
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
         const int t0 = g * G;
-        OwnedStep o2 = o1;
-        if (g + 2 < NG)
-            o2 = owned_step<SOFTPLUS>(xs, dts, zs, (t0 + 2 * G + sub) * CC + c_local, bias, dskip);
-        float2 dxn[G], abn[G][NS / 2];
+        OwnedStep o3 = o2;
+        if (g + 3 < NG)
+            o3 = owned_step<SOFTPLUS>(xs, dts, zs, (t0 + 3 * G + sub) * CC + c_local, bias, dskip);
+        float2 dxc[G], abc[G][NS / 2];
         float yp[G];
 #pragma unroll
         for (int j = 0; j < G; ++j) {
-            if (g + 1 < NG) {
-                const float dl = G == 1 ? o1.dl : __shfl_sync(0xffffffffu, o1.dl, gbase | j);
-                const float dx = G == 1 ? o1.dx : __shfl_sync(0xffffffffu, o1.dx, gbase | j);
-                dxn[j] = make_float2(dx, dx);
+            if (g + 2 < NG) {
+                const float dl = G == 1 ? o2.dl : __shfl_sync(0xffffffffu, o2.dl, gbase | j);
+                const float dx = G == 1 ? o2.dx : __shfl_sync(0xffffffffu, o2.dx, gbase | j);
+                dxc[j] = make_float2(dx, dx);
 #pragma unroll
                 for (int i = 0; i < NS / 2; ++i) {
                     const float2 arg = mul2(make_float2(dl, dl), a2[i]);
-                    abn[j][i] = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+                    abc[j][i] = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
                 }
             }
             const BCPairs<NS> bc = load_bc<NS>(bcs + (t0 + j) * BCROW, sub);
             float2 y2;
 #pragma unroll
             for (int i = 0; i < NS / 2; ++i) {
-                h[i] = fma2(ab[j][i], h[i], mul2(dxp[j], bc.b[i]));
+                h[i] = fma2(aba[j][i], h[i], mul2(dxa[j], bc.b[i]));
                 y2 = i == 0 ? mul2(bc.c[i], h[i]) : fma2(bc.c[i], h[i], y2);
             }
             yp[j] = y2.x + y2.y;
         }
         const float y = reduce_transpose<G>(yp, sub);
         outs[(t0 + sub) * CC + c_local] = from_f32<IoT>(fmaf(y, o0.gate, o0.skg));
-        if (g + 1 < NG) {
 #pragma unroll
-            for (int j = 0; j < G; ++j) {
-                dxp[j] = dxn[j];
+        for (int j = 0; j < G; ++j) {
+            dxa[j] = dxb[j];
+            if (g + 2 < NG) dxb[j] = dxc[j];
 #pragma unroll
-                for (int i = 0; i < NS / 2; ++i) ab[j][i] = abn[j][i];
+            for (int i = 0; i < NS / 2; ++i) {
+                aba[j][i] = abb[j][i];
+                if (g + 2 < NG) abb[j][i] = abc[j][i];
             }
         }
         o0 = o1;
         o1 = o2;
+        o2 = o3;
     }
 }
 
