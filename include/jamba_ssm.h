@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define JAMBA_SSM_ABI_VERSION 1
+#define JAMBA_SSM_ABI_VERSION 2
 
 typedef enum {
     JAMBA_SSM_OK = 0,
@@ -99,9 +99,32 @@ typedef enum {
  *                 overrides the wait limit (SM clock cycles, 0 = ~1 s).
  * Empty input: batch == 0 does nothing; seqlen == 0 copies h0 (or zeros)
  * into h_final.
+ *
+ * Serving layouts (ABI version 2; a caller whose struct_size ends before
+ * these fields gets both off):
+ *   cu_seqlens    device int32 [batch + 1] or NULL.  Non-NULL selects the
+ *                 packed variable-length layout: x, delta, z, out are
+ *                 [total_tokens, d_inner] and B, C [total_tokens, d_state];
+ *                 sequence b is rows cu_seqlens[b] .. cu_seqlens[b+1] - 1
+ *                 (0 = cu_seqlens[0] <= ... <= cu_seqlens[batch] =
+ *                 total_tokens; the kernel clamps every offset to
+ *                 [0, total_tokens]).  `seqlen` is ignored.  An empty
+ *                 sequence copies its initial state to its final state.
+ *   total_tokens  rows of the packed layout (cu_seqlens != NULL), >= 0.
+ *   state_indices device int32 [batch] or NULL.  Non-NULL: h0 and h_final
+ *                 are [num_slots, d_inner, d_state] state caches and
+ *                 sequence b reads / writes row state_indices[b].  A negative
+ *                 index means "no cached state": zero initial state and no
+ *                 final state written (outputs are still computed).  An
+ *                 index >= num_slots is treated the same way and recorded as
+ *                 JAMBA_SSM_ERR_INVALID_ARG in the status word.  Indices of
+ *                 one call must be distinct.
+ *   num_slots     rows of the state caches (state_indices != NULL).
  */
 typedef struct jamba_ssm_scan_params {
-    size_t struct_size;          /* = sizeof(jamba_ssm_scan_params)            */
+    size_t struct_size;          /* = sizeof(jamba_ssm_scan_params); callers of
+                                    ABI version 1 pass the size ending at
+                                    timeout_cycles                             */
     int64_t batch, seqlen, d_inner, d_state;
     int32_t io_dtype;            /* jamba_ssm_dtype                            */
     int32_t delta_softplus;
@@ -116,6 +139,11 @@ typedef struct jamba_ssm_scan_params {
     int32_t kernel_variant;
     uint32_t debug_flags;
     uint64_t timeout_cycles;
+    /* ABI version 2 */
+    const int32_t *cu_seqlens;
+    int64_t total_tokens;
+    const int32_t *state_indices;
+    int64_t num_slots;
 } jamba_ssm_scan_params;
 
 jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream);
@@ -137,9 +165,19 @@ jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream);
  *   B, C       [batch, d_state] io_dtype, 16-byte aligned.
  *   A          [d_inner, d_state] fp32, 16-byte aligned; D, delta_bias as above
  *              (4-byte aligned or NULL).
+ * Serving layout (ABI version 2; absent when struct_size ends before it):
+ *   state_indices device int32 [batch] or NULL.  Non-NULL: `state` is a
+ *              [num_slots, d_inner, d_state] cache and request b updates row
+ *              state_indices[b].  A negative index skips request b (its state
+ *              row and its out row are left untouched: padding in a
+ *              continuous batch); an index >= num_slots is skipped too and
+ *              recorded as JAMBA_SSM_ERR_INVALID_ARG in the status word.
+ *              Indices of one call must be distinct.
+ *   num_slots  rows of the state cache (state_indices != NULL), >= 1.
  */
 typedef struct jamba_ssm_state_update_params {
-    size_t struct_size;          /* = sizeof(jamba_ssm_state_update_params)    */
+    size_t struct_size;          /* = sizeof(jamba_ssm_state_update_params);
+                                    ABI version 1 callers: size ending at out  */
     int64_t batch, d_inner, d_state;
     int32_t io_dtype;
     int32_t delta_softplus;
@@ -150,6 +188,9 @@ typedef struct jamba_ssm_state_update_params {
     const float *D;
     const float *delta_bias;
     void *out;
+    /* ABI version 2 */
+    const int32_t *state_indices;
+    int64_t num_slots;
 } jamba_ssm_state_update_params;
 
 jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, void *stream);
@@ -170,7 +211,8 @@ jamba_ssm_status jamba_ssm_scan_variant_info(int32_t k, int32_t *io_dtype, int32
 
 /* Synchronizes `stream`, then reads and clears the current device's sticky
  * status word: JAMBA_SSM_OK, or the first device-side error recorded since the
- * last call (JAMBA_SSM_ERR_TIMEOUT).  Returns JAMBA_SSM_ERR_CUDA if the
+ * last call (JAMBA_SSM_ERR_TIMEOUT, or JAMBA_SSM_ERR_INVALID_ARG for a state
+ * index past num_slots).  Returns JAMBA_SSM_ERR_CUDA if the
  * synchronization itself failed. */
 jamba_ssm_status jamba_ssm_get_status(void *stream);
 

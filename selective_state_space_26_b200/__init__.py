@@ -51,45 +51,70 @@ def _stream(stream, device):
 
 
 def _scan_params(x, delta, z, B, C, A, D, delta_bias, delta_softplus, h0, out, h_final,
-                 variant, debug_flags, timeout_cycles):
+                 variant, debug_flags, timeout_cycles, cu_seqlens=None, state_indices=None):
     if x.dtype not in _IO:
         raise TypeError(f"x must be bfloat16 or float32, got {x.dtype}")
-    batch, seqlen, d_inner = x.shape
     d_state = A.shape[-1]
     dev = x.device
     io = x.dtype
-    for t, n, s in ((x, "x", (batch, seqlen, d_inner)), (delta, "delta", (batch, seqlen, d_inner)),
-                    (z, "z", (batch, seqlen, d_inner)), (B, "B", (batch, seqlen, d_state)),
-                    (C, "C", (batch, seqlen, d_state)), (out, "out", (batch, seqlen, d_inner))):
+    if cu_seqlens is not None:
+        # packed layout: [total_tokens, d_inner], sequences delimited by cu_seqlens
+        total, d_inner = x.shape
+        _check(cu_seqlens, "cu_seqlens", (cu_seqlens.numel(),), torch.int32, dev)
+        batch, seqlen = cu_seqlens.numel() - 1, 0
+        act, bc = (total, d_inner), (total, d_state)
+    else:
+        batch, seqlen, d_inner = x.shape
+        total = 0
+        act, bc = (batch, seqlen, d_inner), (batch, seqlen, d_state)
+    for t, n, s in ((x, "x", act), (delta, "delta", act), (z, "z", act), (B, "B", bc),
+                    (C, "C", bc), (out, "out", act)):
         _check(t, n, s, io, dev)
     _check(A, "A", (d_inner, d_state), torch.float32, dev)
     _check(D, "D", (d_inner,), torch.float32, dev)
     _check(delta_bias, "delta_bias", (d_inner,), torch.float32, dev)
-    _check(h0, "h0", (batch, d_inner, d_state), torch.float32, dev)
-    _check(h_final, "h_final", (batch, d_inner, d_state), torch.float32, dev)
+    num_slots = 0
+    if state_indices is not None:
+        _check(state_indices, "state_indices", (batch,), torch.int32, dev)
+        caches = [t for t in (h0, h_final) if t is not None]
+        num_slots = caches[0].shape[0] if caches else 1
+    state_shape = (num_slots if state_indices is not None else batch, d_inner, d_state)
+    _check(h0, "h0", state_shape, torch.float32, dev)
+    _check(h_final, "h_final", state_shape, torch.float32, dev)
     return _lib.new_scan_params(
         batch=batch, seqlen=seqlen, d_inner=d_inner, d_state=d_state, io_dtype=_IO[io],
         delta_softplus=int(bool(delta_softplus)), x=_ptr(x), delta=_ptr(delta), z=_ptr(z),
         B=_ptr(B), C=_ptr(C), A=_ptr(A), D=_ptr(D), delta_bias=_ptr(delta_bias), h0=_ptr(h0),
         out=_ptr(out), h_final=_ptr(h_final), kernel_variant=int(variant),
-        debug_flags=int(debug_flags), timeout_cycles=int(timeout_cycles))
+        debug_flags=int(debug_flags), timeout_cycles=int(timeout_cycles),
+        cu_seqlens=_ptr(cu_seqlens), total_tokens=int(total),
+        state_indices=_ptr(state_indices), num_slots=int(num_slots))
 
 
 def jamba_ssm_scan(x, delta, z, B, C, A, D=None, delta_bias=None, delta_softplus=True,
                    h0=None, out=None, h_final=None, return_final_state=True, stream=None,
-                   variant: int = 0, debug_flags: int = 0, timeout_cycles: int = 0):
+                   variant: int = 0, debug_flags: int = 0, timeout_cycles: int = 0,
+                   cu_seqlens=None, state_indices=None):
     """Prefill S6 scan.  Shapes: x, delta, z [batch, seqlen, d_inner] (bf16 or
     fp32), B, C [batch, seqlen, d_state] (same dtype), A [d_inner, d_state]
     fp32, D and delta_bias [d_inner] fp32 or None, h0 [batch, d_inner, d_state]
     fp32 or None.  Returns (out, h_final); h_final is None when
-    return_final_state is False and no buffer was passed."""
+    return_final_state is False and no buffer was passed.
+
+    Serving layouts: with ``cu_seqlens`` (int32 [batch + 1] on the device) the
+    activations are packed [total_tokens, d_inner] / [total_tokens, d_state]
+    and sequence b is rows cu_seqlens[b]:cu_seqlens[b+1].  With
+    ``state_indices`` (int32 [batch]) h0 / h_final are [num_slots, d_inner,
+    d_state] caches and sequence b uses row state_indices[b] (negative: zero
+    initial state, nothing written); pass h_final explicitly in that case."""
     if out is None:
         out = torch.empty_like(x)
-    if h_final is None and return_final_state:
-        h_final = torch.empty(x.shape[0], x.shape[2], A.shape[-1], dtype=torch.float32,
+    if h_final is None and return_final_state and state_indices is None:
+        batch = cu_seqlens.numel() - 1 if cu_seqlens is not None else x.shape[0]
+        h_final = torch.empty(batch, x.shape[-1], A.shape[-1], dtype=torch.float32,
                               device=x.device)
     p = _scan_params(x, delta, z, B, C, A, D, delta_bias, delta_softplus, h0, out, h_final,
-                     variant, debug_flags, timeout_cycles)
+                     variant, debug_flags, timeout_cycles, cu_seqlens, state_indices)
     st = _lib.call_scan(p, _stream(stream, x.device))
     if st != _lib.OK:
         raise JambaSSMError(st, "jamba_ssm_scan")
@@ -106,10 +131,13 @@ def scan_plan(x, A, B=None, variant: int = 0):
 
 
 def jamba_ssm_state_update(state, x, delta, z, B, C, A, D=None, delta_bias=None,
-                           delta_softplus=True, out=None, stream=None):
+                           delta_softplus=True, out=None, stream=None, state_indices=None):
     """One decode step; `state` [batch, d_inner, d_state] fp32 is updated in
     place.  x, delta, z [batch, d_inner]; B, C [batch, d_state].  Returns out
-    [batch, d_inner]."""
+    [batch, d_inner].  With ``state_indices`` (int32 [batch] on the device)
+    `state` is a [num_slots, d_inner, d_state] cache and request b updates row
+    state_indices[b]; a negative index skips the request (its out row is left
+    as it was)."""
     if x.dtype not in _IO:
         raise TypeError(f"x must be bfloat16 or float32, got {x.dtype}")
     batch, d_inner = x.shape
@@ -121,7 +149,12 @@ def jamba_ssm_state_update(state, x, delta, z, B, C, A, D=None, delta_bias=None,
                     (z, "z", (batch, d_inner)), (B, "B", (batch, d_state)),
                     (C, "C", (batch, d_state)), (out, "out", (batch, d_inner))):
         _check(t, n, s, io, dev)
-    _check(state, "state", (batch, d_inner, d_state), torch.float32, dev)
+    num_slots = 0
+    if state_indices is not None:
+        _check(state_indices, "state_indices", (batch,), torch.int32, dev)
+        num_slots = state.shape[0]
+    _check(state, "state", (num_slots if state_indices is not None else batch, d_inner, d_state),
+           torch.float32, dev)
     _check(A, "A", (d_inner, d_state), torch.float32, dev)
     _check(D, "D", (d_inner,), torch.float32, dev)
     _check(delta_bias, "delta_bias", (d_inner,), torch.float32, dev)
@@ -129,7 +162,8 @@ def jamba_ssm_state_update(state, x, delta, z, B, C, A, D=None, delta_bias=None,
         batch=batch, d_inner=d_inner, d_state=d_state, io_dtype=_IO[io],
         delta_softplus=int(bool(delta_softplus)), state=_ptr(state), x=_ptr(x),
         delta=_ptr(delta), z=_ptr(z), B=_ptr(B), C=_ptr(C), A=_ptr(A), D=_ptr(D),
-        delta_bias=_ptr(delta_bias), out=_ptr(out))
+        delta_bias=_ptr(delta_bias), out=_ptr(out), state_indices=_ptr(state_indices),
+        num_slots=int(num_slots))
     st = _lib.call_state_update(p, _stream(stream, dev))
     if st != _lib.OK:
         raise JambaSSMError(st, "jamba_ssm_state_update")

@@ -43,6 +43,9 @@ class ScanParams(ctypes.Structure):
         ("out", _vp), ("h_final", _fp),
         ("kernel_variant", ctypes.c_int32), ("debug_flags", ctypes.c_uint32),
         ("timeout_cycles", ctypes.c_uint64),
+        # ABI version 2
+        ("cu_seqlens", _vp), ("total_tokens", ctypes.c_int64),
+        ("state_indices", _vp), ("num_slots", ctypes.c_int64),
     ]
 
 
@@ -56,6 +59,8 @@ class StateUpdateParams(ctypes.Structure):
         ("B", _vp), ("C", _vp),
         ("A", _fp), ("D", _fp), ("delta_bias", _fp),
         ("out", _vp),
+        # ABI version 2
+        ("state_indices", _vp), ("num_slots", ctypes.c_int64),
     ]
 
 
@@ -107,6 +112,12 @@ def lib():
 
 def status_string(status: int) -> str:
     return lib().jamba_ssm_status_string(int(status)).decode()
+
+
+# struct_size of the ABI version 1 structures (the fields before the
+# version 2 ones), for callers built against version 1
+SCAN_PARAMS_V1_SIZE = ScanParams.cu_seqlens.offset
+STATE_UPDATE_PARAMS_V1_SIZE = StateUpdateParams.state_indices.offset
 
 
 def new_scan_params(**kw) -> ScanParams:

@@ -4,12 +4,14 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstddef>
 #include <cstring>
 #include <mutex>
 
 #include "jamba_ssm.h"
 #include "s6_scan.cuh"
 #include "s6_scan_fused.cuh"
+#include "s6_scan_serving.cuh"
 #include "s6_state_update.cuh"
 
 using jssm::ScanArgs;
@@ -106,9 +108,10 @@ struct ScanVariant {
     int io_dtype, n, g, nw, tt, cw;
     int threads;
     double step_cost;  // measured time per channel-step, relative (multi-task steady state)
-    int smem;
-    const void *kernel;
-    bool attr_set[kMaxDevices];
+    int smem, smem_serving;
+    const void *kernel;          // batched layout
+    const void *kernel_serving;  // packed layout and / or state-cache slots
+    bool attr_set[kMaxDevices], attr_set_serving[kMaxDevices];
 };
 
 // NW compute warps (each does its channels' recurrence, softplus and gate) and
@@ -126,7 +129,10 @@ ScanVariant make_fused(double step_cost) {
     v.threads = (NW + 1) * 32;
     v.step_cost = step_cost;
     v.smem = Cfg::kSmemBytes;
+    v.smem_serving = jssm::ServingCfg<IoT, N, G, NW, TT, S>::kSmemBytes;
     v.kernel = reinterpret_cast<const void *>(&jssm::s6_scan_fused_kernel<IoT, N, G, NW, TT, S>);
+    v.kernel_serving =
+        reinterpret_cast<const void *>(&jssm::s6_scan_serving_kernel<IoT, N, G, NW, TT, S>);
     return v;
 }
 
@@ -190,18 +196,44 @@ bool overlaps(const void *a, size_t an, const void *b, size_t bn) {
 }
 
 constexpr int64_t kMaxElems = int64_t(1) << 40;
+constexpr int64_t kMaxI32 = (int64_t(1) << 31) - 1;
+
+// The caller's parameters as this library version reads them: copied over a
+// zeroed struct, so the fields past a smaller (ABI version 1) struct_size read
+// as zero / NULL.
+constexpr size_t kScanParamsV1 = offsetof(jamba_ssm_scan_params, cu_seqlens);
+constexpr size_t kUpdateParamsV1 = offsetof(jamba_ssm_state_update_params, state_indices);
+
+template <typename P>
+bool read_params(const P *p, size_t v1_size, P *q) {
+    if (!p || p->struct_size < v1_size) return false;
+    std::memset(q, 0, sizeof(P));
+    std::memcpy(q, p, p->struct_size < sizeof(P) ? p->struct_size : sizeof(P));
+    return true;
+}
+
+// Token rows of the activations: batch * seqlen, or the packed total.
+int64_t token_rows(const jamba_ssm_scan_params *p) {
+    return p->cu_seqlens ? p->total_tokens : p->batch * p->seqlen;
+}
 
 jamba_ssm_status validate_scan(const jamba_ssm_scan_params *p) {
-    if (!p || p->struct_size < sizeof(jamba_ssm_scan_params)) return JAMBA_SSM_ERR_INVALID_ARG;
     if (p->batch < 0 || p->seqlen < 0 || p->d_inner < 1 || p->d_state < 1)
         return JAMBA_SSM_ERR_INVALID_ARG;
     if (p->io_dtype != JAMBA_SSM_BF16 && p->io_dtype != JAMBA_SSM_F32)
         return JAMBA_SSM_ERR_INVALID_ARG;
-    if (p->batch > (int64_t(1) << 31) - 1 || p->seqlen > (int64_t(1) << 31) - 1 ||
-        p->d_inner > (int64_t(1) << 30))
+    if (p->cu_seqlens && p->total_tokens < 0) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->state_indices && p->num_slots < 1) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (!aligned(p->cu_seqlens, 4) || !aligned(p->state_indices, 4)) return JAMBA_SSM_ERR_MISALIGNED;
+    // token rows are int32 TMA coordinates, and a tile may start up to one
+    // time tile past the last row
+    const int64_t kMaxRows = kMaxI32 - 256;
+    if (p->batch > kMaxI32 || p->seqlen > kMaxRows || p->d_inner > (int64_t(1) << 30) ||
+        p->total_tokens > kMaxRows || p->num_slots > kMaxI32)
         return JAMBA_SSM_ERR_UNSUPPORTED;
-    if (p->batch && p->seqlen && p->batch * p->seqlen > kMaxElems / p->d_inner)
+    if (!p->cu_seqlens && p->batch && p->seqlen && p->batch > kMaxElems / p->seqlen)
         return JAMBA_SSM_ERR_UNSUPPORTED;
+    if (token_rows(p) > kMaxElems / p->d_inner) return JAMBA_SSM_ERR_UNSUPPORTED;
     const int es = p->io_dtype == JAMBA_SSM_BF16 ? 2 : 4;
     const bool n_ok = p->io_dtype == JAMBA_SSM_BF16 ? (p->d_state == 8 || p->d_state == 16)
                                                     : (p->d_state == 4 || p->d_state == 8 ||
@@ -210,8 +242,9 @@ jamba_ssm_status validate_scan(const jamba_ssm_scan_params *p) {
     if (p->kernel_variant < 0 || p->kernel_variant > kNumVariants) return JAMBA_SSM_ERR_UNSUPPORTED;
     if (p->kernel_variant > 0 && !variant_applies(g_variants[p->kernel_variant - 1], p))
         return JAMBA_SSM_ERR_UNSUPPORTED;
-    const int64_t tok = p->batch * p->seqlen;
-    const size_t state_bytes = size_t(p->batch) * p->d_inner * p->d_state * 4;
+    const int64_t tok = token_rows(p);
+    const int64_t state_rows = p->state_indices ? p->num_slots : p->batch;
+    const size_t state_bytes = size_t(state_rows) * p->d_inner * p->d_state * 4;
     if (tok > 0) {
         if (!p->x || !p->delta || !p->z || !p->B || !p->C || !p->A || !p->out)
             return JAMBA_SSM_ERR_INVALID_ARG;
@@ -226,7 +259,7 @@ jamba_ssm_status validate_scan(const jamba_ssm_scan_params *p) {
         for (int i = 0; i < 5; ++i)
             if (overlaps(p->out, act, ins[i], insz[i])) return JAMBA_SSM_ERR_INVALID_ARG;
         if (overlaps(p->h_final, state_bytes, p->out, act)) return JAMBA_SSM_ERR_INVALID_ARG;
-    } else if (p->batch > 0 && p->seqlen == 0) {
+    } else if (p->batch > 0) {
         if (!aligned(p->h0, 16) || !aligned(p->h_final, 16)) return JAMBA_SSM_ERR_MISALIGNED;
     }
     if (p->h0 && p->h_final && p->h0 != p->h_final &&
@@ -287,9 +320,12 @@ jamba_ssm_status jamba_ssm_scan_variant_info(int32_t k, int32_t *io_dtype, int32
     return JAMBA_SSM_OK;
 }
 
-jamba_ssm_status jamba_ssm_scan_plan(const jamba_ssm_scan_params *p, int32_t *variant,
+jamba_ssm_status jamba_ssm_scan_plan(const jamba_ssm_scan_params *pin, int32_t *variant,
                                      int32_t *lanes_per_channel, int32_t *channels_per_cta_out,
                                      int32_t *grid, int64_t *tasks) {
+    jamba_ssm_scan_params prm;
+    if (!read_params(pin, kScanParamsV1, &prm)) return JAMBA_SSM_ERR_INVALID_ARG;
+    const jamba_ssm_scan_params *p = &prm;
     jamba_ssm_status st = validate_scan(p);
     if (st != JAMBA_SSM_OK) return st;
     const DeviceInfo *dev = current_device(&st);
@@ -305,7 +341,10 @@ jamba_ssm_status jamba_ssm_scan_plan(const jamba_ssm_scan_params *p, int32_t *va
     return JAMBA_SSM_OK;
 }
 
-jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream) {
+jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *pin, void *stream) {
+    jamba_ssm_scan_params prm;
+    if (!read_params(pin, kScanParamsV1, &prm)) return JAMBA_SSM_ERR_INVALID_ARG;
+    const jamba_ssm_scan_params *p = &prm;
     jamba_ssm_status st = validate_scan(p);
     if (st != JAMBA_SSM_OK) return st;
     const DeviceInfo *dev = current_device(&st);
@@ -313,13 +352,25 @@ jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t state_bytes = size_t(p->batch) * p->d_inner * p->d_state * 4;
     if (p->batch == 0) return JAMBA_SSM_OK;
-    if (p->seqlen == 0) {  // no steps: the final state is the initial state
+    const int64_t rows = token_rows(p);
+    if (rows == 0) {  // no steps anywhere: every final state is its initial state
         if (!p->h_final) return JAMBA_SSM_OK;
-        cudaError_t e = p->h0 ? (p->h0 == p->h_final
-                                     ? cudaSuccess
-                                     : cudaMemcpyAsync(p->h_final, p->h0, state_bytes,
-                                                       cudaMemcpyDeviceToDevice, s))
-                              : cudaMemsetAsync(p->h_final, 0, state_bytes, s);
+        if (!p->state_indices) {
+            cudaError_t e = p->h0 ? (p->h0 == p->h_final
+                                         ? cudaSuccess
+                                         : cudaMemcpyAsync(p->h_final, p->h0, state_bytes,
+                                                           cudaMemcpyDeviceToDevice, s))
+                                  : cudaMemsetAsync(p->h_final, 0, state_bytes, s);
+            return e == cudaSuccess ? JAMBA_SSM_OK : cuda_fail(e);
+        }
+        const int64_t per = p->d_inner * p->d_state;
+        const int64_t n = p->batch * per;
+        const int threads = 256;
+        const int64_t blocks = (n + threads - 1) / threads;
+        if (blocks > 0x7fffffff) return JAMBA_SSM_ERR_UNSUPPORTED;
+        jssm::s6_copy_states_kernel<<<static_cast<unsigned>(blocks), threads, 0, s>>>(
+            p->batch, per, p->h0, p->h_final, p->state_indices, p->num_slots);
+        cudaError_t e = cudaGetLastError();
         return e == cudaSuccess ? JAMBA_SSM_OK : cuda_fail(e);
     }
 
@@ -333,26 +384,33 @@ jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream) {
     const int es = p->io_dtype == JAMBA_SSM_BF16 ? 2 : 4;
     const CUtensorMapDataType dt =
         p->io_dtype == JAMBA_SSM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    // [batch][seqlen][channels], or the packed [1][total_tokens][channels]
+    const int64_t dim_t = p->cu_seqlens ? p->total_tokens : p->seqlen;
+    const int64_t dim_b = p->cu_seqlens ? 1 : p->batch;
     CUtensorMap maps[6];
     const void *act_ptrs[4] = {p->x, p->delta, p->z, p->out};
     const int act_idx[4] = {0, 1, 2, 5};
     for (int i = 0; i < 4; ++i)
-        if (!encode_3d(fn, &maps[act_idx[i]], act_ptrs[i], dt, es, p->d_inner, p->seqlen, p->batch,
-                       cc, v.tt))
+        if (!encode_3d(fn, &maps[act_idx[i]], act_ptrs[i], dt, es, p->d_inner, dim_t, dim_b, cc, v.tt))
             return JAMBA_SSM_ERR_UNSUPPORTED;
-    if (!encode_3d(fn, &maps[3], p->B, dt, es, p->d_state, p->seqlen, p->batch, (int)p->d_state, v.tt) ||
-        !encode_3d(fn, &maps[4], p->C, dt, es, p->d_state, p->seqlen, p->batch, (int)p->d_state, v.tt))
+    if (!encode_3d(fn, &maps[3], p->B, dt, es, p->d_state, dim_t, dim_b, (int)p->d_state, v.tt) ||
+        !encode_3d(fn, &maps[4], p->C, dt, es, p->d_state, dim_t, dim_b, (int)p->d_state, v.tt))
         return JAMBA_SSM_ERR_UNSUPPORTED;
 
+    // the serving kernel for packed sequences or cache slots, else the batched one
+    const bool serving = p->cu_seqlens != nullptr || p->state_indices != nullptr;
+    const void *kernel = serving ? v.kernel_serving : v.kernel;
+    const int smem = serving ? v.smem_serving : v.smem;
     int devid = 0;
     cudaGetDevice(&devid);
     {
         std::lock_guard<std::mutex> lock(g_mutex);
-        if (!v.attr_set[devid]) {
-            cudaError_t e = cudaFuncSetAttribute(v.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 v.smem);
+        bool &set = serving ? v.attr_set_serving[devid] : v.attr_set[devid];
+        if (!set) {
+            cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 smem);
             if (e != cudaSuccess) return cuda_fail(e);
-            v.attr_set[devid] = true;
+            set = true;
         }
     }
 
@@ -368,17 +426,27 @@ jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream) {
     args.delta_softplus = p->delta_softplus != 0;
     args.debug_flags = p->debug_flags;
     args.timeout_cycles = p->timeout_cycles ? p->timeout_cycles : (uint64_t(1) << 31);
+    args.cu_seqlens = p->cu_seqlens;
+    args.total_tokens = p->total_tokens;
+    args.state_indices = p->state_indices;
+    args.num_slots = p->num_slots;
+    args.out = p->out;
 
     void *kargs[] = {&maps[0], &maps[1], &maps[2], &maps[3], &maps[4], &maps[5], &args};
-    cudaError_t e = cudaLaunchKernel(v.kernel, dim3(plan.grid), dim3(v.threads), kargs,
-                                     static_cast<size_t>(v.smem), s);
+    cudaError_t e = cudaLaunchKernel(kernel, dim3(plan.grid), dim3(v.threads), kargs,
+                                     static_cast<size_t>(smem), s);
     if (e != cudaSuccess) return cuda_fail(e);
     return JAMBA_SSM_OK;
 }
 
-jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, void *stream) {
-    if (!p || p->struct_size < sizeof(jamba_ssm_state_update_params)) return JAMBA_SSM_ERR_INVALID_ARG;
+jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *pin, void *stream) {
+    jamba_ssm_state_update_params prm;
+    if (!read_params(pin, kUpdateParamsV1, &prm)) return JAMBA_SSM_ERR_INVALID_ARG;
+    const jamba_ssm_state_update_params *p = &prm;
     if (p->batch < 0 || p->d_inner < 1 || p->d_state < 1) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->state_indices && p->num_slots < 1) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->num_slots > kMaxI32) return JAMBA_SSM_ERR_UNSUPPORTED;
+    if (!aligned(p->state_indices, 4)) return JAMBA_SSM_ERR_MISALIGNED;
     if (p->io_dtype != JAMBA_SSM_BF16 && p->io_dtype != JAMBA_SSM_F32) return JAMBA_SSM_ERR_INVALID_ARG;
     if (p->d_state != 4 && p->d_state != 8 && p->d_state != 16) return JAMBA_SSM_ERR_UNSUPPORTED;
     if (p->batch > (int64_t(1) << 31) || p->d_inner > (int64_t(1) << 30)) return JAMBA_SSM_ERR_UNSUPPORTED;
@@ -391,7 +459,7 @@ jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, 
         !aligned(p->D, 4) || !aligned(p->delta_bias, 4))
         return JAMBA_SSM_ERR_MISALIGNED;
     const size_t act = size_t(p->batch) * p->d_inner * es, bc = size_t(p->batch) * p->d_state * es;
-    const size_t sb = size_t(p->batch) * p->d_inner * p->d_state * 4;
+    const size_t sb = size_t(p->state_indices ? p->num_slots : p->batch) * p->d_inner * p->d_state * 4;
     const void *ins[] = {p->x, p->delta, p->z, p->B, p->C, p->state};
     const size_t insz[] = {act, act, act, bc, bc, sb};
     for (int i = 0; i < 6; ++i)
@@ -417,6 +485,8 @@ jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, 
     a.delta_bias = p->delta_bias;
     a.out = p->out;
     a.delta_softplus = p->delta_softplus != 0;
+    a.state_indices = p->state_indices;
+    a.num_slots = p->num_slots;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool bf = p->io_dtype == JAMBA_SSM_BF16;
     // Streaming kernel when every slice is a whole number of 16-byte chunks.
@@ -430,7 +500,9 @@ jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, 
         int threads = 0, smem = 0;
 #define JSSM_STREAM(T, NN)                                                                    \
     do {                                                                                      \
-        k = (const void *)&jssm::s6_state_update_stream_kernel<T, NN, kCPB, kBPC, kS>;        \
+        k = p->state_indices                                                                  \
+                ? (const void *)&jssm::s6_state_update_stream_kernel<T, NN, kCPB, kBPC, kS, true> \
+                : (const void *)&jssm::s6_state_update_stream_kernel<T, NN, kCPB, kBPC, kS, false>; \
         threads = jssm::UpdateCfg<T, NN, kCPB, kS>::kThreads;                                 \
         smem = jssm::UpdateCfg<T, NN, kCPB, kS>::kSmemBytes;                                  \
     } while (0)

@@ -22,7 +22,26 @@ struct ScanArgs {
     int delta_softplus;
     uint32_t debug_flags;
     uint64_t timeout_cycles;
+    const int *cu_seqlens;     // packed layout: sequence offsets [batch + 1], or null
+    int64_t total_tokens;      // rows of the packed layout
+    const int *state_indices;  // state-cache row of each sequence, or null
+    int64_t num_slots;         // rows of the state cache
+    void *out;                 // output base (row-wise stores of short packed tiles)
 };
+
+// No steps at all (every sequence empty) with a state cache: final state =
+// initial state (or zeros) for each sequence's slot; one thread per float.
+// An index past num_slots is recorded as JAMBA_SSM_ERR_INVALID_ARG.
+__global__ void s6_copy_states_kernel(int64_t batch, int64_t per_seq, const float *h0, float *h_final,
+                                      const int *state_indices, int64_t num_slots) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= batch * per_seq) return;
+    const int64_t b = i / per_seq, e = i - b * per_seq;
+    const int64_t row = state_indices[b];
+    if (row >= num_slots && e == 0) atomicCAS(&g_status_word, 0, 1 /* JAMBA_SSM_ERR_INVALID_ARG */);
+    if (row < 0 || row >= num_slots) return;
+    h_final[row * per_seq + e] = h0 ? h0[row * per_seq + e] : 0.0f;
+}
 
 // Staged B / C of one step.  The producer lays each step out in fp32 as G
 // slots, one per lane of a channel: slot s holds the NS values of B and then

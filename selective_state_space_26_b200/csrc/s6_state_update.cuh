@@ -30,7 +30,21 @@ struct UpdateArgs {
     const float *A, *D, *delta_bias;
     void *out;
     int delta_softplus;
+    const int *state_indices;  // state-cache row of each request, or null (row b)
+    int64_t num_slots;         // rows of the state cache
 };
+
+// State-cache row of request b, or -1 when the request is skipped (a negative
+// index: padding; or one past the cache, recorded as an invalid argument).
+__device__ __forceinline__ int64_t state_row(const UpdateArgs &a, int64_t b, bool record) {
+    if (!a.state_indices) return b;
+    const int64_t r = __ldg(a.state_indices + b);
+    if (r >= a.num_slots) {
+        if (record) atomicCAS(&g_status_word, 0, 1 /* JAMBA_SSM_ERR_INVALID_ARG */);
+        return -1;
+    }
+    return r < 0 ? -1 : r;
+}
 
 template <typename IoT>
 __device__ __forceinline__ void load4(const IoT *p, float (&v)[4]);
@@ -82,14 +96,16 @@ __global__ void __launch_bounds__(256) s6_state_update_kernel(const UpdateArgs a
         float4 h4[2];
         float Bv[2][4], Cv[2][4], xv[2], dtv[2], zv[2];
         bool valid[2];
-        int64_t bd[2];
+        int64_t bd[2], sd[2];  // activation row, state row
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int64_t b = b0 + j + u;
-            valid[u] = dvalid && b < a.batch;
             const int64_t bc = b < a.batch ? b : a.batch - 1;
+            const int64_t srow = state_row(a, bc, threadIdx.x == 0 && b < a.batch);
+            valid[u] = dvalid && b < a.batch && srow >= 0;
             bd[u] = bc * a.d_inner + dc;
-            h4[u] = st[bd[u] * Q + q];
+            sd[u] = (srow >= 0 ? srow : 0) * a.d_inner + dc;
+            h4[u] = st[sd[u] * Q + q];
             load4<IoT>(static_cast<const IoT *>(a.B) + bc * N + 4 * q, Bv[u]);
             load4<IoT>(static_cast<const IoT *>(a.C) + bc * N + 4 * q, Cv[u]);
             xv[u] = to_f32(x[bd[u]]);
@@ -111,7 +127,7 @@ __global__ void __launch_bounds__(256) s6_state_update_kernel(const UpdateArgs a
 #pragma unroll
             for (int off = 1; off < Q; off <<= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
             if (valid[u]) {
-                st[bd[u] * Q + q] = make_float4(h[0], h[1], h[2], h[3]);
+                st[sd[u] * Q + q] = make_float4(h[0], h[1], h[2], h[3]);
                 if (q == 0) {
                     const float o = (y + dskip * xv[u]) * silu_f32(zv[u]);
                     static_cast<IoT *>(a.out)[bd[u]] = from_f32<IoT>(o);
@@ -154,7 +170,9 @@ struct UpdateCfg {
     static constexpr int kSmemBytes = kOffBar + 2 * STAGES * 8 + 16;
 };
 
-template <typename IoT, int N, int CPB, int BPC, int STAGES>
+// SLOTS: the state is a cache addressed by state_indices (a template parameter
+// so that the plain kernel carries no per-request lookups).
+template <typename IoT, int N, int CPB, int BPC, int STAGES, bool SLOTS>
 __global__ void __launch_bounds__(UpdateCfg<IoT, N, CPB, STAGES>::kThreads, 4)
     s6_state_update_stream_kernel(const UpdateArgs a, uint64_t limit) {
     using Cfg = UpdateCfg<IoT, N, CPB, STAGES>;
@@ -202,8 +220,10 @@ __global__ void __launch_bounds__(UpdateCfg<IoT, N, CPB, STAGES>::kThreads, 4)
                 }
                 uint8_t *st = smem + s * Cfg::kStage;
                 const int64_t b = breq0 + u, row = b * a.d_inner + d0;
+                const int64_t srow = SLOTS ? state_row(a, b, false) : b;  // skipped: loads row 0
                 mbar_arrive_expect_tx(&full[s], state_bytes + 3 * act_bytes + 2 * Cfg::kBCBytes);
-                bulk_load_1d(st, a.state + row * N, state_bytes, &full[s]);
+                bulk_load_1d(st, a.state + ((srow >= 0 ? srow : 0) * a.d_inner + d0) * N, state_bytes,
+                             &full[s]);
                 bulk_load_1d(st + Cfg::kStateBytes, xg + row, act_bytes, &full[s]);
                 bulk_load_1d(st + Cfg::kStateBytes + Cfg::kActBytes, dtg + row, act_bytes, &full[s]);
                 bulk_load_1d(st + Cfg::kStateBytes + 2 * Cfg::kActBytes, zg + row, act_bytes, &full[s]);
@@ -284,7 +304,9 @@ __global__ void __launch_bounds__(UpdateCfg<IoT, N, CPB, STAGES>::kThreads, 4)
                 float2 y2 = mul2(make_float2(Cv[0], Cv[1]), h0);
                 y2 = fma2(make_float2(Cv[2], Cv[3]), h1, y2);
                 yp[r] = y2.x + y2.y;
-                if (dvalid) stg[((breq0 + r0 + r) * a.d_inner + d) * Q + q] = make_float4(h0.x, h0.y, h1.x, h1.y);
+                const int64_t srow = SLOTS ? state_row(a, breq0 + r0 + r, tid == 0) : breq0 + r0 + r;
+                if (dvalid && srow >= 0)
+                    stg[(srow * a.d_inner + d) * Q + q] = make_float4(h0.x, h0.y, h1.x, h1.y);
             }
         }
         // every lane of the warp has read the group's stages
@@ -292,7 +314,8 @@ __global__ void __launch_bounds__(UpdateCfg<IoT, N, CPB, STAGES>::kThreads, 4)
         if (lane == 0)
             for (int r = 0; r < nr; ++r) mbar_arrive(&empty[(r0 + r) % STAGES]);
         const float y = reduce_transpose<Q>(yp, q);
-        if (dvalid && q < nr) outg[(breq0 + r0 + q) * a.d_inner + d] = from_f32<IoT>(fmaf(y, gate, skg));
+        if (dvalid && q < nr && (!SLOTS || state_row(a, breq0 + r0 + q, false) >= 0))
+            outg[(breq0 + r0 + q) * a.d_inner + d] = from_f32<IoT>(fmaf(y, gate, skg));
         if (*abort_flag) break;
     }
 }

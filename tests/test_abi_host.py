@@ -66,7 +66,7 @@ def test_struct_layout_matches_header(tmp_path):
 
 
 def test_status_strings_and_version(L):
-    assert L.jamba_ssm_abi_version() == 1
+    assert L.jamba_ssm_abi_version() == 2
     for s in range(7):
         assert _lib.status_string(s)
     assert _lib.status_string(99) == "unknown status"
@@ -169,3 +169,49 @@ def test_valid_call_without_device_reports_no_device(L):
     assert _lib.call_state_update(_valid_update(), 0) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
     p = _valid_scan(batch=0)
     assert _scan(p) == _lib.OK or _scan(p) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(cu_seqlens=0x1000, total_tokens=-1), _lib.ERR_INVALID_ARG),
+    (dict(cu_seqlens=0x1002, total_tokens=64), _lib.ERR_MISALIGNED),
+    (dict(state_indices=0x2000, num_slots=0), _lib.ERR_INVALID_ARG),
+    (dict(state_indices=0x2001, num_slots=4), _lib.ERR_MISALIGNED),
+    (dict(cu_seqlens=0x1000, total_tokens=1 << 32), _lib.ERR_UNSUPPORTED),
+    # packed: out overlapping x is measured with total_tokens rows
+    (dict(cu_seqlens=0x1000, total_tokens=64, out=0x10000000 + 256 * 2 * 10),
+     _lib.ERR_INVALID_ARG),
+    # a state cache of num_slots rows that overlaps out
+    (dict(state_indices=0x2000, num_slots=1 << 20, h_final=0x90000000 - 1024),
+     _lib.ERR_INVALID_ARG),
+])
+def test_serving_layout_argument_errors(L, kw, expect):
+    assert _scan(_valid_scan(**kw)) == expect
+
+
+def test_state_update_slot_argument_errors(L):
+    assert _lib.call_state_update(_valid_update(state_indices=0x3000, num_slots=0), 0) == \
+        _lib.ERR_INVALID_ARG
+    assert _lib.call_state_update(_valid_update(state_indices=0x3002, num_slots=8), 0) == \
+        _lib.ERR_MISALIGNED
+    # a cache of num_slots rows is checked for overlap with out
+    assert _lib.call_state_update(_valid_update(state_indices=0x3000, num_slots=1 << 16,
+                                                out=0x10000000 + (1 << 20)), 0) == \
+        _lib.ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_version_1_struct_size_is_accepted(L):
+    """A caller built against ABI version 1 passes the shorter struct: the
+    serving fields read as absent and validation goes on to the device."""
+    p = _valid_scan()
+    p.struct_size = _lib.SCAN_PARAMS_V1_SIZE
+    p.cu_seqlens = 0x1002  # garbage past the version-1 size: must be ignored
+    assert _scan(p) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
+    p.struct_size = _lib.SCAN_PARAMS_V1_SIZE - 8
+    assert _scan(p) == _lib.ERR_INVALID_ARG
+    u = _valid_update()
+    u.struct_size = _lib.STATE_UPDATE_PARAMS_V1_SIZE
+    u.state_indices = 0x3001
+    assert _lib.call_state_update(u, 0) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
+    u.struct_size = _lib.STATE_UPDATE_PARAMS_V1_SIZE - 8
+    assert _lib.call_state_update(u, 0) == _lib.ERR_INVALID_ARG
