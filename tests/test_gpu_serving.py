@@ -231,3 +231,26 @@ def test_batched_layout_with_state_slots():
         if s >= 0:
             assert_state(final[s], ref_h, torch.bfloat16, f"seq {b}")
     assert (final[[1, 2, 3, 4]] == 0).all()
+
+
+def test_serving_kernel_bounded_wait_times_out_and_reports():
+    """The serving kernel's waits are bounded too: with each task's first tile
+    withheld (test hook) the call records TIMEOUT, and the next call is correct."""
+    dev = _dev()
+    lengths = [70, 0, 33]
+    inp = synth.scan_inputs(3, 70, 128, 16, torch.bfloat16, seed=17, device=dev)
+    cu, x, dt, z, B, C = _pack(inp, lengths, dev)
+    assert jamba_ssm_get_status() == _lib.OK
+    jamba_ssm_scan(x, dt, z, B, C, inp.A, D=inp.D, delta_bias=inp.delta_bias, cu_seqlens=cu,
+                   debug_flags=1, timeout_cycles=2_000_000)
+    assert jamba_ssm_get_status() == _lib.ERR_TIMEOUT
+    assert jamba_ssm_get_status() == _lib.OK
+    out, hf = jamba_ssm_scan(x, dt, z, B, C, inp.A, D=inp.D, delta_bias=inp.delta_bias,
+                             cu_seqlens=cu)
+    torch.cuda.synchronize()
+    for b, L in enumerate(lengths):
+        ref_o, ref_h = _oracle_seq(inp, b, L)
+        o0 = int(cu[b])
+        if L:
+            assert_out(out[o0:o0 + L], ref_o, torch.bfloat16, f"seq {b}")
+        assert_state(hf[b], ref_h, torch.bfloat16, f"seq {b}")
