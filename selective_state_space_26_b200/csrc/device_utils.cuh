@@ -57,11 +57,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
     return bits_f2(r);
 }
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-    uint64_t r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
-    return bits_f2(r);
-}
 
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

@@ -122,15 +122,6 @@ __device__ __forceinline__ void stage_slice(T *dst, const T *src) {
                                         reinterpret_cast<const uint32_t *>(src));
 }
 
-// Sum of v over the G lanes of a channel.  Partners are taken in the order
-// reduce_transpose uses (lane ^ G/2 first), so both give bit-identical sums.
-template <int G>
-__device__ __forceinline__ float lane_group_sum(float v) {
-#pragma unroll
-    for (int off = G / 2; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    return v;
-}
-
 // For G consecutive steps held by each of the G lanes of a channel (v[j] is
 // this lane's partial sum of step j), returns the full sum of step `sub` on
 // lane `sub`: a butterfly where each round keeps the half of the values the

@@ -37,11 +37,11 @@ struct TileHdr {
 template <typename IoT, int N, int G, int NW, int TT, int STAGES>
 __global__ void __launch_bounds__((NW + 1) * 32, 1)
     s6_scan_serving_kernel(const __grid_constant__ CUtensorMap tm_x,
-                         const __grid_constant__ CUtensorMap tm_dt,
-                         const __grid_constant__ CUtensorMap tm_z,
-                         const __grid_constant__ CUtensorMap tm_B,
-                         const __grid_constant__ CUtensorMap tm_C,
-                         const __grid_constant__ CUtensorMap tm_out, const ScanArgs args) {
+                           const __grid_constant__ CUtensorMap tm_dt,
+                           const __grid_constant__ CUtensorMap tm_z,
+                           const __grid_constant__ CUtensorMap tm_B,
+                           const __grid_constant__ CUtensorMap tm_C,
+                           const __grid_constant__ CUtensorMap tm_out, const ScanArgs args) {
     using Cfg = ServingCfg<IoT, N, G, NW, TT, STAGES>;
     constexpr int NS = Cfg::NS, CW = Cfg::CW, CC = Cfg::CC, NOUT = Cfg::NOUT;
     extern __shared__ __align__(1024) uint8_t smem[];
