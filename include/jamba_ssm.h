@@ -35,6 +35,9 @@
  *     jamba_ssm_last_cuda_error).  A device-side condition (a bounded wait that
  *     ran out) is recorded in a per-device status word read by
  *     jamba_ssm_get_status.  No C++ exception crosses this interface.
+ *   - Debugging aid: with the environment variable JAMBA_SSM_SYNC_CHECK set
+ *     (and not "0") when the library is first called, every call waits for
+ *     its work and returns jamba_ssm_get_status()'s result itself.
  */
 #ifndef JAMBA_SSM_H
 #define JAMBA_SSM_H

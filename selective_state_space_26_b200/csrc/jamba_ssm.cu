@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cstddef>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -288,6 +289,24 @@ jamba_ssm_status plan_scan(const jamba_ssm_scan_params *p, const DeviceInfo *dev
 
 }  // namespace
 
+extern "C" jamba_ssm_status jamba_ssm_get_status(void *stream);
+
+namespace {
+
+// After an enqueue: with JAMBA_SSM_SYNC_CHECK set (and not "0") in the
+// environment -- a debugging aid, read once per process -- wait for the work
+// and return any device-side condition it recorded (a timeout, a bad state
+// slot) or launch error as this call's own status.
+jamba_ssm_status finish_launch(cudaStream_t s) {
+    static const bool sync_check = [] {
+        const char *v = std::getenv("JAMBA_SSM_SYNC_CHECK");
+        return v != nullptr && *v != '\0' && *v != '0';
+    }();
+    return sync_check ? jamba_ssm_get_status(s) : JAMBA_SSM_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *jamba_ssm_status_string(jamba_ssm_status s) {
@@ -371,7 +390,7 @@ jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *pin, void *stream) 
         jssm::s6_copy_states_kernel<<<static_cast<unsigned>(blocks), threads, 0, s>>>(
             p->batch, per, p->h0, p->h_final, p->state_indices, p->num_slots);
         cudaError_t e = cudaGetLastError();
-        return e == cudaSuccess ? JAMBA_SSM_OK : cuda_fail(e);
+        return e == cudaSuccess ? finish_launch(s) : cuda_fail(e);
     }
 
     ScanPlan plan;
@@ -436,7 +455,7 @@ jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *pin, void *stream) 
     cudaError_t e = cudaLaunchKernel(kernel, dim3(plan.grid), dim3(v.threads), kargs,
                                      static_cast<size_t>(smem), s);
     if (e != cudaSuccess) return cuda_fail(e);
-    return JAMBA_SSM_OK;
+    return finish_launch(s);
 }
 
 jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *pin, void *stream) {
@@ -517,7 +536,7 @@ jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *pin
         cudaError_t e = cudaLaunchKernel(k, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
                                          dim3(threads), kargs, static_cast<size_t>(smem), s);
         if (e != cudaSuccess) return cuda_fail(e);
-        return JAMBA_SSM_OK;
+        return finish_launch(s);
     }
     constexpr int kBPC = 2;  // requests per block (parameters reused across them)
     const int64_t cpb = 256 / (p->d_state / 4);
@@ -536,7 +555,7 @@ jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *pin
     cudaError_t e = cudaLaunchKernel(k, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
                                      dim3(256), kargs, 0, s);
     if (e != cudaSuccess) return cuda_fail(e);
-    return JAMBA_SSM_OK;
+    return finish_launch(s);
 }
 
 jamba_ssm_status jamba_ssm_get_status(void *stream) {

@@ -210,3 +210,33 @@ def test_bounded_wait_times_out_and_reports():
     ref, _ = run_oracle(inp)
     out, _ = run_gpu(inp)
     assert_out(out, ref, torch.bfloat16, "after timeout")
+
+
+def test_sync_check_environment_returns_device_conditions():
+    """With JAMBA_SSM_SYNC_CHECK=1 a call waits for its kernel and returns the
+    device-side condition it recorded (here a withheld tile's timeout) as its
+    own status; a clean call returns OK.  Run in a child process because the
+    variable is read once per process."""
+    _dev()
+    import subprocess
+    import sys
+    code = (
+        "import torch\n"
+        "from selective_state_space_26_b200 import synth, jamba_ssm_scan, JambaSSMError, _lib\n"
+        "dev = torch.device('cuda', 0)\n"
+        "inp = synth.scan_inputs(1, 100, 128, 16, torch.bfloat16, seed=3, device=dev)\n"
+        "args = (inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A)\n"
+        "try:\n"
+        "    jamba_ssm_scan(*args, debug_flags=1, timeout_cycles=2_000_000)\n"
+        "    print('NO-ERROR')\n"
+        "except JambaSSMError as e:\n"
+        "    print('STATUS', e.status)\n"
+        "jamba_ssm_scan(*args)\n"
+        "print('CLEAN-OK')\n")
+    env = dict(os.environ, JAMBA_SSM_SYNC_CHECK="1")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert f"STATUS {_lib.ERR_TIMEOUT}" in r.stdout, r.stdout
+    assert "CLEAN-OK" in r.stdout, r.stdout
