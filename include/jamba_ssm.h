@@ -177,6 +177,11 @@ jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream);
  *              recorded as JAMBA_SSM_ERR_INVALID_ARG in the status word.
  *              Indices of one call must be distinct.
  *   num_slots  rows of the state cache (state_indices != NULL), >= 1.
+ *   debug_flags / timeout_cycles: 0 in production.  Bit 0 of debug_flags
+ *              withholds the first state load of every CTA of the bulk-copy
+ *              kernel so its bounded wait runs out (test of the timeout path;
+ *              rows of 16-byte multiples take that kernel); timeout_cycles
+ *              overrides the wait limit (SM clock cycles, 0 = ~1 s).
  */
 typedef struct jamba_ssm_state_update_params {
     size_t struct_size;          /* = sizeof(jamba_ssm_state_update_params);
@@ -194,6 +199,8 @@ typedef struct jamba_ssm_state_update_params {
     /* ABI version 2 */
     const int32_t *state_indices;
     int64_t num_slots;
+    uint32_t debug_flags;
+    uint64_t timeout_cycles;
 } jamba_ssm_state_update_params;
 
 jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, void *stream);

@@ -131,7 +131,8 @@ def scan_plan(x, A, B=None, variant: int = 0):
 
 
 def jamba_ssm_state_update(state, x, delta, z, B, C, A, D=None, delta_bias=None,
-                           delta_softplus=True, out=None, stream=None, state_indices=None):
+                           delta_softplus=True, out=None, stream=None, state_indices=None,
+                           debug_flags: int = 0, timeout_cycles: int = 0):
     """One decode step; `state` [batch, d_inner, d_state] fp32 is updated in
     place.  x, delta, z [batch, d_inner]; B, C [batch, d_state].  Returns out
     [batch, d_inner].  With ``state_indices`` (int32 [batch] on the device)
@@ -163,7 +164,8 @@ def jamba_ssm_state_update(state, x, delta, z, B, C, A, D=None, delta_bias=None,
         delta_softplus=int(bool(delta_softplus)), state=_ptr(state), x=_ptr(x),
         delta=_ptr(delta), z=_ptr(z), B=_ptr(B), C=_ptr(C), A=_ptr(A), D=_ptr(D),
         delta_bias=_ptr(delta_bias), out=_ptr(out), state_indices=_ptr(state_indices),
-        num_slots=int(num_slots))
+        num_slots=int(num_slots), debug_flags=int(debug_flags),
+        timeout_cycles=int(timeout_cycles))
     st = _lib.call_state_update(p, _stream(stream, dev))
     if st != _lib.OK:
         raise JambaSSMError(st, "jamba_ssm_state_update")

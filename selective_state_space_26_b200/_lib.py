@@ -61,6 +61,7 @@ class StateUpdateParams(ctypes.Structure):
         ("out", _vp),
         # ABI version 2
         ("state_indices", _vp), ("num_slots", ctypes.c_int64),
+        ("debug_flags", ctypes.c_uint32), ("timeout_cycles", ctypes.c_uint64),
     ]
 
 

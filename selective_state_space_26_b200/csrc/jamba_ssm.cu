@@ -506,6 +506,7 @@ jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *pin
     a.delta_softplus = p->delta_softplus != 0;
     a.state_indices = p->state_indices;
     a.num_slots = p->num_slots;
+    a.debug_flags = p->debug_flags;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool bf = p->io_dtype == JAMBA_SSM_BF16;
     // Streaming kernel when every slice is a whole number of 16-byte chunks.
@@ -531,7 +532,7 @@ jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *pin
             default: if (bf) JSSM_STREAM(__nv_bfloat16, 16); else JSSM_STREAM(float, 16); break;
         }
 #undef JSSM_STREAM
-        uint64_t limit = uint64_t(1) << 31;
+        uint64_t limit = p->timeout_cycles ? p->timeout_cycles : (uint64_t(1) << 31);
         void *kargs[] = {&a, &limit};
         cudaError_t e = cudaLaunchKernel(k, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
                                          dim3(threads), kargs, static_cast<size_t>(smem), s);

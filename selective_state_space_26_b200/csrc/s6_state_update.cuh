@@ -32,6 +32,7 @@ struct UpdateArgs {
     int delta_softplus;
     const int *state_indices;  // state-cache row of each request, or null (row b)
     int64_t num_slots;         // rows of the state cache
+    uint32_t debug_flags;      // bit 0: withhold each CTA's first load (tests the bounded waits)
 };
 
 // State-cache row of request b, or -1 when the request is skipped (a negative
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(UpdateCfg<IoT, N, CPB, STAGES>::kThreads, 4)
             const uint32_t state_bytes = static_cast<uint32_t>(nd) * N * 4;
             const uint32_t act_bytes = static_cast<uint32_t>(nd) * sizeof(IoT);
             int issued = 0;
-            bool ok = true;
+            bool ok = true, withheld0 = false;
             for (int u = 0; u < nu; ++u) {
                 const int s = u % STAGES;
                 if (u >= STAGES &&
@@ -217,6 +218,11 @@ __global__ void __launch_bounds__(UpdateCfg<IoT, N, CPB, STAGES>::kThreads, 4)
                                         abort_flag)) {
                     ok = false;
                     break;
+                }
+                if ((a.debug_flags & 1u) && u == 0) {  // test hook: this load never comes
+                    withheld0 = true;
+                    issued = 1;
+                    continue;
                 }
                 uint8_t *st = smem + s * Cfg::kStage;
                 const int64_t b = breq0 + u, row = b * a.d_inner + d0;
@@ -240,7 +246,8 @@ __global__ void __launch_bounds__(UpdateCfg<IoT, N, CPB, STAGES>::kThreads, 4)
             // copies still in flight when the compute warps may have left:
             // wait (bounded) for each stage's last fill before the CTA exits
             for (int u = issued - STAGES > 0 ? issued - STAGES : 0; u < issued; ++u)
-                mbar_wait_bounded(&full[u % STAGES], static_cast<uint32_t>(u / STAGES) & 1u, limit);
+                if (!(withheld0 && u == 0))
+                    mbar_wait_bounded(&full[u % STAGES], static_cast<uint32_t>(u / STAGES) & 1u, limit);
         }
         return;
     }

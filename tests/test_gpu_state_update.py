@@ -73,3 +73,26 @@ def test_odd_sizes_and_ragged_grid():
                                           delta_bias=bias)
     assert_out(out, ref_out, torch.bfloat16)
     assert_state(st, ref_st, torch.bfloat16)
+
+
+def test_bounded_wait_times_out_and_reports():
+    """The bulk-copy decode kernel's waits are bounded: with each CTA's first
+    load withheld (test hook) the call records TIMEOUT and leaves; the context
+    stays usable and the next call matches the oracle."""
+    from selective_state_space_26_b200 import _lib, jamba_ssm_get_status
+    dev = _dev()
+    A, D, bias = _params(128, 16, 3, dev)
+    st = synth.decode_state(40, 128, 16, seed=3, device=dev)
+    s = synth.decode_step(40, 128, 16, 0, 3, torch.bfloat16, dev)
+    assert jamba_ssm_get_status() == _lib.OK
+    work = st.clone()
+    jamba_ssm_state_update(work, s.x, s.delta, s.z, s.B, s.C, A, D=D, delta_bias=bias,
+                           debug_flags=1, timeout_cycles=2_000_000)
+    assert jamba_ssm_get_status() == _lib.ERR_TIMEOUT
+    assert jamba_ssm_get_status() == _lib.OK
+    work = st.clone()
+    out = jamba_ssm_state_update(work, s.x, s.delta, s.z, s.B, s.C, A, D=D, delta_bias=bias)
+    torch.cuda.synchronize()
+    ref_out, ref_st = oracle.state_update(st, s.x, s.delta, s.z, s.B, s.C, A, D=D, delta_bias=bias)
+    assert_out(out, ref_out, torch.bfloat16, "after timeout")
+    assert_state(work, ref_st, torch.bfloat16, "after timeout")
