@@ -1,8 +1,8 @@
 // s6_scan_fused.cuh -- prefill selective scan (S6), fused-warp form (sm_100a).
 //
-// Same computation as s6_scan.cuh (the recurrence of the "Mamba 레이어"
-// section of the Jamba notes, read as h = exp(Delta A) h + Delta B x,
-// out = (C.h + D x) silu(z), Delta = softplus(delta + bias)), organised so
+// The recurrence of the "Mamba 레이어" section of the Jamba notes, read as
+// h = exp(Delta A) h + Delta B x, out = (C.h + D x) silu(z),
+// Delta = softplus(delta + bias) (per-step pieces in s6_scan.cuh), organised so
 // that every warp that carries states also does the per-(t, d) scalar work of
 // its own channels -- no hand-off of Delta or of C.h through shared memory:
 //

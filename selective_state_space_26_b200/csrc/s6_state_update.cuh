@@ -8,13 +8,16 @@
 //     out   = (sum_n C[b,n] h[n] + D[d] x[b,d]) * silu(z[b,d])
 //
 // The fp32 state dominates the bytes (it is read and written once per step),
-// so the kernel is a streaming, HBM-bound pass: Q = N/4 consecutive lanes own
-// one (b, d) and each moves one float4 of its state with a 128-bit load and
-// store (a warp touches 512 contiguous bytes); each thread does UNITS such
-// float4s so enough loads are in flight to cover the HBM latency.  The partial
-// sums of C.h are combined with Q-1 xor-shuffles; the per-(b, d) scalars (softplus, gate) are
-// recomputed by each of the Q lanes, which costs MUFU issue slots that this
-// memory-bound kernel has to spare.
+// so both kernels are streaming, HBM-bound passes in which Q = N/4 lanes own
+// one (request, channel), 4 states each, moved as one 16-byte load and store:
+//  * s6_state_update_stream_kernel (rows of whole 16-byte chunks, the usual
+//    case): a producer warp streams each request's state slab and activations
+//    into a ring of shared-memory stages with 1-D bulk copies; the lanes of a
+//    channel take requests Q at a time, lane q computing request q's softplus
+//    and gate once and handing Delta, Delta x over by shuffles.
+//  * s6_state_update_kernel (any other row size): plain vector loads, two
+//    requests in flight per thread, each of the Q lanes computing the scalars.
+// The partial sums of C.h are combined across the Q lanes with shuffles.
 #pragma once
 
 #include "device_utils.cuh"
