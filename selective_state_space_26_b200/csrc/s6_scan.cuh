@@ -1,6 +1,8 @@
-// s6_scan.cuh -- pieces shared by the S6 prefill kernel (s6_scan_fused.cuh):
-// the device status word, the kernel arguments, B/C widening, and one step of
-// a lane's selective-scan recurrence.
+// s6_scan.cuh -- pieces shared by the S6 prefill kernels (s6_scan_fused.cuh,
+// s6_scan_serving.cuh) and the decode kernels: the scan arguments, the state
+// copy for calls without steps, the staging of B / C into per-lane slots, the
+// transposing butterfly over a channel's lanes, and one step of a lane's
+// selective-scan recurrence.
 //
 // The recurrence (the "Mamba 레이어" section of the Jamba notes, with the
 // discretisation read as exp(Delta A) and Delta B x):
@@ -13,7 +15,6 @@
 #include "s6_math.cuh"
 
 namespace jssm {
-
 
 struct ScanArgs {
     int64_t batch, seqlen, d_inner;
