@@ -1,0 +1,69 @@
+"""Property-based pins of the oracle (CPU): for randomly drawn tiny problems --
+shapes, optional D / delta_bias / h0, softplus on or off, random negative A --
+the sequential fp64 oracle equals the brute-force unrolled sums of the
+recurrence, and the scan is causal and split-invariant."""
+import numpy as np
+from hypothesis import given, settings
+from hypothesis import strategies as st
+
+import oracle
+from tests.oracle_pins import _close, bruteforce
+
+
+@st.composite
+def problems(draw):
+    batch = draw(st.integers(1, 2))
+    seqlen = draw(st.integers(1, 12))
+    d_inner = draw(st.integers(1, 3))
+    d_state = draw(st.sampled_from([1, 2, 4, 8]))
+    seed = draw(st.integers(0, 2**31 - 1))
+    softplus = draw(st.booleans())
+    r = np.random.default_rng(seed)
+    case = dict(
+        x=r.standard_normal((batch, seqlen, d_inner)),
+        delta=r.standard_normal((batch, seqlen, d_inner)),
+        z=r.standard_normal((batch, seqlen, d_inner)),
+        B=r.standard_normal((batch, seqlen, d_state)),
+        C=r.standard_normal((batch, seqlen, d_state)),
+        A=-np.exp(r.standard_normal((d_inner, d_state))),
+        D=r.standard_normal(d_inner) if draw(st.booleans()) else None,
+        delta_bias=r.uniform(-3.0, 0.5, d_inner) if draw(st.booleans()) else None,
+        h0=r.standard_normal((batch, d_inner, d_state)) if draw(st.booleans()) else None,
+    )
+    if not softplus:  # keep Delta positive and O(0.1) without softplus
+        case["delta"] = np.abs(case["delta"]) * 0.1
+        case["delta_bias"] = None
+    return case, softplus
+
+
+@settings(max_examples=60, deadline=None)
+@given(problems())
+def test_oracle_equals_bruteforce(p):
+    case, sp = p
+    out, hf = oracle.scan(**case, delta_softplus=sp)
+    ref_out, ref_hf = bruteforce(case, sp)
+    _close(out, ref_out, 1e-11, "out")
+    _close(hf, ref_hf, 1e-11, "h_final")
+
+
+@settings(max_examples=30, deadline=None)
+@given(problems(), st.integers(0, 11))
+def test_split_and_causality(p, cut):
+    case, sp = p
+    L = case["x"].shape[1]
+    cut = min(cut, L)
+    out, hf = oracle.scan(**case, delta_softplus=sp)
+    # scanning [0, cut) then [cut, L) from the intermediate state is the same scan
+    first = {k: (v[:, :cut] if k in ("x", "delta", "z", "B", "C") else v) for k, v in case.items()}
+    o1, h1 = oracle.scan(**first, delta_softplus=sp)
+    second = {k: (v[:, cut:] if k in ("x", "delta", "z", "B", "C") else v) for k, v in case.items()}
+    second["h0"] = h1
+    o2, h2 = oracle.scan(**second, delta_softplus=sp)
+    _close(np.concatenate([o1, o2], axis=1), out, 1e-12, "split out")
+    _close(h2, hf, 1e-12, "split h_final")
+    # outputs before `cut` do not depend on inputs from `cut` on
+    if cut < L:
+        changed = dict(case, x=case["x"].copy())
+        changed["x"][:, cut:] += 1.0
+        oc, _ = oracle.scan(**changed, delta_softplus=sp)
+        assert np.array_equal(oc[:, :cut], out[:, :cut])
