@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from selective_state_space_26_b200 import (JambaSSMError, jamba_ssm_get_status, jamba_ssm_scan,
-                                           synth)
+                                           scan_plan, synth)
 from selective_state_space_26_b200 import _lib
 from tests.parity import assert_out, assert_state
 
@@ -240,3 +240,19 @@ def test_sync_check_environment_returns_device_conditions():
     assert r.returncode == 0, r.stderr[-2000:]
     assert f"STATUS {_lib.ERR_TIMEOUT}" in r.stdout, r.stdout
     assert "CLEAN-OK" in r.stdout, r.stdout
+
+
+def test_launch_shape_for_jamba_layers():
+    """The cost model picks narrow CTAs for one sequence, so its 8192 channels
+    cover the SMs, and the cheapest per-step variant once the batch fills them."""
+    dev = _dev()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    A = torch.empty(8192, 16, device=dev)
+    one = torch.empty(1, 4096, 8192, dtype=torch.bfloat16, device=dev)
+    plan = scan_plan(one, A)
+    assert plan["channels_per_cta"] == 56 and plan["lanes_per_channel"] == 4
+    assert plan["grid"] == min(sms, 147) and plan["tasks"] == 147
+    many = torch.empty(16, 64, 8192, dtype=torch.bfloat16, device=dev)
+    plan = scan_plan(many, A)
+    assert plan["channels_per_cta"] == 128 and plan["lanes_per_channel"] == 2
+    assert plan["grid"] == sms and plan["tasks"] == 16 * 64
