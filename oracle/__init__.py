@@ -12,6 +12,10 @@ widens inputs to float64 and splits the independent channels across host
 threads (ctypes releases the GIL during the call), which does not change the
 order of any floating-point operation inside a channel.
 
+``scan_packed`` and ``state_update_slots`` define the serving layouts (packed
+variable-length batches, state-cache slots) as loops over the batched
+definitions.
+
 Sources: "Jamba: A Hybrid Transformer-Mamba Language Model" (obsidian-dorae222
 notes), section "Mamba 레이어" -- the S6 recurrence h_t = Abar_t h_{t-1} +
 Bbar_t x_t, y_t = C_t h_t with input-dependent Bbar, C, Delta; and "Jamba --
@@ -151,4 +155,72 @@ def state_update(state, x, delta, z, B, C, A, D=None, delta_bias=None,
                                      int(bool(delta_softplus)), _ptr(out))
     if rc != 0:
         raise ValueError("oracle_state_update_f64 rejected its arguments")
+    return out, st
+
+
+def scan_packed(x, delta, z, B, C, A, cu_seqlens, D=None, delta_bias=None,
+                delta_softplus=True, h0=None, state_indices=None, threads: int = 1, lib=None):
+    """The packed variable-length layout, by definition one `scan` per sequence.
+
+    x, delta, z [total_tokens, d_inner] and B, C [total_tokens, d_state] hold
+    sequence b in rows cu_seqlens[b] .. cu_seqlens[b+1]-1.  Without
+    `state_indices`, h0 is [batch, d_inner, d_state] (or None) and the final
+    states are returned as [batch, d_inner, d_state].  With it, h0 is a
+    [num_slots, d_inner, d_state] cache (or None), sequence b starts from row
+    state_indices[b] (zero for a negative index) and the returned cache is h0
+    with row state_indices[b] replaced by sequence b's final state (rows of
+    negative indices untouched).  An empty sequence's final state is its
+    initial state.  Returns (out [total_tokens, d_inner], final states).
+    """
+    x, delta, z, B, C, A = map(_f64, (x, delta, z, B, C, A))
+    cu = np.asarray(_f64(cu_seqlens), dtype=np.int64)
+    h0 = _f64(h0)
+    batch = cu.size - 1
+    d_inner, d_state = A.shape
+    out = np.zeros((x.shape[0], d_inner), dtype=np.float64)
+    if state_indices is not None:
+        idx = np.asarray(_f64(state_indices), dtype=np.int64)
+        final = (h0.copy() if h0 is not None else None)
+    else:
+        final = np.zeros((batch, d_inner, d_state), dtype=np.float64)
+    for b in range(batch):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        if state_indices is not None:
+            row = int(idx[b])
+            init = h0[row] if (row >= 0 and h0 is not None) else np.zeros((d_inner, d_state))
+        else:
+            init = h0[b] if h0 is not None else np.zeros((d_inner, d_state))
+        if hi > lo:
+            o, hf = scan(x[None, lo:hi], delta[None, lo:hi], z[None, lo:hi], B[None, lo:hi],
+                         C[None, lo:hi], A, D=D, delta_bias=delta_bias,
+                         delta_softplus=delta_softplus, h0=init[None], threads=threads, lib=lib)
+            out[lo:hi] = o[0]
+            hf = hf[0]
+        else:
+            hf = np.array(init, dtype=np.float64)
+        if state_indices is None:
+            final[b] = hf
+        elif row >= 0:
+            if final is None:
+                final = np.zeros((int(idx.max()) + 1, d_inner, d_state), dtype=np.float64)
+            final[row] = hf
+    return out, final
+
+
+def state_update_slots(cache, x, delta, z, B, C, A, state_indices, D=None, delta_bias=None,
+                       delta_softplus=True, lib=None):
+    """One decode step through a state cache: request b updates row
+    state_indices[b]; a negative index skips the request.  Returns (out
+    [batch, d_inner] with NaN rows for skipped requests, the updated cache)."""
+    st = _f64(cache).copy()
+    idx = np.asarray(_f64(state_indices), dtype=np.int64)
+    x, delta, z, B, C = map(_f64, (x, delta, z, B, C))
+    live = [b for b in range(idx.size) if idx[b] >= 0]
+    out = np.full(x.shape, np.nan)
+    if live:
+        rows = idx[live]
+        o, new = state_update(st[rows], x[live], delta[live], z[live], B[live], C[live], A, D=D,
+                              delta_bias=delta_bias, delta_softplus=delta_softplus, lib=lib)
+        out[live] = o
+        st[rows] = new
     return out, st
