@@ -12,7 +12,9 @@ widens inputs to float64 and splits the independent channels across host
 threads (ctypes releases the GIL during the call), which does not change the
 order of any floating-point operation inside a channel.
 
-``scan_packed`` and ``state_update_slots`` define the serving layouts (packed
+``project`` is the step before the scan (Delta, B and C from the scan's
+input through the x / dt projections and RMSNorm).  ``scan_packed`` and
+``state_update_slots`` define the serving layouts (packed
 variable-length batches, state-cache slots) as loops over the batched
 definitions.
 
@@ -57,6 +59,9 @@ def _declare(lib):
     lib.oracle_silu.argtypes = [ctypes.c_double]
     lib.oracle_scan_f64.restype = ctypes.c_int
     lib.oracle_scan_f64.argtypes = [_i64] * 6 + [_dp] * 8 + [ctypes.c_int, _dp, _dp, _dp]
+    lib.oracle_project_f64.restype = ctypes.c_int
+    lib.oracle_project_f64.argtypes = ([_i64] * 6 + [_dp] * 6 + [ctypes.c_double]
+                                       + [_dp] * 3)
     lib.oracle_state_update_f64.restype = ctypes.c_int
     lib.oracle_state_update_f64.argtypes = ([_i64] * 3 + [_dp] * 9
                                             + [ctypes.c_int, _dp])
@@ -156,6 +161,47 @@ def state_update(state, x, delta, z, B, C, A, D=None, delta_bias=None,
     if rc != 0:
         raise ValueError("oracle_state_update_f64 rejected its arguments")
     return out, st
+
+
+def project(u, W_x, W_dt, d_state, w_dt=None, w_B=None, w_C=None, eps=1e-6,
+            threads: int = 1, lib=None):
+    """Delta (raw, before bias and softplus), B and C of every token from the
+    scan's input u, in fp64.
+
+    u [..., d_inner]; W_x [dt_rank + 2 d_state, d_inner]; W_dt [d_inner,
+    dt_rank]; w_dt [dt_rank], w_B / w_C [d_state] are RMSNorm weights (None: that
+    part is not normalised).  Returns (delta [..., d_inner], B [..., d_state],
+    C [..., d_state]).
+    """
+    lib = lib or load()
+    u, W_x, W_dt = map(_f64, (u, W_x, W_dt))
+    w_dt, w_B, w_C = map(_f64, (w_dt, w_B, w_C))
+    lead = u.shape[:-1]
+    d_inner = u.shape[-1]
+    dt_rank = W_dt.shape[1]
+    assert W_x.shape == (dt_rank + 2 * d_state, d_inner) and W_dt.shape == (d_inner, dt_rank)
+    u2 = u.reshape(-1, d_inner)
+    ntok = u2.shape[0]
+    delta = np.empty((ntok, d_inner))
+    B = np.empty((ntok, d_state))
+    C = np.empty((ntok, d_state))
+
+    def run(lo, hi):
+        rc = lib.oracle_project_f64(ntok, d_inner, dt_rank, d_state, lo, hi, _ptr(u2),
+                                    _ptr(W_x), _ptr(W_dt), _ptr(w_dt), _ptr(w_B), _ptr(w_C),
+                                    float(eps), _ptr(delta), _ptr(B), _ptr(C))
+        if rc != 0:
+            raise ValueError("oracle_project_f64 rejected its arguments")
+
+    threads = max(1, min(int(threads), ntok))
+    if threads == 1:
+        run(0, ntok)
+    else:
+        bounds = np.linspace(0, ntok, threads + 1).astype(np.int64)
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(lambda i: run(int(bounds[i]), int(bounds[i + 1])), range(threads)))
+    return (delta.reshape(*lead, d_inner), B.reshape(*lead, d_state),
+            C.reshape(*lead, d_state))
 
 
 def scan_packed(x, delta, z, B, C, A, cu_seqlens, D=None, delta_bias=None,

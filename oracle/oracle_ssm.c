@@ -30,11 +30,14 @@
  *
  * Parity: this file is pinned by tests/test_oracle_pins.py (brute-force
  * unrolled sums, the geometric-series closed form, the Delta->0 and large-Delta
- * limits, libm softplus/silu, split-scan and decode==scan identities).
+ * limits, libm softplus/silu, split-scan and decode==scan identities) and, for
+ * the projection that produces Delta, B and C, by tests/oracle_proj_pins.py
+ * (basis-vector selections, associativity, rank, RMSNorm closed forms).
  */
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 /* softplus(v) = log(1 + e^v), written in the form that does not overflow. */
 double oracle_softplus(double v) {
@@ -137,5 +140,68 @@ int oracle_state_update_f64(int64_t batch, int64_t d_inner, int64_t d_state,
             out[i] = (y + skip) * oracle_silu(z[i]);
         }
     }
+    return 0;
+}
+
+/*
+ * The step before the scan: "Bbar_t, C_t, Delta_t = f(x_t)" (obsidian-dorae222
+ * notes, section "Mamba 레이어"), with the RMSNorm the same section says Jamba
+ * adds to the Mamba layer against training instability.  The pages do not
+ * spell f out; the reading taken is the Mamba-1 one:
+ *   xdbl_t  = W_x u_t                        (one linear map of the token)
+ *   dt_low  = xdbl_t[0 .. R-1],  B_t = xdbl_t[R .. R+N-1],  C_t = xdbl_t[R+N .. R+2N-1]
+ *   each of dt_low, B_t, C_t optionally RMS-normalised over its own entries:
+ *       v_i <- w_i * v_i / sqrt(mean_j v_j^2 + eps)
+ *   delta_t = W_dt dt_low                    (low-rank, rank R = dt_rank)
+ * delta is the raw input of the scan: the per-channel bias and the softplus are
+ * the scan's own first step, so they are not applied here.
+ *   u      : [ntok, d_inner]
+ *   W_x    : [dt_rank + 2 * d_state, d_inner]
+ *   W_dt   : [d_inner, dt_rank]
+ *   w_dt, w_B, w_C : RMSNorm weights [dt_rank], [d_state], [d_state], or NULL
+ *            (no normalisation of that part)
+ *   delta  : [ntok, d_inner]      B, C : [ntok, d_state]
+ * Tokens [t_lo, t_hi) are computed, so a caller may split them across threads.
+ * Returns 0, or -1 on a bad argument.
+ */
+static void oracle_rmsnorm(double *v, int64_t len, const double *w, double eps) {
+    double ss = 0.0;
+    for (int64_t i = 0; i < len; ++i) ss += v[i] * v[i];
+    double inv = 1.0 / sqrt(ss / (double)len + eps);
+    for (int64_t i = 0; i < len; ++i) v[i] = w[i] * (v[i] * inv);
+}
+
+int oracle_project_f64(int64_t ntok, int64_t d_inner, int64_t dt_rank, int64_t d_state,
+                       int64_t t_lo, int64_t t_hi,
+                       const double *u, const double *W_x, const double *W_dt,
+                       const double *w_dt, const double *w_B, const double *w_C, double eps,
+                       double *delta, double *B, double *C) {
+    if (ntok < 0 || d_inner < 1 || dt_rank < 1 || d_state < 1) return -1;
+    if (t_lo < 0 || t_hi > ntok || t_lo > t_hi || !(eps >= 0.0)) return -1;
+    int64_t rows = dt_rank + 2 * d_state;
+    double *xdbl = (double *)malloc((size_t)rows * sizeof(double));
+    if (!xdbl) return -1;
+    for (int64_t t = t_lo; t < t_hi; ++t) {
+        const double *ut = u + t * d_inner;
+        for (int64_t j = 0; j < rows; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < d_inner; ++k) acc += W_x[j * d_inner + k] * ut[k];
+            xdbl[j] = acc;
+        }
+        double *dt_low = xdbl, *Bv = xdbl + dt_rank, *Cv = xdbl + dt_rank + d_state;
+        if (w_dt) oracle_rmsnorm(dt_low, dt_rank, w_dt, eps);
+        if (w_B) oracle_rmsnorm(Bv, d_state, w_B, eps);
+        if (w_C) oracle_rmsnorm(Cv, d_state, w_C, eps);
+        for (int64_t n = 0; n < d_state; ++n) {
+            B[t * d_state + n] = Bv[n];
+            C[t * d_state + n] = Cv[n];
+        }
+        for (int64_t d = 0; d < d_inner; ++d) {
+            double acc = 0.0;
+            for (int64_t r = 0; r < dt_rank; ++r) acc += W_dt[d * dt_rank + r] * dt_low[r];
+            delta[t * d_inner + d] = acc;
+        }
+    }
+    free(xdbl);
     return 0;
 }
