@@ -28,6 +28,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -53,10 +54,20 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_SM_MHZ, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(unit: str = "jamba_ssm.cu"):
+    """Hash of the sources of one translation unit of the library: the .cu
+    file and every csrc header it includes, directly or not."""
     d = os.path.join(ROOT, "selective_state_space_26_b200", "csrc")
+    files, todo = set(), [unit]
+    while todo:
+        f = todo.pop()
+        if f in files or not os.path.exists(os.path.join(d, f)):
+            continue
+        files.add(f)
+        with open(os.path.join(d, f)) as fh:
+            todo += re.findall(r'^#include "([^"]+)"', fh.read(), re.M)
     h = hashlib.sha256()
-    for f in sorted(os.listdir(d)):
+    for f in sorted(files):
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]

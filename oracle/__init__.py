@@ -62,6 +62,8 @@ def _declare(lib):
     lib.oracle_project_f64.restype = ctypes.c_int
     lib.oracle_project_f64.argtypes = ([_i64] * 6 + [_dp] * 6 + [ctypes.c_double]
                                        + [_dp] * 3)
+    lib.oracle_dt_proj_f64.restype = ctypes.c_int
+    lib.oracle_dt_proj_f64.argtypes = [_i64] * 5 + [_dp] * 3
     lib.oracle_state_update_f64.restype = ctypes.c_int
     lib.oracle_state_update_f64.argtypes = ([_i64] * 3 + [_dp] * 9
                                             + [ctypes.c_int, _dp])
@@ -202,6 +204,32 @@ def project(u, W_x, W_dt, d_state, w_dt=None, w_B=None, w_C=None, eps=1e-6,
             list(ex.map(lambda i: run(int(bounds[i]), int(bounds[i + 1])), range(threads)))
     return (delta.reshape(*lead, d_inner), B.reshape(*lead, d_state),
             C.reshape(*lead, d_state))
+
+
+def dt_proj(dt_low, W_dt, threads: int = 1, lib=None):
+    """The last product of `project` alone: delta = dt_low @ W_dt.T in fp64.
+    dt_low [..., dt_rank]; W_dt [d_inner, dt_rank].  Returns delta [..., d_inner]."""
+    lib = lib or load()
+    dt_low, W_dt = _f64(dt_low), _f64(W_dt)
+    d_inner, dt_rank = W_dt.shape
+    lead = dt_low.shape[:-1]
+    a = dt_low.reshape(-1, dt_rank)
+    ntok = a.shape[0]
+    delta = np.empty((ntok, d_inner))
+
+    def run(lo, hi):
+        if lib.oracle_dt_proj_f64(ntok, d_inner, dt_rank, lo, hi, _ptr(a), _ptr(W_dt),
+                                  _ptr(delta)) != 0:
+            raise ValueError("oracle_dt_proj_f64 rejected its arguments")
+
+    threads = max(1, min(int(threads), ntok))
+    if threads == 1:
+        run(0, ntok)
+    else:
+        bounds = np.linspace(0, ntok, threads + 1).astype(np.int64)
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(lambda i: run(int(bounds[i]), int(bounds[i + 1])), range(threads)))
+    return delta.reshape(*lead, d_inner)
 
 
 def scan_packed(x, delta, z, B, C, A, cu_seqlens, D=None, delta_bias=None,

@@ -171,6 +171,16 @@ static void oracle_rmsnorm(double *v, int64_t len, const double *w, double eps) 
     for (int64_t i = 0; i < len; ++i) v[i] = w[i] * (v[i] * inv);
 }
 
+/* delta_row[d] = sum_r W_dt[d, r] * dt_low[r]: the rank-R map of one token. */
+static void oracle_low_rank_row(int64_t d_inner, int64_t dt_rank, const double *W_dt,
+                                const double *dt_low, double *delta_row) {
+    for (int64_t d = 0; d < d_inner; ++d) {
+        double acc = 0.0;
+        for (int64_t r = 0; r < dt_rank; ++r) acc += W_dt[d * dt_rank + r] * dt_low[r];
+        delta_row[d] = acc;
+    }
+}
+
 int oracle_project_f64(int64_t ntok, int64_t d_inner, int64_t dt_rank, int64_t d_state,
                        int64_t t_lo, int64_t t_hi,
                        const double *u, const double *W_x, const double *W_dt,
@@ -196,12 +206,22 @@ int oracle_project_f64(int64_t ntok, int64_t d_inner, int64_t dt_rank, int64_t d
             B[t * d_state + n] = Bv[n];
             C[t * d_state + n] = Cv[n];
         }
-        for (int64_t d = 0; d < d_inner; ++d) {
-            double acc = 0.0;
-            for (int64_t r = 0; r < dt_rank; ++r) acc += W_dt[d * dt_rank + r] * dt_low[r];
-            delta[t * d_inner + d] = acc;
-        }
+        oracle_low_rank_row(d_inner, dt_rank, W_dt, dt_low, delta + t * d_inner);
     }
     free(xdbl);
+    return 0;
+}
+
+/*
+ * The last product of the step alone, for tokens [t_lo, t_hi):
+ *   delta[t, d] = sum_r W_dt[d, r] * dt_low[t, r]
+ *   dt_low : [ntok, dt_rank]   W_dt : [d_inner, dt_rank]   delta : [ntok, d_inner]
+ */
+int oracle_dt_proj_f64(int64_t ntok, int64_t d_inner, int64_t dt_rank, int64_t t_lo,
+                       int64_t t_hi, const double *dt_low, const double *W_dt, double *delta) {
+    if (ntok < 0 || d_inner < 1 || dt_rank < 1) return -1;
+    if (t_lo < 0 || t_hi > ntok || t_lo > t_hi) return -1;
+    for (int64_t t = t_lo; t < t_hi; ++t)
+        oracle_low_rank_row(d_inner, dt_rank, W_dt, dt_low + t * dt_rank, delta + t * d_inner);
     return 0;
 }

@@ -1,12 +1,14 @@
 """B200-native Mamba-1 selective scan (S6): Python binding of the C ABI.
 
-Two calls, with the names of the C entry points:
+The calls, with the names of the C entry points:
 
 * ``jamba_ssm_scan``          -- prefill scan over whole sequences, returning the
   gated output and (for the decode cache) the final state;
-* ``jamba_ssm_state_update``  -- one-token decode step, state updated in place.
+* ``jamba_ssm_state_update``  -- one-token decode step, state updated in place;
+* ``jamba_ssm_dt_proj``       -- the low-rank product that produces the scan's
+  raw Delta from dt_low (libjamba_ssm_proj.so).
 
-Every step of the computation runs in the CUDA kernels of libjamba_ssm.so; this
+Every step of the computation runs in the CUDA kernels of the libraries; this
 module only checks tensor metadata, allocates outputs with PyTorch when the
 caller does not pass them, and hands raw device pointers and the current CUDA
 stream to the library.  There is no CPU fallback: without the built library or
@@ -20,7 +22,7 @@ from . import _lib
 from ._lib import JambaSSMError
 
 __all__ = ["jamba_ssm_scan", "jamba_ssm_state_update", "jamba_ssm_get_status", "scan_plan",
-           "JambaSSMError"]
+           "jamba_ssm_dt_proj", "jamba_ssm_proj_get_status", "JambaSSMError"]
 
 _IO = {torch.bfloat16: _lib.BF16, torch.float32: _lib.F32}
 
@@ -177,3 +179,43 @@ def jamba_ssm_get_status(stream=None, device=None) -> int:
     dev = torch.device(device) if device is not None else torch.device("cuda",
                                                                         torch.cuda.current_device())
     return _lib.get_status(_stream(stream, dev))
+
+
+def jamba_ssm_dt_proj(dt_low_hi, W_dt, dt_low_lo=None, out=None, timeout_cycles=0, stream=None):
+    """delta = (dt_low_hi + dt_low_lo) @ W_dt.T in fp32, rounded once to bf16.
+
+    dt_low_hi / dt_low_lo: [..., dt_rank] bf16, the two planes of the fp32
+    dt_low (lo may be None); W_dt: [d_inner, dt_rank] bf16.  Returns delta
+    [..., d_inner] bf16 (written into ``out`` when given).
+    """
+    dev = dt_low_hi.device
+    if dev.type != "cuda":
+        raise ValueError("jamba_ssm_dt_proj needs CUDA tensors; there is no CPU path")
+    d_inner, dt_rank = W_dt.shape
+    lead = tuple(dt_low_hi.shape[:-1])
+    _check(dt_low_hi, "dt_low_hi", lead + (dt_rank,), torch.bfloat16, dev)
+    _check(dt_low_lo, "dt_low_lo", lead + (dt_rank,), torch.bfloat16, dev)
+    _check(W_dt, "W_dt", (d_inner, dt_rank), torch.bfloat16, dev)
+    if out is None:
+        out = torch.empty(lead + (d_inner,), dtype=torch.bfloat16, device=dev)
+    _check(out, "out", lead + (d_inner,), torch.bfloat16, dev)
+    ntok = 1
+    for n in lead:
+        ntok *= n
+    p = _lib.new_dt_proj_params(ntok=ntok, d_inner=d_inner, dt_rank=dt_rank,
+                                dt_low_hi=_ptr(dt_low_hi), dt_low_lo=_ptr(dt_low_lo),
+                                W_dt=_ptr(W_dt), delta=_ptr(out),
+                                timeout_cycles=int(timeout_cycles))
+    st = _lib.call_dt_proj(p, _stream(stream, dev))
+    if st != _lib.OK:
+        raise JambaSSMError(st, "jamba_ssm_dt_proj",
+                            cuda_error=_lib.proj_lib().jamba_ssm_proj_last_cuda_error())
+    return out
+
+
+def jamba_ssm_proj_get_status(stream=None, device=None):
+    """Wait for the stream and return (and clear) the projection library's
+    device-side status (0 = ok)."""
+    dev = torch.device(device) if device is not None else torch.device("cuda",
+                                                                        torch.cuda.current_device())
+    return _lib.proj_get_status(_stream(stream, dev))

@@ -1,7 +1,8 @@
-"""ctypes view of the C ABI in include/jamba_ssm.h (argument marshalling only).
+"""ctypes view of the C ABIs in include/jamba_ssm.h and include/jamba_ssm_proj.h
+(argument marshalling only).
 
-The structures below mirror the header field by field.  Loading fails loudly
-when libjamba_ssm.so has not been built: there is no fallback path.
+The structures below mirror the headers field by field.  Loading fails loudly
+when a library has not been built: there is no fallback path.
 """
 from __future__ import annotations
 
@@ -11,6 +12,7 @@ import threading
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libjamba_ssm.so")
+PROJ_LIB_PATH = os.path.join(_PKG, "libjamba_ssm_proj.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_NO_DEVICE = range(7)
 BF16, F32 = 0, 1
@@ -25,6 +27,13 @@ EXPORTS = (
     "jamba_ssm_last_cuda_error",
     "jamba_ssm_status_string",
     "jamba_ssm_abi_version",
+)
+# Every symbol jamba_ssm_proj.h declares.
+PROJ_EXPORTS = (
+    "jamba_ssm_dt_proj",
+    "jamba_ssm_proj_get_status",
+    "jamba_ssm_proj_last_cuda_error",
+    "jamba_ssm_proj_abi_version",
 )
 
 _vp = ctypes.c_void_p
@@ -65,17 +74,28 @@ class StateUpdateParams(ctypes.Structure):
     ]
 
 
+class DtProjParams(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t),
+        ("ntok", ctypes.c_int64), ("d_inner", ctypes.c_int64), ("dt_rank", ctypes.c_int64),
+        ("dt_low_hi", _vp), ("dt_low_lo", _vp), ("W_dt", _vp), ("delta", _vp),
+        ("timeout_cycles", ctypes.c_uint64),
+    ]
+
+
 class JambaSSMError(RuntimeError):
-    def __init__(self, status: int, what: str):
+    def __init__(self, status: int, what: str, cuda_error=None):
         self.status = status
         msg = status_string(status)
         if status == ERR_CUDA:
-            msg += f" (cudaError {lib().jamba_ssm_last_cuda_error()})"
+            code = lib().jamba_ssm_last_cuda_error() if cuda_error is None else cuda_error
+            msg += f" (cudaError {code})"
         super().__init__(f"{what}: {msg}")
 
 
 _lock = threading.Lock()
 _lib = None
+_proj_lib = None
 
 
 def lib():
@@ -109,6 +129,29 @@ def lib():
                 L.jamba_ssm_abi_version.argtypes = []
                 _lib = L
     return _lib
+
+
+def proj_lib():
+    """Load libjamba_ssm_proj.so (raises if it is missing: build it first)."""
+    global _proj_lib
+    if _proj_lib is None:
+        with _lock:
+            if _proj_lib is None:
+                if not os.path.exists(PROJ_LIB_PATH):
+                    raise RuntimeError(
+                        f"{PROJ_LIB_PATH} is not built; run selective_state_space_26_b200.build."
+                        "build() (nvcc, sm_100a). There is no CPU fallback.")
+                L = ctypes.CDLL(PROJ_LIB_PATH)
+                L.jamba_ssm_dt_proj.restype = ctypes.c_int
+                L.jamba_ssm_dt_proj.argtypes = [ctypes.POINTER(DtProjParams), _vp]
+                L.jamba_ssm_proj_get_status.restype = ctypes.c_int
+                L.jamba_ssm_proj_get_status.argtypes = [_vp]
+                L.jamba_ssm_proj_last_cuda_error.restype = ctypes.c_int
+                L.jamba_ssm_proj_last_cuda_error.argtypes = []
+                L.jamba_ssm_proj_abi_version.restype = ctypes.c_int
+                L.jamba_ssm_proj_abi_version.argtypes = []
+                _proj_lib = L
+    return _proj_lib
 
 
 def status_string(status: int) -> str:
@@ -167,3 +210,19 @@ def variant_info(k: int):
 
 def get_status(stream: int) -> int:
     return lib().jamba_ssm_get_status(_vp(stream or None))
+
+
+def new_dt_proj_params(**kw) -> DtProjParams:
+    p = DtProjParams()
+    p.struct_size = ctypes.sizeof(DtProjParams)
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def call_dt_proj(p: DtProjParams, stream: int) -> int:
+    return proj_lib().jamba_ssm_dt_proj(ctypes.byref(p), _vp(stream or None))
+
+
+def proj_get_status(stream: int) -> int:
+    return proj_lib().jamba_ssm_proj_get_status(_vp(stream or None))

@@ -1,0 +1,181 @@
+// jamba_ssm_proj.cu -- host side of the C ABI declared in
+// include/jamba_ssm_proj.h: argument validation, TMA tensor-map encoding and
+// the launch of the dt_proj kernel.  Nothing here allocates device memory.
+// Built as its own library, so its kernels and status word form a module of
+// their own.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstring>
+#include <mutex>
+
+#include "jamba_ssm_proj.h"
+#include "s6_dt_proj.cuh"
+
+#define JSSM_PROJ_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+jamba_ssm_status cuda_fail(cudaError_t e) {
+    t_last_cuda_error = static_cast<int>(e);
+    return JAMBA_SSM_ERR_CUDA;
+}
+
+constexpr int kMaxDevices = 64;
+struct DeviceState {
+    bool ready = false;
+    bool usable = false;
+    bool smem_attr = false;
+};
+DeviceState g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+// Checks that the current device is an sm_100 part and, once per device, sets
+// the kernel's dynamic shared-memory limit.
+jamba_ssm_status prepare_device() {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver) return JAMBA_SSM_ERR_NO_DEVICE;
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return JAMBA_SSM_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceState &d = g_devices[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        d.usable = (major == 10 && minor == 0);
+        d.ready = true;
+    }
+    if (!d.usable) return JAMBA_SSM_ERR_NO_DEVICE;
+    if (!d.smem_attr) {
+        e = cudaFuncSetAttribute(reinterpret_cast<const void *>(&jssm::s6_dt_proj_kernel),
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(jssm::DtProjCfg::kSmemBytes));
+        if (e != cudaSuccess) return cuda_fail(e);
+        d.smem_attr = true;
+    }
+    return JAMBA_SSM_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn(jamba_ssm_status *st) {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else if (err == cudaSuccess)
+            err = cudaErrorSymbolNotFound;
+    });
+    if (!fn) *st = cuda_fail(err);
+    return fn;
+}
+
+// 2-D bf16 map over [rows][cols] (cols innermost), box {64 cols, box_rows},
+// 128-byte swizzle, zero fill outside the tensor.
+bool encode_kmajor(EncodeTiledFn fn, CUtensorMap *map, const void *ptr, int64_t cols,
+                   int64_t rows, int box_rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+    cuuint32_t box[2] = {(cuuint32_t)jssm::DtProjCfg::kBK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t an, const void *b, size_t bn) {
+    if (!a || !b || an == 0 || bn == 0) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + bn && y < x + an;
+}
+
+constexpr size_t kDtProjParamsV1 = sizeof(jamba_ssm_dt_proj_params);
+constexpr uint64_t kDefaultTimeoutCycles = 4000000000ull;  // ~2 s at the boost clock
+
+}  // namespace
+
+JSSM_PROJ_API jamba_ssm_status jamba_ssm_dt_proj(const jamba_ssm_dt_proj_params *pin,
+                                                 void *stream) {
+    if (!pin || pin->struct_size < kDtProjParamsV1) return JAMBA_SSM_ERR_INVALID_ARG;
+    jamba_ssm_dt_proj_params p;
+    std::memcpy(&p, pin, sizeof(p));
+    if (p.ntok < 0 || p.d_inner < 1 || p.dt_rank < 1) return JAMBA_SSM_ERR_INVALID_ARG;
+    // d_inner / 256 channel tiles must fit the grid's y dimension
+    if (p.d_inner % 8 != 0 || p.dt_rank % 8 != 0 || p.d_inner > int64_t(65535) * jssm::DtProjCfg::kBN ||
+        p.dt_rank > (int64_t(1) << 16) || p.ntok > int64_t(0x7fffffff) - jssm::DtProjCfg::kBM)
+        return JAMBA_SSM_ERR_UNSUPPORTED;
+    if (p.ntok == 0) return JAMBA_SSM_OK;  // no work; the pointers are not used
+    if (!p.dt_low_hi || !p.W_dt || !p.delta) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (!aligned16(p.dt_low_hi) || !aligned16(p.dt_low_lo) || !aligned16(p.W_dt) ||
+        !aligned16(p.delta))
+        return JAMBA_SSM_ERR_MISALIGNED;
+    const size_t a_bytes = size_t(p.ntok) * size_t(p.dt_rank) * 2;
+    const size_t w_bytes = size_t(p.d_inner) * size_t(p.dt_rank) * 2;
+    const size_t out_bytes = size_t(p.ntok) * size_t(p.d_inner) * 2;
+    if (overlaps(p.delta, out_bytes, p.dt_low_hi, a_bytes) ||
+        overlaps(p.delta, out_bytes, p.dt_low_lo, a_bytes) ||
+        overlaps(p.delta, out_bytes, p.W_dt, w_bytes))
+        return JAMBA_SSM_ERR_INVALID_ARG;
+    jamba_ssm_status st = prepare_device();
+    if (st != JAMBA_SSM_OK) return st;
+
+    EncodeTiledFn fn = encode_fn(&st);
+    if (!fn) return st;
+    CUtensorMap map_hi, map_lo, map_w;
+    const void *lo = p.dt_low_lo ? p.dt_low_lo : p.dt_low_hi;
+    if (!encode_kmajor(fn, &map_hi, p.dt_low_hi, p.dt_rank, p.ntok, jssm::DtProjCfg::kBM) ||
+        !encode_kmajor(fn, &map_lo, lo, p.dt_rank, p.ntok, jssm::DtProjCfg::kBM) ||
+        !encode_kmajor(fn, &map_w, p.W_dt, p.dt_rank, p.d_inner, jssm::DtProjCfg::kBN))
+        return cuda_fail(cudaErrorInvalidValue);
+
+    __nv_bfloat16 *delta = static_cast<__nv_bfloat16 *>(p.delta);
+    int ntok = static_cast<int>(p.ntok), d_inner = static_cast<int>(p.d_inner),
+        dt_rank = static_cast<int>(p.dt_rank), two = p.dt_low_lo ? 1 : 0;
+    uint64_t limit = p.timeout_cycles ? p.timeout_cycles : kDefaultTimeoutCycles;
+    void *args[] = {&map_hi, &map_lo, &map_w, &delta, &ntok, &d_inner, &dt_rank, &two, &limit};
+    const dim3 grid(static_cast<unsigned>((p.ntok + jssm::DtProjCfg::kBM - 1) / jssm::DtProjCfg::kBM),
+                    static_cast<unsigned>((p.d_inner + jssm::DtProjCfg::kBN - 1) / jssm::DtProjCfg::kBN));
+    cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void *>(&jssm::s6_dt_proj_kernel), grid,
+                                     dim3(jssm::DtProjCfg::kThreads), args,
+                                     jssm::DtProjCfg::kSmemBytes, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return JAMBA_SSM_OK;
+}
+
+JSSM_PROJ_API jamba_ssm_status jamba_ssm_proj_get_status(void *stream) {
+    jamba_ssm_status st = prepare_device();
+    if (st != JAMBA_SSM_OK) return st;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    int word = 0;
+    e = cudaMemcpyFromSymbol(&word, jssm::g_status_word, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (word != 0) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(jssm::g_status_word, &zero, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return static_cast<jamba_ssm_status>(word);
+}
+
+JSSM_PROJ_API int jamba_ssm_proj_last_cuda_error(void) { return t_last_cuda_error; }
+
+JSSM_PROJ_API int jamba_ssm_proj_abi_version(void) { return JAMBA_SSM_PROJ_ABI_VERSION; }

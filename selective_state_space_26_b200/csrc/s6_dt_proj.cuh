@@ -1,0 +1,267 @@
+// s6_dt_proj.cuh -- the low-rank step that produces the scan's raw Delta:
+//     delta[t, d] = sum_r W_dt[d, r] * dt_low[t, r]
+// on the sm_100a tensor cores (tcgen05.mma, accumulator in TMEM).
+//
+// Source: "Jamba: A Hybrid Transformer-Mamba Language Model" (obsidian-dorae222
+// notes), section "Mamba 레이어": Bbar_t, C_t and Delta_t are functions of x_t.
+// The pages do not spell the function out; the reading taken is Mamba-1's,
+// where Delta comes from a rank-R vector dt_low_t (R = dt_rank) through one
+// linear map W_dt [d_inner, R].  The per-channel bias and the softplus are the
+// scan's own first step and are not applied here.
+//
+// Precision.  dt_low is an fp32 quantity (it leaves an RMSNorm).  Rounding it
+// to bf16 before this product would add ~1.6e-3 relative error to Delta, more
+// than the layer's bf16 tolerance leaves room for, so it arrives as two bf16
+// planes, hi = bf16(v) and lo = bf16(v - hi), and every k-step issues two MMAs
+// (hi and lo against the same W_dt tile) into one fp32 accumulator.  With lo
+// absent (NULL) only the hi plane is used.
+//
+// Work unit and roles.  One CTA computes a 128-token x 256-channel tile of
+// delta; K = dt_rank runs in 64-wide blocks through a 2-stage ring.
+//   warp 0 (one lane): TMA loads of the hi / lo / W_dt tiles (128-byte swizzle);
+//   warp 1: allocates 256 TMEM columns; one lane issues the MMAs
+//           (M = 128, N = 256, K = 16, bf16 x bf16 -> fp32) and commits each
+//           stage back to the producer, then the finished accumulator;
+//   warps 2-5: epilogue -- each thread owns one token row (TMEM lane), reads
+//           its 256 fp32 columns with tcgen05.ld, rounds to bf16 and stores.
+// Every wait is bounded; a wait that runs out records JAMBA_SSM_ERR_TIMEOUT in
+// the module's status word and the CTA winds down.
+#pragma once
+
+#include "device_utils.cuh"
+
+namespace jssm {
+
+struct DtProjCfg {
+    static constexpr int kBM = 128;  // tokens per tile: the MMA's M (one TMEM lane each)
+    static constexpr int kBN = 256;  // channels per tile: the MMA's N (one TMEM column each)
+    static constexpr int kBK = 64;   // dt_rank per stage: one 128-byte swizzled bf16 row
+    static constexpr int kUK = 16;   // K of one kind::f16 MMA
+    static constexpr int kStages = 2;
+    static constexpr uint32_t kTileA = kBM * kBK * 2;        // 16 KB per plane
+    static constexpr uint32_t kTileW = kBN * kBK * 2;        // 32 KB
+    static constexpr uint32_t kStage = 2 * kTileA + kTileW;  // 64 KB
+    static constexpr uint32_t kOffBar = kStages * kStage;    // barriers after the tiles
+    static constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;  // + room to align to 1 KB
+    static constexpr int kThreads = 192;
+    static constexpr uint32_t kTmemCols = 256;
+    // Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1),
+    // A and B bf16 (bits 7-9 and 10-12 = 1), both K-major (bits 15, 16 = 0),
+    // N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+    static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                                       (uint32_t(kBN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+};
+
+// ------------------------------------------------------------ tcgen05 / TMA
+// Shared-memory matrix descriptor of a K-major operand tile written by TMA with
+// the 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart (the
+// stride-dimension offset), start address in 16-byte units, descriptor version
+// 1 (bits 46-47) and layout type 2 = 128-byte swizzle (bits 61-63).  The
+// leading-dimension offset is unused for swizzled K-major tiles and set to 1.
+// A K offset inside the 128-byte row is applied by advancing the start address;
+// the swizzle is a function of the address bits, so the tile base must be
+// 1024-byte aligned.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) |
+           ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(slot)),
+                 "r"(cols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, one MMA of 128 x N x 16.
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive once on `bar` when every tcgen05 operation this thread issued before
+// has completed.
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+        "[%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// ------------------------------------------------------------------- kernel
+// Grid: x = token tiles of 128, y = channel tiles of 256.  delta is written
+// only inside [ntok, d_inner]; TMA fills out-of-range operand rows and K
+// columns with zeros, so ragged edges need no special case in the MMAs.
+__global__ void __launch_bounds__(DtProjCfg::kThreads, 1)
+    s6_dt_proj_kernel(const __grid_constant__ CUtensorMap map_hi,
+                      const __grid_constant__ CUtensorMap map_lo,
+                      const __grid_constant__ CUtensorMap map_w, __nv_bfloat16 *__restrict__ delta,
+                      int ntok, int d_inner, int dt_rank, int two_planes, uint64_t limit) {
+    using C = DtProjCfg;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
+    uint64_t *empty = full + C::kStages;
+    uint64_t *acc_full = empty + C::kStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * C::kBM, n0 = blockIdx.y * C::kBN;
+    const int kblocks = (dt_rank + C::kBK - 1) / C::kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        fence_mbarrier_init();
+        prefetch_tensormap(&map_hi);
+        prefetch_tensormap(&map_lo);
+        prefetch_tensormap(&map_w);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint32_t bytes = (two_planes ? 2u : 1u) * C::kTileA + C::kTileW;
+            for (int kb = 0; kb < kblocks; ++kb) {
+                const int s = kb % C::kStages;
+                if (kb >= C::kStages &&
+                    !mbar_wait_bounded(&empty[s], ((kb / C::kStages) & 1) ^ 1, limit)) {
+                    atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+                    break;
+                }
+                uint8_t *st = smem + s * C::kStage;
+                mbar_arrive_expect_tx(&full[s], bytes);
+                tma_load_2d(st, &map_hi, kb * C::kBK, m0, &full[s]);
+                if (two_planes) tma_load_2d(st + C::kTileA, &map_lo, kb * C::kBK, m0, &full[s]);
+                tma_load_2d(st + 2 * C::kTileA, &map_w, kb * C::kBK, n0, &full[s]);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int kb = 0; kb < kblocks; ++kb) {
+                const int s = kb % C::kStages;
+                if (!mbar_wait_bounded(&full[s], (kb / C::kStages) & 1, limit)) {
+                    atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a = smem_u32(smem + s * C::kStage);
+#pragma unroll
+                for (int k = 0; k < C::kBK / C::kUK; ++k) {
+                    const uint32_t koff = k * C::kUK * 2;  // bytes along the 128-byte row
+                    const uint64_t bdesc = umma_desc_sw128(a + 2 * C::kTileA + koff);
+                    umma_bf16(tmem, umma_desc_sw128(a + koff), bdesc, C::kIdesc,
+                              (kb | k) != 0 ? 1u : 0u);
+                    if (two_planes)
+                        umma_bf16(tmem, umma_desc_sw128(a + C::kTileA + koff), bdesc, C::kIdesc,
+                                  1u);
+                }
+                tc_commit(&empty[s]);  // the stage is free once these MMAs have read it
+            }
+            tc_commit(acc_full);  // every MMA issued above has completed
+            // Do not leave (and let the accumulator be freed) while MMAs run.
+            if (!mbar_wait_bounded(acc_full, 0, limit))
+                atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+        }
+        __syncwarp();
+    } else {
+        // Epilogue: warp w may read TMEM lanes 32*(w%4) .. 32*(w%4)+31.
+        const int q = warp & 3;
+        const int m = m0 + q * 32 + lane;
+        const bool ok = mbar_wait_bounded(acc_full, 0, limit);
+        tc_fence_after();
+        if (!ok) {
+            if (lane == 0) atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+        } else {
+            __nv_bfloat16 *row = delta + (size_t)(m < ntok ? m : 0) * (size_t)d_inner;
+#pragma unroll 1
+            for (int c = 0; c < C::kBN; c += 32) {
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
+                if (m < ntok) {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const int n = n0 + c + 8 * g;
+                        if (n < d_inner) {
+                            uint4 o;
+                            o.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
+                            o.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
+                            o.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
+                            o.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
+                            *reinterpret_cast<uint4 *>(row + n) = o;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+}  // namespace jssm

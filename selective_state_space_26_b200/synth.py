@@ -33,7 +33,7 @@ import torch
 
 _MASK = (1 << 64) - 1
 # tensor ids of the counter
-T_X, T_DT, T_Z, T_B, T_C, T_H0, T_DT0, T_A = range(8)
+T_X, T_DT, T_Z, T_B, T_C, T_H0, T_DT0, T_A, T_DTLOW, T_WDT = range(10)
 _ROWS_PER_DRAW = 8192  # rows of [seqlen, width] drawn per generator call
 
 
@@ -199,3 +199,28 @@ def workload_inputs(w: Workload, device="cpu", seq_offset: int = 0) -> ScanInput
     assert w.kind == "prefill"
     return scan_inputs(w.batch, w.seqlen, w.d_inner, w.d_state, w.dtype, w.seed, device,
                        seq_offset=seq_offset)
+
+
+@dataclasses.dataclass
+class DtProjInputs:
+    dt_low: torch.Tensor  # [ntok, dt_rank] fp32
+    hi: torch.Tensor      # [ntok, dt_rank] bf16, bf16(dt_low)
+    lo: torch.Tensor      # [ntok, dt_rank] bf16, bf16(dt_low - hi)
+    W_dt: torch.Tensor    # [d_inner, dt_rank] bf16
+
+
+def dt_proj_inputs(ntok: int, d_inner: int, dt_rank: int, seed: int, device) -> DtProjInputs:
+    """Inputs of the low-rank product that produces the scan's raw Delta.
+
+    dt_low ~ N(0, 1) in fp32 (unit RMS, as it leaves an RMSNorm with unit
+    weights), handed over as the two bf16 planes the library takes;
+    W_dt ~ U(-R^-1/2, R^-1/2) rounded to bf16 (R = dt_rank; the scale of
+    Mamba's dt_proj initialisation), so that delta has variance ~1/3.
+    """
+    dt_low = normal((ntok, dt_rank), seed, T_DTLOW, 0, 0, device)
+    hi = dt_low.to(torch.bfloat16)
+    lo = (dt_low - hi.float()).to(torch.bfloat16)
+    g = _gen(device, counter_seed(seed, T_WDT, 0, 0))
+    u = torch.rand((d_inner, dt_rank), generator=g, device=device, dtype=torch.float32)
+    W_dt = ((2.0 * u - 1.0) * dt_rank ** -0.5).to(torch.bfloat16)
+    return DtProjInputs(dt_low, hi, lo, W_dt)

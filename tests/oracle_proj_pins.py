@@ -143,5 +143,27 @@ def pin_proj_norm_off_is_plain(lib):
         assert np.array_equal(p, np.zeros_like(p)), "zero token with eps > 0"
 
 
+def pin_dt_proj_alone(lib):
+    """The last product on its own: one-hot rows of dt_low select the columns
+    of W_dt, the product is linear in dt_low, and it is the delta of the whole
+    step when W_x's first R rows are [I_R 0] and no norm is taken."""
+    d_inner, dt_rank, d_state = 11, 4, 2
+    r = _rng(16)
+    W_x, W_dt = _weights(r, d_inner, dt_rank, d_state)
+    delta = oracle.dt_proj(np.eye(dt_rank), W_dt, lib=lib)
+    for k in range(dt_rank):
+        assert np.array_equal(delta[k], W_dt[:, k]), f"dt_proj of e_{k}"
+    v1, v2 = r.standard_normal((6, dt_rank)), r.standard_normal((6, dt_rank))
+    _close(oracle.dt_proj(0.5 * v1 - 2.0 * v2, W_dt, lib=lib),
+           0.5 * oracle.dt_proj(v1, W_dt, lib=lib) - 2.0 * oracle.dt_proj(v2, W_dt, lib=lib),
+           1e-12, "dt_proj linear in dt_low")
+    W_x[:dt_rank] = 0.0
+    W_x[:dt_rank, :dt_rank] = np.eye(dt_rank)
+    u = r.standard_normal((5, d_inner))
+    d_full, _, _ = oracle.project(u, W_x, W_dt, d_state, lib=lib)
+    assert np.array_equal(d_full, oracle.dt_proj(u[:, :dt_rank], W_dt, lib=lib)), \
+        "dt_proj is the last product of the step"
+
+
 PROJ_PINS = [pin_proj_basis_selection, pin_proj_linearity, pin_proj_low_rank,
-             pin_proj_rmsnorm_closed_forms, pin_proj_norm_off_is_plain]
+             pin_proj_rmsnorm_closed_forms, pin_proj_norm_off_is_plain, pin_dt_proj_alone]

@@ -1,7 +1,8 @@
-"""Host-side checks of the C ABI that need no GPU: the library loads, exports
-every function include/jamba_ssm.h declares, its structures have the layout
-the binding assumes, and argument validation rejects bad calls before any CUDA
-work is enqueued (fake, never-dereferenced pointer values are enough)."""
+"""Host-side checks of the C ABIs that need no GPU: each library loads, exports
+every function its header (include/jamba_ssm.h, include/jamba_ssm_proj.h)
+declares, its structures have the layout the binding assumes, and argument
+validation rejects bad calls before any CUDA work is enqueued (fake,
+never-dereferenced pointer values are enough)."""
 import ctypes
 import os
 import re
@@ -14,6 +15,7 @@ from selective_state_space_26_b200 import _lib, build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "jamba_ssm.h")
+PROJ_HEADER = os.path.join(ROOT, "include", "jamba_ssm_proj.h")
 
 
 @pytest.fixture(scope="module")
@@ -22,8 +24,8 @@ def L():
     return _lib.lib()
 
 
-def declared_functions():
-    text = open(HEADER).read()
+def declared_functions(header=HEADER):
+    text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(jamba_ssm_[a-z_]+)\s*\(", text)))
 
@@ -39,13 +41,33 @@ def test_every_declared_symbol_is_exported(L):
         assert hasattr(L, n)
 
 
+@pytest.fixture(scope="module")
+def P():
+    build.build()
+    return _lib.proj_lib()
+
+
+def test_every_declared_proj_symbol_is_exported(P):
+    names = declared_functions(PROJ_HEADER)
+    assert set(names) == set(_lib.PROJ_EXPORTS), names
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.PROJ_LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    for n in names:
+        assert n in exported, f"{n} declared in the header but not exported"
+    # the projection library keeps its kernels and status word to itself
+    assert not [e for e in exported if "jssm" in e], "internal symbols exported"
+    assert P.jamba_ssm_proj_abi_version() == 1
+
+
 def test_struct_layout_matches_header(tmp_path):
     fields = {
         "jamba_ssm_scan_params": _lib.ScanParams,
         "jamba_ssm_state_update_params": _lib.StateUpdateParams,
+        "jamba_ssm_dt_proj_params": _lib.DtProjParams,
     }
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "jamba_ssm.h"',
-             "int main(void) {"]
+             '#include "jamba_ssm_proj.h"', "int main(void) {"]
     for cname, cls in fields.items():
         lines.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
         for f, _ in cls._fields_:
@@ -215,3 +237,52 @@ def test_version_1_struct_size_is_accepted(L):
     assert _lib.call_state_update(u, 0) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
     u.struct_size = _lib.STATE_UPDATE_PARAMS_V1_SIZE - 8
     assert _lib.call_state_update(u, 0) == _lib.ERR_INVALID_ARG
+
+
+_A16 = 0x7f0000000000  # fake, 16-byte aligned, never dereferenced
+
+
+def _dt_proj_call(P, **kw):
+    base = dict(ntok=300, d_inner=8192, dt_rank=256, dt_low_hi=_A16, dt_low_lo=_A16 + 0x1000000,
+                W_dt=_A16 + 0x2000000, delta=_A16 + 0x10000000)
+    base.update(kw)
+    return _lib.call_dt_proj(_lib.new_dt_proj_params(**base), 0)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ntok=-1), _lib.ERR_INVALID_ARG),
+    (dict(d_inner=0), _lib.ERR_INVALID_ARG),
+    (dict(dt_rank=0), _lib.ERR_INVALID_ARG),
+    (dict(dt_low_hi=None), _lib.ERR_INVALID_ARG),
+    (dict(W_dt=None), _lib.ERR_INVALID_ARG),
+    (dict(delta=None), _lib.ERR_INVALID_ARG),
+    (dict(d_inner=8190), _lib.ERR_UNSUPPORTED),
+    (dict(dt_rank=250), _lib.ERR_UNSUPPORTED),
+    (dict(dt_rank=1 << 17), _lib.ERR_UNSUPPORTED),
+    (dict(ntok=1 << 31), _lib.ERR_UNSUPPORTED),
+    (dict(dt_low_hi=_A16 + 8), _lib.ERR_MISALIGNED),
+    (dict(dt_low_lo=_A16 + 0x1000000 + 2), _lib.ERR_MISALIGNED),
+    (dict(delta=_A16 + 0x10000000 + 4), _lib.ERR_MISALIGNED),
+    (dict(delta=_A16 + 0x2000000), _lib.ERR_INVALID_ARG),  # overlaps W_dt
+])
+def test_dt_proj_argument_errors(P, kw, expect):
+    assert _dt_proj_call(P, **kw) == expect
+
+
+def test_dt_proj_struct_size_and_no_device(P):
+    p = _lib.new_dt_proj_params(ntok=1, d_inner=8, dt_rank=8, dt_low_hi=_A16,
+                                W_dt=_A16 + 0x1000, delta=_A16 + 0x2000)
+    assert P.jamba_ssm_dt_proj(None, None) == _lib.ERR_INVALID_ARG
+    p.struct_size = 8
+    assert _lib.call_dt_proj(p, 0) == _lib.ERR_INVALID_ARG
+    p.struct_size = ctypes.sizeof(_lib.DtProjParams)
+    if not torch.cuda.is_available():
+        assert _lib.call_dt_proj(p, 0) == _lib.ERR_NO_DEVICE
+
+
+def test_dt_proj_empty_batch_needs_no_pointers(P):
+    # an empty torch tensor's data_ptr() is 0: zero tokens must not check pointers
+    assert _lib.call_dt_proj(_lib.new_dt_proj_params(ntok=0, d_inner=256, dt_rank=256), 0) == \
+        _lib.OK
+    assert _lib.call_dt_proj(_lib.new_dt_proj_params(ntok=0, d_inner=250, dt_rank=256), 0) == \
+        _lib.ERR_UNSUPPORTED

@@ -34,8 +34,12 @@ MUTATIONS = [
      "oracle_rmsnorm(Bv, d_state, w_C, eps);"),
     ("norm_without_sqrt", "double inv = 1.0 / sqrt(ss / (double)len + eps);",
      "double inv = 1.0 / (ss / (double)len + eps);"),
-    ("delta_from_B_rows", "acc += W_dt[d * dt_rank + r] * dt_low[r];",
-     "acc += W_dt[d * dt_rank + r] * Bv[r % d_state];"),
+    ("dt_low_slice_off_by_one",
+     "oracle_low_rank_row(d_inner, dt_rank, W_dt, dt_low, delta + t * d_inner);",
+     "oracle_low_rank_row(d_inner, dt_rank, W_dt, xdbl + 1, delta + t * d_inner);"),
+    ("dt_proj_last_token_dropped",
+     "for (int64_t t = t_lo; t < t_hi; ++t)\n        oracle_low_rank_row",
+     "for (int64_t t = t_lo; t + 1 < t_hi; ++t)\n        oracle_low_rank_row"),
 ]
 
 
