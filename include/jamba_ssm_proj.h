@@ -12,10 +12,11 @@
  * where u_t is the scan's input x_t, and delta_t is the scan's raw step input
  * (its per-channel bias and softplus stay the scan's first step).
  *
- * This library provides the last product, delta = dt_low W_dt^T, on the
- * tensor cores.  dt_low is fp32 (it leaves the RMSNorm); a bf16 rounding of it
- * here would add ~1.6e-3 relative error to delta, so it is passed as two bf16
- * planes hi = bf16(v), lo = bf16(v - hi) whose sum is v to ~2^-16 relative.
+ * This library provides both products on the tensor cores: jamba_ssm_x_proj
+ * (W_x u with the three RMSNorms) and jamba_ssm_dt_proj (delta = dt_low W_dt^T).
+ * dt_low is fp32 (it leaves the RMSNorm); a bf16 rounding of it between the two
+ * would add ~1.6e-3 relative error to delta, so it travels as two bf16 planes
+ * hi = bf16(v), lo = bf16(v - hi) whose sum is v to ~2^-16 relative.
  *
  * Conventions are those of jamba_ssm.h: device pointers owned by the caller,
  * nothing allocated, `stream` a cudaStream_t passed as void*, argument errors
@@ -68,6 +69,51 @@ typedef struct {
 } jamba_ssm_dt_proj_params;
 
 jamba_ssm_status jamba_ssm_dt_proj(const jamba_ssm_dt_proj_params *p, void *stream);
+
+/*
+ * [dt_low | B | C] = W_x u for every token, each part then RMS-normalised:
+ * v_i <- w_i * v_i / sqrt(mean_j v_j^2 + eps) (a part whose weight pointer is
+ * NULL is not normalised).  Products accumulate in fp32; B and C are rounded
+ * once to bf16, dt_low is written as its hi / lo planes.
+ *
+ * Sizes: ntok >= 0 (0: nothing is launched, the pointers are not checked and
+ * JAMBA_SSM_OK is returned), ntok <= 2^31 - 129; 8 <= d_inner <= 2^30 with
+ * d_inner % 8 == 0; dt_rank == 256 and d_state == 16 (Jamba's layer; other
+ * values return JAMBA_SSM_ERR_UNSUPPORTED).
+ * Pointers (device, 16-byte aligned unless noted):
+ *   u          [ntok, d_inner] bf16, the scan's input x; required.
+ *   W_x        [dt_rank + 2 d_state, d_inner] bf16 (rows: dt_low, B, C); required.
+ *   w_dt [dt_rank], w_B [d_state], w_C [d_state]: fp32 RMSNorm weights, 4-byte
+ *              aligned, or NULL.
+ *   dt_low_hi, dt_low_lo  [ntok, dt_rank] bf16, written.
+ *   B, C       [ntok, d_state] bf16, written (the scan's B and C layout).
+ * Outputs must not overlap one another or an input.
+ * k_split: CTAs that share one 128-token tile's reduction over d_inner, as a
+ *   thread-block cluster: 1, 2, 4 or 8, or 0 for the library's choice (the
+ *   largest that keeps the grid within one wave of the SMs).
+ * timeout_cycles: as for jamba_ssm_dt_proj.
+ */
+typedef struct {
+    size_t struct_size; /* sizeof(jamba_ssm_x_proj_params) */
+    int64_t ntok;
+    int64_t d_inner;
+    int64_t dt_rank;
+    int64_t d_state;
+    const void *u;
+    const void *W_x;
+    const float *w_dt;
+    const float *w_B;
+    const float *w_C;
+    float eps;
+    int32_t k_split;
+    void *dt_low_hi;
+    void *dt_low_lo;
+    void *B;
+    void *C;
+    uint64_t timeout_cycles;
+} jamba_ssm_x_proj_params;
+
+jamba_ssm_status jamba_ssm_x_proj(const jamba_ssm_x_proj_params *p, void *stream);
 
 /* Waits for `stream`, then returns and clears this library's device-side
  * status word (JAMBA_SSM_OK, or JAMBA_SSM_ERR_TIMEOUT). */

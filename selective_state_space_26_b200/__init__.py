@@ -5,6 +5,8 @@ The calls, with the names of the C entry points:
 * ``jamba_ssm_scan``          -- prefill scan over whole sequences, returning the
   gated output and (for the decode cache) the final state;
 * ``jamba_ssm_state_update``  -- one-token decode step, state updated in place;
+* ``jamba_ssm_x_proj``        -- the projection of the scan's input to dt_low, B
+  and C with their RMSNorms (libjamba_ssm_proj.so);
 * ``jamba_ssm_dt_proj``       -- the low-rank product that produces the scan's
   raw Delta from dt_low (libjamba_ssm_proj.so).
 
@@ -22,7 +24,8 @@ from . import _lib
 from ._lib import JambaSSMError
 
 __all__ = ["jamba_ssm_scan", "jamba_ssm_state_update", "jamba_ssm_get_status", "scan_plan",
-           "jamba_ssm_dt_proj", "jamba_ssm_proj_get_status", "JambaSSMError"]
+           "jamba_ssm_x_proj", "jamba_ssm_dt_proj", "jamba_ssm_proj_get_status",
+           "JambaSSMError"]
 
 _IO = {torch.bfloat16: _lib.BF16, torch.float32: _lib.F32}
 
@@ -179,6 +182,43 @@ def jamba_ssm_get_status(stream=None, device=None) -> int:
     dev = torch.device(device) if device is not None else torch.device("cuda",
                                                                         torch.cuda.current_device())
     return _lib.get_status(_stream(stream, dev))
+
+
+def jamba_ssm_x_proj(u, W_x, w_dt=None, w_B=None, w_C=None, eps=1e-6, d_state=16,
+                     k_split=0, timeout_cycles=0, stream=None):
+    """[dt_low | B | C] = u @ W_x.T, each part RMS-normalised with its weight
+    (None: not normalised).
+
+    u: [..., d_inner] bf16; W_x: [dt_rank + 2 d_state, d_inner] bf16; weights
+    fp32.  Returns (dt_low_hi, dt_low_lo, B, C): the two bf16 planes of dt_low
+    [..., dt_rank] and B, C [..., d_state] bf16.
+    """
+    dev = u.device
+    if dev.type != "cuda":
+        raise ValueError("jamba_ssm_x_proj needs CUDA tensors; there is no CPU path")
+    rows, d_inner = W_x.shape
+    dt_rank = rows - 2 * d_state
+    lead = tuple(u.shape[:-1])
+    _check(u, "u", lead + (d_inner,), torch.bfloat16, dev)
+    _check(W_x, "W_x", (rows, d_inner), torch.bfloat16, dev)
+    _check(w_dt, "w_dt", (dt_rank,), torch.float32, dev)
+    _check(w_B, "w_B", (d_state,), torch.float32, dev)
+    _check(w_C, "w_C", (d_state,), torch.float32, dev)
+    hi, lo = (torch.empty(lead + (dt_rank,), dtype=torch.bfloat16, device=dev) for _ in range(2))
+    B, C = (torch.empty(lead + (d_state,), dtype=torch.bfloat16, device=dev) for _ in range(2))
+    ntok = 1
+    for n in lead:
+        ntok *= n
+    p = _lib.new_x_proj_params(ntok=ntok, d_inner=d_inner, dt_rank=dt_rank, d_state=d_state,
+                               u=_ptr(u), W_x=_ptr(W_x), w_dt=_ptr(w_dt), w_B=_ptr(w_B),
+                               w_C=_ptr(w_C), eps=float(eps), k_split=int(k_split),
+                               dt_low_hi=_ptr(hi), dt_low_lo=_ptr(lo), B=_ptr(B), C=_ptr(C),
+                               timeout_cycles=int(timeout_cycles))
+    st = _lib.call_x_proj(p, _stream(stream, dev))
+    if st != _lib.OK:
+        raise JambaSSMError(st, "jamba_ssm_x_proj",
+                            cuda_error=_lib.proj_lib().jamba_ssm_proj_last_cuda_error())
+    return hi, lo, B, C
 
 
 def jamba_ssm_dt_proj(dt_low_hi, W_dt, dt_low_lo=None, out=None, timeout_cycles=0, stream=None):

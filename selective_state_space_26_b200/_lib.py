@@ -30,6 +30,7 @@ EXPORTS = (
 )
 # Every symbol jamba_ssm_proj.h declares.
 PROJ_EXPORTS = (
+    "jamba_ssm_x_proj",
     "jamba_ssm_dt_proj",
     "jamba_ssm_proj_get_status",
     "jamba_ssm_proj_last_cuda_error",
@@ -79,6 +80,18 @@ class DtProjParams(ctypes.Structure):
         ("struct_size", ctypes.c_size_t),
         ("ntok", ctypes.c_int64), ("d_inner", ctypes.c_int64), ("dt_rank", ctypes.c_int64),
         ("dt_low_hi", _vp), ("dt_low_lo", _vp), ("W_dt", _vp), ("delta", _vp),
+        ("timeout_cycles", ctypes.c_uint64),
+    ]
+
+
+class XProjParams(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t),
+        ("ntok", ctypes.c_int64), ("d_inner", ctypes.c_int64), ("dt_rank", ctypes.c_int64),
+        ("d_state", ctypes.c_int64),
+        ("u", _vp), ("W_x", _vp), ("w_dt", _fp), ("w_B", _fp), ("w_C", _fp),
+        ("eps", ctypes.c_float), ("k_split", ctypes.c_int32),
+        ("dt_low_hi", _vp), ("dt_low_lo", _vp), ("B", _vp), ("C", _vp),
         ("timeout_cycles", ctypes.c_uint64),
     ]
 
@@ -142,6 +155,8 @@ def proj_lib():
                         f"{PROJ_LIB_PATH} is not built; run selective_state_space_26_b200.build."
                         "build() (nvcc, sm_100a). There is no CPU fallback.")
                 L = ctypes.CDLL(PROJ_LIB_PATH)
+                L.jamba_ssm_x_proj.restype = ctypes.c_int
+                L.jamba_ssm_x_proj.argtypes = [ctypes.POINTER(XProjParams), _vp]
                 L.jamba_ssm_dt_proj.restype = ctypes.c_int
                 L.jamba_ssm_dt_proj.argtypes = [ctypes.POINTER(DtProjParams), _vp]
                 L.jamba_ssm_proj_get_status.restype = ctypes.c_int
@@ -218,6 +233,18 @@ def new_dt_proj_params(**kw) -> DtProjParams:
     for k, v in kw.items():
         setattr(p, k, v)
     return p
+
+
+def new_x_proj_params(**kw) -> XProjParams:
+    p = XProjParams()
+    p.struct_size = ctypes.sizeof(XProjParams)
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def call_x_proj(p: XProjParams, stream: int) -> int:
+    return proj_lib().jamba_ssm_x_proj(ctypes.byref(p), _vp(stream or None))
 
 
 def call_dt_proj(p: DtProjParams, stream: int) -> int:

@@ -1,6 +1,6 @@
 // jamba_ssm_proj.cu -- host side of the C ABI declared in
 // include/jamba_ssm_proj.h: argument validation, TMA tensor-map encoding and
-// the launch of the dt_proj kernel.  Nothing here allocates device memory.
+// the launches of the x_proj and dt_proj kernels.  Nothing here allocates device memory.
 // Built as its own library, so its kernels and status word form a module of
 // their own.
 #include <cuda.h>
@@ -12,6 +12,7 @@
 
 #include "jamba_ssm_proj.h"
 #include "s6_dt_proj.cuh"
+#include "s6_x_proj.cuh"
 
 #define JSSM_PROJ_API extern "C" __attribute__((visibility("default")))
 
@@ -28,14 +29,18 @@ constexpr int kMaxDevices = 64;
 struct DeviceState {
     bool ready = false;
     bool usable = false;
-    bool smem_attr = false;
+    bool dt_attr = false;  // s6_dt_proj_kernel's shared-memory limit is set
+    bool x_attr = false;   // s6_x_proj_kernel's
+    int sms = 0;
 };
 DeviceState g_devices[kMaxDevices];
 std::mutex g_mutex;
 
-// Checks that the current device is an sm_100 part and, once per device, sets
-// the kernel's dynamic shared-memory limit.
-jamba_ssm_status prepare_device() {
+// Checks that the current device is an sm_100 part and, once per device and
+// kernel, raises `kernel`'s dynamic shared-memory limit to `smem` bytes (the
+// flag `attr_done` selects which kernel's record).  *sms receives the SM count.
+jamba_ssm_status prepare_device(const void *kernel, int smem, bool DeviceState::*attr_done,
+                                int *sms = nullptr) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver) return JAMBA_SSM_ERR_NO_DEVICE;
@@ -46,19 +51,19 @@ jamba_ssm_status prepare_device() {
     if (!d.ready) {
         int major = 0, minor = 0;
         if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
-            (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+            (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
             return cuda_fail(e);
         d.usable = (major == 10 && minor == 0);
         d.ready = true;
     }
     if (!d.usable) return JAMBA_SSM_ERR_NO_DEVICE;
-    if (!d.smem_attr) {
-        e = cudaFuncSetAttribute(reinterpret_cast<const void *>(&jssm::s6_dt_proj_kernel),
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(jssm::DtProjCfg::kSmemBytes));
+    if (kernel && !(d.*attr_done)) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return cuda_fail(e);
-        d.smem_attr = true;
+        d.*attr_done = true;
     }
+    if (sms) *sms = d.sms;
     return JAMBA_SSM_OK;
 }
 
@@ -85,7 +90,8 @@ EncodeTiledFn encode_fn(jamba_ssm_status *st) {
 }
 
 // 2-D bf16 map over [rows][cols] (cols innermost), box {64 cols, box_rows},
-// 128-byte swizzle, zero fill outside the tensor.
+// 128-byte swizzle, zero fill outside the tensor.  Both kernels take 64-wide
+// K blocks.
 bool encode_kmajor(EncodeTiledFn fn, CUtensorMap *map, const void *ptr, int64_t cols,
                    int64_t rows, int box_rows) {
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -100,6 +106,7 @@ bool encode_kmajor(EncodeTiledFn fn, CUtensorMap *map, const void *ptr, int64_t 
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bool overlaps(const void *a, size_t an, const void *b, size_t bn) {
     if (!a || !b || an == 0 || bn == 0) return false;
@@ -108,6 +115,17 @@ bool overlaps(const void *a, size_t an, const void *b, size_t bn) {
 }
 
 constexpr size_t kDtProjParamsV1 = sizeof(jamba_ssm_dt_proj_params);
+constexpr size_t kXProjParamsV1 = sizeof(jamba_ssm_x_proj_params);
+static_assert(jssm::DtProjCfg::kBK == jssm::XProjCfg::kBK, "one tensor-map box width");
+
+// Cluster size of the x_proj split over d_inner: the largest power of two up
+// to 8 that keeps (token tiles x split) within one wave of the SMs and gives
+// every CTA at least one 64-wide K block.
+int choose_k_split(int64_t m_tiles, int64_t k_blocks, int sms) {
+    int ks = 8;
+    while (ks > 1 && (m_tiles * ks > sms || ks > k_blocks)) ks >>= 1;
+    return ks;
+}
 constexpr uint64_t kDefaultTimeoutCycles = 4000000000ull;  // ~2 s at the boost clock
 
 }  // namespace
@@ -134,7 +152,9 @@ JSSM_PROJ_API jamba_ssm_status jamba_ssm_dt_proj(const jamba_ssm_dt_proj_params 
         overlaps(p.delta, out_bytes, p.dt_low_lo, a_bytes) ||
         overlaps(p.delta, out_bytes, p.W_dt, w_bytes))
         return JAMBA_SSM_ERR_INVALID_ARG;
-    jamba_ssm_status st = prepare_device();
+    jamba_ssm_status st =
+        prepare_device(reinterpret_cast<const void *>(&jssm::s6_dt_proj_kernel),
+                       static_cast<int>(jssm::DtProjCfg::kSmemBytes), &DeviceState::dt_attr);
     if (st != JAMBA_SSM_OK) return st;
 
     EncodeTiledFn fn = encode_fn(&st);
@@ -161,7 +181,7 @@ JSSM_PROJ_API jamba_ssm_status jamba_ssm_dt_proj(const jamba_ssm_dt_proj_params 
 }
 
 JSSM_PROJ_API jamba_ssm_status jamba_ssm_proj_get_status(void *stream) {
-    jamba_ssm_status st = prepare_device();
+    jamba_ssm_status st = prepare_device(nullptr, 0, nullptr);
     if (st != JAMBA_SSM_OK) return st;
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e);
@@ -179,3 +199,84 @@ JSSM_PROJ_API jamba_ssm_status jamba_ssm_proj_get_status(void *stream) {
 JSSM_PROJ_API int jamba_ssm_proj_last_cuda_error(void) { return t_last_cuda_error; }
 
 JSSM_PROJ_API int jamba_ssm_proj_abi_version(void) { return JAMBA_SSM_PROJ_ABI_VERSION; }
+
+JSSM_PROJ_API jamba_ssm_status jamba_ssm_x_proj(const jamba_ssm_x_proj_params *pin,
+                                                void *stream) {
+    using XC = jssm::XProjCfg;
+    if (!pin || pin->struct_size < kXProjParamsV1) return JAMBA_SSM_ERR_INVALID_ARG;
+    jamba_ssm_x_proj_params p;
+    std::memcpy(&p, pin, sizeof(p));
+    if (p.ntok < 0 || p.d_inner < 1 || p.dt_rank < 1 || p.d_state < 1 || !(p.eps >= 0.0f))
+        return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p.k_split != 0 && p.k_split != 1 && p.k_split != 2 && p.k_split != 4 && p.k_split != 8)
+        return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p.dt_rank != XC::kR || p.d_state != XC::kN || p.d_inner % 8 != 0 ||
+        p.d_inner > (int64_t(1) << 30) || p.ntok > int64_t(0x7fffffff) - XC::kBM)
+        return JAMBA_SSM_ERR_UNSUPPORTED;
+    if (p.ntok == 0) return JAMBA_SSM_OK;  // no work; the pointers are not used
+    if (!p.u || !p.W_x || !p.dt_low_hi || !p.dt_low_lo || !p.B || !p.C)
+        return JAMBA_SSM_ERR_INVALID_ARG;
+    if (!aligned16(p.u) || !aligned16(p.W_x) || !aligned16(p.dt_low_hi) ||
+        !aligned16(p.dt_low_lo) || !aligned16(p.B) || !aligned16(p.C) || !aligned4(p.w_dt) ||
+        !aligned4(p.w_B) || !aligned4(p.w_C))
+        return JAMBA_SSM_ERR_MISALIGNED;
+    const size_t u_bytes = size_t(p.ntok) * size_t(p.d_inner) * 2;
+    const size_t w_bytes = size_t(XC::kCols) * size_t(p.d_inner) * 2;
+    const size_t dt_bytes = size_t(p.ntok) * XC::kR * 2, bc_bytes = size_t(p.ntok) * XC::kN * 2;
+    const void *outs[] = {p.dt_low_hi, p.dt_low_lo, p.B, p.C};
+    const size_t outsz[] = {dt_bytes, dt_bytes, bc_bytes, bc_bytes};
+    const void *ins[] = {p.u, p.W_x, p.w_dt, p.w_B, p.w_C};
+    const size_t insz[] = {u_bytes, w_bytes, XC::kR * 4, XC::kN * 4, XC::kN * 4};
+    for (int i = 0; i < 4; ++i) {
+        for (int j = 0; j < 5; ++j)
+            if (overlaps(outs[i], outsz[i], ins[j], insz[j])) return JAMBA_SSM_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 4; ++j)
+            if (overlaps(outs[i], outsz[i], outs[j], outsz[j])) return JAMBA_SSM_ERR_INVALID_ARG;
+    }
+    int sms = 0;
+    jamba_ssm_status st =
+        prepare_device(reinterpret_cast<const void *>(&jssm::s6_x_proj_kernel),
+                       static_cast<int>(XC::kSmemBytes), &DeviceState::x_attr, &sms);
+    if (st != JAMBA_SSM_OK) return st;
+    EncodeTiledFn fn = encode_fn(&st);
+    if (!fn) return st;
+    CUtensorMap map_u, map_w1, map_w2;
+    if (!encode_kmajor(fn, &map_u, p.u, p.d_inner, p.ntok, XC::kBM) ||
+        !encode_kmajor(fn, &map_w1, p.W_x, p.d_inner, XC::kCols, XC::kR) ||
+        !encode_kmajor(fn, &map_w2, p.W_x, p.d_inner, XC::kCols, 2 * XC::kN))
+        return cuda_fail(cudaErrorInvalidValue);
+
+    const int64_t m_tiles = (p.ntok + XC::kBM - 1) / XC::kBM;
+    const int64_t k_blocks = (p.d_inner + XC::kBK - 1) / XC::kBK;
+    const int ks = p.k_split ? p.k_split : choose_k_split(m_tiles, k_blocks, sms);
+    if (m_tiles * ks > int64_t(0x7fffffff)) return JAMBA_SSM_ERR_UNSUPPORTED;
+    jssm::XProjArgs a;
+    a.dt_hi = static_cast<__nv_bfloat16 *>(p.dt_low_hi);
+    a.dt_lo = static_cast<__nv_bfloat16 *>(p.dt_low_lo);
+    a.B = static_cast<__nv_bfloat16 *>(p.B);
+    a.C = static_cast<__nv_bfloat16 *>(p.C);
+    a.w_dt = p.w_dt;
+    a.w_B = p.w_B;
+    a.w_C = p.w_C;
+    a.eps = p.eps;
+    a.ntok = static_cast<int>(p.ntok);
+    a.d_inner = static_cast<int>(p.d_inner);
+    a.ks = ks;
+    a.limit = p.timeout_cycles ? p.timeout_cycles : kDefaultTimeoutCycles;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(m_tiles * ks));
+    cfg.blockDim = dim3(XC::kThreads);
+    cfg.dynamicSmemBytes = XC::kSmemBytes;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(ks);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = ks > 1 ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, jssm::s6_x_proj_kernel, map_u, map_w1, map_w2, a);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return JAMBA_SSM_OK;
+}

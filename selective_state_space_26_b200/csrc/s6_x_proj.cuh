@@ -1,0 +1,287 @@
+// s6_x_proj.cuh -- the first product of the step that feeds the S6 scan:
+//     xdbl_t = W_x u_t,  [dt_low_t | B_t | C_t] = xdbl_t   (R, N, N entries)
+// with each part RMS-normalised (v <- w * v / sqrt(mean(v^2) + eps)), on the
+// sm_100a tensor cores.
+//
+// Source: "Jamba: A Hybrid Transformer-Mamba Language Model" (obsidian-dorae222
+// notes), section "Mamba 레이어": Bbar_t, C_t and Delta_t are functions of x_t,
+// and the layer carries an RMSNorm.  The reading taken (Mamba-1's x_proj, with
+// an RMSNorm on each of its three outputs) is the one the oracle's `project`
+// states.
+//
+// Outputs: B and C in bf16 in the scan's [token, d_state] layout, and dt_low as
+// two bf16 planes hi = bf16(v), lo = bf16(v - hi) for the dt_proj kernel, so
+// that no bf16 rounding of dt_low reaches Delta.
+//
+// Shape handled: R = 256, N = 16 (Jamba), so one CTA's accumulator is 128 tokens
+// x 288 fp32 columns of TMEM, filled by two MMAs per K step (N = 256 for dt_low
+// and N = 32 for B and C) on one u tile.
+//
+// Split K.  With 128 tokens per CTA a 4096-token batch has only 32 row tiles, so
+// K = d_inner is split across the KS CTAs of a thread-block cluster (KS in
+// {1, 2, 4, 8}).  After its MMAs each CTA streams its partial accumulator, row
+// by row from TMEM, into the shared memory of the CTA that owns that row's
+// reduction (rank = row / (128 / KS)), through distributed shared memory; the
+// ring the MMAs used is free by then and holds the receive buffer.  Two cluster
+// barriers order this: one after every CTA's MMAs have completed (so no ring is
+// still being read), one after every partial has been written.  The owners then
+// add the KS partials, normalise, round and store.  No workspace is needed.
+//
+// Roles (192 threads): warp 0 (one lane) TMA loads, warp 1 TMEM allocation and
+// (one lane) the MMAs, warps 2-5 the TMEM read-out and the owners' epilogue.
+// Every mbarrier wait is bounded (a wait that runs out records
+// JAMBA_SSM_ERR_TIMEOUT); every thread reaches both cluster barriers on every
+// path.
+#pragma once
+
+#include "s6_dt_proj.cuh"  // tcgen05 / TMA 2-D helpers and umma_desc_sw128
+
+namespace jssm {
+
+struct XProjCfg {
+    static constexpr int kBM = 128;               // tokens per CTA (the MMA's M)
+    static constexpr int kR = 256;                // dt_rank
+    static constexpr int kN = 16;                 // d_state
+    static constexpr int kCols = kR + 2 * kN;     // 288 accumulator columns
+    static constexpr int kBK = 64;                // d_inner per stage (128-byte rows)
+    static constexpr int kUK = 16;
+    static constexpr int kStages = 4;
+    static constexpr uint32_t kTileA = kBM * kBK * 2;        // 16 KB of u
+    static constexpr uint32_t kTileW1 = kR * kBK * 2;        // 32 KB: W_x rows 0..255
+    static constexpr uint32_t kTileW2 = 2 * kN * kBK * 2;    //  4 KB: W_x rows 256..287
+    static constexpr uint32_t kStage = kTileA + kTileW1 + kTileW2;  // 52 KB, 1 KB multiple
+    static constexpr uint32_t kOffBar = kStages * kStage;
+    static constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;
+    // receive buffer (reuses the ring): [KS][128 / KS rows][kRowWords] fp32;
+    // 288 columns padded to 292 words so that a warp's 16-byte stores to 8
+    // consecutive rows fall in distinct bank groups
+    static constexpr int kRowWords = kCols + 4;
+    static constexpr uint32_t kRecvBytes = kBM * kRowWords * 4;  // 149.5 KB for every KS
+    static constexpr int kThreads = 192;
+    static constexpr uint32_t kTmemCols = 512;  // power of two >= 288
+    static constexpr uint32_t kIdescDt = (1u << 4) | (1u << 7) | (1u << 10) |
+                                         (uint32_t(kR >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+    static constexpr uint32_t kIdescBC = (1u << 4) | (1u << 7) | (1u << 10) |
+                                         (uint32_t((2 * kN) >> 3) << 17) |
+                                         (uint32_t(kBM >> 4) << 24);
+    static_assert(kRecvBytes <= kOffBar, "the receive buffer must fit in the ring");
+    static_assert(kStage % 1024 == 0, "stages must keep the 1 KB swizzle alignment");
+    static_assert(kCols % 32 == 0, "the read-out takes 32 columns at a time");
+};
+
+struct XProjArgs {
+    __nv_bfloat16 *dt_hi, *dt_lo, *B, *C;  // outputs
+    const float *w_dt, *w_B, *w_C;          // RMSNorm weights or nullptr
+    float eps;
+    int ntok, d_inner, ks;
+    uint64_t limit;
+};
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address in CTA `rank`'s shared memory of the location `saddr` names in ours.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Grid: x = KS * token tiles (cluster dims {KS, 1, 1}: one cluster per 128
+// tokens, rank = which K slice).
+__global__ void __launch_bounds__(XProjCfg::kThreads, 1)
+    s6_x_proj_kernel(const __grid_constant__ CUtensorMap map_u,
+                     const __grid_constant__ CUtensorMap map_w1,
+                     const __grid_constant__ CUtensorMap map_w2, const XProjArgs args) {
+    using C = XProjCfg;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
+    uint64_t *empty = full + C::kStages;
+    uint64_t *acc_full = empty + C::kStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    float *recv = reinterpret_cast<float *>(smem);  // valid after cluster barrier 1
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ks = args.ks;
+    const uint32_t rank = ks > 1 ? cluster_ctarank() : 0u;
+    const int m0 = (blockIdx.x / ks) * C::kBM;
+    const int kb_total = (args.d_inner + C::kBK - 1) / C::kBK;
+    const int per = (kb_total + ks - 1) / ks;
+    const int kb0 = min(kb_total, static_cast<int>(rank) * per);
+    const int kb1 = min(kb_total, kb0 + per);
+    const int nkb = kb1 - kb0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        fence_mbarrier_init();
+        prefetch_tensormap(&map_u);
+        prefetch_tensormap(&map_w1);
+        prefetch_tensormap(&map_w2);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % C::kStages;
+                if (i >= C::kStages &&
+                    !mbar_wait_bounded(&empty[s], ((i / C::kStages) & 1) ^ 1, args.limit)) {
+                    atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+                    break;
+                }
+                uint8_t *st = smem + s * C::kStage;
+                const int k = (kb0 + i) * C::kBK;
+                mbar_arrive_expect_tx(&full[s], C::kStage);
+                tma_load_2d(st, &map_u, k, m0, &full[s]);
+                tma_load_2d(st + C::kTileA, &map_w1, k, 0, &full[s]);
+                tma_load_2d(st + C::kTileA + C::kTileW1, &map_w2, k, C::kR, &full[s]);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % C::kStages;
+                if (!mbar_wait_bounded(&full[s], (i / C::kStages) & 1, args.limit)) {
+                    atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a = smem_u32(smem + s * C::kStage);
+#pragma unroll
+                for (int k = 0; k < C::kBK / C::kUK; ++k) {
+                    const uint32_t koff = k * C::kUK * 2;
+                    const uint64_t adesc = umma_desc_sw128(a + koff);
+                    const uint32_t acc = (i | k) != 0 ? 1u : 0u;
+                    umma_bf16(tmem, adesc, umma_desc_sw128(a + C::kTileA + koff), C::kIdescDt,
+                              acc);
+                    umma_bf16(tmem + C::kR, adesc,
+                              umma_desc_sw128(a + C::kTileA + C::kTileW1 + koff), C::kIdescBC,
+                              acc);
+                }
+                tc_commit(&empty[s]);
+            }
+            tc_commit(acc_full);
+            if (!mbar_wait_bounded(acc_full, 0, args.limit))
+                atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+        }
+        __syncwarp();
+    } else {
+        if (!mbar_wait_bounded(acc_full, 0, args.limit) && lane == 0)
+            atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+        tc_fence_after();
+    }
+
+    // Barrier 1: every CTA of the cluster has finished its MMAs, so every ring
+    // may now be overwritten by partial sums.
+    if (ks > 1) cluster_sync_all(); else __syncthreads();
+
+    const int rows_per_owner = C::kBM / ks;
+    if (warp >= 2) {
+        // Each thread sends its token row's 288 partial sums to the row's owner.
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const uint32_t owner = static_cast<uint32_t>(row / rows_per_owner);
+        const uint32_t local = smem_u32(recv) +
+                               4u * static_cast<uint32_t>((rank * rows_per_owner +
+                                                           row % rows_per_owner) * C::kRowWords);
+        const uint32_t dst = ks > 1 ? map_to_rank(local, owner) : local;
+#pragma unroll 1
+        for (int c = 0; c < C::kCols; c += 32) {
+            float v[32];  // kCols is a multiple of 32
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
+            if (nkb == 0) {  // this K slice was empty: the accumulator was never written
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+                st_cluster_v4(dst + 4u * (c + j), v[j], v[j + 1], v[j + 2], v[j + 3]);
+        }
+    }
+    tc_fence_before();
+    // Barrier 2: every partial has landed in its owner's buffer.
+    if (ks > 1) cluster_sync_all(); else __syncthreads();
+
+    if (warp >= 2) {
+        // Owner epilogue: warp w takes rows (w - 2), (w - 2) + 4, ... of this
+        // CTA's share; lane j holds columns j + 32 k (k = 0..7: dt_low; k = 8:
+        // B for j < 16, C for j >= 16).
+        const bool is_b = lane < 16;
+        const float *w8 = is_b ? args.w_B : args.w_C;
+        for (int r = warp - 2; r < rows_per_owner; r += 4) {
+            const int m = m0 + static_cast<int>(rank) * rows_per_owner + r;
+            float v[9];
+#pragma unroll
+            for (int k = 0; k < 9; ++k) v[k] = 0.0f;
+            for (int src = 0; src < ks; ++src) {
+                const float *p = recv + (src * rows_per_owner + r) * C::kRowWords;
+#pragma unroll
+                for (int k = 0; k < 9; ++k) v[k] += p[lane + 32 * k];
+            }
+            if (args.w_dt) {
+                float ss = 0.0f;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) ss += v[k] * v[k];
+                const float inv = rsqrtf(warp_sum(ss) * (1.0f / C::kR) + args.eps);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[k] = args.w_dt[lane + 32 * k] * (v[k] * inv);
+            }
+            const float sq = v[8] * v[8];
+            const float ss_b = warp_sum(is_b ? sq : 0.0f), ss_c = warp_sum(is_b ? 0.0f : sq);
+            if (w8) {
+                const float inv = rsqrtf((is_b ? ss_b : ss_c) * (1.0f / C::kN) + args.eps);
+                v[8] = w8[lane & 15] * (v[8] * inv);
+            }
+            if (m < args.ntok) {
+                __nv_bfloat16 *hi = args.dt_hi + static_cast<size_t>(m) * C::kR;
+                __nv_bfloat16 *lo = args.dt_lo + static_cast<size_t>(m) * C::kR;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const __nv_bfloat16 h = __float2bfloat16_rn(v[k]);
+                    hi[lane + 32 * k] = h;
+                    lo[lane + 32 * k] = __float2bfloat16_rn(v[k] - __bfloat162float(h));
+                }
+                __nv_bfloat16 *bc = (is_b ? args.B : args.C) + static_cast<size_t>(m) * C::kN;
+                bc[lane & 15] = __float2bfloat16_rn(v[8]);
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+}  // namespace jssm

@@ -65,6 +65,7 @@ def test_struct_layout_matches_header(tmp_path):
         "jamba_ssm_scan_params": _lib.ScanParams,
         "jamba_ssm_state_update_params": _lib.StateUpdateParams,
         "jamba_ssm_dt_proj_params": _lib.DtProjParams,
+        "jamba_ssm_x_proj_params": _lib.XProjParams,
     }
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "jamba_ssm.h"',
              '#include "jamba_ssm_proj.h"', "int main(void) {"]
@@ -286,3 +287,40 @@ def test_dt_proj_empty_batch_needs_no_pointers(P):
         _lib.OK
     assert _lib.call_dt_proj(_lib.new_dt_proj_params(ntok=0, d_inner=250, dt_rank=256), 0) == \
         _lib.ERR_UNSUPPORTED
+
+
+def _x_proj_call(P, **kw):
+    base = dict(ntok=4096, d_inner=8192, dt_rank=256, d_state=16, u=_A16,
+                W_x=_A16 + 0x10000000, w_dt=_A16 + 0x11000000, w_B=_A16 + 0x11001000,
+                w_C=_A16 + 0x11002000, eps=1e-6, dt_low_hi=_A16 + 0x20000000,
+                dt_low_lo=_A16 + 0x21000000, B=_A16 + 0x22000000, C=_A16 + 0x22100000)
+    base.update(kw)
+    return _lib.call_x_proj(_lib.new_x_proj_params(**base), 0)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ntok=-1), _lib.ERR_INVALID_ARG),
+    (dict(eps=-1.0), _lib.ERR_INVALID_ARG),
+    (dict(eps=float("nan")), _lib.ERR_INVALID_ARG),
+    (dict(k_split=3), _lib.ERR_INVALID_ARG),
+    (dict(k_split=16), _lib.ERR_INVALID_ARG),
+    (dict(u=None), _lib.ERR_INVALID_ARG),
+    (dict(C=None), _lib.ERR_INVALID_ARG),
+    (dict(dt_rank=128), _lib.ERR_UNSUPPORTED),
+    (dict(d_state=8), _lib.ERR_UNSUPPORTED),
+    (dict(d_inner=8191), _lib.ERR_UNSUPPORTED),
+    (dict(u=_A16 + 8), _lib.ERR_MISALIGNED),
+    (dict(B=_A16 + 0x22000000 + 2), _lib.ERR_MISALIGNED),
+    (dict(w_dt=_A16 + 0x11000000 + 2), _lib.ERR_MISALIGNED),
+    (dict(dt_low_lo=_A16 + 0x20000000), _lib.ERR_INVALID_ARG),  # overlaps dt_low_hi
+    (dict(B=_A16 + 0x100), _lib.ERR_INVALID_ARG),                # overlaps u
+])
+def test_x_proj_argument_errors(P, kw, expect):
+    assert _x_proj_call(P, **kw) == expect
+
+
+def test_x_proj_empty_and_no_device(P):
+    assert _lib.call_x_proj(_lib.new_x_proj_params(ntok=0, d_inner=8192, dt_rank=256,
+                                                   d_state=16), 0) == _lib.OK
+    if not torch.cuda.is_available():
+        assert _x_proj_call(P, w_dt=None, w_B=None, w_C=None) == _lib.ERR_NO_DEVICE
