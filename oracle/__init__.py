@@ -12,6 +12,7 @@ widens inputs to float64 and splits the independent channels across host
 threads (ctypes releases the GIL during the call), which does not change the
 order of any floating-point operation inside a channel.
 
+``scan_bwd`` is the scan's reverse-mode gradient (the backward pass).
 ``project`` is the step before the scan (Delta, B and C from the scan's
 input through the x / dt projections and RMSNorm).  ``scan_packed`` and
 ``state_update_slots`` define the serving layouts (packed
@@ -62,6 +63,9 @@ def _declare(lib):
     lib.oracle_project_f64.restype = ctypes.c_int
     lib.oracle_project_f64.argtypes = ([_i64] * 6 + [_dp] * 6 + [ctypes.c_double]
                                        + [_dp] * 3)
+    lib.oracle_scan_bwd_f64.restype = ctypes.c_int
+    lib.oracle_scan_bwd_f64.argtypes = ([_i64] * 6 + [_dp] * 8 + [ctypes.c_int]
+                                        + [_dp] * 3 + [_dp] * 9)
     lib.oracle_dt_proj_f64.restype = ctypes.c_int
     lib.oracle_dt_proj_f64.argtypes = [_i64] * 5 + [_dp] * 3
     lib.oracle_state_update_f64.restype = ctypes.c_int
@@ -163,6 +167,40 @@ def state_update(state, x, delta, z, B, C, A, D=None, delta_bias=None,
     if rc != 0:
         raise ValueError("oracle_state_update_f64 rejected its arguments")
     return out, st
+
+
+def scan_bwd(x, delta, z, B, C, A, dout, D=None, delta_bias=None, delta_softplus=True,
+             h0=None, dh_final=None, lib=None):
+    """Reverse-mode gradient of `scan` in fp64 for a loss whose gradient is dout
+    with respect to out and dh_final (None: zero) with respect to h_final.
+
+    Returns a dict with dx, ddelta, dz [batch, seqlen, d_inner]; dB, dC [batch,
+    seqlen, d_state]; dA [d_inner, d_state]; dD, ddelta_bias [d_inner]; dh0
+    [batch, d_inner, d_state] (gradients of the parameters that were given;
+    an absent D, bias or h0 still gets its gradient, as if it were zero).
+    """
+    lib = lib or load()
+    x, delta, z, B, C, A, dout = map(_f64, (x, delta, z, B, C, A, dout))
+    D, delta_bias, h0, dh_final = map(_f64, (D, delta_bias, h0, dh_final))
+    batch, seqlen, d_inner = x.shape
+    d_state = A.shape[1]
+    assert dout.shape == x.shape
+    g = dict(dx=np.empty_like(x), ddelta=np.empty_like(x), dz=np.empty_like(x),
+             dB=np.zeros_like(B), dC=np.zeros_like(C), dA=np.zeros_like(A),
+             dD=np.zeros(d_inner), ddelta_bias=np.zeros(d_inner),
+             dh0=np.empty((batch, d_inner, d_state)))
+    # an absent D or bias is zero in the forward pass; its gradient is still defined
+    D0 = D if D is not None else np.zeros(d_inner)
+    b0 = delta_bias if delta_bias is not None else np.zeros(d_inner)
+    rc = lib.oracle_scan_bwd_f64(batch, seqlen, d_inner, d_state, 0, d_inner, _ptr(x),
+                                 _ptr(delta), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(D0),
+                                 _ptr(b0), int(bool(delta_softplus)), _ptr(h0), _ptr(dout),
+                                 _ptr(dh_final), _ptr(g["dx"]), _ptr(g["ddelta"]), _ptr(g["dz"]),
+                                 _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dA"]), _ptr(g["dD"]),
+                                 _ptr(g["ddelta_bias"]), _ptr(g["dh0"]))
+    if rc != 0:
+        raise ValueError("oracle_scan_bwd_f64 rejected its arguments")
+    return g
 
 
 def project(u, W_x, W_dt, d_state, w_dt=None, w_B=None, w_C=None, eps=1e-6,

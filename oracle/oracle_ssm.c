@@ -32,7 +32,9 @@
  * unrolled sums, the geometric-series closed form, the Delta->0 and large-Delta
  * limits, libm softplus/silu, split-scan and decode==scan identities) and, for
  * the projection that produces Delta, B and C, by tests/oracle_proj_pins.py
- * (basis-vector selections, associativity, rank, RMSNorm closed forms).
+ * (basis-vector selections, associativity, rank, RMSNorm closed forms), and the
+ * reverse-mode gradient of the scan by tests/oracle_bwd_pins.py (central finite
+ * differences of the forward scan, closed forms of the state gradient).
  */
 #include <math.h>
 #include <stddef.h>
@@ -223,5 +225,97 @@ int oracle_dt_proj_f64(int64_t ntok, int64_t d_inner, int64_t dt_rank, int64_t t
     if (t_lo < 0 || t_hi > ntok || t_lo > t_hi) return -1;
     for (int64_t t = t_lo; t < t_hi; ++t)
         oracle_low_rank_row(d_inner, dt_rank, W_dt, dt_low + t * dt_rank, delta + t * d_inner);
+    return 0;
+}
+
+/*
+ * Reverse-mode gradient of the prefill scan (training: the backward pass of
+ * the layer).  The caller's scalar loss has gradient dout with respect to out
+ * [batch, seqlen, d_inner] and dh_final with respect to h_final [batch,
+ * d_inner, d_state] (NULL: zero).  For the channels in [d_lo, d_hi):
+ *   written:      dx, ddelta, dz   [batch, seqlen, d_inner]   (ddelta is the
+ *                 gradient of the raw step input)
+ *                 dh0              [batch, d_inner, d_state] or NULL
+ *   accumulated:  dA [d_inner, d_state], dD [d_inner], ddelta_bias [d_inner]
+ *                 (each may be NULL), dB, dC [batch, seqlen, d_state]
+ *                 (summed over the channels in range; the caller zeroes them).
+ * The forward recurrence is re-run per channel, keeping every state, and the
+ * chain rule is applied in reverse time:
+ *   g      = dL/dh_t  = dy_t C_t + Abar_{t+1} * g_{t+1}   (g_L = dh_final)
+ *   dAbar  = g * h_{t-1},  dDelta += dAbar * Abar * A + g * B_t x_t,
+ *   dA    += dAbar * Abar * Delta,  dB_t += g Delta x_t,  dx_t += g Delta B_t,
+ * with dy_t = dout_t silu(z_t), dz_t = dout_t y_t silu'(z_t),
+ * silu'(z) = s (1 + z (1 - s)) for s = 1/(1+e^-z), and softplus'(v) = 1/(1+e^-v).
+ */
+int oracle_scan_bwd_f64(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state,
+                        int64_t d_lo, int64_t d_hi,
+                        const double *x, const double *delta, const double *z,
+                        const double *B, const double *C, const double *A,
+                        const double *D, const double *delta_bias, int delta_softplus,
+                        const double *h0, const double *dout, const double *dh_final,
+                        double *dx, double *ddelta, double *dz, double *dB, double *dC,
+                        double *dA, double *dD, double *ddelta_bias, double *dh0) {
+    if (batch < 0 || seqlen < 0 || d_inner < 0 || d_state < 1 || d_state > 64) return -1;
+    if (d_lo < 0 || d_hi > d_inner || d_lo > d_hi) return -1;
+    double *hs = (double *)malloc((size_t)(seqlen + 1) * (size_t)d_state * sizeof(double));
+    if (!hs) return -1;
+    double g[64];
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = d_lo; d < d_hi; ++d) {
+            /* forward, keeping h_{-1} = h0 in hs[0..N) and h_t in hs[(t+1)N ..) */
+            for (int64_t n = 0; n < d_state; ++n)
+                hs[n] = h0 ? h0[(b * d_inner + d) * d_state + n] : 0.0;
+            for (int64_t t = 0; t < seqlen; ++t) {
+                int64_t i = (b * seqlen + t) * d_inner + d;
+                const double *Bt = B + (b * seqlen + t) * d_state;
+                double dv = oracle_delta(delta[i], delta_bias, d, delta_softplus);
+                for (int64_t n = 0; n < d_state; ++n)
+                    hs[(t + 1) * d_state + n] = exp(dv * A[d * d_state + n]) * hs[t * d_state + n] +
+                                                dv * Bt[n] * x[i];
+            }
+            /* backward */
+            for (int64_t n = 0; n < d_state; ++n)
+                g[n] = dh_final ? dh_final[(b * d_inner + d) * d_state + n] : 0.0;
+            for (int64_t t = seqlen - 1; t >= 0; --t) {
+                int64_t i = (b * seqlen + t) * d_inner + d;
+                const double *Bt = B + (b * seqlen + t) * d_state;
+                const double *Ct = C + (b * seqlen + t) * d_state;
+                double *dBt = dB + (b * seqlen + t) * d_state;
+                double *dCt = dC + (b * seqlen + t) * d_state;
+                const double *h_now = hs + (t + 1) * d_state, *h_prev = hs + t * d_state;
+                double v = delta[i] + (delta_bias ? delta_bias[d] : 0.0);
+                double dv = delta_softplus ? oracle_softplus(v) : v;
+                double xv = x[i], Dd = D ? D[d] : 0.0;
+                double y = Dd * xv;
+                for (int64_t n = 0; n < d_state; ++n) y += Ct[n] * h_now[n];
+                double sz = 1.0 / (1.0 + exp(-z[i]));
+                double dy = dout[i] * (z[i] * sz);
+                dz[i] = dout[i] * y * sz * (1.0 + z[i] * (1.0 - sz));
+                if (dD) dD[d] += dy * xv;
+                double dxi = dy * Dd, dDelta = 0.0;
+                for (int64_t n = 0; n < d_state; ++n) {
+                    g[n] += dy * Ct[n];
+                    dCt[n] += dy * h_now[n];
+                }
+                for (int64_t n = 0; n < d_state; ++n) {
+                    double an = A[d * d_state + n];
+                    double abar = exp(dv * an);
+                    double dabar = g[n] * h_prev[n];
+                    dDelta += dabar * abar * an + g[n] * Bt[n] * xv;
+                    if (dA) dA[d * d_state + n] += dabar * abar * dv;
+                    dBt[n] += g[n] * dv * xv;
+                    dxi += g[n] * dv * Bt[n];
+                    g[n] = abar * g[n];
+                }
+                double draw = delta_softplus ? dDelta / (1.0 + exp(-v)) : dDelta;
+                ddelta[i] = draw;
+                if (ddelta_bias) ddelta_bias[d] += draw;
+                dx[i] = dxi;
+            }
+            if (dh0)
+                for (int64_t n = 0; n < d_state; ++n) dh0[(b * d_inner + d) * d_state + n] = g[n];
+        }
+    }
+    free(hs);
     return 0;
 }
