@@ -91,3 +91,31 @@ def test_reference_arm_under_torchrun_prints_one_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 2
     assert d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_traffic_record_follows_the_scan_library_sources(tmp_path, monkeypatch):
+    """roofline.traffic is reported only while the recorded DRAM counters were
+    taken on the current sources of the translation unit holding the timed
+    kernels: a header it includes changes the hash, a file outside it does not."""
+    csrc = tmp_path / "selective_state_space_26_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "jamba_ssm.cu").write_text('#include "a.cuh"\n#include <cuda.h>\n')
+    (csrc / "a.cuh").write_text('#include "b.cuh"\nint a;\n')
+    (csrc / "b.cuh").write_text("int b;\n")
+    (csrc / "other.cu").write_text("int other;\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash()
+    (csrc / "other.cu").write_text("int other2;\n")
+    (csrc / "unrelated.cuh").write_text("int u;\n")
+    assert bench.kernel_source_hash() == h0
+    (csrc / "b.cuh").write_text("int b2;\n")  # included indirectly
+    h1 = bench.kernel_source_hash()
+    assert h1 != h0
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "dram_traffic.json").write_text(json.dumps(
+        {"k": {"w": {"bytes_per_launch": 123, "source_hash": h1}}}))
+    assert bench.recorded_traffic("k", "w") == 123.0
+    (csrc / "a.cuh").write_text('#include "b.cuh"\nint a2;\n')
+    assert bench.recorded_traffic("k", "w") is None
+
