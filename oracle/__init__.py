@@ -62,7 +62,7 @@ def _declare(lib):
     lib.oracle_scan_f64.argtypes = [_i64] * 6 + [_dp] * 8 + [ctypes.c_int, _dp, _dp, _dp]
     lib.oracle_project_f64.restype = ctypes.c_int
     lib.oracle_project_f64.argtypes = ([_i64] * 6 + [_dp] * 6 + [ctypes.c_double]
-                                       + [_dp] * 3)
+                                       + [_dp] * 4)
     lib.oracle_scan_bwd_f64.restype = ctypes.c_int
     lib.oracle_scan_bwd_f64.argtypes = ([_i64] * 6 + [_dp] * 8 + [ctypes.c_int]
                                         + [_dp] * 3 + [_dp] * 9)
@@ -204,14 +204,15 @@ def scan_bwd(x, delta, z, B, C, A, dout, D=None, delta_bias=None, delta_softplus
 
 
 def project(u, W_x, W_dt, d_state, w_dt=None, w_B=None, w_C=None, eps=1e-6,
-            threads: int = 1, lib=None):
+            threads: int = 1, lib=None, return_dt_low: bool = False):
     """Delta (raw, before bias and softplus), B and C of every token from the
     scan's input u, in fp64.
 
     u [..., d_inner]; W_x [dt_rank + 2 d_state, d_inner]; W_dt [d_inner,
     dt_rank]; w_dt [dt_rank], w_B / w_C [d_state] are RMSNorm weights (None: that
     part is not normalised).  Returns (delta [..., d_inner], B [..., d_state],
-    C [..., d_state]).
+    C [..., d_state]), and with ``return_dt_low`` also dt_low [..., dt_rank]
+    after its RMSNorm (the input of the last product).
     """
     lib = lib or load()
     u, W_x, W_dt = map(_f64, (u, W_x, W_dt))
@@ -225,11 +226,12 @@ def project(u, W_x, W_dt, d_state, w_dt=None, w_B=None, w_C=None, eps=1e-6,
     delta = np.empty((ntok, d_inner))
     B = np.empty((ntok, d_state))
     C = np.empty((ntok, d_state))
+    dt_low = np.empty((ntok, dt_rank)) if return_dt_low else None
 
     def run(lo, hi):
         rc = lib.oracle_project_f64(ntok, d_inner, dt_rank, d_state, lo, hi, _ptr(u2),
                                     _ptr(W_x), _ptr(W_dt), _ptr(w_dt), _ptr(w_B), _ptr(w_C),
-                                    float(eps), _ptr(delta), _ptr(B), _ptr(C))
+                                    float(eps), _ptr(delta), _ptr(B), _ptr(C), _ptr(dt_low))
         if rc != 0:
             raise ValueError("oracle_project_f64 rejected its arguments")
 
@@ -240,8 +242,10 @@ def project(u, W_x, W_dt, d_state, w_dt=None, w_B=None, w_C=None, eps=1e-6,
         bounds = np.linspace(0, ntok, threads + 1).astype(np.int64)
         with ThreadPoolExecutor(threads) as ex:
             list(ex.map(lambda i: run(int(bounds[i]), int(bounds[i + 1])), range(threads)))
-    return (delta.reshape(*lead, d_inner), B.reshape(*lead, d_state),
-            C.reshape(*lead, d_state))
+    res = (delta.reshape(*lead, d_inner), B.reshape(*lead, d_state), C.reshape(*lead, d_state))
+    if return_dt_low:
+        res += (dt_low.reshape(*lead, dt_rank),)
+    return res
 
 
 def dt_proj(dt_low, W_dt, threads: int = 1, lib=None):

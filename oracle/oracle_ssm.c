@@ -163,6 +163,7 @@ int oracle_state_update_f64(int64_t batch, int64_t d_inner, int64_t d_state,
  *   w_dt, w_B, w_C : RMSNorm weights [dt_rank], [d_state], [d_state], or NULL
  *            (no normalisation of that part)
  *   delta  : [ntok, d_inner]      B, C : [ntok, d_state]
+ *   dt_low_out : [ntok, dt_rank] (after its RMSNorm), or NULL
  * Tokens [t_lo, t_hi) are computed, so a caller may split them across threads.
  * Returns 0, or -1 on a bad argument.
  */
@@ -187,7 +188,7 @@ int oracle_project_f64(int64_t ntok, int64_t d_inner, int64_t dt_rank, int64_t d
                        int64_t t_lo, int64_t t_hi,
                        const double *u, const double *W_x, const double *W_dt,
                        const double *w_dt, const double *w_B, const double *w_C, double eps,
-                       double *delta, double *B, double *C) {
+                       double *delta, double *B, double *C, double *dt_low_out) {
     if (ntok < 0 || d_inner < 1 || dt_rank < 1 || d_state < 1) return -1;
     if (t_lo < 0 || t_hi > ntok || t_lo > t_hi || !(eps >= 0.0)) return -1;
     int64_t rows = dt_rank + 2 * d_state;
@@ -208,6 +209,8 @@ int oracle_project_f64(int64_t ntok, int64_t d_inner, int64_t dt_rank, int64_t d
             B[t * d_state + n] = Bv[n];
             C[t * d_state + n] = Cv[n];
         }
+        if (dt_low_out)
+            for (int64_t r = 0; r < dt_rank; ++r) dt_low_out[t * dt_rank + r] = dt_low[r];
         oracle_low_rank_row(d_inner, dt_rank, W_dt, dt_low, delta + t * d_inner);
     }
     free(xdbl);

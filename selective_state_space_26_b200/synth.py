@@ -33,7 +33,7 @@ import torch
 
 _MASK = (1 << 64) - 1
 # tensor ids of the counter
-T_X, T_DT, T_Z, T_B, T_C, T_H0, T_DT0, T_A, T_DTLOW, T_WDT = range(10)
+T_X, T_DT, T_Z, T_B, T_C, T_H0, T_DT0, T_A, T_DTLOW, T_WDT, T_WX, T_NORMW = range(12)
 _ROWS_PER_DRAW = 8192  # rows of [seqlen, width] drawn per generator call
 
 
@@ -224,3 +224,30 @@ def dt_proj_inputs(ntok: int, d_inner: int, dt_rank: int, seed: int, device) -> 
     u = torch.rand((d_inner, dt_rank), generator=g, device=device, dtype=torch.float32)
     W_dt = ((2.0 * u - 1.0) * dt_rank ** -0.5).to(torch.bfloat16)
     return DtProjInputs(dt_low, hi, lo, W_dt)
+
+
+@dataclasses.dataclass
+class XProjInputs:
+    u: torch.Tensor      # [ntok, d_inner] bf16 (the scan's x)
+    W_x: torch.Tensor    # [dt_rank + 2 d_state, d_inner] bf16
+    w_dt: torch.Tensor   # [dt_rank] fp32 RMSNorm weights
+    w_B: torch.Tensor    # [d_state] fp32
+    w_C: torch.Tensor    # [d_state] fp32
+
+
+def x_proj_inputs(ntok: int, d_inner: int, dt_rank: int, d_state: int, seed: int,
+                  device) -> XProjInputs:
+    """Inputs of the projection before the scan.
+
+    u ~ N(0, 1) rounded to bf16 (the scan's x recipe); W_x ~ N(0, 1/d_inner)
+    rounded to bf16, so each projected entry is ~N(0, 1) before its norm; the
+    three RMSNorm weights ~ U(0.5, 1.5) in fp32 (a trained norm's weights sit
+    near 1; the spread makes a swapped or ignored weight visible).
+    """
+    u = normal((ntok, d_inner), seed, T_X, 0, 0, device).to(torch.bfloat16)
+    W_x = normal((dt_rank + 2 * d_state, d_inner), seed, T_WX, 0, 0, device,
+                 std=d_inner ** -0.5).to(torch.bfloat16)
+    g = _gen(device, counter_seed(seed, T_NORMW, 0, 0))
+    w = 0.5 + torch.rand(dt_rank + 2 * d_state, generator=g, device=device, dtype=torch.float32)
+    return XProjInputs(u, W_x, w[:dt_rank].contiguous(), w[dt_rank:dt_rank + d_state].contiguous(),
+                       w[dt_rank + d_state:].contiguous())

@@ -165,5 +165,24 @@ def pin_dt_proj_alone(lib):
         "dt_proj is the last product of the step"
 
 
+def pin_proj_dt_low_output(lib):
+    """The dt_low the step returns is the one its delta was made from
+    (delta == dt_proj(dt_low)); without a norm a one-hot token selects column k
+    of W_x's first R rows; with unit weights and eps = 0 its RMS is 1."""
+    d_inner, dt_rank, d_state = 10, 4, 3
+    r = _rng(17)
+    W_x, W_dt = _weights(r, d_inner, dt_rank, d_state)
+    _, _, _, low = oracle.project(np.eye(d_inner), W_x, W_dt, d_state, return_dt_low=True,
+                                  lib=lib)
+    for k in range(d_inner):
+        assert np.array_equal(low[k], W_x[:dt_rank, k]), f"dt_low of e_{k}"
+    u = r.standard_normal((7, d_inner))
+    delta, _, _, low = oracle.project(u, W_x, W_dt, d_state, w_dt=np.ones(dt_rank), eps=0.0,
+                                      return_dt_low=True, lib=lib)
+    _close(np.mean(low * low, axis=1), np.ones(7), 1e-14, "unit RMS of the returned dt_low")
+    _close(delta, oracle.dt_proj(low, W_dt, lib=lib), 1e-14, "delta == dt_proj(dt_low)")
+
+
 PROJ_PINS = [pin_proj_basis_selection, pin_proj_linearity, pin_proj_low_rank,
-             pin_proj_rmsnorm_closed_forms, pin_proj_norm_off_is_plain, pin_dt_proj_alone]
+             pin_proj_rmsnorm_closed_forms, pin_proj_norm_off_is_plain, pin_dt_proj_alone,
+             pin_proj_dt_low_output]
