@@ -324,3 +324,18 @@ def test_x_proj_empty_and_no_device(P):
                                                    d_state=16), 0) == _lib.OK
     if not torch.cuda.is_available():
         assert _x_proj_call(P, w_dt=None, w_B=None, w_C=None) == _lib.ERR_NO_DEVICE
+
+
+def test_proj_abi_from_plain_c(P, tmp_path):
+    """The projection library's boundary is C: a gcc-built program with no
+    Python in it includes the header, links the library and gets the
+    documented statuses back (host-side paths only; no GPU needed)."""
+    exe = tmp_path / "proj_abi_check"
+    libdir = os.path.dirname(_lib.PROJ_LIB_PATH)
+    subprocess.run(["gcc", "-O1", "-Wall", "-Werror", "-o", str(exe),
+                    os.path.join(ROOT, "tests", "c", "proj_abi_check.c"), "-I",
+                    os.path.join(ROOT, "include"), "-L", libdir, "-ljamba_ssm_proj",
+                    f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert "passed" in r.stdout
