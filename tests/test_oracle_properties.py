@@ -67,3 +67,29 @@ def test_split_and_causality(p, cut):
         changed["x"][:, cut:] += 1.0
         oc, _ = oracle.scan(**changed, delta_softplus=sp)
         assert np.array_equal(oc[:, :cut], out[:, :cut])
+
+
+@settings(max_examples=25, deadline=None)
+@given(problems(), st.integers(0, 2**31 - 1))
+def test_backward_equals_finite_differences(p, seed):
+    """On random tiny problems the backward oracle's gradient, projected on a
+    random direction of every input at once, equals the central finite
+    difference of the forward oracle along that direction."""
+    case, sp = p
+    r = np.random.default_rng(seed)
+    out, hf = oracle.scan(**case, delta_softplus=sp)
+    dout, dhf = r.standard_normal(out.shape), r.standard_normal(hf.shape)
+    g = oracle.scan_bwd(dout=dout, dh_final=dhf, delta_softplus=sp, **case)
+    names = {"x": "dx", "delta": "ddelta", "z": "dz", "B": "dB", "C": "dC", "A": "dA",
+             "D": "dD", "delta_bias": "ddelta_bias", "h0": "dh0"}
+    dirs = {k: r.standard_normal(np.shape(case[k])) for k in names if case[k] is not None}
+    eps = 1e-6
+
+    def loss(sign):
+        moved = {k: (v + sign * eps * dirs[k] if k in dirs else v) for k, v in case.items()}
+        o, h = oracle.scan(**moved, delta_softplus=sp)
+        return float(np.sum(o * dout) + np.sum(h * dhf))
+
+    fd = (loss(1.0) - loss(-1.0)) / (2 * eps)
+    an = sum(float(np.sum(g[names[k]] * dirs[k])) for k in dirs)
+    assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (fd, an)
