@@ -82,3 +82,13 @@ def test_dt_proj_full_size_sampled_rows():
                                                               replace=False))])
     got = out[torch.as_tensor(rows, device=dev)]
     assert_out(got, _ref(inp, rows=rows), torch.bfloat16, "dt_proj full size")
+
+
+def test_dt_proj_is_deterministic():
+    """A fixed MMA order and no atomics: two launches give the same bits."""
+    dev = _dev()
+    inp = synth.dt_proj_inputs(300, 776, 256, seed=36, device=dev)
+    a = jamba_ssm_dt_proj(inp.hi, inp.W_dt, dt_low_lo=inp.lo)
+    b = jamba_ssm_dt_proj(inp.hi, inp.W_dt, dt_low_lo=inp.lo)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
