@@ -248,7 +248,7 @@ JSSM_PROJ_API jamba_ssm_status jamba_ssm_x_proj(const jamba_ssm_x_proj_params *p
 
     const int64_t m_tiles = (p.ntok + XC::kBM - 1) / XC::kBM;
     const int64_t k_blocks = (p.d_inner + XC::kBK - 1) / XC::kBK;
-    const int ks = p.k_split ? p.k_split : choose_k_split(m_tiles, k_blocks, sms);
+    int ks = p.k_split ? p.k_split : choose_k_split(m_tiles, k_blocks, sms);
     if (m_tiles * ks > int64_t(0x7fffffff)) return JAMBA_SSM_ERR_UNSUPPORTED;
     jssm::XProjArgs a;
     a.dt_hi = static_cast<__nv_bfloat16 *>(p.dt_low_hi);
@@ -261,21 +261,34 @@ JSSM_PROJ_API jamba_ssm_status jamba_ssm_x_proj(const jamba_ssm_x_proj_params *p
     a.eps = p.eps;
     a.ntok = static_cast<int>(p.ntok);
     a.d_inner = static_cast<int>(p.d_inner);
-    a.ks = ks;
     a.limit = p.timeout_cycles ? p.timeout_cycles : kDefaultTimeoutCycles;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(m_tiles * ks));
     cfg.blockDim = dim3(XC::kThreads);
     cfg.dynamicSmemBytes = XC::kSmemBytes;
     cfg.stream = static_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(ks);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = ks > 1 ? 1 : 0;
+    // The library's own choice falls back to smaller clusters if the device
+    // cannot co-schedule this many CTAs of this size; an explicit k_split is
+    // launched as asked (and fails as a launch error if it cannot run).
+    for (;;) {
+        a.ks = ks;
+        cfg.gridDim = dim3(static_cast<unsigned>(m_tiles * ks));
+        attr[0].val.clusterDim.x = static_cast<unsigned>(ks);
+        cfg.numAttrs = ks > 1 ? 1 : 0;
+        if (ks == 1 || p.k_split != 0) break;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, jssm::s6_x_proj_kernel, &cfg) ==
+                cudaSuccess &&
+            clusters > 0)
+            break;
+        (void)cudaGetLastError();  // clear a failed query before trying a smaller cluster
+        ks >>= 1;
+    }
     cudaError_t e = cudaLaunchKernelEx(&cfg, jssm::s6_x_proj_kernel, map_u, map_w1, map_w2, a);
     if (e != cudaSuccess) return cuda_fail(e);
     return JAMBA_SSM_OK;
