@@ -93,3 +93,28 @@ def test_backward_equals_finite_differences(p, seed):
     fd = (loss(1.0) - loss(-1.0)) / (2 * eps)
     an = sum(float(np.sum(g[names[k]] * dirs[k])) for k in dirs)
     assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (fd, an)
+
+
+@settings(max_examples=40, deadline=None)
+@given(st.integers(1, 6), st.integers(1, 9), st.integers(1, 5), st.integers(1, 4),
+       st.integers(0, 2**31 - 1), st.booleans())
+def test_projection_is_rms_normalised_low_rank_map(ntok, d_inner, dt_rank, d_state, seed, norm):
+    """For random shapes: delta has rank <= dt_rank and equals dt_proj of the
+    returned dt_low; with the norm and unit weights at eps = 0 every part has
+    unit RMS; without it, B and C of a one-hot token are W_x's columns."""
+    r = np.random.default_rng(seed)
+    W_x = r.standard_normal((dt_rank + 2 * d_state, d_inner))
+    W_dt = r.standard_normal((d_inner, dt_rank))
+    u = r.standard_normal((ntok, d_inner))
+    ws = dict(w_dt=np.ones(dt_rank), w_B=np.ones(d_state), w_C=np.ones(d_state)) if norm else {}
+    delta, B, C, low = oracle.project(u, W_x, W_dt, d_state, eps=0.0, return_dt_low=True, **ws)
+    _close(delta, oracle.dt_proj(low, W_dt), 1e-13, "delta from dt_low")
+    assert np.linalg.matrix_rank(delta, tol=1e-9 * max(1.0, np.abs(delta).max())) <= dt_rank
+    if norm:
+        for part in (low, B, C):
+            _close(np.mean(part * part, axis=1), np.ones(ntok), 1e-12, "unit RMS")
+    else:
+        k = int(r.integers(0, d_inner))
+        _, Bk, Ck = oracle.project(np.eye(d_inner)[k:k + 1], W_x, W_dt, d_state)
+        assert np.array_equal(Bk[0], W_x[dt_rank:dt_rank + d_state, k])
+        assert np.array_equal(Ck[0], W_x[dt_rank + d_state:, k])
