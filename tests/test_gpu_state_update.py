@@ -4,7 +4,7 @@ import torch
 
 import oracle
 from selective_state_space_26_b200 import jamba_ssm_scan, jamba_ssm_state_update, synth
-from tests.parity import assert_out, assert_state, compare_out, rel_l2
+from tests.parity import assert_out, assert_state, rel_l2
 
 pytestmark = pytest.mark.gpu
 
