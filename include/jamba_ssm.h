@@ -33,8 +33,19 @@
  *     returned as a status; nothing is launched then.  A failed launch returns
  *     JAMBA_SSM_ERR_CUDA (the CUDA error code is kept per host thread, see
  *     jamba_ssm_last_cuda_error).  A device-side condition (a bounded wait that
- *     ran out) is recorded in a per-device status word read by
- *     jamba_ssm_get_status.  No C++ exception crosses this interface.
+ *     ran out, a state slot past the cache) is recorded in a status word: the
+ *     first word of the caller's workspace when the call was given one, else
+ *     a per-device word of the library; jamba_ssm_get_status reads it.  No C++
+ *     exception crosses this interface.
+ *   - Workspace: the calls take an optional caller-owned device buffer of at
+ *     least jamba_ssm_scan_workspace_size() bytes (16-byte aligned).  The
+ *     scan needs no scratch of its own -- every lane carries its channel's
+ *     states through the whole sequence in registers, so no carry between
+ *     chunks of a sequence is ever stored -- and the workspace holds only the
+ *     call's status word.  A caller that gives each stream its own workspace
+ *     keeps the streams' device-side conditions apart.  The caller zero-fills
+ *     a workspace once before its first use; jamba_ssm_get_status clears it
+ *     again after reading a condition.
  *   - Debugging aid: with the environment variable JAMBA_SSM_SYNC_CHECK set
  *     (and not "0") when the library is first called, every call waits for
  *     its work and returns jamba_ssm_get_status()'s result itself.
@@ -49,16 +60,24 @@
 extern "C" {
 #endif
 
-#define JAMBA_SSM_ABI_VERSION 2
+/* Version 3: the workspace fields, jamba_ssm_scan_workspace_size, the
+ * (workspace, stream) form of jamba_ssm_get_status, d_state 1 and 2 (and 4 in
+ * bf16), and the status codes renumbered so that ERR_WORKSPACE is 4: a caller
+ * built against an earlier version of this header must be rebuilt. */
+#define JAMBA_SSM_ABI_VERSION 3
+
+/* Bytes of the status block at the start of a workspace. */
+#define JAMBA_SSM_STATUS_BYTES 16
 
 typedef enum {
     JAMBA_SSM_OK = 0,
     JAMBA_SSM_ERR_INVALID_ARG = 1,  /* NULL pointer, negative size, aliasing, bad struct_size */
     JAMBA_SSM_ERR_UNSUPPORTED = 2,  /* d_state / dtype / d_inner combination not built        */
     JAMBA_SSM_ERR_MISALIGNED = 3,   /* a pointer is not aligned as documented below            */
-    JAMBA_SSM_ERR_CUDA = 4,         /* a CUDA runtime/driver call or the launch failed         */
-    JAMBA_SSM_ERR_TIMEOUT = 5,      /* device side: a bounded wait ran out (get_status only)   */
-    JAMBA_SSM_ERR_NO_DEVICE = 6     /* no usable sm_100 device is current                      */
+    JAMBA_SSM_ERR_WORKSPACE = 4,    /* workspace given but smaller than required               */
+    JAMBA_SSM_ERR_CUDA = 5,         /* a CUDA runtime/driver call or the launch failed         */
+    JAMBA_SSM_ERR_TIMEOUT = 6,      /* device side: a bounded wait ran out (get_status only)   */
+    JAMBA_SSM_ERR_NO_DEVICE = 7     /* no usable sm_100 device is current                      */
 } jamba_ssm_status;
 
 typedef enum {
@@ -70,11 +89,13 @@ typedef enum {
  * Prefill scan over whole sequences (the S6 recurrence of "Mamba 레이어",
  * evaluated for t = 0 .. seqlen-1 from the initial state h0).
  *
- * Sizes: batch >= 0, seqlen >= 0, d_inner >= 1, d_state in the supported set:
- *   bf16 I/O: d_state in {8, 16} and d_inner % 8 == 0;
- *   f32  I/O: d_state in {4, 8, 16} and d_inner % 4 == 0.
- * (Each activation row must be a multiple of 16 bytes.)  Jamba's layer is
- * d_inner = 8192, d_state = 16.
+ * Sizes: batch >= 0, seqlen >= 0, d_inner >= 1, d_state in {1, 2, 4, 8, 16},
+ * and d_inner % 8 == 0 for bf16 I/O, d_inner % 4 == 0 for f32 I/O (each
+ * activation row is a multiple of 16 bytes).  Jamba's layer is d_inner = 8192,
+ * d_state = 16.  State sizes whose B / C rows are shorter than 16 bytes (bf16
+ * d_state 1, 2, 4; f32 d_state 1, 2) take a one-thread-per-channel kernel
+ * with plain loads, at most 65535 sequences per call; the others take the
+ * TMA-fed kernels.
  * Pointers (device):
  *   x, delta, z   [batch, seqlen, d_inner] io_dtype, 16-byte aligned, required.
  *                 delta is the raw step input; Delta is formed in the kernel.
@@ -123,6 +144,12 @@ typedef enum {
  *                 JAMBA_SSM_ERR_INVALID_ARG in the status word.  Indices of
  *                 one call must be distinct.
  *   num_slots     rows of the state caches (state_indices != NULL).
+ *
+ * Workspace (ABI version 3; absent -- NULL -- for a shorter struct_size):
+ *   workspace     device buffer of workspace_bytes >= the size
+ *                 jamba_ssm_scan_workspace_size returns, 16-byte aligned, or
+ *                 NULL (the status goes to the library's per-device word).
+ *                 Too small: JAMBA_SSM_ERR_WORKSPACE.
  */
 typedef struct jamba_ssm_scan_params {
     size_t struct_size;          /* = sizeof(jamba_ssm_scan_params); callers of
@@ -147,7 +174,15 @@ typedef struct jamba_ssm_scan_params {
     int64_t total_tokens;
     const int32_t *state_indices;
     int64_t num_slots;
+    /* ABI version 3 */
+    void *workspace;
+    size_t workspace_bytes;
 } jamba_ssm_scan_params;
+
+/* Bytes of workspace a scan of these sizes may use: the status block
+ * (JAMBA_SSM_STATUS_BYTES) at any size, since nothing else is stored. */
+size_t jamba_ssm_scan_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner,
+                                     int64_t d_state);
 
 jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream);
 
@@ -158,16 +193,19 @@ jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream);
  *   out   = (sum_n C[b,n] h'[n] + D[d] x) * silu(z),
  * and the state is overwritten with h' IN PLACE.
  * Sizes: as jamba_ssm_scan with seqlen = 1, except d_inner only needs
- * d_inner >= 1 and d_state in {4, 8, 16} for both dtypes.
+ * d_inner >= 1; d_state in {1, 2, 4, 8, 16} for both dtypes (1 and 2: at most
+ * 65535 requests per call).
  * Pointers (device):
- *   state      [batch, d_inner, d_state] fp32, 16-byte aligned, read + written.
+ *   state      [batch, d_inner, d_state] fp32, 16-byte aligned (4-byte for
+ *              d_state 1 and 2), read + written.
  *   x, delta, z, out [batch, d_inner] io_dtype, aligned to the element size;
  *              out must not overlap an input.  (When x, delta and z are
  *              16-byte aligned and the rows are multiples of 16 bytes, a
  *              bulk-copy kernel is used; otherwise a plain-load kernel.)
- *   B, C       [batch, d_state] io_dtype, 16-byte aligned.
- *   A          [d_inner, d_state] fp32, 16-byte aligned; D, delta_bias as above
- *              (4-byte aligned or NULL).
+ *   B, C       [batch, d_state] io_dtype, 16-byte aligned (element-aligned
+ *              for d_state 1 and 2).
+ *   A          [d_inner, d_state] fp32, 16-byte aligned (4-byte for d_state 1
+ *              and 2); D, delta_bias as above (4-byte aligned or NULL).
  * Serving layout (ABI version 2; absent when struct_size ends before it):
  *   state_indices device int32 [batch] or NULL.  Non-NULL: `state` is a
  *              [num_slots, d_inner, d_state] cache and request b updates row
@@ -182,6 +220,7 @@ jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *p, void *stream);
  *              kernel so its bounded wait runs out (test of the timeout path;
  *              rows of 16-byte multiples take that kernel); timeout_cycles
  *              overrides the wait limit (SM clock cycles, 0 = ~1 s).
+ * Workspace (ABI version 3): as jamba_ssm_scan (status word only), or NULL.
  */
 typedef struct jamba_ssm_state_update_params {
     size_t struct_size;          /* = sizeof(jamba_ssm_state_update_params);
@@ -201,12 +240,16 @@ typedef struct jamba_ssm_state_update_params {
     int64_t num_slots;
     uint32_t debug_flags;
     uint64_t timeout_cycles;
+    /* ABI version 3 */
+    void *workspace;
+    size_t workspace_bytes;
 } jamba_ssm_state_update_params;
 
 jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, void *stream);
 
 /* Launch shape the scan would use for these parameters (no launch).  Any of
- * the out pointers may be NULL.  variant: the built variant chosen;
+ * the out pointers may be NULL.  variant: the built variant chosen (0 for the
+ * one-thread-per-channel kernel of the small state sizes);
  * lanes_per_channel: lanes sharing one channel's states; channels_per_cta;
  * grid: CTAs launched; tasks: (sequence, channel-group) units. */
 jamba_ssm_status jamba_ssm_scan_plan(const jamba_ssm_scan_params *p, int32_t *variant,
@@ -219,12 +262,15 @@ jamba_ssm_status jamba_ssm_scan_variant_info(int32_t k, int32_t *io_dtype, int32
                                              int32_t *lanes_per_channel, int32_t *warps_per_cta,
                                              int32_t *time_tile);
 
-/* Synchronizes `stream`, then reads and clears the current device's sticky
- * status word: JAMBA_SSM_OK, or the first device-side error recorded since the
- * last call (JAMBA_SSM_ERR_TIMEOUT, or JAMBA_SSM_ERR_INVALID_ARG for a state
- * index past num_slots).  Returns JAMBA_SSM_ERR_CUDA if the
- * synchronization itself failed. */
-jamba_ssm_status jamba_ssm_get_status(void *stream);
+/* Synchronizes `stream`, then reads and clears a sticky status word: the
+ * first word of `workspace` (the calls that were given this workspace), or,
+ * for workspace == NULL, the current device's word of the library (the calls
+ * given none).  Returns JAMBA_SSM_OK, or the first device-side error recorded
+ * there since the last read (JAMBA_SSM_ERR_TIMEOUT, or
+ * JAMBA_SSM_ERR_INVALID_ARG for a state index past num_slots).  Returns
+ * JAMBA_SSM_ERR_CUDA if the synchronization or the read itself failed, and
+ * JAMBA_SSM_ERR_MISALIGNED for a workspace that is not 16-byte aligned. */
+jamba_ssm_status jamba_ssm_get_status(void *workspace, void *stream);
 
 /* CUDA error code (cudaError_t as int) behind the last JAMBA_SSM_ERR_CUDA
  * returned on this host thread, 0 if none. */

@@ -24,6 +24,7 @@ from . import _lib
 from ._lib import JambaSSMError
 
 __all__ = ["jamba_ssm_scan", "jamba_ssm_state_update", "jamba_ssm_get_status", "scan_plan",
+           "jamba_ssm_scan_workspace_size",
            "jamba_ssm_x_proj", "jamba_ssm_dt_proj", "jamba_ssm_proj_get_status",
            "JambaSSMError"]
 
@@ -55,8 +56,18 @@ def _stream(stream, device):
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _workspace(ws, device):
+    """(pointer, bytes) of an optional workspace tensor (the call's status word)."""
+    if ws is None:
+        return None, 0
+    if not isinstance(ws, torch.Tensor) or ws.device != device or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor on the device of the inputs")
+    return ws.data_ptr(), ws.numel() * ws.element_size()
+
+
 def _scan_params(x, delta, z, B, C, A, D, delta_bias, delta_softplus, h0, out, h_final,
-                 variant, debug_flags, timeout_cycles, cu_seqlens=None, state_indices=None):
+                 variant, debug_flags, timeout_cycles, cu_seqlens=None, state_indices=None,
+                 workspace=None):
     if x.dtype not in _IO:
         raise TypeError(f"x must be bfloat16 or float32, got {x.dtype}")
     d_state = A.shape[-1]
@@ -86,6 +97,7 @@ def _scan_params(x, delta, z, B, C, A, D, delta_bias, delta_softplus, h0, out, h
     state_shape = (num_slots if state_indices is not None else batch, d_inner, d_state)
     _check(h0, "h0", state_shape, torch.float32, dev)
     _check(h_final, "h_final", state_shape, torch.float32, dev)
+    ws, ws_bytes = _workspace(workspace, dev)
     return _lib.new_scan_params(
         batch=batch, seqlen=seqlen, d_inner=d_inner, d_state=d_state, io_dtype=_IO[io],
         delta_softplus=int(bool(delta_softplus)), x=_ptr(x), delta=_ptr(delta), z=_ptr(z),
@@ -93,13 +105,14 @@ def _scan_params(x, delta, z, B, C, A, D, delta_bias, delta_softplus, h0, out, h
         out=_ptr(out), h_final=_ptr(h_final), kernel_variant=int(variant),
         debug_flags=int(debug_flags), timeout_cycles=int(timeout_cycles),
         cu_seqlens=_ptr(cu_seqlens), total_tokens=int(total),
-        state_indices=_ptr(state_indices), num_slots=int(num_slots))
+        state_indices=_ptr(state_indices), num_slots=int(num_slots), workspace=ws,
+        workspace_bytes=ws_bytes)
 
 
 def jamba_ssm_scan(x, delta, z, B, C, A, D=None, delta_bias=None, delta_softplus=True,
                    h0=None, out=None, h_final=None, return_final_state=True, stream=None,
                    variant: int = 0, debug_flags: int = 0, timeout_cycles: int = 0,
-                   cu_seqlens=None, state_indices=None):
+                   cu_seqlens=None, state_indices=None, workspace=None):
     """Prefill S6 scan.  Shapes: x, delta, z [batch, seqlen, d_inner] (bf16 or
     fp32), B, C [batch, seqlen, d_state] (same dtype), A [d_inner, d_state]
     fp32, D and delta_bias [d_inner] fp32 or None, h0 [batch, d_inner, d_state]
@@ -111,7 +124,11 @@ def jamba_ssm_scan(x, delta, z, B, C, A, D=None, delta_bias=None, delta_softplus
     and sequence b is rows cu_seqlens[b]:cu_seqlens[b+1].  With
     ``state_indices`` (int32 [batch]) h0 / h_final are [num_slots, d_inner,
     d_state] caches and sequence b uses row state_indices[b] (negative: zero
-    initial state, nothing written); pass h_final explicitly in that case."""
+    initial state, nothing written); pass h_final explicitly in that case.
+
+    ``workspace``: an optional zero-filled device tensor of at least
+    ``jamba_ssm_scan_workspace_size(...)`` bytes that holds this call's status
+    word (read with ``jamba_ssm_get_status(workspace=...)``)."""
     if out is None:
         out = torch.empty_like(x)
     if h_final is None and return_final_state and state_indices is None:
@@ -119,7 +136,7 @@ def jamba_ssm_scan(x, delta, z, B, C, A, D=None, delta_bias=None, delta_softplus
         h_final = torch.empty(batch, x.shape[-1], A.shape[-1], dtype=torch.float32,
                               device=x.device)
     p = _scan_params(x, delta, z, B, C, A, D, delta_bias, delta_softplus, h0, out, h_final,
-                     variant, debug_flags, timeout_cycles, cu_seqlens, state_indices)
+                     variant, debug_flags, timeout_cycles, cu_seqlens, state_indices, workspace)
     st = _lib.call_scan(p, _stream(stream, x.device))
     if st != _lib.OK:
         raise JambaSSMError(st, "jamba_ssm_scan")
@@ -137,7 +154,7 @@ def scan_plan(x, A, B=None, variant: int = 0):
 
 def jamba_ssm_state_update(state, x, delta, z, B, C, A, D=None, delta_bias=None,
                            delta_softplus=True, out=None, stream=None, state_indices=None,
-                           debug_flags: int = 0, timeout_cycles: int = 0):
+                           debug_flags: int = 0, timeout_cycles: int = 0, workspace=None):
     """One decode step; `state` [batch, d_inner, d_state] fp32 is updated in
     place.  x, delta, z [batch, d_inner]; B, C [batch, d_state].  Returns out
     [batch, d_inner].  With ``state_indices`` (int32 [batch] on the device)
@@ -164,28 +181,36 @@ def jamba_ssm_state_update(state, x, delta, z, B, C, A, D=None, delta_bias=None,
     _check(A, "A", (d_inner, d_state), torch.float32, dev)
     _check(D, "D", (d_inner,), torch.float32, dev)
     _check(delta_bias, "delta_bias", (d_inner,), torch.float32, dev)
+    ws, ws_bytes = _workspace(workspace, dev)
     p = _lib.new_state_update_params(
         batch=batch, d_inner=d_inner, d_state=d_state, io_dtype=_IO[io],
         delta_softplus=int(bool(delta_softplus)), state=_ptr(state), x=_ptr(x),
         delta=_ptr(delta), z=_ptr(z), B=_ptr(B), C=_ptr(C), A=_ptr(A), D=_ptr(D),
         delta_bias=_ptr(delta_bias), out=_ptr(out), state_indices=_ptr(state_indices),
         num_slots=int(num_slots), debug_flags=int(debug_flags),
-        timeout_cycles=int(timeout_cycles))
+        timeout_cycles=int(timeout_cycles), workspace=ws, workspace_bytes=ws_bytes)
     st = _lib.call_state_update(p, _stream(stream, dev))
     if st != _lib.OK:
         raise JambaSSMError(st, "jamba_ssm_state_update")
     return out
 
 
-def jamba_ssm_get_status(stream=None, device=None) -> int:
-    """Synchronize the stream and read-and-clear the device status word."""
+def jamba_ssm_get_status(stream=None, device=None, workspace=None) -> int:
+    """Synchronize the stream and read-and-clear a status word: the
+    workspace's, or the device's word of the library when none is given."""
     dev = torch.device(device) if device is not None else torch.device("cuda",
                                                                         torch.cuda.current_device())
-    return _lib.get_status(_stream(stream, dev))
+    ws, _ = _workspace(workspace, workspace.device if workspace is not None else dev)
+    return _lib.get_status(_stream(stream, dev), ws or 0)
+
+
+def jamba_ssm_scan_workspace_size(batch: int, seqlen: int, d_inner: int, d_state: int) -> int:
+    """Bytes of the optional workspace of a scan (its status block)."""
+    return _lib.scan_workspace_size(int(batch), int(seqlen), int(d_inner), int(d_state))
 
 
 def jamba_ssm_x_proj(u, W_x, w_dt=None, w_B=None, w_C=None, eps=1e-6, d_state=16,
-                     k_split=0, timeout_cycles=0, stream=None):
+                     k_split=0, timeout_cycles=0, stream=None, debug_flags=0):
     """[dt_low | B | C] = u @ W_x.T, each part RMS-normalised with its weight
     (None: not normalised).
 
@@ -213,7 +238,7 @@ def jamba_ssm_x_proj(u, W_x, w_dt=None, w_B=None, w_C=None, eps=1e-6, d_state=16
                                u=_ptr(u), W_x=_ptr(W_x), w_dt=_ptr(w_dt), w_B=_ptr(w_B),
                                w_C=_ptr(w_C), eps=float(eps), k_split=int(k_split),
                                dt_low_hi=_ptr(hi), dt_low_lo=_ptr(lo), B=_ptr(B), C=_ptr(C),
-                               timeout_cycles=int(timeout_cycles))
+                               timeout_cycles=int(timeout_cycles), debug_flags=int(debug_flags))
     st = _lib.call_x_proj(p, _stream(stream, dev))
     if st != _lib.OK:
         raise JambaSSMError(st, "jamba_ssm_x_proj",
@@ -221,7 +246,8 @@ def jamba_ssm_x_proj(u, W_x, w_dt=None, w_B=None, w_C=None, eps=1e-6, d_state=16
     return hi, lo, B, C
 
 
-def jamba_ssm_dt_proj(dt_low_hi, W_dt, dt_low_lo=None, out=None, timeout_cycles=0, stream=None):
+def jamba_ssm_dt_proj(dt_low_hi, W_dt, dt_low_lo=None, out=None, timeout_cycles=0, stream=None,
+                      debug_flags=0):
     """delta = (dt_low_hi + dt_low_lo) @ W_dt.T in fp32, rounded once to bf16.
 
     dt_low_hi / dt_low_lo: [..., dt_rank] bf16, the two planes of the fp32
@@ -245,7 +271,7 @@ def jamba_ssm_dt_proj(dt_low_hi, W_dt, dt_low_lo=None, out=None, timeout_cycles=
     p = _lib.new_dt_proj_params(ntok=ntok, d_inner=d_inner, dt_rank=dt_rank,
                                 dt_low_hi=_ptr(dt_low_hi), dt_low_lo=_ptr(dt_low_lo),
                                 W_dt=_ptr(W_dt), delta=_ptr(out),
-                                timeout_cycles=int(timeout_cycles))
+                                timeout_cycles=int(timeout_cycles), debug_flags=int(debug_flags))
     st = _lib.call_dt_proj(p, _stream(stream, dev))
     if st != _lib.OK:
         raise JambaSSMError(st, "jamba_ssm_dt_proj",

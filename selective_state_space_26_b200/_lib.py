@@ -14,12 +14,15 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libjamba_ssm.so")
 PROJ_LIB_PATH = os.path.join(_PKG, "libjamba_ssm_proj.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_NO_DEVICE = range(7)
+(OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT,
+ ERR_NO_DEVICE) = range(8)
+STATUS_BYTES = 16  # JAMBA_SSM_STATUS_BYTES
 BF16, F32 = 0, 1
 
 # Every symbol the header declares.
 EXPORTS = (
     "jamba_ssm_scan",
+    "jamba_ssm_scan_workspace_size",
     "jamba_ssm_state_update",
     "jamba_ssm_scan_plan",
     "jamba_ssm_scan_variant_info",
@@ -56,6 +59,8 @@ class ScanParams(ctypes.Structure):
         # ABI version 2
         ("cu_seqlens", _vp), ("total_tokens", ctypes.c_int64),
         ("state_indices", _vp), ("num_slots", ctypes.c_int64),
+        # ABI version 3
+        ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
     ]
 
 
@@ -72,6 +77,8 @@ class StateUpdateParams(ctypes.Structure):
         # ABI version 2
         ("state_indices", _vp), ("num_slots", ctypes.c_int64),
         ("debug_flags", ctypes.c_uint32), ("timeout_cycles", ctypes.c_uint64),
+        # ABI version 3
+        ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
     ]
 
 
@@ -81,6 +88,7 @@ class DtProjParams(ctypes.Structure):
         ("ntok", ctypes.c_int64), ("d_inner", ctypes.c_int64), ("dt_rank", ctypes.c_int64),
         ("dt_low_hi", _vp), ("dt_low_lo", _vp), ("W_dt", _vp), ("delta", _vp),
         ("timeout_cycles", ctypes.c_uint64),
+        ("debug_flags", ctypes.c_uint32),  # version 2
     ]
 
 
@@ -93,6 +101,7 @@ class XProjParams(ctypes.Structure):
         ("eps", ctypes.c_float), ("k_split", ctypes.c_int32),
         ("dt_low_hi", _vp), ("dt_low_lo", _vp), ("B", _vp), ("C", _vp),
         ("timeout_cycles", ctypes.c_uint64),
+        ("debug_flags", ctypes.c_uint32),  # version 2
     ]
 
 
@@ -133,7 +142,9 @@ def lib():
                 L.jamba_ssm_scan_variant_info.restype = ctypes.c_int
                 L.jamba_ssm_scan_variant_info.argtypes = [ctypes.c_int32] + [i32p] * 5
                 L.jamba_ssm_get_status.restype = ctypes.c_int
-                L.jamba_ssm_get_status.argtypes = [_vp]
+                L.jamba_ssm_get_status.argtypes = [_vp, _vp]
+                L.jamba_ssm_scan_workspace_size.restype = ctypes.c_size_t
+                L.jamba_ssm_scan_workspace_size.argtypes = [ctypes.c_int64] * 4
                 L.jamba_ssm_last_cuda_error.restype = ctypes.c_int
                 L.jamba_ssm_last_cuda_error.argtypes = []
                 L.jamba_ssm_status_string.restype = ctypes.c_char_p
@@ -173,10 +184,12 @@ def status_string(status: int) -> str:
     return lib().jamba_ssm_status_string(int(status)).decode()
 
 
-# struct_size of the ABI version 1 structures (the fields before the
-# version 2 ones), for callers built against version 1
+# struct_size of the ABI version 1 and 2 structures (the fields before the
+# next version's), for callers built against those versions
 SCAN_PARAMS_V1_SIZE = ScanParams.cu_seqlens.offset
 STATE_UPDATE_PARAMS_V1_SIZE = StateUpdateParams.state_indices.offset
+SCAN_PARAMS_V2_SIZE = ScanParams.workspace.offset
+STATE_UPDATE_PARAMS_V2_SIZE = StateUpdateParams.workspace.offset
 
 
 def new_scan_params(**kw) -> ScanParams:
@@ -223,8 +236,12 @@ def variant_info(k: int):
     return dict(zip(keys, (v.value for v in vals)))
 
 
-def get_status(stream: int) -> int:
-    return lib().jamba_ssm_get_status(_vp(stream or None))
+def get_status(stream: int, workspace: int = 0) -> int:
+    return lib().jamba_ssm_get_status(_vp(workspace or None), _vp(stream or None))
+
+
+def scan_workspace_size(batch: int, seqlen: int, d_inner: int, d_state: int) -> int:
+    return lib().jamba_ssm_scan_workspace_size(batch, seqlen, d_inner, d_state)
 
 
 def new_dt_proj_params(**kw) -> DtProjParams:

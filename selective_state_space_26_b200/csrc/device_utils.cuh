@@ -10,8 +10,19 @@
 namespace jssm {
 
 // Sticky device-side status word of the library (0 = ok), one per device; a
-// kernel whose bounded wait runs out writes JAMBA_SSM_ERR_TIMEOUT here.
+// kernel whose bounded wait runs out writes JAMBA_SSM_ERR_TIMEOUT here, unless
+// the caller passed a workspace, whose first word then takes its place.
 __device__ int g_status_word;
+
+// Device-side status codes (the values of jamba_ssm_status).
+constexpr int kStInvalidArg = 1;  // JAMBA_SSM_ERR_INVALID_ARG
+constexpr int kStTimeout = 6;     // JAMBA_SSM_ERR_TIMEOUT
+
+// Records `code` in the call's status word (the caller's workspace, or the
+// library's own word when there is none) unless an error is already there.
+__device__ __forceinline__ void record_status(int *workspace_word, int code) {
+    atomicCAS(workspace_word ? workspace_word : &g_status_word, 0, code);
+}
 
 // ---------------------------------------------------------------- conversions
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }

@@ -28,18 +28,19 @@ struct ScanArgs {
     const int *state_indices;  // state-cache row of each sequence, or null
     int64_t num_slots;         // rows of the state cache
     void *out;                 // output base (row-wise stores of short packed tiles)
+    int *status;               // the call's status word (caller workspace), or null
 };
 
 // No steps at all (every sequence empty) with a state cache: final state =
 // initial state (or zeros) for each sequence's slot; one thread per float.
 // An index past num_slots is recorded as JAMBA_SSM_ERR_INVALID_ARG.
 __global__ void s6_copy_states_kernel(int64_t batch, int64_t per_seq, const float *h0, float *h_final,
-                                      const int *state_indices, int64_t num_slots) {
+                                      const int *state_indices, int64_t num_slots, int *status) {
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= batch * per_seq) return;
     const int64_t b = i / per_seq, e = i - b * per_seq;
     const int64_t row = state_indices[b];
-    if (row >= num_slots && e == 0) atomicCAS(&g_status_word, 0, 1 /* JAMBA_SSM_ERR_INVALID_ARG */);
+    if (row >= num_slots && e == 0) record_status(status, kStInvalidArg);
     if (row < 0 || row >= num_slots) return;
     h_final[row * per_seq + e] = h0 ? h0[row * per_seq + e] : 0.0f;
 }

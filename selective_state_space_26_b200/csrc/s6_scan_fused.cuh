@@ -218,7 +218,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
 
     auto fail = [&]() {
         *abort_flag = 1;
-        atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+        record_status(args.status, kStTimeout);
     };
     // (sequence, first channel, tile index) of the CTA's g-th tile.  Callers
     // walk g upward, so the cursor advances without 64-bit divisions except

@@ -107,7 +107,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
 
     auto fail = [&]() {
         *abort_flag = 1;
-        atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+        record_status(args.status, kStTimeout);
     };
     // The CTA's g-th tile: task (sequence b, channels from c0), tile k of the
     // task.  Every caller walks g upward one at a time, so the cursor only
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             srow = __ldg(args.state_indices + b);
             svalid = srow >= 0 && srow < args.num_slots;
             if (srow >= args.num_slots && tid == 0)
-                atomicCAS(&g_status_word, 0, 1 /* JAMBA_SSM_ERR_INVALID_ARG */);
+                record_status(args.status, kStInvalidArg);
         }
 #pragma unroll
         for (int i = 0; i < NS / 2; ++i) {

@@ -36,6 +36,7 @@ struct UpdateArgs {
     const int *state_indices;  // state-cache row of each request, or null (row b)
     int64_t num_slots;         // rows of the state cache
     uint32_t debug_flags;      // bit 0: withhold each CTA's first load (tests the bounded waits)
+    int *status;               // the call's status word (caller workspace), or null
 };
 
 // State-cache row of request b, or -1 when the request is skipped (a negative
@@ -44,7 +45,7 @@ __device__ __forceinline__ int64_t state_row(const UpdateArgs &a, int64_t b, boo
     if (!a.state_indices) return b;
     const int64_t r = __ldg(a.state_indices + b);
     if (r >= a.num_slots) {
-        if (record) atomicCAS(&g_status_word, 0, 1 /* JAMBA_SSM_ERR_INVALID_ARG */);
+        if (record) record_status(a.status, kStInvalidArg);
         return -1;
     }
     return r < 0 ? -1 : r;
@@ -244,7 +245,7 @@ __global__ void __launch_bounds__(UpdateCfg<IoT, N, CPB, STAGES>::kThreads, 4)
             }
             if (!ok) {
                 *abort_flag = 1;
-                atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+                record_status(a.status, kStTimeout);
             }
             // copies still in flight when the compute warps may have left:
             // wait (bounded) for each stage's last fill before the CTA exits
@@ -282,7 +283,7 @@ __global__ void __launch_bounds__(UpdateCfg<IoT, N, CPB, STAGES>::kThreads, 4)
                                     limit, abort_flag);
         if (!ok) {
             *abort_flag = 1;
-            atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+            record_status(a.status, kStTimeout);
             break;
         }
         // this lane's owned request r0 + q (a copy of request r0 when q >= nr)

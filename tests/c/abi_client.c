@@ -76,7 +76,15 @@ int main(int argc, char **argv) {
     p.x = dx; p.delta = ddt; p.z = dz; p.B = dB; p.C = dC;
     p.A = (const float *)dA; p.D = (const float *)dD; p.delta_bias = (const float *)dbias;
     p.out = dout; p.h_final = (float *)dhf;
+    /* the optional workspace: the call's status word, zero-filled once */
+    const size_t ws_bytes = jamba_ssm_scan_workspace_size(b, l, d, n);
+    void *ws = NULL;
+    if (ws_bytes < JAMBA_SSM_STATUS_BYTES || cudaMalloc(&ws, ws_bytes) != cudaSuccess ||
+        cudaMemset(ws, 0, ws_bytes) != cudaSuccess)
+        return 4;
+    p.workspace = ws; p.workspace_bytes = ws_bytes;
     if (check(jamba_ssm_scan(&p, NULL), "jamba_ssm_scan")) return 5;
+    if (check(jamba_ssm_get_status(ws, NULL), "jamba_ssm_get_status (workspace)")) return 5;
 
     jamba_ssm_state_update_params u = {0};
     u.struct_size = sizeof(u);
@@ -92,7 +100,7 @@ int main(int argc, char **argv) {
     float *hf = (float *)malloc(st * sizeof(float));
     if (!hf || cudaMemcpy(hf, dhf, st * sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess) return 6;
     if (check(jamba_ssm_state_update(&u, NULL), "jamba_ssm_state_update")) return 5;
-    if (check(jamba_ssm_get_status(NULL), "jamba_ssm_get_status")) return 5;
+    if (check(jamba_ssm_get_status(NULL, NULL), "jamba_ssm_get_status")) return 5;
 
     float *out = (float *)malloc(act * sizeof(float)), *out1 = (float *)malloc((size_t)(b * d) * sizeof(float));
     float *st1 = (float *)malloc(st * sizeof(float));

@@ -57,7 +57,7 @@ def test_every_declared_proj_symbol_is_exported(P):
         assert n in exported, f"{n} declared in the header but not exported"
     # the projection library keeps its kernels and status word to itself
     assert not [e for e in exported if "jssm" in e], "internal symbols exported"
-    assert P.jamba_ssm_proj_abi_version() == 1
+    assert P.jamba_ssm_proj_abi_version() == 2
 
 
 def test_struct_layout_matches_header(tmp_path):
@@ -89,10 +89,37 @@ def test_struct_layout_matches_header(tmp_path):
 
 
 def test_status_strings_and_version(L):
-    assert L.jamba_ssm_abi_version() == 2
-    for s in range(7):
-        assert _lib.status_string(s)
+    assert L.jamba_ssm_abi_version() == 3
+    for s in range(8):
+        assert _lib.status_string(s) != "unknown status"
     assert _lib.status_string(99) == "unknown status"
+
+
+def test_status_codes_match_header(tmp_path):
+    """The binding's status constants are the header's enum values (the
+    contract's order: ERR_WORKSPACE = 4, ERR_CUDA = 5, ERR_TIMEOUT = 6)."""
+    names = ["OK", "ERR_INVALID_ARG", "ERR_UNSUPPORTED", "ERR_MISALIGNED", "ERR_WORKSPACE",
+             "ERR_CUDA", "ERR_TIMEOUT", "ERR_NO_DEVICE"]
+    body = "".join(f'printf("{n} %d\\n", (int)JAMBA_SSM_{n});' for n in names)
+    src = tmp_path / "enums.c"
+    src.write_text('#include <stdio.h>\n#include "jamba_ssm.h"\nint main(void) {' + body +
+                   'printf("STATUS_BYTES %d\\n", JAMBA_SSM_STATUS_BYTES); return 0; }')
+    exe = tmp_path / "enums"
+    subprocess.run(["gcc", "-I", os.path.dirname(HEADER), "-o", str(exe), str(src)], check=True)
+    got = dict(line.split() for line in subprocess.run(
+        [str(exe)], capture_output=True, text=True, check=True).stdout.splitlines())
+    for n in names:
+        assert int(got[n]) == getattr(_lib, n), n
+    assert (_lib.ERR_WORKSPACE, _lib.ERR_CUDA, _lib.ERR_TIMEOUT) == (4, 5, 6)
+    assert int(got["STATUS_BYTES"]) == _lib.STATUS_BYTES
+
+
+def test_scan_workspace_size(L):
+    """The scan stores no carry between chunks of a sequence, so its workspace
+    is the status block at every size."""
+    for sizes in [(1, 4096, 8192, 16), (16, 16384, 8192, 16), (1, 1 << 18, 8192, 16),
+                  (0, 0, 8, 1), (3, 77, 64, 4)]:
+        assert _lib.scan_workspace_size(*sizes) == _lib.STATUS_BYTES
 
 
 def test_variant_table(L):
@@ -130,8 +157,9 @@ def _scan(p):
     (dict(d_inner=0), _lib.ERR_INVALID_ARG),
     (dict(io_dtype=7), _lib.ERR_INVALID_ARG),
     (dict(d_state=5), _lib.ERR_UNSUPPORTED),
-    (dict(d_state=4), _lib.ERR_UNSUPPORTED),          # bf16 rows of 8 bytes: not TMA-able
+    (dict(d_state=3), _lib.ERR_UNSUPPORTED),
     (dict(d_state=32), _lib.ERR_UNSUPPORTED),
+    (dict(d_state=4, batch=70000, seqlen=1), _lib.ERR_UNSUPPORTED),  # small-state grid
     (dict(d_inner=12), _lib.ERR_UNSUPPORTED),         # bf16 row not a multiple of 16 bytes
     (dict(kernel_variant=99), _lib.ERR_UNSUPPORTED),
     (dict(kernel_variant=8), _lib.ERR_UNSUPPORTED),   # an fp32 variant for bf16 data
@@ -147,8 +175,11 @@ def _scan(p):
     (dict(h_final=0x90000000 + 1024), _lib.ERR_INVALID_ARG),  # h_final inside out
     (dict(h0=0xA0000000 + 16), _lib.ERR_INVALID_ARG),  # h0 partially overlaps h_final
     (dict(batch=1 << 20, seqlen=1 << 20, d_inner=1 << 12), _lib.ERR_UNSUPPORTED),
-    (dict(io_dtype=_lib.F32, d_state=2), _lib.ERR_UNSUPPORTED),
+    (dict(io_dtype=_lib.F32, d_state=6), _lib.ERR_UNSUPPORTED),
     (dict(io_dtype=_lib.F32, d_inner=10), _lib.ERR_UNSUPPORTED),
+    (dict(workspace=0xC0000008, workspace_bytes=64), _lib.ERR_MISALIGNED),
+    (dict(workspace=0xC0000000, workspace_bytes=8), _lib.ERR_WORKSPACE),
+    (dict(workspace=0xC0000000, workspace_bytes=0), _lib.ERR_WORKSPACE),
 ])
 def test_scan_argument_errors(L, kw, expect):
     assert _scan(_valid_scan(**kw)) == expect
@@ -173,8 +204,12 @@ def _valid_update(**kw):
 
 @pytest.mark.parametrize("kw,expect", [
     (dict(batch=-1), _lib.ERR_INVALID_ARG),
-    (dict(d_state=2), _lib.ERR_UNSUPPORTED),
+    (dict(d_state=3), _lib.ERR_UNSUPPORTED),
     (dict(d_state=12), _lib.ERR_UNSUPPORTED),
+    (dict(d_state=2, batch=70000), _lib.ERR_UNSUPPORTED),  # small-state grid
+    (dict(d_state=2, state=0x10000002), _lib.ERR_MISALIGNED),
+    (dict(workspace=0x90000004, workspace_bytes=16), _lib.ERR_MISALIGNED),
+    (dict(workspace=0x90000000, workspace_bytes=4), _lib.ERR_WORKSPACE),
     (dict(state=None), _lib.ERR_INVALID_ARG),
     (dict(state=0x10000008), _lib.ERR_MISALIGNED),
     (dict(x=0x20000001), _lib.ERR_MISALIGNED),
@@ -190,6 +225,16 @@ def test_state_update_argument_errors(L, kw, expect):
 def test_valid_call_without_device_reports_no_device(L):
     assert _scan(_valid_scan()) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
     assert _lib.call_state_update(_valid_update(), 0) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
+    # every d_state of the contract passes validation (the small ones too)
+    for n in (1, 2, 4, 8, 16):
+        for io in (_lib.BF16, _lib.F32):
+            assert _scan(_valid_scan(d_state=n, io_dtype=io)) in \
+                (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA), (n, io)
+            assert _lib.call_state_update(_valid_update(d_state=n, io_dtype=io), 0) in \
+                (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA), (n, io)
+    # a big enough, aligned workspace is accepted
+    assert _scan(_valid_scan(workspace=0xC0000000, workspace_bytes=16)) in \
+        (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
     p = _valid_scan(batch=0)
     assert _scan(p) == _lib.OK or _scan(p) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
 
@@ -238,6 +283,18 @@ def test_version_1_struct_size_is_accepted(L):
     assert _lib.call_state_update(u, 0) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
     u.struct_size = _lib.STATE_UPDATE_PARAMS_V1_SIZE - 8
     assert _lib.call_state_update(u, 0) == _lib.ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_version_2_struct_size_is_accepted(L):
+    """A version-2 caller's struct ends before the workspace fields: whatever
+    lies past it is ignored (no workspace)."""
+    p = _valid_scan(workspace=0xC0000004, workspace_bytes=1)  # invalid if it were read
+    p.struct_size = _lib.SCAN_PARAMS_V2_SIZE
+    assert _scan(p) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
+    u = _valid_update(workspace=0x90000004, workspace_bytes=1)
+    u.struct_size = _lib.STATE_UPDATE_PARAMS_V2_SIZE
+    assert _lib.call_state_update(u, 0) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
 
 
 _A16 = 0x7f0000000000  # fake, 16-byte aligned, never dereferenced
