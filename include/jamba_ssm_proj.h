@@ -22,7 +22,10 @@
  * nothing allocated, `stream` a cudaStream_t passed as void*, argument errors
  * returned before anything is enqueued, no C++ exception across the interface.
  * Device-side conditions of this library are read with
- * jamba_ssm_proj_get_status (this library keeps its own status word).
+ * jamba_ssm_proj_get_status (this library keeps its own status word): a call
+ * returns as soon as its kernel is enqueued, so a caller that must know the
+ * outputs are valid checks that status after the stream's work.  With
+ * JAMBA_SSM_SYNC_CHECK set (and not "0") every call waits and returns it.
  */
 #ifndef JAMBA_SSM_PROJ_H
 #define JAMBA_SSM_PROJ_H
@@ -36,7 +39,8 @@
 extern "C" {
 #endif
 
-#define JAMBA_SSM_PROJ_ABI_VERSION 1
+/* Version 2 appends debug_flags to both parameter structs. */
+#define JAMBA_SSM_PROJ_ABI_VERSION 2
 
 /*
  * delta[t, d] = sum_r W_dt[d, r] * (dt_low_hi[t, r] + dt_low_lo[t, r]),
@@ -53,6 +57,9 @@ extern "C" {
  *   delta      [ntok, d_inner]   bf16, written; must not overlap an input.
  * timeout_cycles: SM clock cycles a bounded wait may spin before the kernel
  *   gives up and records JAMBA_SSM_ERR_TIMEOUT (0 = the default, ~2 s).
+ * debug_flags (version 2; 0 in production): bit 0 withholds every CTA's first
+ *   k-block of operands so that its bounded wait runs out (a test of the
+ *   timeout path); the tiles of such a call are not written.
  * Errors: INVALID_ARG (NULL, bad size or struct_size, overlap), UNSUPPORTED
  * (sizes out of range or not multiples of 8), MISALIGNED, NO_DEVICE, CUDA.
  */
@@ -66,6 +73,7 @@ typedef struct {
     const void *W_dt;
     void *delta;
     uint64_t timeout_cycles;
+    uint32_t debug_flags; /* version 2 */
 } jamba_ssm_dt_proj_params;
 
 jamba_ssm_status jamba_ssm_dt_proj(const jamba_ssm_dt_proj_params *p, void *stream);
@@ -91,7 +99,8 @@ jamba_ssm_status jamba_ssm_dt_proj(const jamba_ssm_dt_proj_params *p, void *stre
  * k_split: CTAs that share one 128-token tile's reduction over d_inner, as a
  *   thread-block cluster: 1, 2, 4 or 8, or 0 for the library's choice (the
  *   largest that keeps the grid within one wave of the SMs).
- * timeout_cycles: as for jamba_ssm_dt_proj.
+ * timeout_cycles, debug_flags: as for jamba_ssm_dt_proj (a withheld k-block
+ *   of one CTA leaves its whole cluster's rows unwritten).
  */
 typedef struct {
     size_t struct_size; /* sizeof(jamba_ssm_x_proj_params) */
@@ -111,6 +120,7 @@ typedef struct {
     void *B;
     void *C;
     uint64_t timeout_cycles;
+    uint32_t debug_flags; /* version 2 */
 } jamba_ssm_x_proj_params;
 
 jamba_ssm_status jamba_ssm_x_proj(const jamba_ssm_x_proj_params *p, void *stream);

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <cstddef>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -91,7 +92,7 @@ EncodeTiledFn encode_fn(jamba_ssm_status *st) {
 
 // 2-D bf16 map over [rows][cols] (cols innermost), box {64 cols, box_rows},
 // 128-byte swizzle, zero fill outside the tensor.  Both kernels take 64-wide
-// K blocks.
+// K blocks, and dt_proj stores its output tile as 64-column slabs.
 bool encode_kmajor(EncodeTiledFn fn, CUtensorMap *map, const void *ptr, int64_t cols,
                    int64_t rows, int box_rows) {
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -114,8 +115,17 @@ bool overlaps(const void *a, size_t an, const void *b, size_t bn) {
     return x < y + bn && y < x + an;
 }
 
-constexpr size_t kDtProjParamsV1 = sizeof(jamba_ssm_dt_proj_params);
-constexpr size_t kXProjParamsV1 = sizeof(jamba_ssm_x_proj_params);
+// Version 1 structs end before debug_flags; a caller's shorter struct is copied
+// over a zeroed one, so its missing fields read as zero.
+constexpr size_t kDtProjParamsV1 = offsetof(jamba_ssm_dt_proj_params, debug_flags);
+constexpr size_t kXProjParamsV1 = offsetof(jamba_ssm_x_proj_params, debug_flags);
+template <typename P>
+bool read_params(const P *pin, size_t v1_size, P *p) {
+    if (!pin || pin->struct_size < v1_size) return false;
+    std::memset(p, 0, sizeof(P));
+    std::memcpy(p, pin, pin->struct_size < sizeof(P) ? pin->struct_size : sizeof(P));
+    return true;
+}
 static_assert(jssm::DtProjCfg::kBK == jssm::XProjCfg::kBK, "one tensor-map box width");
 
 // Cluster size of the x_proj split over d_inner: the largest power of two up
@@ -130,11 +140,26 @@ constexpr uint64_t kDefaultTimeoutCycles = 4000000000ull;  // ~2 s at the boost 
 
 }  // namespace
 
+JSSM_PROJ_API jamba_ssm_status jamba_ssm_proj_get_status(void *stream);
+
+namespace {
+// After an enqueue: with JAMBA_SSM_SYNC_CHECK set (and not "0") in the
+// environment -- a debugging aid, read once per process -- wait for the work
+// and return any device-side condition it recorded as this call's own status.
+jamba_ssm_status finish_launch(void *stream) {
+    static const bool sync_check = [] {
+        const char *v = std::getenv("JAMBA_SSM_SYNC_CHECK");
+        return v != nullptr && *v != '\0' && *v != '0';
+    }();
+    return sync_check ? jamba_ssm_proj_get_status(stream) : JAMBA_SSM_OK;
+}
+
+}  // namespace
+
 JSSM_PROJ_API jamba_ssm_status jamba_ssm_dt_proj(const jamba_ssm_dt_proj_params *pin,
                                                  void *stream) {
-    if (!pin || pin->struct_size < kDtProjParamsV1) return JAMBA_SSM_ERR_INVALID_ARG;
     jamba_ssm_dt_proj_params p;
-    std::memcpy(&p, pin, sizeof(p));
+    if (!read_params(pin, kDtProjParamsV1, &p)) return JAMBA_SSM_ERR_INVALID_ARG;
     if (p.ntok < 0 || p.d_inner < 1 || p.dt_rank < 1) return JAMBA_SSM_ERR_INVALID_ARG;
     // d_inner / 256 channel tiles must fit the grid's y dimension
     if (p.d_inner % 8 != 0 || p.dt_rank % 8 != 0 || p.d_inner > int64_t(65535) * jssm::DtProjCfg::kBN ||
@@ -159,25 +184,24 @@ JSSM_PROJ_API jamba_ssm_status jamba_ssm_dt_proj(const jamba_ssm_dt_proj_params 
 
     EncodeTiledFn fn = encode_fn(&st);
     if (!fn) return st;
-    CUtensorMap map_hi, map_lo, map_w;
+    CUtensorMap map_hi, map_lo, map_w, map_out;
     const void *lo = p.dt_low_lo ? p.dt_low_lo : p.dt_low_hi;
     if (!encode_kmajor(fn, &map_hi, p.dt_low_hi, p.dt_rank, p.ntok, jssm::DtProjCfg::kBM) ||
         !encode_kmajor(fn, &map_lo, lo, p.dt_rank, p.ntok, jssm::DtProjCfg::kBM) ||
-        !encode_kmajor(fn, &map_w, p.W_dt, p.dt_rank, p.d_inner, jssm::DtProjCfg::kBN))
+        !encode_kmajor(fn, &map_w, p.W_dt, p.dt_rank, p.d_inner, jssm::DtProjCfg::kBN) ||
+        !encode_kmajor(fn, &map_out, p.delta, p.d_inner, p.ntok, jssm::DtProjCfg::kBM))
         return cuda_fail(cudaErrorInvalidValue);
-
-    __nv_bfloat16 *delta = static_cast<__nv_bfloat16 *>(p.delta);
-    int ntok = static_cast<int>(p.ntok), d_inner = static_cast<int>(p.d_inner),
-        dt_rank = static_cast<int>(p.dt_rank), two = p.dt_low_lo ? 1 : 0;
+    int dt_rank = static_cast<int>(p.dt_rank), two = p.dt_low_lo ? 1 : 0;
     uint64_t limit = p.timeout_cycles ? p.timeout_cycles : kDefaultTimeoutCycles;
-    void *args[] = {&map_hi, &map_lo, &map_w, &delta, &ntok, &d_inner, &dt_rank, &two, &limit};
+    uint32_t debug_flags = p.debug_flags;
+    void *args[] = {&map_hi, &map_lo, &map_w, &map_out, &dt_rank, &two, &limit, &debug_flags};
     const dim3 grid(static_cast<unsigned>((p.ntok + jssm::DtProjCfg::kBM - 1) / jssm::DtProjCfg::kBM),
                     static_cast<unsigned>((p.d_inner + jssm::DtProjCfg::kBN - 1) / jssm::DtProjCfg::kBN));
     cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void *>(&jssm::s6_dt_proj_kernel), grid,
                                      dim3(jssm::DtProjCfg::kThreads), args,
                                      jssm::DtProjCfg::kSmemBytes, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e);
-    return JAMBA_SSM_OK;
+    return finish_launch(stream);
 }
 
 JSSM_PROJ_API jamba_ssm_status jamba_ssm_proj_get_status(void *stream) {
@@ -203,9 +227,8 @@ JSSM_PROJ_API int jamba_ssm_proj_abi_version(void) { return JAMBA_SSM_PROJ_ABI_V
 JSSM_PROJ_API jamba_ssm_status jamba_ssm_x_proj(const jamba_ssm_x_proj_params *pin,
                                                 void *stream) {
     using XC = jssm::XProjCfg;
-    if (!pin || pin->struct_size < kXProjParamsV1) return JAMBA_SSM_ERR_INVALID_ARG;
     jamba_ssm_x_proj_params p;
-    std::memcpy(&p, pin, sizeof(p));
+    if (!read_params(pin, kXProjParamsV1, &p)) return JAMBA_SSM_ERR_INVALID_ARG;
     if (p.ntok < 0 || p.d_inner < 1 || p.dt_rank < 1 || p.d_state < 1 || !(p.eps >= 0.0f))
         return JAMBA_SSM_ERR_INVALID_ARG;
     if (p.k_split != 0 && p.k_split != 1 && p.k_split != 2 && p.k_split != 4 && p.k_split != 8)
@@ -262,6 +285,7 @@ JSSM_PROJ_API jamba_ssm_status jamba_ssm_x_proj(const jamba_ssm_x_proj_params *p
     a.ntok = static_cast<int>(p.ntok);
     a.d_inner = static_cast<int>(p.d_inner);
     a.limit = p.timeout_cycles ? p.timeout_cycles : kDefaultTimeoutCycles;
+    a.debug_flags = p.debug_flags;
 
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(XC::kThreads);
@@ -291,5 +315,5 @@ JSSM_PROJ_API jamba_ssm_status jamba_ssm_x_proj(const jamba_ssm_x_proj_params *p
     }
     cudaError_t e = cudaLaunchKernelEx(&cfg, jssm::s6_x_proj_kernel, map_u, map_w1, map_w2, a);
     if (e != cudaSuccess) return cuda_fail(e);
-    return JAMBA_SSM_OK;
+    return finish_launch(stream);
 }

@@ -23,9 +23,19 @@
 //           (M = 128, N = 256, K = 16, bf16 x bf16 -> fp32) and commits each
 //           stage back to the producer, then the finished accumulator;
 //   warps 2-5: epilogue -- each thread owns one token row (TMEM lane), reads
-//           its 256 fp32 columns with tcgen05.ld, rounds to bf16 and stores.
+//           its 256 fp32 columns with tcgen05.ld, rounds them to bf16 into a
+//           staged copy of the output tile in shared memory (the operand ring,
+//           free once every MMA has completed), laid out as four 64-column
+//           slabs with the 128-byte swizzle so that the 32 rows a warp writes
+//           at once fall in distinct banks; one thread then writes the tile
+//           with four TMA stores, which clip it to [ntok, d_inner].
 // Every wait is bounded; a wait that runs out records JAMBA_SSM_ERR_TIMEOUT in
-// the module's status word and the CTA winds down.
+// the module's status word and sets a CTA abort flag.  The CTA then winds down
+// in order: the producer waits (bounded) for every TMA load it issued to land,
+// the MMA thread for every MMA it issued to complete, and only then -- past a
+// CTA barrier, and only if nothing aborted -- is the accumulator read out; the
+// TMEM is freed last.  Bit 0 of debug_flags withholds the first k-block's
+// loads so that the MMA thread's wait runs out (a test of this path).
 #pragma once
 
 #include "device_utils.cuh"
@@ -42,6 +52,7 @@ struct DtProjCfg {
     static constexpr uint32_t kTileW = kBN * kBK * 2;        // 32 KB
     static constexpr uint32_t kStage = 2 * kTileA + kTileW;  // 64 KB
     static constexpr uint32_t kOffBar = kStages * kStage;    // barriers after the tiles
+    // full[2], empty[2], acc_full (40 bytes), the TMEM slot, the abort flag
     static constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;  // + room to align to 1 KB
     static constexpr int kThreads = 192;
     static constexpr uint32_t kTmemCols = 256;
@@ -137,15 +148,35 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int c0,
+                                             int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(src)), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+// Barrier over the `count` threads of the epilogue warps only (id 1).
+__device__ __forceinline__ void epilogue_sync(int count) {
+    asm volatile("bar.sync 1, %0;" ::"r"(count) : "memory");
+}
+
 // ------------------------------------------------------------------- kernel
 // Grid: x = token tiles of 128, y = channel tiles of 256.  delta is written
-// only inside [ntok, d_inner]; TMA fills out-of-range operand rows and K
-// columns with zeros, so ragged edges need no special case in the MMAs.
+// only inside [ntok, d_inner] (the TMA stores clip the tile); TMA fills
+// out-of-range operand rows and K columns with zeros, so ragged edges need no
+// special case in the MMAs.
 __global__ void __launch_bounds__(DtProjCfg::kThreads, 1)
     s6_dt_proj_kernel(const __grid_constant__ CUtensorMap map_hi,
                       const __grid_constant__ CUtensorMap map_lo,
-                      const __grid_constant__ CUtensorMap map_w, __nv_bfloat16 *__restrict__ delta,
-                      int ntok, int d_inner, int dt_rank, int two_planes, uint64_t limit) {
+                      const __grid_constant__ CUtensorMap map_w,
+                      const __grid_constant__ CUtensorMap map_out, int dt_rank, int two_planes,
+                      uint64_t limit, uint32_t debug_flags) {
     using C = DtProjCfg;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -154,10 +185,15 @@ __global__ void __launch_bounds__(DtProjCfg::kThreads, 1)
     uint64_t *empty = full + C::kStages;
     uint64_t *acc_full = empty + C::kStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.x * C::kBM, n0 = blockIdx.y * C::kBN;
     const int kblocks = (dt_rank + C::kBK - 1) / C::kBK;
+    auto fail = [&]() {
+        if (!*abort_flag) record_status(nullptr, kStTimeout);
+        *abort_flag = 1;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -165,10 +201,12 @@ __global__ void __launch_bounds__(DtProjCfg::kThreads, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
+        *abort_flag = 0;
         fence_mbarrier_init();
         prefetch_tensormap(&map_hi);
         prefetch_tensormap(&map_lo);
         prefetch_tensormap(&map_w);
+        prefetch_tensormap(&map_out);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -182,27 +220,36 @@ __global__ void __launch_bounds__(DtProjCfg::kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             const uint32_t bytes = (two_planes ? 2u : 1u) * C::kTileA + C::kTileW;
+            int last_kb[C::kStages];  // the last k-block whose loads each stage was armed for
+            for (int s = 0; s < C::kStages; ++s) last_kb[s] = -1;
             for (int kb = 0; kb < kblocks; ++kb) {
                 const int s = kb % C::kStages;
                 if (kb >= C::kStages &&
-                    !mbar_wait_bounded(&empty[s], ((kb / C::kStages) & 1) ^ 1, limit)) {
-                    atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+                    !mbar_wait_or_abort(&empty[s], ((kb / C::kStages) & 1) ^ 1, limit, abort_flag)) {
+                    fail();
                     break;
                 }
+                if ((debug_flags & 1u) && kb == 0) continue;  // test hook: withhold k-block 0
                 uint8_t *st = smem + s * C::kStage;
                 mbar_arrive_expect_tx(&full[s], bytes);
                 tma_load_2d(st, &map_hi, kb * C::kBK, m0, &full[s]);
                 if (two_planes) tma_load_2d(st + C::kTileA, &map_lo, kb * C::kBK, m0, &full[s]);
                 tma_load_2d(st + 2 * C::kTileA, &map_w, kb * C::kBK, n0, &full[s]);
+                last_kb[s] = kb;
             }
+            // No load may still be landing in the ring when the CTA moves on.
+            for (int s = 0; s < C::kStages; ++s)
+                if (last_kb[s] >= 0 &&
+                    !mbar_wait_bounded(&full[s], (last_kb[s] / C::kStages) & 1, limit))
+                    fail();
         }
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
             for (int kb = 0; kb < kblocks; ++kb) {
                 const int s = kb % C::kStages;
-                if (!mbar_wait_bounded(&full[s], (kb / C::kStages) & 1, limit)) {
-                    atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+                if (!mbar_wait_or_abort(&full[s], (kb / C::kStages) & 1, limit, abort_flag)) {
+                    fail();
                     break;
                 }
                 tc_fence_after();
@@ -221,39 +268,49 @@ __global__ void __launch_bounds__(DtProjCfg::kThreads, 1)
             }
             tc_commit(acc_full);  // every MMA issued above has completed
             // Do not leave (and let the accumulator be freed) while MMAs run.
-            if (!mbar_wait_bounded(acc_full, 0, limit))
-                atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+            if (!mbar_wait_bounded(acc_full, 0, limit)) fail();
         }
         __syncwarp();
-    } else {
+    }
+    // Every load has landed and every MMA has completed (or the CTA aborted).
+    tc_fence_before();
+    __syncthreads();
+    if (warp >= 2) {
         // Epilogue: warp w may read TMEM lanes 32*(w%4) .. 32*(w%4)+31.
         const int q = warp & 3;
-        const int m = m0 + q * 32 + lane;
-        const bool ok = mbar_wait_bounded(acc_full, 0, limit);
+        const int r = q * 32 + lane;  // this thread's token row of the tile
+        const bool ok = !*abort_flag && mbar_wait_bounded(acc_full, 0, limit);
         tc_fence_after();
-        if (!ok) {
-            if (lane == 0) atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
-        } else {
-            __nv_bfloat16 *row = delta + (size_t)(m < ntok ? m : 0) * (size_t)d_inner;
+        if (ok) {
+            // The bf16 tile as 4 slabs of [128 rows][64 columns] (16 KB each)
+            // in ring stage 0: 16-byte chunk j of row r at r * 128 + ((j ^ (r
+            // % 8)) * 16), the TMA 128-byte swizzle.
+            const uint32_t stage = smem_u32(smem);
 #pragma unroll 1
             for (int c = 0; c < C::kBN; c += 32) {
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
-                if (m < ntok) {
+                const uint32_t slab = stage + (uint32_t)(c / 64) * (C::kBM * 128u) + r * 128u;
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const int n = n0 + c + 8 * g;
-                        if (n < d_inner) {
-                            uint4 o;
-                            o.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
-                            o.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
-                            o.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
-                            o.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
-                            *reinterpret_cast<uint4 *>(row + n) = o;
-                        }
-                    }
+                for (int g = 0; g < 4; ++g) {
+                    const uint32_t j = (uint32_t)((c % 64) / 8 + g);
+                    uint4 o;
+                    o.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
+                    o.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
+                    o.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
+                    o.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
+                    st_shared_v4(slab + ((j ^ (uint32_t)(r & 7)) * 16u), o);
                 }
             }
+            fence_proxy_async_smem();  // the staged tile, before the TMA engine reads it
+        }
+        epilogue_sync(128);
+        if (ok && warp == 2 && lane == 0) {
+#pragma unroll
+            for (int s = 0; s < C::kBN / 64; ++s)
+                tma_store_2d(&map_out, smem + s * (C::kBM * 128), n0 + 64 * s, m0);
+            bulk_commit();
+            bulk_wait<0>();  // the stores are done before the CTA (and its smem) goes
         }
     }
     tc_fence_before();

@@ -29,9 +29,15 @@
 //
 // Roles (192 threads): warp 0 (one lane) TMA loads, warp 1 TMEM allocation and
 // (one lane) the MMAs, warps 2-5 the TMEM read-out and the owners' epilogue.
-// Every mbarrier wait is bounded (a wait that runs out records
-// JAMBA_SSM_ERR_TIMEOUT); every thread reaches both cluster barriers on every
-// path.
+// Every mbarrier wait is bounded; a wait that runs out records
+// JAMBA_SSM_ERR_TIMEOUT and sets the CTA's abort flag.  Before cluster barrier
+// 1 the producer waits (bounded) for every load it issued to land and the MMA
+// thread for every MMA to complete, so the ring holds no copy in flight when it
+// becomes the receive buffer.  An aborted CTA sends no partials, every CTA
+// tells every other CTA of the cluster whether it aborted (before barrier 2),
+// and owners write no output row when any CTA of their cluster aborted.  Every
+// thread reaches both cluster barriers on every path.  Bit 0 of debug_flags
+// withholds each CTA's first k-block (a test of the timeout path).
 #pragma once
 
 #include "s6_dt_proj.cuh"  // tcgen05 / TMA 2-D helpers and umma_desc_sw128
@@ -51,6 +57,9 @@ struct XProjCfg {
     static constexpr uint32_t kTileW2 = 2 * kN * kBK * 2;    //  4 KB: W_x rows 256..287
     static constexpr uint32_t kStage = kTileA + kTileW1 + kTileW2;  // 52 KB, 1 KB multiple
     static constexpr uint32_t kOffBar = kStages * kStage;
+    // full[4], empty[4], acc_full (72 bytes), the TMEM slot (4), the CTA's abort
+    // flag (at +80) and the cluster's abort flags (8 words at +96)
+    static constexpr uint32_t kOffAbort = kOffBar + 80, kOffAbortAll = kOffBar + 96;
     static constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;
     // receive buffer (reuses the ring): [KS][128 / KS rows][kRowWords] fp32;
     // 288 columns padded to 292 words so that a warp's 16-byte stores to 8
@@ -75,6 +84,7 @@ struct XProjArgs {
     float eps;
     int ntok, d_inner, ks;
     uint64_t limit;
+    uint32_t debug_flags;  // bit 0: withhold each CTA's first k-block (tests the timeout path)
 };
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -91,6 +101,9 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
     return r;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
     asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
@@ -118,6 +131,8 @@ __global__ void __launch_bounds__(XProjCfg::kThreads, 1)
     uint64_t *empty = full + C::kStages;
     uint64_t *acc_full = empty + C::kStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffAbort);
+    volatile int *abort_all = reinterpret_cast<volatile int *>(smem + C::kOffAbortAll);
     float *recv = reinterpret_cast<float *>(smem);  // valid after cluster barrier 1
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -129,6 +144,10 @@ __global__ void __launch_bounds__(XProjCfg::kThreads, 1)
     const int kb0 = min(kb_total, static_cast<int>(rank) * per);
     const int kb1 = min(kb_total, kb0 + per);
     const int nkb = kb1 - kb0;
+    auto fail = [&]() {
+        if (!*abort_flag) record_status(nullptr, kStTimeout);
+        *abort_flag = 1;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -136,6 +155,7 @@ __global__ void __launch_bounds__(XProjCfg::kThreads, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
+        *abort_flag = 0;
         fence_mbarrier_init();
         prefetch_tensormap(&map_u);
         prefetch_tensormap(&map_w1);
@@ -152,28 +172,39 @@ __global__ void __launch_bounds__(XProjCfg::kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
+            int last_i[C::kStages];  // the last k-block whose loads each stage was armed for
+            for (int s = 0; s < C::kStages; ++s) last_i[s] = -1;
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % C::kStages;
                 if (i >= C::kStages &&
-                    !mbar_wait_bounded(&empty[s], ((i / C::kStages) & 1) ^ 1, args.limit)) {
-                    atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+                    !mbar_wait_or_abort(&empty[s], ((i / C::kStages) & 1) ^ 1, args.limit,
+                                        abort_flag)) {
+                    fail();
                     break;
                 }
+                if ((args.debug_flags & 1u) && i == 0) continue;  // test hook: withhold k-block 0
                 uint8_t *st = smem + s * C::kStage;
                 const int k = (kb0 + i) * C::kBK;
                 mbar_arrive_expect_tx(&full[s], C::kStage);
                 tma_load_2d(st, &map_u, k, m0, &full[s]);
                 tma_load_2d(st + C::kTileA, &map_w1, k, 0, &full[s]);
                 tma_load_2d(st + C::kTileA + C::kTileW1, &map_w2, k, C::kR, &full[s]);
+                last_i[s] = i;
             }
+            // The ring becomes the receive buffer after barrier 1: no load may
+            // still be landing in it.
+            for (int s = 0; s < C::kStages; ++s)
+                if (last_i[s] >= 0 &&
+                    !mbar_wait_bounded(&full[s], (last_i[s] / C::kStages) & 1, args.limit))
+                    fail();
         }
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % C::kStages;
-                if (!mbar_wait_bounded(&full[s], (i / C::kStages) & 1, args.limit)) {
-                    atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+                if (!mbar_wait_or_abort(&full[s], (i / C::kStages) & 1, args.limit, abort_flag)) {
+                    fail();
                     break;
                 }
                 tc_fence_after();
@@ -192,22 +223,32 @@ __global__ void __launch_bounds__(XProjCfg::kThreads, 1)
                 tc_commit(&empty[s]);
             }
             tc_commit(acc_full);
-            if (!mbar_wait_bounded(acc_full, 0, args.limit))
-                atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+            if (!mbar_wait_bounded(acc_full, 0, args.limit)) fail();
         }
         __syncwarp();
     } else {
-        if (!mbar_wait_bounded(acc_full, 0, args.limit) && lane == 0)
-            atomicCAS(&g_status_word, 0, 5 /* JAMBA_SSM_ERR_TIMEOUT */);
+        if (!mbar_wait_bounded(acc_full, 0, args.limit)) fail();
         tc_fence_after();
     }
 
-    // Barrier 1: every CTA of the cluster has finished its MMAs, so every ring
-    // may now be overwritten by partial sums.
+    // Barrier 1: every CTA of the cluster has finished its MMAs and its loads,
+    // so every ring may now be overwritten by partial sums.
+    tc_fence_before();
     if (ks > 1) cluster_sync_all(); else __syncthreads();
+    tc_fence_after();
 
     const int rows_per_owner = C::kBM / ks;
-    if (warp >= 2) {
+    const bool aborted = *abort_flag != 0;
+    if (threadIdx.x == 0) {  // tell every CTA of the cluster (self included)
+        if (ks > 1) {
+            const uint32_t slot = smem_u32(const_cast<int *>(abort_all)) + 4u * rank;
+            for (int r = 0; r < ks; ++r)
+                st_cluster_u32(map_to_rank(slot, static_cast<uint32_t>(r)), aborted ? 1u : 0u);
+        } else {
+            abort_all[0] = aborted ? 1 : 0;
+        }
+    }
+    if (warp >= 2 && !aborted) {
         // Each thread sends its token row's 288 partial sums to the row's owner.
         const int q = warp & 3;
         const int row = q * 32 + lane;
@@ -230,10 +271,12 @@ __global__ void __launch_bounds__(XProjCfg::kThreads, 1)
         }
     }
     tc_fence_before();
-    // Barrier 2: every partial has landed in its owner's buffer.
+    // Barrier 2: every partial (and every CTA's abort flag) has landed.
     if (ks > 1) cluster_sync_all(); else __syncthreads();
+    bool cluster_aborted = false;
+    for (int r = 0; r < ks; ++r) cluster_aborted |= abort_all[r] != 0;
 
-    if (warp >= 2) {
+    if (warp >= 2 && !cluster_aborted) {
         // Owner epilogue: warp w takes rows (w - 2), (w - 2) + 4, ... of this
         // CTA's share; lane j holds columns j + 32 k (k = 0..7: dt_low; k = 8:
         // B for j < 16, C for j >= 16).
