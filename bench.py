@@ -39,9 +39,13 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-MUFU_OPS_PER_CLK_PER_SM = 16   # exp2 / rcp throughput per SM per clock (sm_100)
+# exp2 / rcp throughput per SM per clock on sm_100: the unit count of the
+# special-function pipe, confirmed by the ex2 microbenchmark
+# tests/c/mufu_rate.cu (profiles/mufu_peak.md)
+MUFU_OPS_PER_CLK_PER_SM = 16
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_SM_MHZ = 1965.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 # ----------------------------------------------------------------- helpers
@@ -52,6 +56,15 @@ def peaks():
         return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", FALLBACK_SM_MHZ)), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, FALLBACK_SM_MHZ, "fallback"
+
+
+def bf16_peak():
+    """Dense bf16 tensor-core peak (TFLOP/s) for a kernel timed alone (burst)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def kernel_source_hash(unit: str = "jamba_ssm.cu"):
@@ -107,6 +120,45 @@ def exp_ops(tokens, d_inner, d_state):
     """Transcendental ops the method needs per (token, channel): d_state exps
     for Abar, exp + log for softplus, exp + reciprocal for the gate."""
     return tokens * d_inner * (d_state + 4)
+
+
+def x_proj_work(ntok, d_inner, dt_rank, d_state):
+    """FLOPs and minimum bytes of [dt_low | B | C] = W_x u: u and W_x read once,
+    dt_low written as two bf16 planes, B and C in bf16."""
+    rows = dt_rank + 2 * d_state
+    flops = 2 * ntok * d_inner * rows
+    nbytes = 2 * (ntok * d_inner + rows * d_inner + 2 * ntok * dt_rank + 2 * ntok * d_state)
+    return flops, nbytes
+
+
+def dt_proj_work(ntok, d_inner, dt_rank):
+    """FLOPs of Delta_raw = dt_low W_dt^T (the method's, counting dt_low once)
+    and minimum bytes: the two dt_low planes and W_dt read, Delta_raw written."""
+    flops = 2 * ntok * d_inner * dt_rank
+    nbytes = 2 * (2 * ntok * dt_rank + d_inner * dt_rank + ntok * d_inner)
+    return flops, nbytes
+
+
+def time_launches(fn, reps, stream, dev, flush=None, warmup=1):
+    """Mean device time (s) of `fn` over `reps` launches, each bracketed by
+    CUDA events on `stream`, after `warmup` untimed launches; `flush` (if
+    given) runs before every launch, outside the events."""
+    for _ in range(warmup):
+        if flush:
+            flush()
+        fn()
+    torch.cuda.synchronize(dev)
+    tot = 0.0
+    for _ in range(reps):
+        if flush:
+            flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        tot += a.elapsed_time(b) / 1e3
+    return tot / reps
 
 
 class ClockSampler:
@@ -183,6 +235,111 @@ def replica_seq_offset(rank, batch):
     """First sequence index of this rank's replica: rank r scans sequences
     r*batch .. r*batch+batch-1 of the workload's seeded stream."""
     return rank * batch
+
+
+# ------------------------------------------------------------- the other configs
+def per_workload(args, dev, stream, flush_l2, sms, world):
+    """The other BASELINE configurations, each timed on its own with CUDA
+    events (the max over ranks) against its own bound, plus the two projection
+    kernels that feed the scan: {name: {kernel_us, tokens_per_s, roofline}}."""
+    import selective_state_space_26_b200 as jssm
+    from selective_state_space_26_b200 import synth
+
+    hbm_gbs, sm_mhz, peak_kind = peaks()
+    mufu_peak = sms * MUFU_OPS_PER_CLK_PER_SM * sm_mhz * 1e6
+    res = {}
+    names, times, meta = [], [], []
+
+    # prefill configs: 256K tokens in one sequence, and 16 sequences of 16K
+    for wname in ("s6_prefill_bf16_b1_l262144_d8192_n16", "s6_prefill_bf16_b16_l16384_d8192_n16"):
+        w = synth.WORKLOADS[wname]
+        inp = synth.workload_inputs(w, device=dev, seq_offset=replica_seq_offset(args.rank, w.batch))
+        out = torch.empty_like(inp.x)
+        hf = torch.empty(w.batch, w.d_inner, w.d_state, dtype=torch.float32, device=dev)
+
+        def scan():
+            jssm.jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, D=inp.D,
+                                delta_bias=inp.delta_bias, out=out, h_final=hf)
+        t = time_launches(scan, args.pw_reps, stream, dev, flush=flush_l2)
+        names.append(wname)
+        times.append(t)
+        meta.append((w, "scan"))
+        del inp, out, hf
+        torch.cuda.empty_cache()
+
+    # decode: 256 requests, 128 sequential single-token updates of the cache
+    w = synth.WORKLOADS["s6_decode_bf16_b256_d8192_n16_x128"]
+    A = synth.make_A(w.d_inner, w.d_state).to(dev)
+    Dv = torch.ones(w.d_inner, device=dev)
+    bias = synth.dt_bias_for(w.d_inner, w.seed).to(dev)
+    st = synth.decode_state(w.batch, w.d_inner, w.d_state, w.seed + 1000 * args.rank, device=dev)
+    steps = [synth.decode_step(w.batch, w.d_inner, w.d_state, k, w.seed, w.dtype, dev)
+             for k in range(w.seqlen)]
+    dec_out = torch.empty(w.batch, w.d_inner, dtype=w.dtype, device=dev)
+
+    def decode_all():  # every pass continues the cache from the previous one
+        for s in steps:
+            jssm.jamba_ssm_state_update(st, s.x, s.delta, s.z, s.B, s.C, A, D=Dv,
+                                        delta_bias=bias, out=dec_out)
+    names.append(w.name)
+    times.append(time_launches(decode_all, args.pw_reps, stream, dev, flush=flush_l2))
+    meta.append((w, "decode"))
+    del steps, st
+
+    # the projections that feed the scan, at the headline's 4096 tokens
+    ntok, d_inner, R, N = 4096, 8192, 256, 16
+    xp = synth.x_proj_inputs(ntok, d_inner, R, N, seed=5, device=dev)
+    dp = synth.dt_proj_inputs(ntok, d_inner, R, seed=5, device=dev)
+    dl = torch.empty(ntok, d_inner, dtype=torch.bfloat16, device=dev)
+    t_x = time_launches(lambda: jssm.jamba_ssm_x_proj(xp.u, xp.W_x, w_dt=xp.w_dt, w_B=xp.w_B,
+                                                      w_C=xp.w_C),
+                        max(args.pw_reps, 10), stream, dev, flush=flush_l2)
+    t_d = time_launches(lambda: jssm.jamba_ssm_dt_proj(dp.hi, dp.W_dt, dt_low_lo=dp.lo, out=dl),
+                        max(args.pw_reps, 10), stream, dev, flush=flush_l2)
+    names += ["x_proj_bf16_t4096_d8192_r256_n16", "dt_proj_bf16_t4096_d8192_r256"]
+    times += [t_x, t_d]
+    meta += [(None, "x_proj"), (None, "dt_proj")]
+
+    times = max_over_ranks(times, world, dev)
+    tc_peak, tc_kind = bf16_peak()
+    for name, t, (w, kind) in zip(names, times, meta):
+        if kind == "scan":
+            ops = exp_ops(w.batch * w.seqlen, w.d_inner, w.d_state)
+            nbytes = prefill_bytes(w.batch, w.seqlen, w.d_inner, w.d_state, 2)
+            res[name] = {
+                "kernel_us": t * 1e6, "tokens_per_s": w.batch * w.seqlen * world / t,
+                "roofline": {"bound": "alu", "achieved": ops / t / 1e12,
+                             "peak": mufu_peak / 1e12, "unit": "Top/s (exp-class, MUFU)",
+                             "frac": ops / t / mufu_peak,
+                             "hbm_gbs": nbytes / t / 1e9, "hbm_frac": nbytes / t / 1e9 / hbm_gbs},
+                "timing": f"{args.pw_reps} launches after 1 warm-up, L2 flushed before each"}
+        elif kind == "decode":
+            nbytes = decode_bytes(w.batch, w.d_inner, w.d_state, 2)
+            per = t / w.seqlen
+            res[name] = {
+                "kernel_us": per * 1e6, "tokens_per_s": w.batch * world / per,
+                "roofline": {"bound": "hbm", "achieved": nbytes / per / 1e9, "peak": hbm_gbs,
+                             "unit": "GB/s", "frac": nbytes / per / 1e9 / hbm_gbs},
+                "timing": f"mean over {w.seqlen} back-to-back updates of one pass, "
+                          f"{args.pw_reps} passes, L2 flushed before each pass"}
+        else:
+            flops, nbytes = (x_proj_work(ntok, d_inner, R, N) if kind == "x_proj"
+                             else dt_proj_work(ntok, d_inner, R))
+            t_tc = flops / (tc_peak * 1e12)
+            t_mem = nbytes / (hbm_gbs * 1e9)
+            bound = "tensor" if t_tc >= t_mem else "hbm"
+            res[name] = {
+                "kernel_us": t * 1e6, "tokens_per_s": ntok * world / t,
+                "roofline": {"bound": bound,
+                             "achieved": flops / t / 1e12 if bound == "tensor" else nbytes / t / 1e9,
+                             "peak": tc_peak if bound == "tensor" else hbm_gbs,
+                             "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
+                             "frac": max(t_tc, t_mem) / t, "flops": flops, "bytes": nbytes,
+                             "tflops": flops / t / 1e12, "hbm_gbs": nbytes / t / 1e9},
+                "timing": f"{max(args.pw_reps, 10)} launches after 1 warm-up, L2 flushed before each"}
+    res["_peaks"] = {"hbm_gbs": hbm_gbs, "hbm_kind": peak_kind, "bf16_tflops": tc_peak,
+                     "bf16_kind": tc_kind, "mufu_top_s": mufu_peak / 1e12}
+    return res
 
 
 # ------------------------------------------------------------- our arm
@@ -397,6 +554,12 @@ def run_ours(args, rank, world, local_rank):
                 "peak_basis": f"{peak_kind} copy bandwidth",
                 "algorithmic_bytes_per_launch": dom_bytes, "launch_us": dom_launch_s * 1e6}
 
+    pw = None
+    if not args.no_per_workload:
+        with ClockSampler(props, period=0.01) as clk_pw:
+            pw = per_workload(args, dev, stream, flush_l2, sms, world)
+        pw["_clocks"] = clk_pw.summary()
+
     line = {
         "metric": "selective-scan tokens/s & HBM GB/s (fraction of roofline) at d_inner=8192, N=16",
         "value": job_tokens_per_s(tokens, world, ms_per_step / 1e3),
@@ -419,6 +582,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
+        "per_workload": pw,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp if w.kind == "prefill" else None,
@@ -541,11 +705,16 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling)")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the other configurations and the projection kernels")
+    ap.add_argument("--pw-reps", type=int, default=3,
+                    help="timed launches of each other configuration")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    args.rank = rank
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         if rank == 0:

@@ -247,6 +247,73 @@ typedef struct jamba_ssm_state_update_params {
 
 jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, void *stream);
 
+/*
+ * Backward pass of jamba_ssm_scan (training): the gradients of a loss L with
+ * respect to every input of the scan, given dout = dL/dout and, optionally,
+ * dL/dh_final.  The chain rule through the recurrence of "Mamba 레이어" in
+ * reverse time, with g = dL/dh_t:  g += dy C_t (dy = dout silu(z)); then per
+ * state dC_t += dy h_t, dB_t += g Delta x, dDelta += g h_{t-1} Abar A + g B x,
+ * dx += g Delta B, dA += g h_{t-1} Abar Delta, g <- Abar g; dz and dD from the
+ * gate and the skip; ddelta = dDelta * d softplus(v)/dv; dh0 = the final g.
+ *
+ * Sizes: as jamba_ssm_scan (batched layout only; no cu_seqlens or state
+ * slots), with d_state in {8, 16} for bf16 I/O and {4, 8, 16} for f32 I/O.
+ * Pointers (device; the forward's inputs as given to jamba_ssm_scan):
+ *   x, delta, z, B, C, A, D, delta_bias, h0, delta_softplus: as the forward.
+ *   dout       [batch, seqlen, d_inner] io_dtype, 16-byte aligned, required.
+ *   dh_final   [batch, d_inner, d_state] fp32 or NULL (zero).
+ *   dx, ddelta, dz  [batch, seqlen, d_inner] io_dtype, 16-byte aligned,
+ *              written (ddelta is the gradient of the raw step input delta).
+ *   dB, dC     [batch, seqlen, d_state] io_dtype, 16-byte aligned, written.
+ *   dA         [d_inner, d_state] fp32 (summed over the batch), or NULL.
+ *   dD, ddelta_bias [d_inner] fp32 (summed over the batch), or NULL.
+ *   dh0        [batch, d_inner, d_state] fp32, or NULL.
+ *   Outputs must not overlap one another or an input.
+ *   workspace  REQUIRED: device buffer of at least
+ *              jamba_ssm_scan_bwd_workspace_size() bytes, 16-byte aligned, its
+ *              first JAMBA_SSM_STATUS_BYTES zero-filled before first use (the
+ *              status word, read with jamba_ssm_get_status(workspace, ...)).
+ *              The rest is scratch: the states every 16 steps (recomputed from
+ *              the inputs), per-CTA partial sums of dB and dC, and per-sequence
+ *              partials of dA, dD, ddelta_bias.
+ * The result does not depend on the launch shape or on timing: every sum is
+ * taken in a fixed order (no atomics).  Calls sharing one workspace must not
+ * overlap on the GPU.
+ * debug_flags / timeout_cycles: as jamba_ssm_scan (bit 0 withholds each
+ * CTA's first tile of the backward kernel).
+ */
+typedef struct jamba_ssm_scan_bwd_params {
+    size_t struct_size;          /* = sizeof(jamba_ssm_scan_bwd_params)       */
+    int64_t batch, seqlen, d_inner, d_state;
+    int32_t io_dtype;
+    int32_t delta_softplus;
+    const void *x, *delta, *z;
+    const void *B, *C;
+    const float *A;
+    const float *D;
+    const float *delta_bias;
+    const float *h0;
+    const void *dout;
+    const float *dh_final;
+    void *dx, *ddelta, *dz;
+    void *dB, *dC;
+    float *dA;
+    float *dD;
+    float *ddelta_bias;
+    float *dh0;
+    void *workspace;
+    size_t workspace_bytes;
+    uint32_t debug_flags;
+    uint64_t timeout_cycles;
+} jamba_ssm_scan_bwd_params;
+
+/* Bytes of workspace jamba_ssm_scan_bwd needs for these sizes (0 for an
+ * unsupported d_state). */
+size_t jamba_ssm_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner,
+                                         int64_t d_state);
+
+jamba_ssm_status jamba_ssm_scan_bwd(const jamba_ssm_scan_bwd_params *p, void *stream);
+
 /* Launch shape the scan would use for these parameters (no launch).  Any of
  * the out pointers may be NULL.  variant: the built variant chosen (0 for the
  * one-thread-per-channel kernel of the small state sizes);

@@ -5,6 +5,8 @@ The calls, with the names of the C entry points:
 * ``jamba_ssm_scan``          -- prefill scan over whole sequences, returning the
   gated output and (for the decode cache) the final state;
 * ``jamba_ssm_state_update``  -- one-token decode step, state updated in place;
+* ``jamba_ssm_scan_bwd``      -- the scan's backward pass (gradients of every
+  input, for training);
 * ``jamba_ssm_x_proj``        -- the projection of the scan's input to dt_low, B
   and C with their RMSNorms (libjamba_ssm_proj.so);
 * ``jamba_ssm_dt_proj``       -- the low-rank product that produces the scan's
@@ -24,7 +26,8 @@ from . import _lib
 from ._lib import JambaSSMError
 
 __all__ = ["jamba_ssm_scan", "jamba_ssm_state_update", "jamba_ssm_get_status", "scan_plan",
-           "jamba_ssm_scan_workspace_size",
+           "jamba_ssm_scan_workspace_size", "jamba_ssm_scan_bwd",
+           "jamba_ssm_scan_bwd_workspace_size",
            "jamba_ssm_x_proj", "jamba_ssm_dt_proj", "jamba_ssm_proj_get_status",
            "JambaSSMError"]
 
@@ -141,6 +144,64 @@ def jamba_ssm_scan(x, delta, z, B, C, A, D=None, delta_bias=None, delta_softplus
     if st != _lib.OK:
         raise JambaSSMError(st, "jamba_ssm_scan")
     return out, h_final
+
+
+def jamba_ssm_scan_bwd_workspace_size(batch: int, seqlen: int, d_inner: int,
+                                      d_state: int) -> int:
+    """Bytes of the workspace the backward pass needs (0: d_state unsupported)."""
+    return _lib.scan_bwd_workspace_size(int(batch), int(seqlen), int(d_inner), int(d_state))
+
+
+def jamba_ssm_scan_bwd(x, delta, z, B, C, A, dout, D=None, delta_bias=None,
+                       delta_softplus=True, h0=None, dh_final=None, workspace=None,
+                       stream=None, debug_flags: int = 0, timeout_cycles: int = 0):
+    """Backward pass of jamba_ssm_scan: the gradients of a loss with respect to
+    every input, given dout = dL/dout [batch, seqlen, d_inner] (the dtype of x)
+    and optionally dh_final = dL/dh_final [batch, d_inner, d_state] fp32.
+
+    Returns a dict: dx, ddelta, dz [batch, seqlen, d_inner] and dB, dC [batch,
+    seqlen, d_state] in x's dtype; dA [d_inner, d_state], dD, ddelta_bias
+    [d_inner] fp32 (summed over the batch); dh0 [batch, d_inner, d_state] fp32.
+    ``workspace``: a device tensor of at least
+    ``jamba_ssm_scan_bwd_workspace_size(...)`` bytes whose first 16 bytes are
+    zero (allocated here when None; its status word is read with
+    ``jamba_ssm_get_status(workspace=...)``)."""
+    if x.dtype not in _IO:
+        raise TypeError(f"x must be bfloat16 or float32, got {x.dtype}")
+    batch, seqlen, d_inner = x.shape
+    d_state = A.shape[-1]
+    dev, io = x.device, x.dtype
+    act, bc = (batch, seqlen, d_inner), (batch, seqlen, d_state)
+    for t, n, s in ((x, "x", act), (delta, "delta", act), (z, "z", act), (B, "B", bc),
+                    (C, "C", bc), (dout, "dout", act)):
+        _check(t, n, s, io, dev)
+    _check(A, "A", (d_inner, d_state), torch.float32, dev)
+    _check(D, "D", (d_inner,), torch.float32, dev)
+    _check(delta_bias, "delta_bias", (d_inner,), torch.float32, dev)
+    _check(h0, "h0", (batch, d_inner, d_state), torch.float32, dev)
+    _check(dh_final, "dh_final", (batch, d_inner, d_state), torch.float32, dev)
+    if workspace is None:
+        need = jamba_ssm_scan_bwd_workspace_size(batch, seqlen, d_inner, d_state)
+        workspace = torch.zeros(max(need, _lib.STATUS_BYTES), dtype=torch.uint8, device=dev)
+    ws, ws_bytes = _workspace(workspace, dev)
+    g = dict(dx=torch.empty_like(x), ddelta=torch.empty_like(x), dz=torch.empty_like(x),
+             dB=torch.empty_like(B), dC=torch.empty_like(C),
+             dA=torch.empty(d_inner, d_state, dtype=torch.float32, device=dev),
+             dD=torch.empty(d_inner, dtype=torch.float32, device=dev),
+             ddelta_bias=torch.empty(d_inner, dtype=torch.float32, device=dev),
+             dh0=torch.empty(batch, d_inner, d_state, dtype=torch.float32, device=dev))
+    p = _lib.new_scan_bwd_params(
+        batch=batch, seqlen=seqlen, d_inner=d_inner, d_state=d_state, io_dtype=_IO[io],
+        delta_softplus=int(bool(delta_softplus)), x=_ptr(x), delta=_ptr(delta), z=_ptr(z),
+        B=_ptr(B), C=_ptr(C), A=_ptr(A), D=_ptr(D), delta_bias=_ptr(delta_bias), h0=_ptr(h0),
+        dout=_ptr(dout), dh_final=_ptr(dh_final),
+        **{k: _ptr(v) for k, v in g.items()},
+        workspace=ws, workspace_bytes=ws_bytes, debug_flags=int(debug_flags),
+        timeout_cycles=int(timeout_cycles))
+    st = _lib.call_scan_bwd(p, _stream(stream, dev))
+    if st != _lib.OK:
+        raise JambaSSMError(st, "jamba_ssm_scan_bwd")
+    return g
 
 
 def scan_plan(x, A, B=None, variant: int = 0):

@@ -23,6 +23,8 @@ BF16, F32 = 0, 1
 EXPORTS = (
     "jamba_ssm_scan",
     "jamba_ssm_scan_workspace_size",
+    "jamba_ssm_scan_bwd",
+    "jamba_ssm_scan_bwd_workspace_size",
     "jamba_ssm_state_update",
     "jamba_ssm_scan_plan",
     "jamba_ssm_scan_variant_info",
@@ -79,6 +81,24 @@ class StateUpdateParams(ctypes.Structure):
         ("debug_flags", ctypes.c_uint32), ("timeout_cycles", ctypes.c_uint64),
         # ABI version 3
         ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class ScanBwdParams(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t),
+        ("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+        ("d_inner", ctypes.c_int64), ("d_state", ctypes.c_int64),
+        ("io_dtype", ctypes.c_int32), ("delta_softplus", ctypes.c_int32),
+        ("x", _vp), ("delta", _vp), ("z", _vp),
+        ("B", _vp), ("C", _vp),
+        ("A", _fp), ("D", _fp), ("delta_bias", _fp), ("h0", _fp),
+        ("dout", _vp), ("dh_final", _fp),
+        ("dx", _vp), ("ddelta", _vp), ("dz", _vp),
+        ("dB", _vp), ("dC", _vp),
+        ("dA", _fp), ("dD", _fp), ("ddelta_bias", _fp), ("dh0", _fp),
+        ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+        ("debug_flags", ctypes.c_uint32), ("timeout_cycles", ctypes.c_uint64),
     ]
 
 
@@ -145,6 +165,10 @@ def lib():
                 L.jamba_ssm_get_status.argtypes = [_vp, _vp]
                 L.jamba_ssm_scan_workspace_size.restype = ctypes.c_size_t
                 L.jamba_ssm_scan_workspace_size.argtypes = [ctypes.c_int64] * 4
+                L.jamba_ssm_scan_bwd.restype = ctypes.c_int
+                L.jamba_ssm_scan_bwd.argtypes = [ctypes.POINTER(ScanBwdParams), _vp]
+                L.jamba_ssm_scan_bwd_workspace_size.restype = ctypes.c_size_t
+                L.jamba_ssm_scan_bwd_workspace_size.argtypes = [ctypes.c_int64] * 4
                 L.jamba_ssm_last_cuda_error.restype = ctypes.c_int
                 L.jamba_ssm_last_cuda_error.argtypes = []
                 L.jamba_ssm_status_string.restype = ctypes.c_char_p
@@ -242,6 +266,22 @@ def get_status(stream: int, workspace: int = 0) -> int:
 
 def scan_workspace_size(batch: int, seqlen: int, d_inner: int, d_state: int) -> int:
     return lib().jamba_ssm_scan_workspace_size(batch, seqlen, d_inner, d_state)
+
+
+def scan_bwd_workspace_size(batch: int, seqlen: int, d_inner: int, d_state: int) -> int:
+    return lib().jamba_ssm_scan_bwd_workspace_size(batch, seqlen, d_inner, d_state)
+
+
+def new_scan_bwd_params(**kw) -> ScanBwdParams:
+    p = ScanBwdParams()
+    p.struct_size = ctypes.sizeof(ScanBwdParams)
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def call_scan_bwd(p: ScanBwdParams, stream: int) -> int:
+    return lib().jamba_ssm_scan_bwd(ctypes.byref(p), _vp(stream or None))
 
 
 def new_dt_proj_params(**kw) -> DtProjParams:

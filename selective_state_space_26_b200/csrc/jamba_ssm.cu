@@ -11,6 +11,7 @@
 
 #include "jamba_ssm.h"
 #include "s6_scan.cuh"
+#include "s6_scan_bwd.cuh"
 #include "s6_scan_fused.cuh"
 #include "s6_scan_serving.cuh"
 #include "s6_scan_small.cuh"
@@ -312,6 +313,66 @@ jamba_ssm_status plan_scan(const jamba_ssm_scan_params *p, const DeviceInfo *dev
     plan->grid = static_cast<int>(g < 1 ? 1 : g);
     return JAMBA_SSM_OK;
 }
+
+// ------------------------------------------------------------ backward pass
+// Launch shape of the backward per (io dtype, d_state): G lanes per channel,
+// NW compute warps, TT-step tiles (fp32 tiles are half as long so that the
+// stage ring, the output tiles and the dB / dC partials fit in shared memory).
+struct BwdShape {
+    int g, nw, tt, cc;
+};
+bool bwd_shape(int io_dtype, int64_t n, BwdShape *s) {
+    const bool bf = io_dtype == JAMBA_SSM_BF16;
+    if (n == 16 || n == 8) *s = {4, 7, bf ? 64 : 32, 7 * 8};
+    else if (n == 4 && !bf) *s = {2, 4, 32, 4 * 16};
+    else return false;
+    return true;
+}
+constexpr int kCkChannels = 32;  // channels per block of the checkpoint pass
+
+// Workspace of the backward: the status block, then the checkpoints, the
+// per-CTA dB | dC partials and the per-sequence parameter partials.
+struct BwdLayout {
+    int64_t nck, ngroups;
+    size_t off_ckpt, off_bc, off_par, total;
+};
+size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
+BwdLayout bwd_layout(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state, int cc) {
+    BwdLayout l;
+    l.nck = (seqlen + jssm::kCk - 1) / jssm::kCk;
+    l.ngroups = (d_inner + cc - 1) / cc;
+    l.off_ckpt = 256;
+    l.off_bc = l.off_ckpt + round256(size_t(batch) * l.nck * d_inner * d_state * 4);
+    l.off_par = l.off_bc + round256(size_t(batch) * l.ngroups * seqlen * 2 * d_state * 4);
+    l.total = l.off_par + round256(size_t(batch) * d_inner * (d_state + 2) * 4);
+    return l;
+}
+
+struct BwdKernels {
+    const void *ckpt, *bwd, *reduce;
+    int smem;
+    bool attr[kMaxDevices];
+};
+
+template <typename IoT, int N, int G, int NW, int TT, bool SP>
+BwdKernels make_bwd() {
+    BwdKernels k{};
+    k.ckpt = reinterpret_cast<const void *>(&jssm::s6_bwd_ckpt_kernel<IoT, N, G, kCkChannels>);
+    k.bwd = reinterpret_cast<const void *>(&jssm::s6_bwd_kernel<IoT, N, G, NW, TT, SP>);
+    k.reduce = reinterpret_cast<const void *>(&jssm::s6_bwd_reduce_kernel<IoT, N>);
+    k.smem = jssm::BwdCfg<IoT, N, G, NW, TT>::kSmemBytes;
+    return k;
+}
+
+// [dtype][d_state 16, 8, 4][softplus off, on]
+BwdKernels g_bwd[2][3][2] = {
+    {{make_bwd<__nv_bfloat16, 16, 4, 7, 64, false>(), make_bwd<__nv_bfloat16, 16, 4, 7, 64, true>()},
+     {make_bwd<__nv_bfloat16, 8, 4, 7, 64, false>(), make_bwd<__nv_bfloat16, 8, 4, 7, 64, true>()},
+     {BwdKernels{}, BwdKernels{}}},
+    {{make_bwd<float, 16, 4, 7, 32, false>(), make_bwd<float, 16, 4, 7, 32, true>()},
+     {make_bwd<float, 8, 4, 7, 32, false>(), make_bwd<float, 8, 4, 7, 32, true>()},
+     {make_bwd<float, 4, 2, 4, 32, false>(), make_bwd<float, 4, 2, 4, 32, true>()}},
+};
 
 }  // namespace
 
@@ -648,6 +709,161 @@ jamba_ssm_status jamba_ssm_get_status(void *workspace, void *stream) {
         if (e != cudaSuccess) return cuda_fail(e);
     }
     return static_cast<jamba_ssm_status>(word);
+}
+
+size_t jamba_ssm_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner,
+                                         int64_t d_state) {
+    BwdShape sh;
+    if (batch < 0 || seqlen < 0 || d_inner < 1 || !bwd_shape(JAMBA_SSM_F32, d_state, &sh))
+        return 0;
+    // the layout depends on the channel-group width, which is the same for
+    // both dtypes at a given d_state
+    return bwd_layout(batch, seqlen, d_inner, d_state, sh.cc).total;
+}
+
+jamba_ssm_status jamba_ssm_scan_bwd(const jamba_ssm_scan_bwd_params *p, void *stream) {
+    if (!p || p->struct_size < sizeof(jamba_ssm_scan_bwd_params)) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->batch < 0 || p->seqlen < 0 || p->d_inner < 1 || p->d_state < 1)
+        return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->io_dtype != JAMBA_SSM_BF16 && p->io_dtype != JAMBA_SSM_F32) return JAMBA_SSM_ERR_INVALID_ARG;
+    BwdShape sh;
+    const int es = p->io_dtype == JAMBA_SSM_BF16 ? 2 : 4;
+    if (!bwd_shape(p->io_dtype, p->d_state, &sh) || (p->d_inner * es) % 16 != 0)
+        return JAMBA_SSM_ERR_UNSUPPORTED;
+    const int64_t kMaxRows = kMaxI32 - 256;
+    if (p->batch > 65535 || p->seqlen > kMaxRows || p->d_inner > (int64_t(1) << 30) ||
+        (p->batch && p->seqlen && p->batch > kMaxElems / p->seqlen) ||
+        p->batch * p->seqlen > kMaxElems / p->d_inner)
+        return JAMBA_SSM_ERR_UNSUPPORTED;
+    if (!p->workspace) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (!aligned(p->workspace, 16)) return JAMBA_SSM_ERR_MISALIGNED;
+    const BwdLayout lay = bwd_layout(p->batch, p->seqlen, p->d_inner, p->d_state, sh.cc);
+    if (p->workspace_bytes < lay.total) return JAMBA_SSM_ERR_WORKSPACE;
+    const int64_t tok = p->batch * p->seqlen;
+    const size_t act = size_t(tok) * p->d_inner * es, bc = size_t(tok) * p->d_state * es;
+    const size_t st = size_t(p->batch) * p->d_inner * p->d_state * 4;
+    const size_t pn = size_t(p->d_inner) * 4, an = size_t(p->d_inner) * p->d_state * 4;
+    if (tok > 0) {
+        if (!p->x || !p->delta || !p->z || !p->B || !p->C || !p->A || !p->dout || !p->dx ||
+            !p->ddelta || !p->dz || !p->dB || !p->dC)
+            return JAMBA_SSM_ERR_INVALID_ARG;
+        const void *a16[] = {p->x, p->delta, p->z, p->B, p->C, p->A, p->dout, p->dx, p->ddelta,
+                             p->dz, p->dB, p->dC, p->h0, p->dh_final, p->dh0};
+        for (const void *q : a16)
+            if (!aligned(q, 16)) return JAMBA_SSM_ERR_MISALIGNED;
+    }
+    if (!aligned(p->D, 4) || !aligned(p->delta_bias, 4) || !aligned(p->dA, 4) ||
+        !aligned(p->dD, 4) || !aligned(p->ddelta_bias, 4) || !aligned(p->h0, 4) ||
+        !aligned(p->dh_final, 4) || !aligned(p->dh0, 4))
+        return JAMBA_SSM_ERR_MISALIGNED;
+    // no output may overlap an input, another output or the workspace
+    const void *outs[] = {p->dx, p->ddelta, p->dz, p->dB, p->dC, p->dA, p->dD, p->ddelta_bias,
+                          p->dh0};
+    const size_t outsz[] = {act, act, act, bc, bc, an, pn, pn, st};
+    const void *ins[] = {p->x, p->delta, p->z, p->B, p->C, p->A, p->D, p->delta_bias, p->h0,
+                         p->dout, p->dh_final, p->workspace};
+    const size_t insz[] = {act, act, act, bc, bc, an, pn, pn, st, act, st, lay.total};
+    for (int i = 0; i < 9; ++i) {
+        for (int j = 0; j < 12; ++j)
+            if (overlaps(outs[i], outsz[i], ins[j], insz[j])) return JAMBA_SSM_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 9; ++j)
+            if (overlaps(outs[i], outsz[i], outs[j], outsz[j])) return JAMBA_SSM_ERR_INVALID_ARG;
+    }
+    jamba_ssm_status stt;
+    const DeviceInfo *dev = current_device(&stt);
+    if (!dev) return stt;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int *status = static_cast<int *>(p->workspace);
+    uint8_t *ws = static_cast<uint8_t *>(p->workspace);
+    cudaError_t e;
+    if (tok == 0) {  // no steps: the parameter gradients are zero and dh0 = dh_final
+        if (p->dA && (e = cudaMemsetAsync(p->dA, 0, an, s)) != cudaSuccess) return cuda_fail(e);
+        if (p->dD && (e = cudaMemsetAsync(p->dD, 0, pn, s)) != cudaSuccess) return cuda_fail(e);
+        if (p->ddelta_bias && (e = cudaMemsetAsync(p->ddelta_bias, 0, pn, s)) != cudaSuccess)
+            return cuda_fail(e);
+        if (p->dh0 && st) {
+            e = p->dh_final ? cudaMemcpyAsync(p->dh0, p->dh_final, st, cudaMemcpyDeviceToDevice, s)
+                            : cudaMemsetAsync(p->dh0, 0, st, s);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        return finish_launch(s, p->workspace);
+    }
+    const int di = p->io_dtype == JAMBA_SSM_BF16 ? 0 : 1;
+    const int ni = p->d_state == 16 ? 0 : (p->d_state == 8 ? 1 : 2);
+    BwdKernels &K = g_bwd[di][ni][p->delta_softplus ? 1 : 0];
+    EncodeTiledFn fn = encode_fn(&stt);
+    if (!fn) return stt;
+    int devid = 0;
+    cudaGetDevice(&devid);
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!K.attr[devid]) {
+            e = cudaFuncSetAttribute(K.bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, K.smem);
+            if (e != cudaSuccess) return cuda_fail(e);
+            K.attr[devid] = true;
+        }
+    }
+    jssm::BwdArgs a{};
+    a.batch = p->batch;
+    a.seqlen = p->seqlen;
+    a.d_inner = p->d_inner;
+    a.A = p->A;
+    a.D = p->D;
+    a.delta_bias = p->delta_bias;
+    a.h0 = p->h0;
+    a.dh_final = p->dh_final;
+    a.delta_softplus = p->delta_softplus != 0;
+    a.x = p->x;
+    a.delta = p->delta;
+    a.B = p->B;
+    a.ckpt = reinterpret_cast<float *>(ws + lay.off_ckpt);
+    a.part_bc = reinterpret_cast<float *>(ws + lay.off_bc);
+    a.part_par = reinterpret_cast<float *>(ws + lay.off_par);
+    a.dh0 = p->dh0;
+    a.status = status;
+    a.debug_flags = p->debug_flags;
+    a.timeout_cycles = p->timeout_cycles ? p->timeout_cycles : (uint64_t(1) << 31);
+
+    // 1. checkpoints
+    {
+        const dim3 grid(static_cast<unsigned>((p->d_inner + kCkChannels - 1) / kCkChannels),
+                        static_cast<unsigned>(p->batch));
+        void *kargs[] = {&a};
+        e = cudaLaunchKernel(K.ckpt, grid, dim3(kCkChannels * sh.g), kargs, 0, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    // 2. the reverse walk
+    {
+        const CUtensorMapDataType dt = p->io_dtype == JAMBA_SSM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+        jssm::BwdMaps m;
+        CUtensorMap *acts[] = {&m.x, &m.dt, &m.z, &m.dout, &m.dx, &m.ddt, &m.dz};
+        const void *aptr[] = {p->x, p->delta, p->z, p->dout, p->dx, p->ddelta, p->dz};
+        for (int i = 0; i < 7; ++i)
+            if (!encode_3d(fn, acts[i], aptr[i], dt, es, p->d_inner, p->seqlen, p->batch, sh.cc, sh.tt))
+                return JAMBA_SSM_ERR_UNSUPPORTED;
+        if (!encode_3d(fn, &m.B, p->B, dt, es, p->d_state, p->seqlen, p->batch, (int)p->d_state, sh.tt) ||
+            !encode_3d(fn, &m.C, p->C, dt, es, p->d_state, p->seqlen, p->batch, (int)p->d_state, sh.tt))
+            return JAMBA_SSM_ERR_UNSUPPORTED;
+        const dim3 grid(static_cast<unsigned>(lay.ngroups), static_cast<unsigned>(p->batch));
+        void *kargs[] = {&m, &a};
+        e = cudaLaunchKernel(K.bwd, grid, dim3((sh.nw + 1) * 32), kargs, static_cast<size_t>(K.smem), s);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    // 3. sums over CTAs and sequences
+    {
+        const int64_t total = tok * 2 * p->d_state + p->d_inner * (p->d_state + 2);
+        int64_t blocks = (total + 255) / 256;
+        if (blocks > int64_t(dev->sms) * 16) blocks = int64_t(dev->sms) * 16;
+        const float *pbc = a.part_bc, *ppar = a.part_par;
+        int64_t batch = p->batch, seqlen = p->seqlen, d_inner = p->d_inner, ng = lay.ngroups;
+        void *dB = p->dB, *dC = p->dC;
+        float *dA = p->dA, *dD = p->dD, *db = p->ddelta_bias;
+        void *kargs[] = {&pbc, &ppar, &batch, &seqlen, &d_inner, &ng, &dB, &dC, &dA, &dD, &db};
+        e = cudaLaunchKernel(K.reduce, dim3(static_cast<unsigned>(blocks)), dim3(256), kargs, 0, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return finish_launch(s, p->workspace);
 }
 
 size_t jamba_ssm_scan_workspace_size(int64_t batch, int64_t seqlen, int64_t d_inner,

@@ -1,0 +1,589 @@
+// s6_scan_bwd.cuh -- backward pass (reverse-mode gradient) of the S6 prefill
+// scan on sm_100a, for training.
+//
+// The forward recurrence is the one of the "Mamba 레이어" section of the
+// Jamba notes, read as h_t = exp(Delta_t A) h_{t-1} + Delta_t B_t x_t,
+// y_t = C_t . h_t + D x_t, out_t = y_t silu(z_t), Delta = softplus(delta +
+// bias).  Given dout = dL/dout (and dL/dh_final), the chain rule in reverse
+// time with the carry g = dL/dh_t gives, per channel d and step t (g first
+// takes the readout's share, g += dy C_t, with dy = dout silu(z)):
+//   dz       = dout y sigma(z) (1 + z (1 - sigma(z)))
+//   dC_t[n] += dy h_t[n]               dB_t[n] += g_n Delta x      (summed over d)
+//   dDelta   = sum_n g_n h_{t-1}[n] Abar_n A_n + x sum_n g_n B_n
+//   dx       = dy D + Delta sum_n g_n B_n
+//   dA[n]   += g_n h_{t-1}[n] Abar_n Delta,  dD += dy x,  ddelta = dDelta sigma(v)
+//   g_n     <- Abar_n g_n                  (and dh0 = g after step 0)
+// where sigma(v) = d softplus / dv for v = delta + bias.  (This is the
+// derivative the fp64 oracle's scan_bwd takes, step for step.)
+//
+// Three kernels, all deterministic (no atomics, fixed summation orders):
+//  1. s6_bwd_ckpt_kernel: the forward recurrence once more, storing the state
+//     before every kCk-th step (the checkpoints) in the workspace.
+//  2. s6_bwd_kernel: per (sequence, channel group), 64-step tiles from the last
+//     to the first, fed by TMA (x, delta, z, dout, B, C) like the forward.  In
+//     each tile, segments of kCk steps from the last to the first: the lanes
+//     recompute the segment's states from its checkpoint into registers, then
+//     walk it backwards with g in registers.  The lane layout is the forward's:
+//     G lanes per channel, NS = N / G states per lane, lane `sub` owning the
+//     per-(t, d) scalars of steps sub, sub + G, ...; sums over a channel's
+//     states go through the transposing butterfly.  dB and dC, sums over
+//     channels, are reduced over a warp's channels with a transposing
+//     butterfly on the lane bits that select the channel, then over the CTA's
+//     warps in shared memory, and written as one partial per CTA.  dx, ddelta
+//     and dz leave through shared memory and TMA stores.
+//  3. s6_bwd_reduce_kernel: dB and dC = the sum of the CTA partials, and dA,
+//     dD, dbias = the sum over sequences, in a fixed order in fp64.
+// Every mbarrier wait is bounded; a wait that runs out records
+// JAMBA_SSM_ERR_TIMEOUT, sets the CTA's abort flag, and every warp winds down
+// after the producer has waited (bounded) for the copies it issued.
+#pragma once
+
+#include "device_utils.cuh"
+#include "s6_math.cuh"
+#include "s6_scan.cuh"
+
+namespace jssm {
+
+constexpr int kCk = 16;  // steps between checkpoints (= the backward's segment)
+
+struct BwdArgs {
+    int64_t batch, seqlen, d_inner;
+    const float *A, *D, *delta_bias, *h0, *dh_final;
+    int delta_softplus;
+    const void *x, *delta, *B;  // for the checkpoint pass (plain loads of B)
+    float *ckpt;                // [batch, nck, d_inner, N] fp32
+    float *part_bc;             // [batch, ngroups, seqlen, 2N] fp32: CTA partials of dB | dC
+    float *part_par;            // [batch, d_inner, N + 2] fp32: dA[N], dD, dbias per sequence
+    float *dh0;                 // [batch, d_inner, N] or null
+    int *status;
+    uint32_t debug_flags;
+    uint64_t timeout_cycles;
+};
+
+template <typename IoT, int N, int G, int NW, int TT>
+struct BwdCfg {
+    static constexpr int NS = N / G, CW = 32 / G, CC = NW * CW;
+    static_assert(NS == 2 || NS == 4, "two or four states per lane");
+    static_assert(TT % kCk == 0 && kCk % G == 0, "segments of whole step groups");
+    static constexpr int kAct = TT * CC * (int)sizeof(IoT);   // one [TT x CC] tile
+    static constexpr int kBC = TT * N * (int)sizeof(IoT);     // one [TT x N] tile
+    static constexpr int kStage = 4 * kAct + 2 * kBC;         // x, delta, z, dout, B, C
+    static constexpr int STAGES = 2;
+    static constexpr int NOUT = 2;                            // output tile sets in flight
+    static constexpr int kOffOut = STAGES * kStage;           // dx, ddelta, dz per set
+    static constexpr int kOffPart = kOffOut + NOUT * 3 * kAct;  // [NW][TT][2N] fp32
+    static constexpr int kPart = NW * TT * 2 * N * 4;
+    static constexpr int kOffBar = kOffPart + kPart;
+    static constexpr int kNumBars = 2 * STAGES + 2 * NOUT;    // full, empty, out_full, out_free
+    static constexpr int kOffFlag = kOffBar + kNumBars * 8;
+    static constexpr int kSmemBytes = kOffFlag + 16;
+    static_assert(kAct % 128 == 0 && kBC % 128 == 0, "TMA boxes 128-byte aligned");
+};
+
+// Sum over the CW channels of a warp: each lane holds V = 2 NS partial sums
+// (its states' dB then dC) of one step; after log2(CW) rounds over the lane
+// bits that select the channel, lane (c, sub) holds the sum over the warp's
+// channels of value index `bc_index<...>(lane)` of its sub's V values (while
+// there are values to split, each round keeps the half its bit selects and
+// trades the other; once one value is left the rounds just add).
+template <int V, int G>
+__device__ __forceinline__ float reduce_channels(float (&v)[V], int lane) {
+    constexpr int CW = 32 / G;
+    float w[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) w[i] = v[i];
+    int n = V;
+#pragma unroll
+    for (int m = G; m < 32; m <<= 1) {
+        const bool upper = (lane & m) != 0;
+        if (n > 1) {
+            const int h = n / 2;
+#pragma unroll
+            for (int i = 0; i < V / 2; ++i) {
+                if (i < h) {
+                    const float keep = upper ? w[i + h] : w[i];
+                    const float send = upper ? w[i] : w[i + h];
+                    w[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
+            }
+            n = h;
+        } else {
+            w[0] += __shfl_xor_sync(0xffffffffu, w[0], m);
+        }
+    }
+    static_assert(CW >= 1, "");
+    return w[0];
+}
+// Which of the V values lane `lane` holds after reduce_channels.
+template <int V, int G>
+__device__ __forceinline__ int bc_index(int lane) {
+    int idx = 0, n = V;
+#pragma unroll
+    for (int m = G; m < 32 && n > 1; m <<= 1) {
+        n /= 2;
+        if (lane & m) idx += n;
+    }
+    return idx;
+}
+
+// ------------------------------------------------------------ checkpoints
+// grid (ceil(d_inner / CC), batch), threads CC * G: thread (d, sub) carries
+// NS states of channel d through the whole sequence and stores them before
+// every kCk-th step.  Plain loads: x, delta of the owned step per lane (the
+// G lanes of a channel own consecutive steps), B slices broadcast over the
+// warp; each segment's loads are issued before its arithmetic.
+template <typename IoT, int N, int G, int CC>
+__global__ void __launch_bounds__(CC *G) s6_bwd_ckpt_kernel(const BwdArgs a) {
+    constexpr int NS = N / G;
+    const int lane = threadIdx.x & 31, sub = lane % G;
+    const int gbase = lane & ~(G - 1);
+    const int64_t b = blockIdx.y;
+    const int64_t d = static_cast<int64_t>(blockIdx.x) * CC + threadIdx.x / G;
+    const bool dvalid = d < a.d_inner;
+    const int64_t dc = dvalid ? d : a.d_inner - 1;  // invalid lanes still join the shuffles
+    const int64_t D = a.d_inner, L = a.seqlen;
+    const int64_t nck = (L + kCk - 1) / kCk;
+    float h[NS], a2[NS];
+#pragma unroll
+    for (int i = 0; i < NS; ++i) {
+        a2[i] = __ldg(a.A + dc * N + sub * NS + i) * kLog2e;
+        h[i] = a.h0 ? __ldg(a.h0 + (b * D + dc) * N + sub * NS + i) : 0.0f;
+    }
+    const float bias = a.delta_bias ? __ldg(a.delta_bias + dc) : 0.0f;
+    const bool sp = a.delta_softplus != 0;
+    const IoT *x = static_cast<const IoT *>(a.x) + b * L * D;
+    const IoT *dt = static_cast<const IoT *>(a.delta) + b * L * D;
+    const IoT *Bm = static_cast<const IoT *>(a.B) + b * L * N;
+    for (int64_t k = 0; k < nck; ++k) {
+        if (dvalid) {
+            float *o = a.ckpt + ((b * nck + k) * D + d) * N + sub * NS;
+#pragma unroll
+            for (int i = 0; i < NS; ++i) o[i] = h[i];
+        }
+        const int64_t t0 = k * kCk;
+        const int nst = static_cast<int>(L - t0 < kCk ? L - t0 : kCk);
+        float xo[kCk / G], vo[kCk / G], bv[kCk][NS];
+#pragma unroll
+        for (int q = 0; q < kCk / G; ++q) {
+            const int j = q * G + sub;
+            const bool ok = j < nst;
+            xo[q] = ok ? to_f32(x[(t0 + j) * D + dc]) : 0.0f;
+            vo[q] = ok ? to_f32(dt[(t0 + j) * D + dc]) : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < kCk; ++j)
+#pragma unroll
+            for (int i = 0; i < NS; ++i)
+                bv[j][i] = j < nst ? to_f32(Bm[(t0 + j) * N + sub * NS + i]) : 0.0f;
+#pragma unroll
+        for (int q = 0; q < kCk / G; ++q) {
+            const float dl_o = delta_f32(vo[q], bias, sp);
+            const float dx_o = dl_o * xo[q];
+#pragma unroll
+            for (int jj = 0; jj < G; ++jj) {
+                const int j = q * G + jj;
+                const float dl = __shfl_sync(0xffffffffu, dl_o, gbase | jj);
+                const float dx = __shfl_sync(0xffffffffu, dx_o, gbase | jj);
+                if (j < nst) {
+#pragma unroll
+                    for (int i = 0; i < NS; ++i) h[i] = fmaf(ex2_mufu(dl * a2[i]), h[i], dx * bv[j][i]);
+                }
+            }
+        }
+    }
+}
+
+// --------------------------------------------------------------- backward
+// Lanes that write the channel-reduced dB / dC values: after log2(V) splitting
+// rounds every further round only adds, so the lanes that differ in those
+// later bits hold the same sums and only the first of them writes.
+template <int V, int G>
+__device__ __forceinline__ bool bc_writer(int lane) {
+    constexpr int kSplit = (V >= 8 ? 3 : (V >= 4 ? 2 : (V >= 2 ? 1 : 0)));
+    return (G << kSplit) >= 32 || lane < (G << kSplit);
+}
+
+// One segment of kCk steps (starting at tile step s0, `nst` of them valid),
+// recomputed from h_in and walked backwards.  Owner scalars come from the
+// stage's x / delta / z / dout tiles; B / C from the stage's [TT][N] tiles.
+// `part` is the warp's [TT][2N] slab of the CTA's dB | dC partial sums.
+template <bool FULL, bool SP, typename IoT, int N, int G, int CC>
+__device__ __forceinline__ void bwd_segment(
+    const float (&h_in)[N / G], float (&g)[N / G], float (&dA)[N / G], float &dD_acc,
+    float &dbias_acc, const float (&a2)[N / G], const float (&Araw)[N / G], float bias, float dskip,
+    const IoT *xs, const IoT *dts, const IoT *zs, const IoT *dos, const IoT *Bs, const IoT *Cs,
+    IoT *dxs, IoT *dds, IoT *dzs, float *part, int s0, int nst, int c_local, int sub, int gbase,
+    int lane) {
+    constexpr int NS = N / G, NQ = kCk / G, V = 2 * NS;
+    // ---- recompute: the state after every step of the segment, and the
+    // steps' Delta and Delta x on every lane of the channel
+    float hs[kCk][NS];
+    float dl[kCk], dxv[kCk];
+    float dl_own[NQ], w_own[NQ], v_own[NQ];  // owned steps: Delta, e^{-|v|}, v
+    float h[NS];
+#pragma unroll
+    for (int i = 0; i < NS; ++i) h[i] = h_in[i];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+        const int idx = (s0 + q * G + sub) * CC + c_local;
+        const float xo = to_f32(xs[idx]);
+        const float v = to_f32(dts[idx]) + bias;
+        const float dlo = SP ? softplus_f32(v) : v;
+        dl_own[q] = dlo;
+        v_own[q] = v;
+        w_own[q] = SP ? ex2_mufu(-fabsf(v) * kLog2e) : 0.0f;
+        const float dxo = dlo * xo;
+#pragma unroll
+        for (int jj = 0; jj < G; ++jj) {
+            const int j = q * G + jj;
+            dl[j] = G == 1 ? dlo : __shfl_sync(0xffffffffu, dlo, gbase | jj);
+            dxv[j] = G == 1 ? dxo : __shfl_sync(0xffffffffu, dxo, gbase | jj);
+            if (FULL || j < nst) {
+                const IoT *bj = Bs + (s0 + j) * N + sub * NS;
+#pragma unroll
+                for (int i = 0; i < NS; ++i)
+                    h[i] = fmaf(ex2_mufu(dl[j] * a2[i]), h[i], dxv[j] * to_f32(bj[i]));
+            }
+#pragma unroll
+            for (int i = 0; i < NS; ++i) hs[j][i] = h[i];
+        }
+    }
+    // ---- backward walk, groups of G steps from the last
+#pragma unroll
+    for (int q = NQ - 1; q >= 0; --q) {
+        const int jo = q * G + sub;
+        const int idx = (s0 + jo) * CC + c_local;
+        const bool own_ok = FULL || jo < nst;
+        const float zo = to_f32(zs[idx]);
+        const float doo = own_ok ? to_f32(dos[idx]) : 0.0f;
+        const float xo = to_f32(xs[idx]);
+        const float sz = rcp_mufu(1.0f + ex2_mufu(-zo * kLog2e));  // sigma(z)
+        const float dy_o = doo * zo * sz;
+        float yp[G], pa[G], gb[G];
+#pragma unroll
+        for (int jj = G - 1; jj >= 0; --jj) {
+            const int j = q * G + jj;
+            const float dy = G == 1 ? dy_o : __shfl_sync(0xffffffffu, dy_o, gbase | jj);
+            float bcv[V];
+            yp[jj] = 0.0f;
+            pa[jj] = 0.0f;
+            gb[jj] = 0.0f;
+#pragma unroll
+            for (int i = 0; i < V; ++i) bcv[i] = 0.0f;
+            if (FULL || j < nst) {
+                const IoT *bj = Bs + (s0 + j) * N + sub * NS;
+                const IoT *cj = Cs + (s0 + j) * N + sub * NS;
+#pragma unroll
+                for (int i = 0; i < NS; ++i) {
+                    const float cv = to_f32(cj[i]), bv = to_f32(bj[i]);
+                    const float hprev = j > 0 ? hs[j - 1][i] : h_in[i];
+                    yp[jj] = fmaf(cv, hs[j][i], yp[jj]);
+                    g[i] = fmaf(dy, cv, g[i]);           // dL/dh_t: the readout's share
+                    bcv[NS + i] = dy * hs[j][i];         // dC_t[n], this channel
+                    const float abar = ex2_mufu(dl[j] * a2[i]);
+                    const float P = g[i] * hprev * abar;  // dL/dAbar * Abar
+                    pa[jj] = fmaf(P, Araw[i], pa[jj]);
+                    dA[i] = fmaf(P, dl[j], dA[i]);
+                    gb[jj] = fmaf(g[i], bv, gb[jj]);
+                    bcv[i] = g[i] * dxv[j];              // dB_t[n], this channel
+                    g[i] *= abar;                        // dL/dh_{t-1}
+                }
+            }
+            // dB / dC of this step summed over the warp's channels
+            const float s = reduce_channels<V, G>(bcv, lane);
+            if ((FULL || j < nst) && bc_writer<V, G>(lane)) {
+                const int vi = bc_index<V, G>(lane);
+                const int slot = (vi < NS ? 0 : N) + sub * NS + (vi % NS);
+                part[(s0 + j) * 2 * N + slot] = s;
+            }
+        }
+        // the owner's totals for its step: y (pre-gate), sum P A, sum g B
+        const float ys = reduce_transpose<G>(yp, sub);
+        const float pas = reduce_transpose<G>(pa, sub);
+        const float gbs = reduce_transpose<G>(gb, sub);
+        if (own_ok) {
+            const float y = fmaf(dskip, xo, ys);
+            const float dz = doo * y * sz * (1.0f + zo * (1.0f - sz));
+            const float dDelta = fmaf(xo, gbs, pas);
+            float ddr = dDelta;
+            if (SP) {  // d softplus / dv = sigma(v), from w = e^{-|v|}
+                const float r = rcp_mufu(1.0f + w_own[q]);
+                ddr = dDelta * (v_own[q] >= 0.0f ? r : w_own[q] * r);
+            }
+            dbias_acc += ddr;
+            dD_acc = fmaf(dy_o, xo, dD_acc);
+            dxs[idx] = from_f32<IoT>(fmaf(dy_o, dskip, dl_own[q] * gbs));
+            dds[idx] = from_f32<IoT>(ddr);
+            dzs[idx] = from_f32<IoT>(dz);
+        }
+    }
+}
+
+struct BwdMaps {
+    CUtensorMap x, dt, z, dout, B, C, dx, ddt, dz;
+};
+
+// grid (ceil(d_inner / CC), batch); NW compute warps + 1 producer warp.  SP:
+// Delta = softplus(delta + bias) (else delta + bias).
+template <typename IoT, int N, int G, int NW, int TT, bool SP>
+__global__ void __launch_bounds__((NW + 1) * 32, 1)
+    s6_bwd_kernel(const __grid_constant__ BwdMaps maps, const BwdArgs a) {
+    using Cfg = BwdCfg<IoT, N, G, NW, TT>;
+    constexpr int NS = Cfg::NS, CW = Cfg::CW, CC = Cfg::CC, STAGES = Cfg::STAGES,
+                  NOUT = Cfg::NOUT;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
+    uint64_t *empty = full + STAGES;
+    uint64_t *out_full = empty + STAGES;
+    uint64_t *out_free = out_full + NOUT;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffFlag);
+    float *part_all = reinterpret_cast<float *>(smem + Cfg::kOffPart);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t b = blockIdx.y;
+    const int c0 = blockIdx.x * CC;
+    const int64_t D = a.d_inner, L = a.seqlen;
+    const int ntiles = static_cast<int>((L + TT - 1) / TT);
+    const int64_t nck = (L + kCk - 1) / kCk;
+    const uint64_t limit = a.timeout_cycles;
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NW * 32);
+        }
+        for (int o = 0; o < NOUT; ++o) {
+            mbar_init(&out_full[o], NW * 32);
+            mbar_init(&out_free[o], 1);
+        }
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    auto fail = [&]() {
+        if (!*abort_flag) record_status(a.status, kStTimeout);
+        *abort_flag = 1;
+    };
+
+    if (warp == NW) {
+        // ===================== producer: TMA loads and stores =====================
+        if (lane == 0) {
+            prefetch_tensormap(&maps.x);
+            prefetch_tensormap(&maps.dt);
+            prefetch_tensormap(&maps.z);
+            prefetch_tensormap(&maps.dout);
+            prefetch_tensormap(&maps.B);
+            prefetch_tensormap(&maps.C);
+            prefetch_tensormap(&maps.dx);
+            prefetch_tensormap(&maps.ddt);
+            prefetch_tensormap(&maps.dz);
+            const int bb = static_cast<int>(b);
+            int last_i[STAGES];
+            for (int s = 0; s < STAGES; ++s) last_i[s] = -1;
+            bool ok = true;
+            // the i-th tile walked is tile ntiles - 1 - i
+            auto issue = [&](int i) -> bool {
+                const int s = i % STAGES;
+                if (i >= STAGES &&
+                    !mbar_wait_or_abort(&empty[s], ((i / STAGES) & 1) ^ 1, limit, abort_flag))
+                    return false;
+                if ((a.debug_flags & 1u) && i == 0) return true;  // test hook: withhold tile 0
+                uint8_t *st = smem + s * Cfg::kStage;
+                const int t0 = (ntiles - 1 - i) * TT;
+                mbar_arrive_expect_tx(&full[s], Cfg::kStage);
+                tma_load_3d(st, &maps.x, c0, t0, bb, &full[s]);
+                tma_load_3d(st + Cfg::kAct, &maps.dt, c0, t0, bb, &full[s]);
+                tma_load_3d(st + 2 * Cfg::kAct, &maps.z, c0, t0, bb, &full[s]);
+                tma_load_3d(st + 3 * Cfg::kAct, &maps.dout, c0, t0, bb, &full[s]);
+                tma_load_3d(st + 4 * Cfg::kAct, &maps.B, 0, t0, bb, &full[s]);
+                tma_load_3d(st + 4 * Cfg::kAct + Cfg::kBC, &maps.C, 0, t0, bb, &full[s]);
+                last_i[s] = i;
+                return true;
+            };
+            int next = 0;
+            for (; next < STAGES && next < ntiles && ok; ++next) ok = issue(next);
+            for (int i = 0; i < ntiles && ok; ++i) {
+                // outputs of walked tile i are complete: store them, then refill
+                const int slot = i % NOUT;
+                if (!mbar_wait_or_abort(&out_full[slot], (i / NOUT) & 1, limit, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *ob = smem + Cfg::kOffOut + slot * 3 * Cfg::kAct;
+                const int t0 = (ntiles - 1 - i) * TT;
+                tma_store_3d(&maps.dx, ob, c0, t0, bb);
+                tma_store_3d(&maps.ddt, ob + Cfg::kAct, c0, t0, bb);
+                tma_store_3d(&maps.dz, ob + 2 * Cfg::kAct, c0, t0, bb);
+                bulk_commit();
+                if (next < ntiles) ok = issue(next++);
+                if (i > 0) {
+                    bulk_wait_read<1>();  // the stores of tile i-1 have read their buffers
+                    mbar_arrive(&out_free[(i - 1) % NOUT]);
+                }
+            }
+            if (!ok) fail();
+            // nothing in flight may outlive the CTA
+            for (int s = 0; s < STAGES; ++s)
+                if (last_i[s] >= 0 && !mbar_wait_bounded(&full[s], (last_i[s] / STAGES) & 1, limit))
+                    fail();
+            bulk_wait<0>();
+        }
+        __syncwarp();
+        return;
+    }
+
+    // ============================ compute warps ============================
+    const int c_local = warp * CW + lane / G;
+    const int sub = lane % G;
+    const int gbase = lane & ~(G - 1);
+    const int64_t d = c0 + c_local;
+    const bool dvalid = d < D;
+    const int64_t dc = dvalid ? d : D - 1;
+    float a2[NS], Araw[NS], g[NS], dA[NS];
+#pragma unroll
+    for (int i = 0; i < NS; ++i) {
+        Araw[i] = __ldg(a.A + dc * N + sub * NS + i);
+        a2[i] = Araw[i] * kLog2e;
+        g[i] = a.dh_final ? __ldg(a.dh_final + (b * D + dc) * N + sub * NS + i) : 0.0f;
+        dA[i] = 0.0f;
+    }
+    const float bias = a.delta_bias ? __ldg(a.delta_bias + dc) : 0.0f;
+    const float dskip = a.D ? __ldg(a.D + dc) : 0.0f;
+    float dD_acc = 0.0f, dbias_acc = 0.0f;
+    float *part = part_all + warp * TT * 2 * N;
+    // checkpoints are consumed from the last to the first; the next one is
+    // loaded one segment ahead
+    const float *ck = a.ckpt + (b * nck * D + dc) * N + sub * NS;  // + c * D * N
+    int64_t c_next = nck - 1;
+    float hnext[NS];
+#pragma unroll
+    for (int i = 0; i < NS; ++i) hnext[i] = ck[c_next * D * N + i];
+
+    // Every compute warp makes every iteration and reaches both named
+    // barriers of each, doing the work only while nothing has aborted.
+    bool ok = true;
+    for (int it = 0; it < ntiles; ++it) {
+        const int k = ntiles - 1 - it;
+        const int s = it % STAGES, slot = it % NOUT;
+        if (ok && (!mbar_wait_or_abort(&full[s], (it / STAGES) & 1, limit, abort_flag) ||
+                   (it >= NOUT && !mbar_wait_or_abort(&out_free[slot], ((it / NOUT) - 1) & 1,
+                                                      limit, abort_flag)))) {
+            ok = false;
+            fail();
+        }
+        const int64_t t_tile = int64_t(k) * TT;
+        const int nsteps = static_cast<int>(L - t_tile < TT ? L - t_tile : TT);
+        if (ok) {
+            const uint8_t *st = smem + s * Cfg::kStage;
+            const IoT *xs = reinterpret_cast<const IoT *>(st);
+            const IoT *dts = reinterpret_cast<const IoT *>(st + Cfg::kAct);
+            const IoT *zs = reinterpret_cast<const IoT *>(st + 2 * Cfg::kAct);
+            const IoT *dos = reinterpret_cast<const IoT *>(st + 3 * Cfg::kAct);
+            const IoT *Bs = reinterpret_cast<const IoT *>(st + 4 * Cfg::kAct);
+            const IoT *Cs = reinterpret_cast<const IoT *>(st + 4 * Cfg::kAct + Cfg::kBC);
+            uint8_t *ob = smem + Cfg::kOffOut + slot * 3 * Cfg::kAct;
+            IoT *dxs = reinterpret_cast<IoT *>(ob);
+            IoT *dds = reinterpret_cast<IoT *>(ob + Cfg::kAct);
+            IoT *dzs = reinterpret_cast<IoT *>(ob + 2 * Cfg::kAct);
+            const int nseg = (nsteps + kCk - 1) / kCk;
+#pragma unroll 1
+            for (int sg = nseg - 1; sg >= 0; --sg) {
+                float hcur[NS];
+#pragma unroll
+                for (int i = 0; i < NS; ++i) hcur[i] = hnext[i];
+                if (c_next > 0) {
+                    --c_next;
+#pragma unroll
+                    for (int i = 0; i < NS; ++i) hnext[i] = ck[c_next * D * N + i];
+                }
+                const int rem = nsteps - sg * kCk;
+                if (rem >= kCk)
+                    bwd_segment<true, SP, IoT, N, G, CC>(hcur, g, dA, dD_acc, dbias_acc, a2, Araw,
+                                                         bias, dskip, xs, dts, zs, dos, Bs, Cs, dxs,
+                                                         dds, dzs, part, sg * kCk, kCk, c_local, sub,
+                                                         gbase, lane);
+                else
+                    bwd_segment<false, SP, IoT, N, G, CC>(hcur, g, dA, dD_acc, dbias_acc, a2, Araw,
+                                                          bias, dskip, xs, dts, zs, dos, Bs, Cs,
+                                                          dxs, dds, dzs, part, sg * kCk, rem,
+                                                          c_local, sub, gbase, lane);
+            }
+            mbar_arrive(&empty[s]);    // the input stage may be refilled
+            fence_proxy_async_smem();  // output tiles, before the TMA engine reads them
+            mbar_arrive(&out_full[slot]);
+        }
+        // this tile's dB | dC partials: the sum over the CTA's warps, to global
+        asm volatile("bar.sync 1, %0;" ::"r"(NW * 32) : "memory");
+        if (ok) {
+            float *dst = a.part_bc + ((b * gridDim.x + blockIdx.x) * L + t_tile) * 2 * N;
+            for (int e = tid; e < nsteps * 2 * N; e += NW * 32) {
+                float acc = 0.0f;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) acc += part_all[w * TT * 2 * N + e];
+                dst[e] = acc;
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(NW * 32) : "memory");
+    }
+    if (!ok) return;
+    // per-sequence parameter partials, and dL/dh0
+    float dD_sum = dD_acc, db_sum = dbias_acc;
+#pragma unroll
+    for (int m = 1; m < G; m <<= 1) {
+        dD_sum += __shfl_xor_sync(0xffffffffu, dD_sum, m);
+        db_sum += __shfl_xor_sync(0xffffffffu, db_sum, m);
+    }
+    if (dvalid) {
+        float *pp = a.part_par + (b * D + d) * (N + 2);
+#pragma unroll
+        for (int i = 0; i < NS; ++i) pp[sub * NS + i] = dA[i];
+        if (sub == 0) {
+            pp[N] = dD_sum;
+            pp[N + 1] = db_sum;
+        }
+        if (a.dh0) {
+#pragma unroll
+            for (int i = 0; i < NS; ++i) a.dh0[(b * D + d) * N + sub * NS + i] = g[i];
+        }
+    }
+}
+
+// --------------------------------------------------------------- reduction
+// dB, dC [batch, seqlen, N] = the sum of the ngroups CTA partials; dA [D, N],
+// dD, dbias [D] = the sums over the batch; fp64 accumulation in a fixed order.
+// grid-stride over (batch * seqlen * 2N) + (D * (N + 2)) elements.
+template <typename IoT, int N>
+__global__ void __launch_bounds__(256)
+    s6_bwd_reduce_kernel(const float *__restrict__ part_bc, const float *__restrict__ part_par,
+                         int64_t batch, int64_t seqlen, int64_t d_inner, int64_t ngroups, IoT *dB,
+                         IoT *dC, float *dA, float *dD, float *dbias) {
+    const int64_t n_bc = batch * seqlen * 2 * N;
+    const int64_t n_par = d_inner * (N + 2);
+    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n_bc + n_par;
+         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        if (e < n_bc) {
+            const int64_t slot = e % (2 * N), bt = e / (2 * N);
+            const int64_t b = bt / seqlen, t = bt % seqlen;
+            double acc = 0.0;
+            for (int64_t gi = 0; gi < ngroups; ++gi)
+                acc += part_bc[((b * ngroups + gi) * seqlen + t) * 2 * N + slot];
+            IoT *o = slot < N ? dB : dC;
+            o[bt * N + (slot % N)] = from_f32<IoT>(static_cast<float>(acc));
+        } else {
+            const int64_t f = e - n_bc;
+            const int64_t dd = f / (N + 2), j = f % (N + 2);
+            double acc = 0.0;
+            for (int64_t b = 0; b < batch; ++b) acc += part_par[(b * d_inner + dd) * (N + 2) + j];
+            if (j < N) {
+                if (dA) dA[dd * N + j] = static_cast<float>(acc);
+            }
+            else if (j == N) {
+                if (dD) dD[dd] = static_cast<float>(acc);
+            } else if (dbias) {
+                dbias[dd] = static_cast<float>(acc);
+            }
+        }
+    }
+}
+
+}  // namespace jssm
