@@ -168,7 +168,7 @@ class ClockSampler:
              0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
              0x100: "display_clock_setting"}
 
-    def __init__(self, props, period=0.002):
+    def __init__(self, props, period=0.0002):
         self.period = period
         self.samples, self.reasons, self.ok = [], 0, False
         self._stop = threading.Event()
@@ -299,6 +299,16 @@ def per_workload(args, dev, stream, flush_l2, sms, world):
     names += ["x_proj_bf16_t4096_d8192_r256_n16", "dt_proj_bf16_t4096_d8192_r256"]
     times += [t_x, t_d]
     meta += [(None, "x_proj"), (None, "dt_proj")]
+    del xp, dp, dl
+
+    # the backward pass of the headline layer (training): all three kernels
+    wb = synth.WORKLOADS["s6_prefill_bf16_b1_l4096_d8192_n16"]
+    bw = _bwd_inputs(wb, dev, args.rank)
+    t_b = time_launches(bw["call"], args.pw_reps, stream, dev, flush=flush_l2)
+    names.append("scan_bwd_bf16_b1_l4096_d8192_n16")
+    times.append(t_b)
+    meta.append((wb, "bwd"))
+    del bw
 
     times = max_over_ranks(times, world, dev)
     tc_peak, tc_kind = bf16_peak()
@@ -313,6 +323,23 @@ def per_workload(args, dev, stream, flush_l2, sms, world):
                              "frac": ops / t / mufu_peak,
                              "hbm_gbs": nbytes / t / 1e9, "hbm_frac": nbytes / t / 1e9 / hbm_gbs},
                 "timing": f"{args.pw_reps} launches after 1 warm-up, L2 flushed before each"}
+        elif kind == "bwd":
+            tok = w.batch * w.seqlen
+            ops = tok * w.d_inner * (w.d_state + 5)
+            issued = tok * w.d_inner * (3 * w.d_state + 6)
+            res[name] = {
+                "kernel_us": t * 1e6, "tokens_per_s": tok * world / t,
+                "roofline": {"bound": "alu", "achieved": ops / t / 1e12,
+                             "peak": mufu_peak / 1e12, "unit": "Top/s (exp-class, MUFU)",
+                             "frac": ops / t / mufu_peak,
+                             "algorithmic_ops": ops, "issued_ops": issued,
+                             "issued_frac": issued / t / mufu_peak},
+                "ops_basis": "algorithmic: d_state + 5 exp-class ops per (token, channel) "
+                             "(Abar for the carry, softplus exp + log, sigma(z) exp + rcp, "
+                             "sigma(v) rcp); issued: 3 d_state + 6 (the 16-step checkpoints "
+                             "and the per-segment recompute add 2 d_state + 1)",
+                "timing": f"{args.pw_reps} calls (checkpoint, backward and reduction kernels) "
+                          "after 1 warm-up, L2 flushed before each"}
         elif kind == "decode":
             nbytes = decode_bytes(w.batch, w.d_inner, w.d_state, 2)
             per = t / w.seqlen
@@ -340,6 +367,54 @@ def per_workload(args, dev, stream, flush_l2, sms, world):
     res["_peaks"] = {"hbm_gbs": hbm_gbs, "hbm_kind": peak_kind, "bf16_tflops": tc_peak,
                      "bf16_kind": tc_kind, "mufu_top_s": mufu_peak / 1e12}
     return res
+
+
+def _bwd_inputs(w, dev, rank):
+    """Inputs, dout and workspace of one backward call of workload w; returns
+    {"call": fn} launching jamba_ssm_scan_bwd on them."""
+    import selective_state_space_26_b200 as jssm
+    from selective_state_space_26_b200 import synth
+    inp = synth.workload_inputs(w, device=dev, seq_offset=replica_seq_offset(rank, w.batch))
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 77)
+    dout = torch.randn(inp.x.shape, generator=g, device=dev).to(w.dtype)
+    ws = torch.zeros(jssm.jamba_ssm_scan_bwd_workspace_size(w.batch, w.seqlen, w.d_inner,
+                                                            w.d_state),
+                     dtype=torch.uint8, device=dev)
+
+    def call():
+        jssm.jamba_ssm_scan_bwd(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, dout, D=inp.D,
+                                delta_bias=inp.delta_bias, workspace=ws)
+    return {"call": call, "inp": inp, "dout": dout, "ws": ws}
+
+
+def profile_one(args):
+    """--kernel K: warm up, then launch only kernel K (at the sizes the bench
+    times) args.steps times, for a profiler to capture; prints nothing."""
+    import selective_state_space_26_b200 as jssm
+    from selective_state_space_26_b200 import build, synth
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[args.workload]
+    if args.kernel == "scan":
+        inp = synth.workload_inputs(w, device=dev)
+        fn = lambda: jssm.jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A,  # noqa
+                                         D=inp.D, delta_bias=inp.delta_bias)
+    elif args.kernel == "scan_bwd":
+        fn = _bwd_inputs(w, dev, 0)["call"]
+    elif args.kernel == "x_proj":
+        xp = synth.x_proj_inputs(4096, 8192, 256, 16, seed=5, device=dev)
+        fn = lambda: jssm.jamba_ssm_x_proj(xp.u, xp.W_x, w_dt=xp.w_dt, w_B=xp.w_B,  # noqa
+                                           w_C=xp.w_C)
+    elif args.kernel == "dt_proj":
+        dp = synth.dt_proj_inputs(4096, 8192, 256, seed=5, device=dev)
+        fn = lambda: jssm.jamba_ssm_dt_proj(dp.hi, dp.W_dt, dt_low_lo=dp.lo)  # noqa
+    else:
+        raise ValueError(f"unknown kernel {args.kernel}")
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize(dev)
 
 
 # ------------------------------------------------------------- our arm
@@ -709,6 +784,10 @@ def main():
                     help="skip the other configurations and the projection kernels")
     ap.add_argument("--pw-reps", type=int, default=3,
                     help="timed launches of each other configuration")
+    ap.add_argument("--kernel", default=None,
+                    choices=["scan", "scan_bwd", "x_proj", "dt_proj"],
+                    help="profiling aid: launch only this kernel (warmup + steps times), "
+                         "print nothing")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -719,6 +798,9 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.kernel:
+        profile_one(args)
         return
     if world > 1:
         import datetime

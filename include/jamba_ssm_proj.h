@@ -48,7 +48,7 @@ extern "C" {
  *
  * Sizes: ntok >= 0 (0: nothing is launched, the pointers are not checked and
  * may be NULL, and JAMBA_SSM_OK is returned), ntok <= 2^31 - 129;
- * 1 <= d_inner <= 65535 * 256 with d_inner % 8 == 0; 1 <= dt_rank <= 2^16
+ * 1 <= d_inner <= 65535 * 128 with d_inner % 8 == 0; 1 <= dt_rank <= 2^16
  * with dt_rank % 8 == 0 (Jamba: d_inner 8192, dt_rank 256).
  * Pointers (device, 16-byte aligned):
  *   dt_low_hi  [ntok, dt_rank]   bf16, required.

@@ -16,19 +16,21 @@
 // (hi and lo against the same W_dt tile) into one fp32 accumulator.  With lo
 // absent (NULL) only the hi plane is used.
 //
-// Work unit and roles.  One CTA computes a 128-token x 256-channel tile of
-// delta; K = dt_rank runs in 64-wide blocks through a 2-stage ring.
+// Work unit and roles.  One CTA computes a 128-token x 128-channel tile of
+// delta; K = dt_rank runs in 64-wide blocks through a 2-stage ring.  A CTA
+// takes 97 KB of shared memory and 128 TMEM columns, so two run on each SM and
+// one's loads and epilogue overlap the other's MMAs.
 //   warp 0 (one lane): TMA loads of the hi / lo / W_dt tiles (128-byte swizzle);
-//   warp 1: allocates 256 TMEM columns; one lane issues the MMAs
-//           (M = 128, N = 256, K = 16, bf16 x bf16 -> fp32) and commits each
+//   warp 1: allocates 128 TMEM columns; one lane issues the MMAs
+//           (M = 128, N = 128, K = 16, bf16 x bf16 -> fp32) and commits each
 //           stage back to the producer, then the finished accumulator;
 //   warps 2-5: epilogue -- each thread owns one token row (TMEM lane), reads
-//           its 256 fp32 columns with tcgen05.ld, rounds them to bf16 into a
+//           its 128 fp32 columns with tcgen05.ld, rounds them to bf16 into a
 //           staged copy of the output tile in shared memory (the operand ring,
-//           free once every MMA has completed), laid out as four 64-column
+//           free once every MMA has completed), laid out as two 64-column
 //           slabs with the 128-byte swizzle so that the 32 rows a warp writes
 //           at once fall in distinct banks; one thread then writes the tile
-//           with four TMA stores, which clip it to [ntok, d_inner].
+//           with two TMA stores, which clip it to [ntok, d_inner].
 // Every wait is bounded; a wait that runs out records JAMBA_SSM_ERR_TIMEOUT in
 // the module's status word and sets a CTA abort flag.  The CTA then winds down
 // in order: the producer waits (bounded) for every TMA load it issued to land,
@@ -44,18 +46,20 @@ namespace jssm {
 
 struct DtProjCfg {
     static constexpr int kBM = 128;  // tokens per tile: the MMA's M (one TMEM lane each)
-    static constexpr int kBN = 256;  // channels per tile: the MMA's N (one TMEM column each)
+    static constexpr int kBN = 128;  // channels per tile: the MMA's N (one TMEM column each)
     static constexpr int kBK = 64;   // dt_rank per stage: one 128-byte swizzled bf16 row
     static constexpr int kUK = 16;   // K of one kind::f16 MMA
     static constexpr int kStages = 2;
     static constexpr uint32_t kTileA = kBM * kBK * 2;        // 16 KB per plane
-    static constexpr uint32_t kTileW = kBN * kBK * 2;        // 32 KB
-    static constexpr uint32_t kStage = 2 * kTileA + kTileW;  // 64 KB
+    static constexpr uint32_t kTileW = kBN * kBK * 2;        // 16 KB
+    static constexpr uint32_t kStage = 2 * kTileA + kTileW;  // 48 KB
     static constexpr uint32_t kOffBar = kStages * kStage;    // barriers after the tiles
     // full[2], empty[2], acc_full (40 bytes), the TMEM slot, the abort flag
     static constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;  // + room to align to 1 KB
     static constexpr int kThreads = 192;
-    static constexpr uint32_t kTmemCols = 256;
+    static constexpr uint32_t kTmemCols = kBN;
+    static_assert(kStage % 1024 == 0, "stages keep the 1 KB swizzle alignment");
+    static_assert(kBM * kBN * 2 <= kStage, "the staged output tile fits in ring stage 0");
     // Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1),
     // A and B bf16 (bits 7-9 and 10-12 = 1), both K-major (bits 15, 16 = 0),
     // N >> 3 in bits 17-22, M >> 4 in bits 24-28.
@@ -167,11 +171,11 @@ __device__ __forceinline__ void epilogue_sync(int count) {
 }
 
 // ------------------------------------------------------------------- kernel
-// Grid: x = token tiles of 128, y = channel tiles of 256.  delta is written
+// Grid: x = token tiles of 128, y = channel tiles of 128.  delta is written
 // only inside [ntok, d_inner] (the TMA stores clip the tile); TMA fills
 // out-of-range operand rows and K columns with zeros, so ragged edges need no
 // special case in the MMAs.
-__global__ void __launch_bounds__(DtProjCfg::kThreads, 1)
+__global__ void __launch_bounds__(DtProjCfg::kThreads, 2)
     s6_dt_proj_kernel(const __grid_constant__ CUtensorMap map_hi,
                       const __grid_constant__ CUtensorMap map_lo,
                       const __grid_constant__ CUtensorMap map_w,
