@@ -314,6 +314,35 @@ size_t jamba_ssm_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t 
 
 jamba_ssm_status jamba_ssm_scan_bwd(const jamba_ssm_scan_bwd_params *p, void *stream);
 
+/*
+ * jamba_ssm_scan_bwd for callers that cannot allocate device memory where
+ * they run it -- for instance a plug-in whose host framework owns every device
+ * allocation and fixes its memory plan before the run, or code on a path where
+ * cudaMalloc's implicit device synchronisation is not acceptable.  The source
+ * pages have no counterpart of this call; it is a deployment convenience.
+ *
+ * Same parameters and results as jamba_ssm_scan_bwd, except that `workspace`
+ * must be NULL and `workspace_bytes` 0: the scratch is a fixed array of
+ * JAMBA_SSM_BWD_NOALLOC_SCRATCH_BYTES that the library reserves in the memory
+ * of every device it is loaded on and keeps until the process exits.  Nothing
+ * is allocated or freed by this call.
+ *   - Sizes whose jamba_ssm_scan_bwd_workspace_size exceeds that array return
+ *     JAMBA_SSM_ERR_WORKSPACE before anything is enqueued (at Jamba's width,
+ *     d_inner 8192 and d_state 16, about 1300 tokens fit).
+ *   - Every call shares the one array of its device: calls that overlap on the
+ *     GPU (other streams, other host threads) race on it and must be ordered
+ *     by the caller.  The array keeps the last call's contents; each call
+ *     clears the part that must start at zero (its status word) itself.
+ *   - A device-side condition (a bounded wait that ran out) is moved into the
+ *     library's per-device status word: read it with
+ *     jamba_ssm_get_status(NULL, stream).
+ *   - The first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress), once; make that first call before any stream
+ *     capture on that device.
+ */
+#define JAMBA_SSM_BWD_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+jamba_ssm_status jamba_ssm_scan_bwd_noalloc(const jamba_ssm_scan_bwd_params *p, void *stream);
+
 /* Launch shape the scan would use for these parameters (no launch).  Any of
  * the out pointers may be NULL.  variant: the built variant chosen (0 for the
  * one-thread-per-channel kernel of the small state sizes);

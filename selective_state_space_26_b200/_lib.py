@@ -25,6 +25,7 @@ EXPORTS = (
     "jamba_ssm_scan_workspace_size",
     "jamba_ssm_scan_bwd",
     "jamba_ssm_scan_bwd_workspace_size",
+    "jamba_ssm_scan_bwd_noalloc",
     "jamba_ssm_state_update",
     "jamba_ssm_scan_plan",
     "jamba_ssm_scan_variant_info",
@@ -167,6 +168,8 @@ def lib():
                 L.jamba_ssm_scan_workspace_size.argtypes = [ctypes.c_int64] * 4
                 L.jamba_ssm_scan_bwd.restype = ctypes.c_int
                 L.jamba_ssm_scan_bwd.argtypes = [ctypes.POINTER(ScanBwdParams), _vp]
+                L.jamba_ssm_scan_bwd_noalloc.restype = ctypes.c_int
+                L.jamba_ssm_scan_bwd_noalloc.argtypes = [ctypes.POINTER(ScanBwdParams), _vp]
                 L.jamba_ssm_scan_bwd_workspace_size.restype = ctypes.c_size_t
                 L.jamba_ssm_scan_bwd_workspace_size.argtypes = [ctypes.c_int64] * 4
                 L.jamba_ssm_last_cuda_error.restype = ctypes.c_int

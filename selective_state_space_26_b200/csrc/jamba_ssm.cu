@@ -879,3 +879,70 @@ size_t jamba_ssm_scan_workspace_size(int64_t batch, int64_t seqlen, int64_t d_in
 }
 
 }  // extern "C"
+
+// ------------------------------------------- backward without a caller workspace
+// Some callers cannot allocate device memory where they run the backward pass:
+// a plug-in whose host framework owns every device allocation and fixes its
+// memory plan before the run, or code on a path where cudaMalloc's implicit
+// device synchronisation is not acceptable.  jamba_ssm_scan_bwd_noalloc serves
+// them with scratch the library owns: this array, reserved in every device's
+// memory when the library's module is loaded and kept until the process exits.
+static __device__ __align__(256) uint8_t g_bwd_noalloc_scratch[JAMBA_SSM_BWD_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of the array above on each device.  In host code the
+// array's name only stands in for the symbol (it is not a device address), so
+// the address is looked up once per device, with that device current.
+void *g_noalloc_ptr[kMaxDevices];
+
+// Moves a condition the backward recorded in the scratch's status word into
+// the library's per-device word, where jamba_ssm_get_status(NULL, ...) reads it.
+__global__ void s6_noalloc_status_kernel(const int *word) {
+    const int w = *word;
+    if (w != 0) atomicCAS(&jssm::g_status_word, 0, w);
+}
+
+}  // namespace
+
+extern "C" jamba_ssm_status jamba_ssm_scan_bwd_noalloc(const jamba_ssm_scan_bwd_params *pin,
+                                                       void *stream) {
+    if (!pin || pin->struct_size < sizeof(jamba_ssm_scan_bwd_params)) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (pin->workspace || pin->workspace_bytes) return JAMBA_SSM_ERR_INVALID_ARG;
+    const size_t need =
+        jamba_ssm_scan_bwd_workspace_size(pin->batch, pin->seqlen, pin->d_inner, pin->d_state);
+    if (need == 0)  // sizes the backward does not take
+        return (pin->batch < 0 || pin->seqlen < 0 || pin->d_inner < 1 || pin->d_state < 1)
+                   ? JAMBA_SSM_ERR_INVALID_ARG
+                   : JAMBA_SSM_ERR_UNSUPPORTED;
+    if (need > JAMBA_SSM_BWD_NOALLOC_SCRATCH_BYTES) return JAMBA_SSM_ERR_WORKSPACE;
+    jamba_ssm_status st;
+    if (!current_device(&st)) return st;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!g_noalloc_ptr[dev]) {  // set-up, once per device, on this call
+            void *ptr = nullptr;
+            e = cudaGetSymbolAddress(&ptr, g_bwd_noalloc_scratch);
+            if (e != cudaSuccess || !ptr) return cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+            g_noalloc_ptr[dev] = ptr;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the array keeps the previous call's contents; only its status word has to
+    // start at zero (every other part is written before it is read)
+    e = cudaMemsetAsync(scratch, 0, JAMBA_SSM_STATUS_BYTES, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    jamba_ssm_scan_bwd_params q = *pin;
+    q.workspace = scratch;
+    q.workspace_bytes = JAMBA_SSM_BWD_NOALLOC_SCRATCH_BYTES;
+    st = jamba_ssm_scan_bwd(&q, stream);
+    if (st != JAMBA_SSM_OK) return st;
+    s6_noalloc_status_kernel<<<1, 1, 0, s>>>(static_cast<const int *>(scratch));
+    e = cudaGetLastError();
+    return e == cudaSuccess ? JAMBA_SSM_OK : cuda_fail(e);
+}
