@@ -13,6 +13,8 @@ threads (ctypes releases the GIL during the call), which does not change the
 order of any floating-point operation inside a channel.
 
 ``scan_bwd`` is the scan's reverse-mode gradient (the backward pass).
+``ssd_scan`` is the scalar-identity variant (Mamba-2's state matrix: one decay
+per head and step, shared by all of the head's channels and states).
 ``project`` is the step before the scan (Delta, B and C from the scan's
 input through the x / dt projections and RMSNorm).  ``scan_packed`` and
 ``state_update_slots`` define the serving layouts (packed
@@ -71,6 +73,9 @@ def _declare(lib):
     lib.oracle_state_update_f64.restype = ctypes.c_int
     lib.oracle_state_update_f64.argtypes = ([_i64] * 3 + [_dp] * 9
                                             + [ctypes.c_int, _dp])
+    lib.oracle_ssd_scan_f64.restype = ctypes.c_int
+    lib.oracle_ssd_scan_f64.argtypes = ([_i64] * 7 + [_dp] * 8 + [ctypes.c_int]
+                                        + [_dp] * 3)
     return lib
 
 
@@ -340,3 +345,41 @@ def state_update_slots(cache, x, delta, z, B, C, A, state_indices, D=None, delta
         out[live] = o
         st[rows] = new
     return out, st
+
+
+def ssd_scan(x, delta, z, B, C, A, nheads, D=None, delta_bias=None, delta_softplus=True,
+             h0=None, threads: int = 1, lib=None):
+    """Sequential fp64 scan of the scalar-identity (Mamba-2) variant.
+
+    Shapes: x, z [batch, seqlen, nheads * headdim]; delta [batch, seqlen,
+    nheads]; B, C [batch, seqlen, d_state]; A, delta_bias [nheads]; D
+    [nheads * headdim]; h0 [batch, nheads * headdim, d_state].  Returns (out,
+    h_final) as float64 arrays.  Heads are independent and split across host
+    threads.
+    """
+    lib = lib or load()
+    x, delta, z, B, C, A = map(_f64, (x, delta, z, B, C, A))
+    D, delta_bias, h0 = _f64(D), _f64(delta_bias), _f64(h0)
+    batch, seqlen, d_inner = x.shape
+    d_state = B.shape[-1]
+    assert d_inner % nheads == 0 and A.shape == (nheads,)
+    assert delta.shape == (batch, seqlen, nheads) and z.shape == x.shape
+    headdim = d_inner // nheads
+    out = np.empty_like(x)
+    h_final = np.empty((batch, d_inner, d_state), dtype=np.float64)
+
+    def run(lo, hi):
+        if lib.oracle_ssd_scan_f64(batch, seqlen, nheads, headdim, d_state, lo, hi, _ptr(x),
+                                   _ptr(delta), _ptr(z), _ptr(B), _ptr(C), _ptr(A), _ptr(D),
+                                   _ptr(delta_bias), int(bool(delta_softplus)), _ptr(h0),
+                                   _ptr(out), _ptr(h_final)) != 0:
+            raise ValueError("oracle_ssd_scan_f64 rejected its arguments")
+
+    threads = max(1, min(int(threads), nheads))
+    if threads == 1:
+        run(0, nheads)
+    else:
+        bounds = np.linspace(0, nheads, threads + 1).astype(np.int64)
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(lambda i: run(int(bounds[i]), int(bounds[i + 1])), range(threads)))
+    return out, h_final

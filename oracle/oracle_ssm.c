@@ -322,3 +322,65 @@ int oracle_scan_bwd_f64(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t 
     free(hs);
     return 0;
 }
+
+/*
+ * The scalar-identity variant of the selective SSM (Mamba-2's state matrix):
+ * "Jamba -- Hybrid SSM-Transformer" (factory.pai-world.com lesson), section
+ * "Mamba-3: 2026년의 순수 SSM 기준선", item 2: the state matrix went from
+ * complex (S4) to real diagonal (Mamba) to a scaled identity (Mamba-2); item 1
+ * of the same list: Mamba-2 discretises with the Euler method.  Reading (the
+ * pages print no equations of this variant): d_inner = nheads * headdim
+ * channels, channel d = head * headdim + p; each head has one scalar A[head]
+ * and one step size per token, Delta[t, head] = softplus(delta[t, head] +
+ * delta_bias[head]) (or without softplus); every channel of the head keeps
+ * d_state states
+ *     h[n] = exp(Delta A[head]) h[n] + Delta B[t, n] x[t, d],
+ *     out  = (sum_n C[t, n] h[n] + D[d] x[t, d]) silu(z[t, d]).
+ *
+ * Heads [h_lo, h_hi) of every sequence; layouts:
+ *   x, z, out : [batch, seqlen, nheads * headdim]
+ *   delta     : [batch, seqlen, nheads]
+ *   B, C      : [batch, seqlen, d_state]
+ *   A, delta_bias : [nheads] (delta_bias may be NULL)
+ *   D         : [nheads * headdim] or NULL
+ *   h0, h_final : [batch, nheads * headdim, d_state] (h0, h_final may be NULL)
+ */
+int oracle_ssd_scan_f64(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim,
+                        int64_t d_state, int64_t h_lo, int64_t h_hi, const double *x,
+                        const double *delta, const double *z, const double *B, const double *C,
+                        const double *A, const double *D, const double *delta_bias,
+                        int delta_softplus, const double *h0, double *out, double *h_final) {
+    if (batch < 0 || seqlen < 0 || nheads < 0 || headdim < 1 || d_state < 1 || d_state > 64)
+        return -1;
+    if (h_lo < 0 || h_hi > nheads || h_lo > h_hi) return -1;
+    const int64_t d_inner = nheads * headdim;
+    double h[64];
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t hd = h_lo; hd < h_hi; ++hd) {
+            for (int64_t p = 0; p < headdim; ++p) {
+                const int64_t d = hd * headdim + p;
+                for (int64_t n = 0; n < d_state; ++n)
+                    h[n] = h0 ? h0[(b * d_inner + d) * d_state + n] : 0.0;
+                for (int64_t t = 0; t < seqlen; ++t) {
+                    const double v = delta[(b * seqlen + t) * nheads + hd] +
+                                     (delta_bias ? delta_bias[hd] : 0.0);
+                    const double dv = delta_softplus ? oracle_softplus(v) : v;
+                    const double decay = exp(dv * A[hd]);  /* one scalar for every state */
+                    const int64_t i = (b * seqlen + t) * d_inner + d;
+                    const double *Bt = B + (b * seqlen + t) * d_state;
+                    const double *Ct = C + (b * seqlen + t) * d_state;
+                    double y = 0.0;
+                    for (int64_t n = 0; n < d_state; ++n) {
+                        h[n] = decay * h[n] + dv * Bt[n] * x[i];
+                        y += Ct[n] * h[n];
+                    }
+                    y += (D ? D[d] : 0.0) * x[i];
+                    out[i] = y * oracle_silu(z[i]);
+                }
+                if (h_final)
+                    for (int64_t n = 0; n < d_state; ++n) h_final[(b * d_inner + d) * d_state + n] = h[n];
+            }
+        }
+    }
+    return 0;
+}
