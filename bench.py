@@ -301,6 +301,20 @@ def per_workload(args, dev, stream, flush_l2, sms, world):
     meta += [(None, "x_proj"), (None, "dt_proj")]
     del xp, dp, dl
 
+    # the scalar-identity (Mamba-2) variant at Jamba's width: 128 heads of 64
+    ssd = synth.ssd_inputs(1, 4096, 128, 64, 16, torch.bfloat16, seed=6, device=dev,
+                           seq_offset=args.rank)
+    ssd_out = torch.empty_like(ssd.x)
+    ssd_hf = torch.empty(1, 8192, 16, dtype=torch.float32, device=dev)
+    t_s = time_launches(lambda: jssm.jamba_ssm_ssd_scan(ssd.x, ssd.delta, ssd.z, ssd.B, ssd.C,
+                                                        ssd.A, D=ssd.D, delta_bias=ssd.delta_bias,
+                                                        out=ssd_out, h_final=ssd_hf),
+                        max(args.pw_reps, 10), stream, dev, flush=flush_l2)
+    names.append("ssd_bf16_b1_l4096_h128_p64_n16")
+    times.append(t_s)
+    meta.append((None, "ssd"))
+    del ssd, ssd_out, ssd_hf
+
     # the backward pass of the headline layer (training): all three kernels
     wb = synth.WORKLOADS["s6_prefill_bf16_b1_l4096_d8192_n16"]
     bw = _bwd_inputs(wb, dev, args.rank)
@@ -340,6 +354,16 @@ def per_workload(args, dev, stream, flush_l2, sms, world):
                              "and the per-segment recompute add 2 d_state + 1)",
                 "timing": f"{args.pw_reps} calls (checkpoint, backward and reduction kernels) "
                           "after 1 warm-up, L2 flushed before each"}
+        elif kind == "ssd":
+            tok, d_inner, H, N = 4096, 8192, 128, 16
+            nbytes = (tok * (3 * d_inner + H + 2 * N) * 2 + (H * 2 + d_inner) * 4
+                      + d_inner * N * 4)
+            res[name] = {
+                "kernel_us": t * 1e6, "tokens_per_s": tok * world / t,
+                "roofline": {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": hbm_gbs,
+                             "unit": "GB/s", "frac": nbytes / t / 1e9 / hbm_gbs,
+                             "algorithmic_bytes": nbytes},
+                "timing": f"{max(args.pw_reps, 10)} launches after 1 warm-up, L2 flushed before each"}
         elif kind == "decode":
             nbytes = decode_bytes(w.batch, w.d_inner, w.d_state, 2)
             per = t / w.seqlen

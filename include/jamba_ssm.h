@@ -343,6 +343,51 @@ jamba_ssm_status jamba_ssm_scan_bwd(const jamba_ssm_scan_bwd_params *p, void *st
 #define JAMBA_SSM_BWD_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 jamba_ssm_status jamba_ssm_scan_bwd_noalloc(const jamba_ssm_scan_bwd_params *p, void *stream);
 
+/*
+ * The scalar-identity variant of the selective scan (Mamba-2's state matrix).
+ * Sources: "Jamba -- Hybrid SSM-Transformer" (factory.pai-world.com), section
+ * "Mamba-3: 2026년의 순수 SSM 기준선", items 1-2: the state matrix is a scaled
+ * identity, discretised by Euler's method.  Reading: d_inner = nheads *
+ * headdim channels, channel d = head * headdim + p; per head and token
+ *     Delta = softplus(delta[t, head] + delta_bias[head]) (or without softplus),
+ *     h[n]  = exp(Delta A[head]) h[n] + Delta B[t, n] x[t, d],
+ *     out   = (sum_n C[t, n] h[n] + D[d] x[t, d]) silu(z[t, d]).
+ *
+ * Sizes: batch in [0, 65535], seqlen >= 0, headdim a multiple of 32, nheads a
+ * multiple of 8 (bf16) or 4 (f32), d_state in {8, 16}.
+ * Pointers (device, 16-byte aligned unless noted):
+ *   x, z, out   [batch, seqlen, nheads * headdim] io_dtype (out written; it must
+ *               not overlap an input).
+ *   delta       [batch, seqlen, nheads] io_dtype: one raw step size per head.
+ *   B, C        [batch, seqlen, d_state] io_dtype.
+ *   A           [nheads] fp32 (4-byte aligned); delta_bias [nheads] fp32 or NULL;
+ *               D [nheads * headdim] fp32 or NULL.
+ *   h0, h_final [batch, nheads * headdim, d_state] fp32 or NULL (the same
+ *               state layout as jamba_ssm_scan's).
+ *   workspace   optional status block, as for jamba_ssm_scan.
+ * debug_flags / timeout_cycles: as jamba_ssm_scan.
+ */
+typedef struct jamba_ssm_ssd_params {
+    size_t struct_size;          /* = sizeof(jamba_ssm_ssd_params)            */
+    int64_t batch, seqlen, nheads, headdim, d_state;
+    int32_t io_dtype;
+    int32_t delta_softplus;
+    const void *x, *delta, *z;
+    const void *B, *C;
+    const float *A;
+    const float *D;
+    const float *delta_bias;
+    const float *h0;
+    void *out;
+    float *h_final;
+    void *workspace;
+    size_t workspace_bytes;
+    uint32_t debug_flags;
+    uint64_t timeout_cycles;
+} jamba_ssm_ssd_params;
+
+jamba_ssm_status jamba_ssm_ssd_scan(const jamba_ssm_ssd_params *p, void *stream);
+
 /* Launch shape the scan would use for these parameters (no launch).  Any of
  * the out pointers may be NULL.  variant: the built variant chosen (0 for the
  * one-thread-per-channel kernel of the small state sizes);

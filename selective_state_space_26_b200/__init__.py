@@ -7,6 +7,8 @@ The calls, with the names of the C entry points:
 * ``jamba_ssm_state_update``  -- one-token decode step, state updated in place;
 * ``jamba_ssm_scan_bwd``      -- the scan's backward pass (gradients of every
   input, for training);
+* ``jamba_ssm_ssd_scan``      -- the scalar-identity (Mamba-2) variant of the
+  scan: one decay per head and token;
 * ``jamba_ssm_x_proj``        -- the projection of the scan's input to dt_low, B
   and C with their RMSNorms (libjamba_ssm_proj.so);
 * ``jamba_ssm_dt_proj``       -- the low-rank product that produces the scan's
@@ -27,7 +29,7 @@ from ._lib import JambaSSMError
 
 __all__ = ["jamba_ssm_scan", "jamba_ssm_state_update", "jamba_ssm_get_status", "scan_plan",
            "jamba_ssm_scan_workspace_size", "jamba_ssm_scan_bwd",
-           "jamba_ssm_scan_bwd_workspace_size",
+           "jamba_ssm_scan_bwd_workspace_size", "jamba_ssm_ssd_scan",
            "jamba_ssm_x_proj", "jamba_ssm_dt_proj", "jamba_ssm_proj_get_status",
            "JambaSSMError"]
 
@@ -202,6 +204,49 @@ def jamba_ssm_scan_bwd(x, delta, z, B, C, A, dout, D=None, delta_bias=None,
     if st != _lib.OK:
         raise JambaSSMError(st, "jamba_ssm_scan_bwd")
     return g
+
+
+def jamba_ssm_ssd_scan(x, delta, z, B, C, A, D=None, delta_bias=None, delta_softplus=True,
+                       h0=None, out=None, h_final=None, return_final_state=True, stream=None,
+                       debug_flags: int = 0, timeout_cycles: int = 0, workspace=None):
+    """Scan of the scalar-identity (Mamba-2) variant.  x, z [batch, seqlen,
+    nheads * headdim]; delta [batch, seqlen, nheads] (one step size per head);
+    B, C [batch, seqlen, d_state]; A, delta_bias [nheads] fp32; D [nheads *
+    headdim] fp32; h0 [batch, nheads * headdim, d_state] fp32.  Returns (out,
+    h_final)."""
+    if x.dtype not in _IO:
+        raise TypeError(f"x must be bfloat16 or float32, got {x.dtype}")
+    batch, seqlen, d_inner = x.shape
+    nheads = A.shape[0]
+    d_state = B.shape[-1]
+    if nheads < 1 or d_inner % nheads:
+        raise ValueError("d_inner must be a multiple of the number of heads")
+    dev, io = x.device, x.dtype
+    if out is None:
+        out = torch.empty_like(x)
+    if h_final is None and return_final_state:
+        h_final = torch.empty(batch, d_inner, d_state, dtype=torch.float32, device=dev)
+    for t, n, sh in ((x, "x", (batch, seqlen, d_inner)), (z, "z", (batch, seqlen, d_inner)),
+                     (out, "out", (batch, seqlen, d_inner)),
+                     (delta, "delta", (batch, seqlen, nheads)),
+                     (B, "B", (batch, seqlen, d_state)), (C, "C", (batch, seqlen, d_state))):
+        _check(t, n, sh, io, dev)
+    _check(A, "A", (nheads,), torch.float32, dev)
+    _check(delta_bias, "delta_bias", (nheads,), torch.float32, dev)
+    _check(D, "D", (d_inner,), torch.float32, dev)
+    _check(h0, "h0", (batch, d_inner, d_state), torch.float32, dev)
+    _check(h_final, "h_final", (batch, d_inner, d_state), torch.float32, dev)
+    ws, ws_bytes = _workspace(workspace, dev)
+    p = _lib.new_ssd_params(
+        batch=batch, seqlen=seqlen, nheads=nheads, headdim=d_inner // nheads, d_state=d_state,
+        io_dtype=_IO[io], delta_softplus=int(bool(delta_softplus)), x=_ptr(x), delta=_ptr(delta),
+        z=_ptr(z), B=_ptr(B), C=_ptr(C), A=_ptr(A), D=_ptr(D), delta_bias=_ptr(delta_bias),
+        h0=_ptr(h0), out=_ptr(out), h_final=_ptr(h_final), workspace=ws, workspace_bytes=ws_bytes,
+        debug_flags=int(debug_flags), timeout_cycles=int(timeout_cycles))
+    st = _lib.call_ssd(p, _stream(stream, dev))
+    if st != _lib.OK:
+        raise JambaSSMError(st, "jamba_ssm_ssd_scan")
+    return out, h_final
 
 
 def scan_plan(x, A, B=None, variant: int = 0):

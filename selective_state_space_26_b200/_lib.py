@@ -26,6 +26,7 @@ EXPORTS = (
     "jamba_ssm_scan_bwd",
     "jamba_ssm_scan_bwd_workspace_size",
     "jamba_ssm_scan_bwd_noalloc",
+    "jamba_ssm_ssd_scan",
     "jamba_ssm_state_update",
     "jamba_ssm_scan_plan",
     "jamba_ssm_scan_variant_info",
@@ -103,6 +104,21 @@ class ScanBwdParams(ctypes.Structure):
     ]
 
 
+class SsdParams(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t),
+        ("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
+        ("headdim", ctypes.c_int64), ("d_state", ctypes.c_int64),
+        ("io_dtype", ctypes.c_int32), ("delta_softplus", ctypes.c_int32),
+        ("x", _vp), ("delta", _vp), ("z", _vp),
+        ("B", _vp), ("C", _vp),
+        ("A", _fp), ("D", _fp), ("delta_bias", _fp), ("h0", _fp),
+        ("out", _vp), ("h_final", _fp),
+        ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+        ("debug_flags", ctypes.c_uint32), ("timeout_cycles", ctypes.c_uint64),
+    ]
+
+
 class DtProjParams(ctypes.Structure):
     _fields_ = [
         ("struct_size", ctypes.c_size_t),
@@ -168,6 +184,8 @@ def lib():
                 L.jamba_ssm_scan_workspace_size.argtypes = [ctypes.c_int64] * 4
                 L.jamba_ssm_scan_bwd.restype = ctypes.c_int
                 L.jamba_ssm_scan_bwd.argtypes = [ctypes.POINTER(ScanBwdParams), _vp]
+                L.jamba_ssm_ssd_scan.restype = ctypes.c_int
+                L.jamba_ssm_ssd_scan.argtypes = [ctypes.POINTER(SsdParams), _vp]
                 L.jamba_ssm_scan_bwd_noalloc.restype = ctypes.c_int
                 L.jamba_ssm_scan_bwd_noalloc.argtypes = [ctypes.POINTER(ScanBwdParams), _vp]
                 L.jamba_ssm_scan_bwd_workspace_size.restype = ctypes.c_size_t
@@ -281,6 +299,18 @@ def new_scan_bwd_params(**kw) -> ScanBwdParams:
     for k, v in kw.items():
         setattr(p, k, v)
     return p
+
+
+def new_ssd_params(**kw) -> SsdParams:
+    p = SsdParams()
+    p.struct_size = ctypes.sizeof(SsdParams)
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def call_ssd(p: SsdParams, stream: int) -> int:
+    return lib().jamba_ssm_ssd_scan(ctypes.byref(p), _vp(stream or None))
 
 
 def call_scan_bwd(p: ScanBwdParams, stream: int) -> int:

@@ -15,6 +15,7 @@
 #include "s6_scan_fused.cuh"
 #include "s6_scan_serving.cuh"
 #include "s6_scan_small.cuh"
+#include "s6_ssd.cuh"
 #include "s6_state_update.cuh"
 
 using jssm::ScanArgs;
@@ -372,6 +373,31 @@ BwdKernels g_bwd[2][3][2] = {
     {{make_bwd<float, 16, 4, 7, 32, false>(), make_bwd<float, 16, 4, 7, 32, true>()},
      {make_bwd<float, 8, 4, 7, 32, false>(), make_bwd<float, 8, 4, 7, 32, true>()},
      {make_bwd<float, 4, 2, 4, 32, false>(), make_bwd<float, 4, 2, 4, 32, true>()}},
+};
+
+// ------------------------------------------------------- scalar-identity scan
+// 4 lanes per channel, 4 compute warps: 32 channels of one head per CTA.
+constexpr int kSsdNW = 4, kSsdG = 4, kSsdTT = 64, kSsdStages = 3;
+constexpr int kSsdCC = kSsdNW * (32 / kSsdG);
+struct SsdKernel {
+    const void *k;
+    int smem;
+    bool attr[kMaxDevices];
+};
+template <typename IoT, int N, bool SP>
+SsdKernel make_ssd() {
+    SsdKernel k{};
+    k.k = reinterpret_cast<const void *>(
+        &jssm::s6_ssd_kernel<IoT, N, kSsdG, kSsdNW, kSsdTT, kSsdStages, SP>);
+    k.smem = jssm::SsdCfg<IoT, N, kSsdG, kSsdNW, kSsdTT, kSsdStages>::kSmemBytes;
+    return k;
+}
+// [dtype][d_state 16, 8][softplus off, on]
+SsdKernel g_ssd[2][2][2] = {
+    {{make_ssd<__nv_bfloat16, 16, false>(), make_ssd<__nv_bfloat16, 16, true>()},
+     {make_ssd<__nv_bfloat16, 8, false>(), make_ssd<__nv_bfloat16, 8, true>()}},
+    {{make_ssd<float, 16, false>(), make_ssd<float, 16, true>()},
+     {make_ssd<float, 8, false>(), make_ssd<float, 8, true>()}},
 };
 
 }  // namespace
@@ -863,6 +889,102 @@ jamba_ssm_status jamba_ssm_scan_bwd(const jamba_ssm_scan_bwd_params *p, void *st
         e = cudaLaunchKernel(K.reduce, dim3(static_cast<unsigned>(blocks)), dim3(256), kargs, 0, s);
         if (e != cudaSuccess) return cuda_fail(e);
     }
+    return finish_launch(s, p->workspace);
+}
+
+jamba_ssm_status jamba_ssm_ssd_scan(const jamba_ssm_ssd_params *p, void *stream) {
+    if (!p || p->struct_size < sizeof(jamba_ssm_ssd_params)) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->batch < 0 || p->seqlen < 0 || p->nheads < 1 || p->headdim < 1 || p->d_state < 1)
+        return JAMBA_SSM_ERR_INVALID_ARG;
+    if (p->io_dtype != JAMBA_SSM_BF16 && p->io_dtype != JAMBA_SSM_F32) return JAMBA_SSM_ERR_INVALID_ARG;
+    const int es = p->io_dtype == JAMBA_SSM_BF16 ? 2 : 4;
+    if ((p->d_state != 8 && p->d_state != 16) || p->headdim % kSsdCC != 0 ||
+        (p->nheads * es) % 16 != 0)
+        return JAMBA_SSM_ERR_UNSUPPORTED;
+    const int64_t D = p->nheads * p->headdim;
+    const int64_t kMaxRows = kMaxI32 - 256;
+    if (p->batch > 65535 || p->seqlen > kMaxRows || D > (int64_t(1) << 30) ||
+        (p->batch && p->seqlen && p->batch > kMaxElems / p->seqlen) ||
+        p->batch * p->seqlen > kMaxElems / D)
+        return JAMBA_SSM_ERR_UNSUPPORTED;
+    {
+        const jamba_ssm_status ws = check_workspace(p->workspace, p->workspace_bytes);
+        if (ws != JAMBA_SSM_OK) return ws;
+    }
+    const int64_t tok = p->batch * p->seqlen;
+    const size_t act = size_t(tok) * D * es, dts = size_t(tok) * p->nheads * es;
+    const size_t bc = size_t(tok) * p->d_state * es, st = size_t(p->batch) * D * p->d_state * 4;
+    if (tok > 0) {
+        if (!p->x || !p->delta || !p->z || !p->B || !p->C || !p->A || !p->out)
+            return JAMBA_SSM_ERR_INVALID_ARG;
+        const void *a16[] = {p->x, p->delta, p->z, p->B, p->C, p->out, p->h0, p->h_final};
+        for (const void *q : a16)
+            if (!aligned(q, 16)) return JAMBA_SSM_ERR_MISALIGNED;
+        const void *ins[] = {p->x, p->delta, p->z, p->B, p->C};
+        const size_t insz[] = {act, dts, act, bc, bc};
+        for (int i = 0; i < 5; ++i)
+            if (overlaps(p->out, act, ins[i], insz[i])) return JAMBA_SSM_ERR_INVALID_ARG;
+        if (overlaps(p->h_final, st, p->out, act)) return JAMBA_SSM_ERR_INVALID_ARG;
+    }
+    if (!aligned(p->A, 4) || !aligned(p->D, 4) || !aligned(p->delta_bias, 4) ||
+        !aligned(p->h0, 16) || !aligned(p->h_final, 16))
+        return JAMBA_SSM_ERR_MISALIGNED;
+    if (p->h0 && p->h_final && p->h0 != p->h_final && overlaps(p->h0, st, p->h_final, st))
+        return JAMBA_SSM_ERR_INVALID_ARG;
+    jamba_ssm_status stt;
+    const DeviceInfo *dev = current_device(&stt);
+    if (!dev) return stt;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (p->batch == 0) return JAMBA_SSM_OK;
+    if (tok == 0) {  // no steps: the final state is the initial state
+        if (!p->h_final || p->h0 == p->h_final) return JAMBA_SSM_OK;
+        cudaError_t e = p->h0 ? cudaMemcpyAsync(p->h_final, p->h0, st, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(p->h_final, 0, st, s);
+        return e == cudaSuccess ? finish_launch(s, p->workspace) : cuda_fail(e);
+    }
+    SsdKernel &K = g_ssd[p->io_dtype == JAMBA_SSM_BF16 ? 0 : 1][p->d_state == 16 ? 0 : 1]
+                        [p->delta_softplus ? 1 : 0];
+    EncodeTiledFn fn = encode_fn(&stt);
+    if (!fn) return stt;
+    const CUtensorMapDataType dt =
+        p->io_dtype == JAMBA_SSM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    jssm::SsdMaps m;
+    if (!encode_3d(fn, &m.x, p->x, dt, es, D, p->seqlen, p->batch, kSsdCC, kSsdTT) ||
+        !encode_3d(fn, &m.z, p->z, dt, es, D, p->seqlen, p->batch, kSsdCC, kSsdTT) ||
+        !encode_3d(fn, &m.out, p->out, dt, es, D, p->seqlen, p->batch, kSsdCC, kSsdTT) ||
+        !encode_3d(fn, &m.dt, p->delta, dt, es, p->nheads, p->seqlen, p->batch, 16 / es, kSsdTT) ||
+        !encode_3d(fn, &m.B, p->B, dt, es, p->d_state, p->seqlen, p->batch, (int)p->d_state, kSsdTT) ||
+        !encode_3d(fn, &m.C, p->C, dt, es, p->d_state, p->seqlen, p->batch, (int)p->d_state, kSsdTT))
+        return JAMBA_SSM_ERR_UNSUPPORTED;
+    int devid = 0;
+    cudaGetDevice(&devid);
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!K.attr[devid]) {
+            cudaError_t e = cudaFuncSetAttribute(K.k, cudaFuncAttributeMaxDynamicSharedMemorySize, K.smem);
+            if (e != cudaSuccess) return cuda_fail(e);
+            K.attr[devid] = true;
+        }
+    }
+    jssm::SsdArgs a{};
+    a.batch = p->batch;
+    a.seqlen = p->seqlen;
+    a.nheads = p->nheads;
+    a.headdim = p->headdim;
+    a.A = p->A;
+    a.D = p->D;
+    a.delta_bias = p->delta_bias;
+    a.h0 = p->h0;
+    a.h_final = p->h_final;
+    a.delta_softplus = p->delta_softplus != 0;
+    a.status = static_cast<int *>(p->workspace);
+    a.debug_flags = p->debug_flags;
+    a.timeout_cycles = p->timeout_cycles ? p->timeout_cycles : (uint64_t(1) << 31);
+    const dim3 grid(static_cast<unsigned>(D / kSsdCC), static_cast<unsigned>(p->batch));
+    void *kargs[] = {&m, &a};
+    cudaError_t e = cudaLaunchKernel(K.k, grid, dim3((kSsdNW + 1) * 32), kargs,
+                                     static_cast<size_t>(K.smem), s);
+    if (e != cudaSuccess) return cuda_fail(e);
     return finish_launch(s, p->workspace);
 }
 

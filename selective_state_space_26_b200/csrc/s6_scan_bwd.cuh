@@ -26,11 +26,12 @@
 //     walk it backwards with g in registers.  The lane layout is the forward's:
 //     G lanes per channel, NS = N / G states per lane, lane `sub` owning the
 //     per-(t, d) scalars of steps sub, sub + G, ...; sums over a channel's
-//     states go through the transposing butterfly.  dB and dC, sums over
-//     channels, are reduced over a warp's channels with a transposing
-//     butterfly on the lane bits that select the channel, then over the CTA's
-//     warps in shared memory, and written as one partial per CTA.  dx, ddelta
-//     and dz leave through shared memory and TMA stores.
+//     states go through the transposing butterfly; the state math runs on
+//     fp32 pairs.  dB and dC, sums over channels, are summed over a warp's
+//     channels through a small per-warp shared-memory scratch (each lane
+//     stores its slices, then lane k adds slot k), then over the CTA's warps,
+//     and written as one partial per CTA.  dx, ddelta and dz leave through
+//     shared memory and TMA stores.
 //  3. s6_bwd_reduce_kernel: dB and dC = the sum of the CTA partials, and dA,
 //     dD, dbias = the sum over sequences, in a fixed order in fp64.
 // Every mbarrier wait is bounded; a wait that runs out records
@@ -73,57 +74,39 @@ struct BwdCfg {
     static constexpr int kOffOut = STAGES * kStage;           // dx, ddelta, dz per set
     static constexpr int kOffPart = kOffOut + NOUT * 3 * kAct;  // [NW][TT][2N] fp32
     static constexpr int kPart = NW * TT * 2 * N * 4;
-    static constexpr int kOffBar = kOffPart + kPart;
+    // per warp, one step's [channel][dB | dC] scratch (see BcScratch)
+    static constexpr int kOffScr = kOffPart + kPart;
+    static constexpr int kScrWords = CW * (N == 16 ? 48 : (N == 8 ? 24 : 12));
+    static constexpr int kOffBar = kOffScr + NW * kScrWords * 4;
     static constexpr int kNumBars = 2 * STAGES + 2 * NOUT;    // full, empty, out_full, out_free
     static constexpr int kOffFlag = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffFlag + 16;
     static_assert(kAct % 128 == 0 && kBC % 128 == 0, "TMA boxes 128-byte aligned");
 };
 
-// Sum over the CW channels of a warp: each lane holds V = 2 NS partial sums
-// (its states' dB then dC) of one step; after log2(CW) rounds over the lane
-// bits that select the channel, lane (c, sub) holds the sum over the warp's
-// channels of value index `bc_index<...>(lane)` of its sub's V values (while
-// there are values to split, each round keeps the half its bit selects and
-// trades the other; once one value is left the rounds just add).
-template <int V, int G>
-__device__ __forceinline__ float reduce_channels(float (&v)[V], int lane) {
-    constexpr int CW = 32 / G;
-    float w[V];
-#pragma unroll
-    for (int i = 0; i < V; ++i) w[i] = v[i];
-    int n = V;
-#pragma unroll
-    for (int m = G; m < 32; m <<= 1) {
-        const bool upper = (lane & m) != 0;
-        if (n > 1) {
-            const int h = n / 2;
-#pragma unroll
-            for (int i = 0; i < V / 2; ++i) {
-                if (i < h) {
-                    const float keep = upper ? w[i + h] : w[i];
-                    const float send = upper ? w[i] : w[i + h];
-                    w[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-                }
-            }
-            n = h;
-        } else {
-            w[0] += __shfl_xor_sync(0xffffffffu, w[0], m);
-        }
+// NS consecutive values (one lane's B or C slice of one step) as NS / 2 fp32
+// pairs, read with one vector load: 4 or 8 bytes of bf16, 8 or 16 of fp32.
+template <int NS>
+__device__ __forceinline__ void load_pairs(const __nv_bfloat16 *p, float2 (&v)[NS / 2]) {
+    if constexpr (NS == 4) {
+        const uint2 w = *reinterpret_cast<const uint2 *>(p);
+        v[0] = bf16x2_to_f2(w.x);
+        v[1] = bf16x2_to_f2(w.y);
+    } else {
+        static_assert(NS == 2, "two or four values");
+        v[0] = bf16x2_to_f2(*reinterpret_cast<const uint32_t *>(p));
     }
-    static_assert(CW >= 1, "");
-    return w[0];
 }
-// Which of the V values lane `lane` holds after reduce_channels.
-template <int V, int G>
-__device__ __forceinline__ int bc_index(int lane) {
-    int idx = 0, n = V;
-#pragma unroll
-    for (int m = G; m < 32 && n > 1; m <<= 1) {
-        n /= 2;
-        if (lane & m) idx += n;
+template <int NS>
+__device__ __forceinline__ void load_pairs(const float *p, float2 (&v)[NS / 2]) {
+    if constexpr (NS == 4) {
+        const float4 w = *reinterpret_cast<const float4 *>(p);
+        v[0] = make_float2(w.x, w.y);
+        v[1] = make_float2(w.z, w.w);
+    } else {
+        static_assert(NS == 2, "two or four values");
+        v[0] = *reinterpret_cast<const float2 *>(p);
     }
-    return idx;
 }
 
 // ------------------------------------------------------------ checkpoints
@@ -134,7 +117,7 @@ __device__ __forceinline__ int bc_index(int lane) {
 // warp; each segment's loads are issued before its arithmetic.
 template <typename IoT, int N, int G, int CC>
 __global__ void __launch_bounds__(CC *G) s6_bwd_ckpt_kernel(const BwdArgs a) {
-    constexpr int NS = N / G;
+    constexpr int NS = N / G, NP = NS / 2;
     const int lane = threadIdx.x & 31, sub = lane % G;
     const int gbase = lane & ~(G - 1);
     const int64_t b = blockIdx.y;
@@ -143,26 +126,34 @@ __global__ void __launch_bounds__(CC *G) s6_bwd_ckpt_kernel(const BwdArgs a) {
     const int64_t dc = dvalid ? d : a.d_inner - 1;  // invalid lanes still join the shuffles
     const int64_t D = a.d_inner, L = a.seqlen;
     const int64_t nck = (L + kCk - 1) / kCk;
-    float h[NS], a2[NS];
+    float2 h[NP], a2[NP];
 #pragma unroll
-    for (int i = 0; i < NS; ++i) {
-        a2[i] = __ldg(a.A + dc * N + sub * NS + i) * kLog2e;
-        h[i] = a.h0 ? __ldg(a.h0 + (b * D + dc) * N + sub * NS + i) : 0.0f;
+    for (int i = 0; i < NP; ++i) {
+        const int n = sub * NS + 2 * i;
+        a2[i] = make_float2(__ldg(a.A + dc * N + n) * kLog2e, __ldg(a.A + dc * N + n + 1) * kLog2e);
+        h[i] = a.h0 ? make_float2(__ldg(a.h0 + (b * D + dc) * N + n), __ldg(a.h0 + (b * D + dc) * N + n + 1))
+                    : make_float2(0.0f, 0.0f);
     }
     const float bias = a.delta_bias ? __ldg(a.delta_bias + dc) : 0.0f;
     const bool sp = a.delta_softplus != 0;
     const IoT *x = static_cast<const IoT *>(a.x) + b * L * D;
     const IoT *dt = static_cast<const IoT *>(a.delta) + b * L * D;
-    const IoT *Bm = static_cast<const IoT *>(a.B) + b * L * N;
+    const IoT *Bm = static_cast<const IoT *>(a.B) + b * L * N + sub * NS;
     for (int64_t k = 0; k < nck; ++k) {
         if (dvalid) {
             float *o = a.ckpt + ((b * nck + k) * D + d) * N + sub * NS;
 #pragma unroll
-            for (int i = 0; i < NS; ++i) o[i] = h[i];
+            for (int i = 0; i < NP; ++i) {
+                o[2 * i] = h[i].x;
+                o[2 * i + 1] = h[i].y;
+            }
         }
         const int64_t t0 = k * kCk;
         const int nst = static_cast<int>(L - t0 < kCk ? L - t0 : kCk);
-        float xo[kCk / G], vo[kCk / G], bv[kCk][NS];
+        // every load of the segment first: the owned steps' x, delta, and every
+        // step's B slice
+        float xo[kCk / G], vo[kCk / G];
+        float2 bv[kCk][NP];
 #pragma unroll
         for (int q = 0; q < kCk / G; ++q) {
             const int j = q * G + sub;
@@ -171,10 +162,12 @@ __global__ void __launch_bounds__(CC *G) s6_bwd_ckpt_kernel(const BwdArgs a) {
             vo[q] = ok ? to_f32(dt[(t0 + j) * D + dc]) : 0.0f;
         }
 #pragma unroll
-        for (int j = 0; j < kCk; ++j)
+        for (int j = 0; j < kCk; ++j) {
+            if (j < nst) load_pairs<NS>(Bm + (t0 + j) * N, bv[j]);
+            else
 #pragma unroll
-            for (int i = 0; i < NS; ++i)
-                bv[j][i] = j < nst ? to_f32(Bm[(t0 + j) * N + sub * NS + i]) : 0.0f;
+                for (int i = 0; i < NP; ++i) bv[j][i] = make_float2(0.0f, 0.0f);
+        }
 #pragma unroll
         for (int q = 0; q < kCk / G; ++q) {
             const float dl_o = delta_f32(vo[q], bias, sp);
@@ -186,7 +179,11 @@ __global__ void __launch_bounds__(CC *G) s6_bwd_ckpt_kernel(const BwdArgs a) {
                 const float dx = __shfl_sync(0xffffffffu, dx_o, gbase | jj);
                 if (j < nst) {
 #pragma unroll
-                    for (int i = 0; i < NS; ++i) h[i] = fmaf(ex2_mufu(dl * a2[i]), h[i], dx * bv[j][i]);
+                    for (int i = 0; i < NP; ++i) {
+                        const float2 arg = mul2(make_float2(dl, dl), a2[i]);
+                        const float2 ab = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+                        h[i] = fma2(ab, h[i], mul2(make_float2(dx, dx), bv[j][i]));
+                    }
                 }
             }
         }
@@ -194,35 +191,39 @@ __global__ void __launch_bounds__(CC *G) s6_bwd_ckpt_kernel(const BwdArgs a) {
 }
 
 // --------------------------------------------------------------- backward
-// Lanes that write the channel-reduced dB / dC values: after log2(V) splitting
-// rounds every further round only adds, so the lanes that differ in those
-// later bits hold the same sums and only the first of them writes.
-template <int V, int G>
-__device__ __forceinline__ bool bc_writer(int lane) {
-    constexpr int kSplit = (V >= 8 ? 3 : (V >= 4 ? 2 : (V >= 2 ? 1 : 0)));
-    return (G << kSplit) >= 32 || lane < (G << kSplit);
-}
+// Row stride (in words) of a warp's [channel][dB | dC] scratch: 2N values plus
+// padding chosen so that the lanes of one vector-store wavefront (the slices of
+// 2, 4 or 8 channels) land in distinct banks.
+template <int N, int G>
+struct BcScratch {
+    static constexpr int CW = 32 / G;
+    static constexpr int RS = N == 16 ? 48 : (N == 8 ? 24 : 12);
+    static constexpr int kWords = CW * RS;
+};
 
 // One segment of kCk steps (starting at tile step s0, `nst` of them valid),
 // recomputed from h_in and walked backwards.  Owner scalars come from the
-// stage's x / delta / z / dout tiles; B / C from the stage's [TT][N] tiles.
-// `part` is the warp's [TT][2N] slab of the CTA's dB | dC partial sums.
+// stage's x / delta / z / dout tiles; B / C slices from the stage's [TT][N]
+// tiles, one vector load each; the state math is on fp32 pairs.  `part` is
+// the warp's [TT][2N] slab of the CTA's dB | dC partial sums and `bcs` its
+// [CW][RS] scratch for summing one step over the warp's channels.
 template <bool FULL, bool SP, typename IoT, int N, int G, int CC>
 __device__ __forceinline__ void bwd_segment(
-    const float (&h_in)[N / G], float (&g)[N / G], float (&dA)[N / G], float &dD_acc,
-    float &dbias_acc, const float (&a2)[N / G], const float (&Araw)[N / G], float bias, float dskip,
-    const IoT *xs, const IoT *dts, const IoT *zs, const IoT *dos, const IoT *Bs, const IoT *Cs,
-    IoT *dxs, IoT *dds, IoT *dzs, float *part, int s0, int nst, int c_local, int sub, int gbase,
-    int lane) {
-    constexpr int NS = N / G, NQ = kCk / G, V = 2 * NS;
+    const float2 (&h_in)[N / G / 2], float2 (&g)[N / G / 2], float2 (&dA)[N / G / 2],
+    float &dD_acc, float &dbias_acc, const float2 (&a2)[N / G / 2], const float2 (&Araw)[N / G / 2],
+    float bias, float dskip, const IoT *xs, const IoT *dts, const IoT *zs, const IoT *dos,
+    const IoT *Bs, const IoT *Cs, IoT *dxs, IoT *dds, IoT *dzs, float *part, float *bcs, int s0,
+    int nst, int c_local, int sub, int gbase, int lane) {
+    constexpr int NS = N / G, NP = NS / 2, NQ = kCk / G;
+    using SC = BcScratch<N, G>;
     // ---- recompute: the state after every step of the segment, and the
     // steps' Delta and Delta x on every lane of the channel
-    float hs[kCk][NS];
+    float2 hs[kCk][NP];
     float dl[kCk], dxv[kCk];
     float dl_own[NQ], w_own[NQ], v_own[NQ];  // owned steps: Delta, e^{-|v|}, v
-    float h[NS];
+    float2 h[NP];
 #pragma unroll
-    for (int i = 0; i < NS; ++i) h[i] = h_in[i];
+    for (int i = 0; i < NP; ++i) h[i] = h_in[i];
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
         const int idx = (s0 + q * G + sub) * CC + c_local;
@@ -236,19 +237,25 @@ __device__ __forceinline__ void bwd_segment(
 #pragma unroll
         for (int jj = 0; jj < G; ++jj) {
             const int j = q * G + jj;
-            dl[j] = G == 1 ? dlo : __shfl_sync(0xffffffffu, dlo, gbase | jj);
-            dxv[j] = G == 1 ? dxo : __shfl_sync(0xffffffffu, dxo, gbase | jj);
+            dl[j] = __shfl_sync(0xffffffffu, dlo, gbase | jj);
+            dxv[j] = __shfl_sync(0xffffffffu, dxo, gbase | jj);
             if (FULL || j < nst) {
-                const IoT *bj = Bs + (s0 + j) * N + sub * NS;
+                float2 bv[NP];
+                load_pairs<NS>(Bs + (s0 + j) * N + sub * NS, bv);
 #pragma unroll
-                for (int i = 0; i < NS; ++i)
-                    h[i] = fmaf(ex2_mufu(dl[j] * a2[i]), h[i], dxv[j] * to_f32(bj[i]));
+                for (int i = 0; i < NP; ++i) {
+                    const float2 arg = mul2(make_float2(dl[j], dl[j]), a2[i]);
+                    const float2 ab = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+                    h[i] = fma2(ab, h[i], mul2(make_float2(dxv[j], dxv[j]), bv[i]));
+                }
             }
 #pragma unroll
-            for (int i = 0; i < NS; ++i) hs[j][i] = h[i];
+            for (int i = 0; i < NP; ++i) hs[j][i] = h[i];
         }
     }
     // ---- backward walk, groups of G steps from the last
+    const int c_in_warp = lane / G;
+    float *my_row = bcs + c_in_warp * SC::RS + sub * NS;
 #pragma unroll
     for (int q = NQ - 1; q >= 0; --q) {
         const int jo = q * G + sub;
@@ -263,38 +270,53 @@ __device__ __forceinline__ void bwd_segment(
 #pragma unroll
         for (int jj = G - 1; jj >= 0; --jj) {
             const int j = q * G + jj;
-            const float dy = G == 1 ? dy_o : __shfl_sync(0xffffffffu, dy_o, gbase | jj);
-            float bcv[V];
-            yp[jj] = 0.0f;
-            pa[jj] = 0.0f;
-            gb[jj] = 0.0f;
+            const float dy = __shfl_sync(0xffffffffu, dy_o, gbase | jj);
+            float2 dBp[NP], dCp[NP];
+            float2 y2 = make_float2(0.0f, 0.0f), pa2 = y2, gb2 = y2;
 #pragma unroll
-            for (int i = 0; i < V; ++i) bcv[i] = 0.0f;
+            for (int i = 0; i < NP; ++i) dBp[i] = dCp[i] = make_float2(0.0f, 0.0f);
             if (FULL || j < nst) {
-                const IoT *bj = Bs + (s0 + j) * N + sub * NS;
-                const IoT *cj = Cs + (s0 + j) * N + sub * NS;
+                float2 bv[NP], cv[NP];
+                load_pairs<NS>(Bs + (s0 + j) * N + sub * NS, bv);
+                load_pairs<NS>(Cs + (s0 + j) * N + sub * NS, cv);
+                const float2 dy2 = make_float2(dy, dy), dl2 = make_float2(dl[j], dl[j]);
+                const float2 dx2 = make_float2(dxv[j], dxv[j]);
 #pragma unroll
-                for (int i = 0; i < NS; ++i) {
-                    const float cv = to_f32(cj[i]), bv = to_f32(bj[i]);
-                    const float hprev = j > 0 ? hs[j - 1][i] : h_in[i];
-                    yp[jj] = fmaf(cv, hs[j][i], yp[jj]);
-                    g[i] = fmaf(dy, cv, g[i]);           // dL/dh_t: the readout's share
-                    bcv[NS + i] = dy * hs[j][i];         // dC_t[n], this channel
-                    const float abar = ex2_mufu(dl[j] * a2[i]);
-                    const float P = g[i] * hprev * abar;  // dL/dAbar * Abar
-                    pa[jj] = fmaf(P, Araw[i], pa[jj]);
-                    dA[i] = fmaf(P, dl[j], dA[i]);
-                    gb[jj] = fmaf(g[i], bv, gb[jj]);
-                    bcv[i] = g[i] * dxv[j];              // dB_t[n], this channel
-                    g[i] *= abar;                        // dL/dh_{t-1}
+                for (int i = 0; i < NP; ++i) {
+                    const float2 hprev = j > 0 ? hs[j - 1][i] : h_in[i];
+                    y2 = fma2(cv[i], hs[j][i], y2);
+                    g[i] = fma2(dy2, cv[i], g[i]);           // dL/dh_t: the readout's share
+                    dCp[i] = mul2(dy2, hs[j][i]);            // dC_t[n], this channel
+                    const float2 arg = mul2(dl2, a2[i]);
+                    const float2 ab = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+                    const float2 P = mul2(mul2(g[i], hprev), ab);  // dL/dAbar * Abar
+                    pa2 = fma2(P, Araw[i], pa2);
+                    dA[i] = fma2(P, dl2, dA[i]);
+                    gb2 = fma2(g[i], bv[i], gb2);
+                    dBp[i] = mul2(g[i], dx2);                // dB_t[n], this channel
+                    g[i] = mul2(g[i], ab);                   // dL/dh_{t-1}
                 }
             }
-            // dB / dC of this step summed over the warp's channels
-            const float s = reduce_channels<V, G>(bcv, lane);
-            if ((FULL || j < nst) && bc_writer<V, G>(lane)) {
-                const int vi = bc_index<V, G>(lane);
-                const int slot = (vi < NS ? 0 : N) + sub * NS + (vi % NS);
-                part[(s0 + j) * 2 * N + slot] = s;
+            yp[jj] = y2.x + y2.y;
+            pa[jj] = pa2.x + pa2.y;
+            gb[jj] = gb2.x + gb2.y;
+            // dB / dC of this step summed over the warp's channels, through the
+            // warp's scratch: each lane stores its slices, then lane k adds
+            // slot k over the channels
+            if (FULL || j < nst) {
+#pragma unroll
+                for (int i = 0; i < NP; ++i) {
+                    reinterpret_cast<float2 *>(my_row)[i] = dBp[i];
+                    reinterpret_cast<float2 *>(my_row + N)[i] = dCp[i];
+                }
+                __syncwarp();
+                if (lane < 2 * N) {
+                    float acc = bcs[lane];
+#pragma unroll
+                    for (int c = 1; c < SC::CW; ++c) acc += bcs[c * SC::RS + lane];
+                    part[(s0 + j) * 2 * N + lane] = acc;
+                }
+                __syncwarp();
             }
         }
         // the owner's totals for its step: y (pre-gate), sum P A, sum g B
@@ -338,6 +360,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
     uint64_t *out_free = out_full + NOUT;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffFlag);
     float *part_all = reinterpret_cast<float *>(smem + Cfg::kOffPart);
+    static_assert(Cfg::kScrWords == BcScratch<N, G>::kWords, "scratch layout");
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t b = blockIdx.y;
@@ -439,25 +462,30 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
     const int64_t d = c0 + c_local;
     const bool dvalid = d < D;
     const int64_t dc = dvalid ? d : D - 1;
-    float a2[NS], Araw[NS], g[NS], dA[NS];
+    constexpr int NP = NS / 2;
+    float2 a2[NP], Araw[NP], g[NP], dA[NP];
 #pragma unroll
-    for (int i = 0; i < NS; ++i) {
-        Araw[i] = __ldg(a.A + dc * N + sub * NS + i);
-        a2[i] = Araw[i] * kLog2e;
-        g[i] = a.dh_final ? __ldg(a.dh_final + (b * D + dc) * N + sub * NS + i) : 0.0f;
-        dA[i] = 0.0f;
+    for (int i = 0; i < NP; ++i) {
+        const int n = sub * NS + 2 * i;
+        Araw[i] = make_float2(__ldg(a.A + dc * N + n), __ldg(a.A + dc * N + n + 1));
+        a2[i] = make_float2(Araw[i].x * kLog2e, Araw[i].y * kLog2e);
+        g[i] = a.dh_final ? make_float2(__ldg(a.dh_final + (b * D + dc) * N + n),
+                                        __ldg(a.dh_final + (b * D + dc) * N + n + 1))
+                          : make_float2(0.0f, 0.0f);
+        dA[i] = make_float2(0.0f, 0.0f);
     }
     const float bias = a.delta_bias ? __ldg(a.delta_bias + dc) : 0.0f;
     const float dskip = a.D ? __ldg(a.D + dc) : 0.0f;
     float dD_acc = 0.0f, dbias_acc = 0.0f;
     float *part = part_all + warp * TT * 2 * N;
+    float *bcs = reinterpret_cast<float *>(smem + Cfg::kOffScr) + warp * Cfg::kScrWords;
     // checkpoints are consumed from the last to the first; the next one is
     // loaded one segment ahead
     const float *ck = a.ckpt + (b * nck * D + dc) * N + sub * NS;  // + c * D * N
     int64_t c_next = nck - 1;
-    float hnext[NS];
+    float2 hnext[NP];
 #pragma unroll
-    for (int i = 0; i < NS; ++i) hnext[i] = ck[c_next * D * N + i];
+    for (int i = 0; i < NP; ++i) hnext[i] = *reinterpret_cast<const float2 *>(ck + c_next * D * N + 2 * i);
 
     // Every compute warp makes every iteration and reaches both named
     // barriers of each, doing the work only while nothing has aborted.
@@ -488,24 +516,25 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             const int nseg = (nsteps + kCk - 1) / kCk;
 #pragma unroll 1
             for (int sg = nseg - 1; sg >= 0; --sg) {
-                float hcur[NS];
+                float2 hcur[NP];
 #pragma unroll
-                for (int i = 0; i < NS; ++i) hcur[i] = hnext[i];
+                for (int i = 0; i < NP; ++i) hcur[i] = hnext[i];
                 if (c_next > 0) {
                     --c_next;
 #pragma unroll
-                    for (int i = 0; i < NS; ++i) hnext[i] = ck[c_next * D * N + i];
+                    for (int i = 0; i < NP; ++i)
+                        hnext[i] = *reinterpret_cast<const float2 *>(ck + c_next * D * N + 2 * i);
                 }
                 const int rem = nsteps - sg * kCk;
                 if (rem >= kCk)
                     bwd_segment<true, SP, IoT, N, G, CC>(hcur, g, dA, dD_acc, dbias_acc, a2, Araw,
                                                          bias, dskip, xs, dts, zs, dos, Bs, Cs, dxs,
-                                                         dds, dzs, part, sg * kCk, kCk, c_local, sub,
-                                                         gbase, lane);
+                                                         dds, dzs, part, bcs, sg * kCk, kCk, c_local,
+                                                         sub, gbase, lane);
                 else
                     bwd_segment<false, SP, IoT, N, G, CC>(hcur, g, dA, dD_acc, dbias_acc, a2, Araw,
                                                           bias, dskip, xs, dts, zs, dos, Bs, Cs,
-                                                          dxs, dds, dzs, part, sg * kCk, rem,
+                                                          dxs, dds, dzs, part, bcs, sg * kCk, rem,
                                                           c_local, sub, gbase, lane);
             }
             mbar_arrive(&empty[s]);    // the input stage may be refilled
@@ -536,14 +565,20 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
     if (dvalid) {
         float *pp = a.part_par + (b * D + d) * (N + 2);
 #pragma unroll
-        for (int i = 0; i < NS; ++i) pp[sub * NS + i] = dA[i];
+        for (int i = 0; i < NP; ++i) {
+            pp[sub * NS + 2 * i] = dA[i].x;
+            pp[sub * NS + 2 * i + 1] = dA[i].y;
+        }
         if (sub == 0) {
             pp[N] = dD_sum;
             pp[N + 1] = db_sum;
         }
         if (a.dh0) {
 #pragma unroll
-            for (int i = 0; i < NS; ++i) a.dh0[(b * D + d) * N + sub * NS + i] = g[i];
+            for (int i = 0; i < NP; ++i) {
+                a.dh0[(b * D + d) * N + sub * NS + 2 * i] = g[i].x;
+                a.dh0[(b * D + d) * N + sub * NS + 2 * i + 1] = g[i].y;
+            }
         }
     }
 }

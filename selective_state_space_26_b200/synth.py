@@ -167,6 +167,49 @@ def decode_step(batch: int, d_inner: int, d_state: int, step: int, seed: int,
                       B=draw(d_state, T_B), C=draw(d_state, T_C))
 
 
+@dataclasses.dataclass
+class SsdInputs:
+    x: torch.Tensor           # [batch, seqlen, nheads * headdim]
+    delta: torch.Tensor       # [batch, seqlen, nheads]
+    z: torch.Tensor
+    B: torch.Tensor           # [batch, seqlen, d_state]
+    C: torch.Tensor
+    A: torch.Tensor           # [nheads] fp32
+    D: torch.Tensor           # [nheads * headdim] fp32
+    delta_bias: torch.Tensor  # [nheads] fp32
+    h0: torch.Tensor | None
+    delta_softplus: bool = True
+
+
+def ssd_inputs(batch: int, seqlen: int, nheads: int, headdim: int, d_state: int,
+               dtype=torch.bfloat16, seed: int = 0, device="cpu", h0_std: float = 0.0,
+               seq_offset: int = 0) -> SsdInputs:
+    """Inputs of the scalar-identity (Mamba-2) scan, drawn like the diagonal
+    scan's: x, z, delta, B, C ~ N(0, 1) rounded to the I/O dtype (delta one
+    column per head), a per-head bias that centres Delta on a log-uniform dt0,
+    A[head] = -U(1, 16) (a head's decay rate; Mamba-2 draws its A in that
+    range), D = 1."""
+    dev = torch.device(device)
+    d_inner = nheads * headdim
+
+    def act(width, tensor):
+        t = torch.empty(batch, seqlen, width, dtype=dtype, device=dev)
+        for b in range(batch):
+            _fill_sequence(t[b], seed, tensor, seq_offset + b)
+        return t
+    x, dt, z = act(d_inner, T_X), act(nheads, T_DT), act(d_inner, T_Z)
+    Bm, Cm = act(d_state, T_B), act(d_state, T_C)
+    g = _gen("cpu", counter_seed(seed, T_A, 1, 0))
+    A = -(1.0 + 15.0 * torch.rand(nheads, generator=g, dtype=torch.float32))
+    h0 = None
+    if h0_std > 0:
+        h0 = torch.stack([normal((d_inner, d_state), seed, T_H0, seq_offset + b, 0, dev,
+                                 std=h0_std) for b in range(batch)])
+    return SsdInputs(x=x, delta=dt, z=z, B=Bm, C=Cm, A=A.to(dev),
+                     D=torch.ones(d_inner, dtype=torch.float32, device=dev),
+                     delta_bias=dt_bias_for(nheads, seed).to(dev), h0=h0)
+
+
 # Named workloads (the S6 layer at Jamba's sizes, plus a tiny fp32 case).
 @dataclasses.dataclass(frozen=True)
 class Workload:

@@ -1,0 +1,126 @@
+"""Parity of the scalar-identity (Mamba-2) scan kernel with the fp64 oracle's
+ssd_scan (needs a B200), under the layer's comparison rules (tests/parity.py),
+and its agreement with the diagonal scan kernel when the diagonal scan's
+parameters are tied across each head."""
+import os
+
+import pytest
+import torch
+
+import oracle
+from selective_state_space_26_b200 import (_lib, jamba_ssm_get_status, jamba_ssm_scan,
+                                           jamba_ssm_ssd_scan, synth)
+from tests.parity import assert_out, assert_state, compare_out
+
+pytestmark = pytest.mark.gpu
+THREADS = max(1, min(32, os.cpu_count() or 1))
+
+
+def _dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda", 0)
+
+
+def _gpu(inp, **kw):
+    out, hf = jamba_ssm_ssd_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, D=inp.D,
+                                 delta_bias=inp.delta_bias, delta_softplus=inp.delta_softplus,
+                                 h0=inp.h0, **kw)
+    torch.cuda.synchronize()
+    return out, hf
+
+
+def _oracle(inp):
+    return oracle.ssd_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, inp.A.shape[0],
+                           D=inp.D, delta_bias=inp.delta_bias, delta_softplus=inp.delta_softplus,
+                           h0=inp.h0, threads=THREADS)
+
+
+@pytest.mark.parametrize("dtype,n", [(torch.bfloat16, 16), (torch.bfloat16, 8),
+                                     (torch.float32, 16), (torch.float32, 8)])
+def test_ssd_matches_oracle_ragged(dtype, n):
+    """Several 64-step tiles and a ragged tail, 8 heads of 64 channels (two
+    CTAs per head), two sequences, a nonzero initial state."""
+    dev = _dev()
+    inp = synth.ssd_inputs(2, 203, 8, 64, n, dtype, seed=71, device=dev, h0_std=0.5)
+    out, hf = _gpu(inp)
+    ref, ref_h = _oracle(inp)
+    assert_out(out, ref, dtype, f"ssd {dtype} N={n}")
+    assert_state(hf, ref_h, dtype, f"ssd {dtype} N={n}")
+
+
+@pytest.mark.parametrize("seqlen", [1, 63, 64, 65])
+def test_ssd_boundary_lengths_and_heads_of_32(seqlen):
+    dev = _dev()
+    inp = synth.ssd_inputs(1, seqlen, 16, 32, 16, torch.bfloat16, seed=72, device=dev, h0_std=0.3)
+    out, hf = _gpu(inp)
+    ref, ref_h = _oracle(inp)
+    assert_out(out, ref, torch.bfloat16, f"L={seqlen}")
+    assert_state(hf, ref_h, torch.bfloat16, f"L={seqlen}")
+
+
+def test_ssd_without_softplus_split_and_empty():
+    dev = _dev()
+    inp = synth.ssd_inputs(1, 150, 8, 32, 16, torch.bfloat16, seed=73, device=dev, h0_std=0.3)
+    inp.delta.copy_((inp.delta.float().abs() * 0.05).to(torch.bfloat16))
+    inp.delta_bias.fill_(0.01)
+    inp.delta_softplus = False
+    out, hf = _gpu(inp)
+    ref, ref_h = _oracle(inp)
+    assert_out(out, ref, torch.bfloat16, "no softplus")
+    # chunked: the first 70 steps, then the rest from their final state, is the whole scan
+    cut = 70
+    part = lambda t, sl: t[:, sl].contiguous()  # noqa: E731
+    a = synth.SsdInputs(*(part(getattr(inp, k), slice(0, cut)) for k in ("x", "delta", "z", "B", "C")),
+                        inp.A, inp.D, inp.delta_bias, inp.h0, False)
+    o1, h1 = _gpu(a)
+    b = synth.SsdInputs(*(part(getattr(inp, k), slice(cut, None)) for k in ("x", "delta", "z", "B", "C")),
+                        inp.A, inp.D, inp.delta_bias, h1, False)
+    o2, h2 = _gpu(b)
+    assert torch.equal(torch.cat([o1, o2], 1), out) and torch.equal(h2, hf)
+    e = synth.ssd_inputs(1, 0, 8, 32, 16, torch.bfloat16, seed=74, device=dev, h0_std=1.0)
+    _, he = _gpu(e)
+    assert torch.equal(he, e.h0)
+
+
+def test_ssd_agrees_with_the_diagonal_kernel_on_tied_parameters():
+    """The diagonal scan with A[d, n] = A[head(d)] and Delta[t, d] = Delta[t,
+    head(d)] is the same map; the two kernels agree under the bf16 rule."""
+    dev = _dev()
+    H, P, N = 8, 64, 16
+    inp = synth.ssd_inputs(1, 130, H, P, N, torch.bfloat16, seed=75, device=dev, h0_std=0.2)
+    out, hf = _gpu(inp)
+    head = torch.arange(H * P, device=dev) // P
+    A_diag = inp.A[head][:, None].expand(H * P, N).contiguous()
+    out_d, hf_d = jamba_ssm_scan(inp.x, inp.delta[:, :, head].contiguous(), inp.z, inp.B, inp.C,
+                                 A_diag, D=inp.D, delta_bias=inp.delta_bias[head].contiguous(),
+                                 h0=inp.h0)
+    torch.cuda.synchronize()
+    m = compare_out(out, out_d.double(), torch.bfloat16)
+    assert m["ok"], m
+    assert_state(hf, hf_d, torch.bfloat16, "tied parameters")
+
+
+def test_ssd_full_size_jamba_width():
+    """Jamba's layer width as 128 heads of 64 channels, d_state 16, 4096
+    tokens: every output against the oracle."""
+    dev = _dev()
+    inp = synth.ssd_inputs(1, 4096, 128, 64, 16, torch.bfloat16, seed=76, device=dev)
+    out, hf = _gpu(inp)
+    ref, ref_h = _oracle(inp)
+    assert_out(out, ref, torch.bfloat16, "ssd full size")
+    assert_state(hf, ref_h, torch.bfloat16, "ssd full size")
+
+
+def test_ssd_deterministic_and_timeout():
+    dev = _dev()
+    inp = synth.ssd_inputs(2, 140, 8, 32, 16, torch.bfloat16, seed=77, device=dev)
+    a = _gpu(inp)
+    b = _gpu(inp)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    assert jamba_ssm_get_status() == _lib.OK
+    _gpu(inp, debug_flags=1, timeout_cycles=2_000_000)
+    assert jamba_ssm_get_status() == _lib.ERR_TIMEOUT
+    assert jamba_ssm_get_status() == _lib.OK
+    c = _gpu(inp)
+    assert torch.equal(c[0], a[0])
