@@ -67,11 +67,17 @@ def bf16_peak():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_source_hash(unit: str = "jamba_ssm.cu"):
-    """Hash of the sources of one translation unit of the library: the .cu
-    file and every csrc header it includes, directly or not."""
+# The device code of each kernel whose DRAM traffic is recorded: its header
+# and every csrc header that header includes, directly or not.
+KERNEL_HEADER = {"s6_scan_fused_kernel": "s6_scan_fused.cuh",
+                 "s6_state_update_kernel": "s6_state_update.cuh",
+                 "s6_ssd_kernel": "s6_ssd.cuh"}
+
+
+def kernel_source_hash(kernel: str):
+    """Hash of the device sources of one kernel (KERNEL_HEADER's closure)."""
     d = os.path.join(ROOT, "selective_state_space_26_b200", "csrc")
-    files, todo = set(), [unit]
+    files, todo = set(), [KERNEL_HEADER[kernel]]
     while todo:
         f = todo.pop()
         if f in files or not os.path.exists(os.path.join(d, f)):
@@ -86,19 +92,30 @@ def kernel_source_hash(unit: str = "jamba_ssm.cu"):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, workload: str):
+def plan_launch(plan):
+    """A scan plan's launch shape, as recorded beside the traffic it was taken on."""
+    if not plan:
+        return None
+    return (f"variant {plan['variant']}, grid {plan['grid']}, "
+            f"{plan['channels_per_cta']} channels per CTA")
+
+
+def recorded_traffic(kernel: str, workload: str, launch=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    the current device code of the kernel and (when given) the same launch
+    shape; else None."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
         r = rec[kernel][workload]
-        if r.get("source_hash") == kernel_source_hash():
-            return float(r["bytes_per_launch"])
+        if r.get("source_hash") != kernel_source_hash(kernel):
+            return None
+        if launch is not None and r.get("launch") != launch:
+            return None
+        return float(r["bytes_per_launch"])
     except Exception:
-        pass
-    return None
+        return None
 
 
 def prefill_bytes(batch, seqlen, d_inner, d_state, io_bytes):
@@ -434,6 +451,10 @@ def profile_one(args):
     elif args.kernel == "dt_proj":
         dp = synth.dt_proj_inputs(4096, 8192, 256, seed=5, device=dev)
         fn = lambda: jssm.jamba_ssm_dt_proj(dp.hi, dp.W_dt, dt_low_lo=dp.lo)  # noqa
+    elif args.kernel == "ssd":
+        sd = synth.ssd_inputs(1, 4096, 128, 64, 16, torch.bfloat16, seed=6, device=dev)
+        fn = lambda: jssm.jamba_ssm_ssd_scan(sd.x, sd.delta, sd.z, sd.B, sd.C, sd.A,  # noqa
+                                             D=sd.D, delta_bias=sd.delta_bias)
     else:
         raise ValueError(f"unknown kernel {args.kernel}")
     for _ in range(args.warmup + args.steps):
@@ -629,7 +650,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- roofline of the dominant kernel
     hbm_gbs, sm_mhz_peak, peak_kind = peaks()
     clocks = clk.summary()
-    traffic = recorded_traffic(dom_name, w.name)
+    traffic = recorded_traffic(dom_name, w.name, plan_launch(plan))
     if w.kind == "prefill":
         ops = exp_ops(w.batch * w.seqlen, w.d_inner, w.d_state)
         peak = sms * MUFU_OPS_PER_CLK_PER_SM * sm_mhz_peak * 1e6 / 1e12
@@ -809,7 +830,7 @@ def main():
     ap.add_argument("--pw-reps", type=int, default=3,
                     help="timed launches of each other configuration")
     ap.add_argument("--kernel", default=None,
-                    choices=["scan", "scan_bwd", "x_proj", "dt_proj"],
+                    choices=["scan", "scan_bwd", "x_proj", "dt_proj", "ssd"],
                     help="profiling aid: launch only this kernel (warmup + steps times), "
                          "print nothing")
     args = ap.parse_args()

@@ -148,6 +148,12 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
+// The lanes of a warp agree on the outcome of their waits: true only if every
+// lane saw true.  A wait can end one way in one lane and the other way in the
+// next (the phase completes just as another warp raises the abort flag); the
+// shuffles that follow a wait must then not run with part of the warp gone.
+__device__ __forceinline__ bool warp_agree(bool v) { return __all_sync(0xffffffffu, v) != 0; }
+
 // ----------------------------------------------------------------------- TMA
 // 3-D tiled load global -> shared, completion signalled on `bar` (bytes).
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1,

@@ -115,12 +115,14 @@ struct ScanVariant {
     int smem, smem_serving;
     const void *kernel;          // batched layout
     const void *kernel_serving;  // packed layout and / or state-cache slots
+    const void *kernel_ckpt;     // the backward's checkpoint pass, or null
+    bool attr_set_ckpt[kMaxDevices];
     bool attr_set[kMaxDevices], attr_set_serving[kMaxDevices];
 };
 
 // NW compute warps (each does its channels' recurrence, softplus and gate) and
 // one producer warp (TMA, B/C widening).
-template <typename IoT, int N, int G, int NW, int TT, int S>
+template <typename IoT, int N, int G, int NW, int TT, int S, bool CKPT = false>
 ScanVariant make_fused(double step_cost) {
     using Cfg = jssm::FusedCfg<IoT, N, G, NW, TT, S>;
     ScanVariant v{};
@@ -137,6 +139,9 @@ ScanVariant make_fused(double step_cost) {
     v.kernel = reinterpret_cast<const void *>(&jssm::s6_scan_fused_kernel<IoT, N, G, NW, TT, S>);
     v.kernel_serving =
         reinterpret_cast<const void *>(&jssm::s6_scan_serving_kernel<IoT, N, G, NW, TT, S>);
+    if (CKPT)
+        v.kernel_ckpt =
+            reinterpret_cast<const void *>(&jssm::s6_scan_fused_kernel<IoT, N, G, NW, TT, S, true>);
     return v;
 }
 
@@ -145,18 +150,21 @@ ScanVariant make_fused(double step_cost) {
 // is busy (measured on B200 at Jamba's sizes, bf16 I/O; the fp32 ones serve
 // small and test shapes).  Fewer lanes per channel cost less per step; more
 // lanes give narrower CTAs, so a single sequence's 8192 channels still cover
-// the 148 SMs (56 channels per CTA -> 147 CTAs).
+// the 148 SMs (56 channels per CTA -> 147 CTAs).  The variants marked `true`
+// also serve the backward's checkpoint pass (the states alone, stored every
+// kCk steps), chosen by the same cost model.
 ScanVariant g_variants[] = {
-    make_fused<__nv_bfloat16, 16, 2, 8, 64, 2>(1.00),   // 1: 128 channels / CTA
-    make_fused<__nv_bfloat16, 16, 4, 7, 64, 3>(1.33),   // 2:  56 channels / CTA
-    make_fused<__nv_bfloat16, 16, 4, 8, 64, 3>(1.35),   // 3:  64 channels / CTA
-    make_fused<__nv_bfloat16, 16, 4, 7, 32, 4>(1.47),   // 4:  56 channels / CTA
-    make_fused<__nv_bfloat16, 8, 2, 8, 32, 4>(1.00),    // 5: 128 channels / CTA
-    make_fused<__nv_bfloat16, 8, 1, 4, 32, 4>(1.70),    // 6: 128 channels / CTA
-    make_fused<__nv_bfloat16, 8, 4, 7, 64, 3>(1.29),    // 7:  56 channels / CTA
-    make_fused<float, 16, 1, 2, 32, 3>(1.00),           // 8:  64 channels / CTA
-    make_fused<float, 8, 1, 2, 32, 3>(1.00),            // 9:  64 channels / CTA
-    make_fused<float, 4, 1, 2, 32, 3>(1.00),            // 10: 64 channels / CTA
+    make_fused<__nv_bfloat16, 16, 2, 8, 64, 2, true>(1.00),  // 1: 128 channels / CTA
+    make_fused<__nv_bfloat16, 16, 4, 7, 64, 3, true>(1.33),  // 2:  56 channels / CTA
+    make_fused<__nv_bfloat16, 16, 4, 8, 64, 3>(1.35),        // 3:  64 channels / CTA
+    make_fused<__nv_bfloat16, 16, 4, 7, 32, 4>(1.47),        // 4:  56 channels / CTA
+    make_fused<__nv_bfloat16, 8, 2, 8, 32, 4, true>(1.00),   // 5: 128 channels / CTA
+    make_fused<__nv_bfloat16, 8, 1, 4, 32, 4>(1.70),         // 6: 128 channels / CTA
+    make_fused<__nv_bfloat16, 8, 4, 7, 64, 3, true>(1.29),   // 7:  56 channels / CTA
+    make_fused<float, 16, 1, 2, 32, 3, true>(1.00),          // 8:  64 channels / CTA
+    make_fused<float, 8, 1, 2, 32, 3, true>(1.00),           // 9:  64 channels / CTA
+    make_fused<float, 4, 1, 2, 32, 3, true>(1.00),           // 10: 64 channels / CTA
+    make_fused<__nv_bfloat16, 16, 8, 14, 64, 3>(1.40),       // 11:  56 channels / CTA
 };
 constexpr int kNumVariants = sizeof(g_variants) / sizeof(g_variants[0]);
 
@@ -184,11 +192,12 @@ double variant_cost(const ScanVariant &v, const jamba_ssm_scan_params *p, int sm
     return double(per_cta) * cc * v.step_cost;
 }
 
-int choose_variant(const jamba_ssm_scan_params *p, int sms) {
+int choose_variant(const jamba_ssm_scan_params *p, int sms, bool ckpt = false) {
     int best = -1;
     double best_cost = 0;
     for (int i = 0; i < kNumVariants; ++i) {
         if (!variant_applies(g_variants[i], p)) continue;
+        if (ckpt && !g_variants[i].kernel_ckpt) continue;
         const double c = variant_cost(g_variants[i], p, sms);
         if (best < 0 || c < best_cost) {
             best = i;
@@ -329,7 +338,6 @@ bool bwd_shape(int io_dtype, int64_t n, BwdShape *s) {
     else return false;
     return true;
 }
-constexpr int kCkChannels = 32;  // channels per block of the checkpoint pass
 
 // Workspace of the backward: the status block, then the checkpoints, the
 // per-CTA dB | dC partials and the per-sequence parameter partials.
@@ -350,7 +358,7 @@ BwdLayout bwd_layout(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_s
 }
 
 struct BwdKernels {
-    const void *ckpt, *bwd, *reduce;
+    const void *bwd, *reduce;
     int smem;
     bool attr[kMaxDevices];
 };
@@ -358,7 +366,6 @@ struct BwdKernels {
 template <typename IoT, int N, int G, int NW, int TT, bool SP>
 BwdKernels make_bwd() {
     BwdKernels k{};
-    k.ckpt = reinterpret_cast<const void *>(&jssm::s6_bwd_ckpt_kernel<IoT, N, G, kCkChannels>);
     k.bwd = reinterpret_cast<const void *>(&jssm::s6_bwd_kernel<IoT, N, G, NW, TT, SP>);
     k.reduce = reinterpret_cast<const void *>(&jssm::s6_bwd_reduce_kernel<IoT, N>);
     k.smem = jssm::BwdCfg<IoT, N, G, NW, TT>::kSmemBytes;
@@ -839,10 +846,8 @@ jamba_ssm_status jamba_ssm_scan_bwd(const jamba_ssm_scan_bwd_params *p, void *st
     a.h0 = p->h0;
     a.dh_final = p->dh_final;
     a.delta_softplus = p->delta_softplus != 0;
-    a.x = p->x;
-    a.delta = p->delta;
-    a.B = p->B;
-    a.ckpt = reinterpret_cast<float *>(ws + lay.off_ckpt);
+    float *ckpt = reinterpret_cast<float *>(ws + lay.off_ckpt);
+    a.ckpt = ckpt;
     a.part_bc = reinterpret_cast<float *>(ws + lay.off_bc);
     a.part_par = reinterpret_cast<float *>(ws + lay.off_par);
     a.dh0 = p->dh0;
@@ -850,18 +855,61 @@ jamba_ssm_status jamba_ssm_scan_bwd(const jamba_ssm_scan_bwd_params *p, void *st
     a.debug_flags = p->debug_flags;
     a.timeout_cycles = p->timeout_cycles ? p->timeout_cycles : (uint64_t(1) << 31);
 
-    // 1. checkpoints
+    const CUtensorMapDataType dt = p->io_dtype == JAMBA_SSM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                                 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    // 1. checkpoints: the forward kernel in its checkpoint mode, the variant
+    //    the forward's cost model picks for this shape
     {
-        const dim3 grid(static_cast<unsigned>((p->d_inner + kCkChannels - 1) / kCkChannels),
-                        static_cast<unsigned>(p->batch));
-        void *kargs[] = {&a};
-        e = cudaLaunchKernel(K.ckpt, grid, dim3(kCkChannels * sh.g), kargs, 0, s);
+        jamba_ssm_scan_params fp{};
+        fp.struct_size = sizeof(fp);
+        fp.batch = p->batch;
+        fp.seqlen = p->seqlen;
+        fp.d_inner = p->d_inner;
+        fp.d_state = p->d_state;
+        fp.io_dtype = p->io_dtype;
+        const int vi = choose_variant(&fp, dev->sms, true);
+        if (vi < 0) return JAMBA_SSM_ERR_UNSUPPORTED;
+        ScanVariant &v = g_variants[vi];
+        const int cc = channels_per_cta(v);
+        CUtensorMap maps[6];
+        if (!encode_3d(fn, &maps[0], p->x, dt, es, p->d_inner, p->seqlen, p->batch, cc, v.tt) ||
+            !encode_3d(fn, &maps[1], p->delta, dt, es, p->d_inner, p->seqlen, p->batch, cc, v.tt) ||
+            !encode_3d(fn, &maps[3], p->B, dt, es, p->d_state, p->seqlen, p->batch, (int)p->d_state,
+                       v.tt))
+            return JAMBA_SSM_ERR_UNSUPPORTED;
+        maps[2] = maps[0];  // z, C and the output are not read or written in this mode
+        maps[4] = maps[3];
+        maps[5] = maps[0];
+        {
+            std::lock_guard<std::mutex> lock(g_mutex);
+            if (!v.attr_set_ckpt[devid]) {
+                e = cudaFuncSetAttribute(v.kernel_ckpt, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         v.smem);
+                if (e != cudaSuccess) return cuda_fail(e);
+                v.attr_set_ckpt[devid] = true;
+            }
+        }
+        jssm::ScanArgs fa{};
+        fa.batch = p->batch;
+        fa.seqlen = p->seqlen;
+        fa.d_inner = p->d_inner;
+        fa.A = p->A;
+        fa.delta_bias = p->delta_bias;
+        fa.h0 = p->h0;
+        fa.delta_softplus = p->delta_softplus != 0;
+        fa.debug_flags = p->debug_flags;
+        fa.timeout_cycles = a.timeout_cycles;
+        fa.status = status;
+        fa.ckpt = ckpt;
+        const int64_t tasks = p->batch * ((p->d_inner + cc - 1) / cc);
+        const int grid = static_cast<int>(tasks < dev->sms ? tasks : dev->sms);
+        void *kargs[] = {&maps[0], &maps[1], &maps[2], &maps[3], &maps[4], &maps[5], &fa};
+        e = cudaLaunchKernel(v.kernel_ckpt, dim3(grid < 1 ? 1 : grid), dim3(v.threads), kargs,
+                             static_cast<size_t>(v.smem), s);
         if (e != cudaSuccess) return cuda_fail(e);
     }
     // 2. the reverse walk
     {
-        const CUtensorMapDataType dt = p->io_dtype == JAMBA_SSM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
         jssm::BwdMaps m;
         CUtensorMap *acts[] = {&m.x, &m.dt, &m.z, &m.dout, &m.dx, &m.ddt, &m.dz};
         const void *aptr[] = {p->x, p->delta, p->z, p->dout, p->dx, p->ddelta, p->dz};

@@ -16,6 +16,9 @@
 
 namespace jssm {
 
+// Steps between the backward's checkpoints (and the length of its segments).
+constexpr int kCk = 16;
+
 struct ScanArgs {
     int64_t batch, seqlen, d_inner;
     const float *A, *D, *delta_bias, *h0;
@@ -29,7 +32,15 @@ struct ScanArgs {
     int64_t num_slots;         // rows of the state cache
     void *out;                 // output base (row-wise stores of short packed tiles)
     int *status;               // the call's status word (caller workspace), or null
+    float *ckpt;               // checkpoint pass: [batch, ceil(seqlen / kCk), d_inner, N]
 };
+
+// A lane's NS states (fp32 pairs) to global memory.
+template <int NS>
+__device__ __forceinline__ void store_states(float *dst, const float2 (&h)[NS / 2]) {
+#pragma unroll
+    for (int i = 0; i < NS / 2; ++i) reinterpret_cast<float2 *>(dst)[i] = h[i];
+}
 
 // No steps at all (every sequence empty) with a state cache: final state =
 // initial state (or zeros) for each sequence's slot; one thread per float.
@@ -78,6 +89,51 @@ __device__ __forceinline__ BCPairs<NS> load_bc(const float *row, int sub) {
         r.c[i] = make_float2(f[NS + 2 * i], f[NS + 2 * i + 1]);
     }
     return r;
+}
+
+// The same slot read with explicit shared-space loads, and explicit
+// shared-space accesses of the bf16 / fp32 activation tiles.  Kept in program
+// order (volatile) and named as shared memory rather than left to generic
+// addressing; with 2 lanes per channel the tile loop ran 2-4% faster this way
+// on B200, with 4 lanes 2% slower, so only the 2-lane form uses them.
+template <int NS>
+__device__ __forceinline__ BCPairs<NS> load_bc_shared(const float *row, int sub) {
+    const uint32_t a = smem_u32(row + sub * 2 * NS);
+    float f[2 * NS];
+#pragma unroll
+    for (int q = 0; q < NS / 2; ++q) {
+        float4 v;
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                     : "r"(a + 16 * q));
+        f[4 * q] = v.x;
+        f[4 * q + 1] = v.y;
+        f[4 * q + 2] = v.z;
+        f[4 * q + 3] = v.w;
+    }
+    BCPairs<NS> r;
+#pragma unroll
+    for (int i = 0; i < NS / 2; ++i) {
+        r.b[i] = make_float2(f[2 * i], f[2 * i + 1]);
+        r.c[i] = make_float2(f[NS + 2 * i], f[NS + 2 * i + 1]);
+    }
+    return r;
+}
+__device__ __forceinline__ float lds_f32(const __nv_bfloat16 *p) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_u32(p)));
+    return __uint_as_float(uint32_t(v) << 16);
+}
+__device__ __forceinline__ float lds_f32(const float *p) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(smem_u32(p)));
+    return v;
+}
+__device__ __forceinline__ void sts_io(__nv_bfloat16 *p, __nv_bfloat16 v) {
+    asm volatile("st.shared.b16 [%0], %1;" ::"r"(smem_u32(p)), "h"(__bfloat16_as_ushort(v)));
+}
+__device__ __forceinline__ void sts_io(float *p, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(smem_u32(p)), "f"(v));
 }
 
 // One B or C slice of NS values from the TMA tile into its staged slot: a

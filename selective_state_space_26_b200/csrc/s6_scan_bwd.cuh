@@ -17,8 +17,9 @@
 // derivative the fp64 oracle's scan_bwd takes, step for step.)
 //
 // Three kernels, all deterministic (no atomics, fixed summation orders):
-//  1. s6_bwd_ckpt_kernel: the forward recurrence once more, storing the state
-//     before every kCk-th step (the checkpoints) in the workspace.
+//  1. the checkpoint pass: the forward kernel (s6_scan_fused_kernel) in its
+//     checkpoint mode runs the recurrence once more, TMA-fed, storing the
+//     state before every kCk-th step in the workspace (no readout, no output).
 //  2. s6_bwd_kernel: per (sequence, channel group), 64-step tiles from the last
 //     to the first, fed by TMA (x, delta, z, dout, B, C) like the forward.  In
 //     each tile, segments of kCk steps from the last to the first: the lanes
@@ -45,14 +46,11 @@
 
 namespace jssm {
 
-constexpr int kCk = 16;  // steps between checkpoints (= the backward's segment)
-
 struct BwdArgs {
     int64_t batch, seqlen, d_inner;
     const float *A, *D, *delta_bias, *h0, *dh_final;
     int delta_softplus;
-    const void *x, *delta, *B;  // for the checkpoint pass (plain loads of B)
-    float *ckpt;                // [batch, nck, d_inner, N] fp32
+    const float *ckpt;          // [batch, nck, d_inner, N] fp32, from the checkpoint pass
     float *part_bc;             // [batch, ngroups, seqlen, 2N] fp32: CTA partials of dB | dC
     float *part_par;            // [batch, d_inner, N + 2] fp32: dA[N], dD, dbias per sequence
     float *dh0;                 // [batch, d_inner, N] or null
@@ -106,87 +104,6 @@ __device__ __forceinline__ void load_pairs(const float *p, float2 (&v)[NS / 2]) 
     } else {
         static_assert(NS == 2, "two or four values");
         v[0] = *reinterpret_cast<const float2 *>(p);
-    }
-}
-
-// ------------------------------------------------------------ checkpoints
-// grid (ceil(d_inner / CC), batch), threads CC * G: thread (d, sub) carries
-// NS states of channel d through the whole sequence and stores them before
-// every kCk-th step.  Plain loads: x, delta of the owned step per lane (the
-// G lanes of a channel own consecutive steps), B slices broadcast over the
-// warp; each segment's loads are issued before its arithmetic.
-template <typename IoT, int N, int G, int CC>
-__global__ void __launch_bounds__(CC *G) s6_bwd_ckpt_kernel(const BwdArgs a) {
-    constexpr int NS = N / G, NP = NS / 2;
-    const int lane = threadIdx.x & 31, sub = lane % G;
-    const int gbase = lane & ~(G - 1);
-    const int64_t b = blockIdx.y;
-    const int64_t d = static_cast<int64_t>(blockIdx.x) * CC + threadIdx.x / G;
-    const bool dvalid = d < a.d_inner;
-    const int64_t dc = dvalid ? d : a.d_inner - 1;  // invalid lanes still join the shuffles
-    const int64_t D = a.d_inner, L = a.seqlen;
-    const int64_t nck = (L + kCk - 1) / kCk;
-    float2 h[NP], a2[NP];
-#pragma unroll
-    for (int i = 0; i < NP; ++i) {
-        const int n = sub * NS + 2 * i;
-        a2[i] = make_float2(__ldg(a.A + dc * N + n) * kLog2e, __ldg(a.A + dc * N + n + 1) * kLog2e);
-        h[i] = a.h0 ? make_float2(__ldg(a.h0 + (b * D + dc) * N + n), __ldg(a.h0 + (b * D + dc) * N + n + 1))
-                    : make_float2(0.0f, 0.0f);
-    }
-    const float bias = a.delta_bias ? __ldg(a.delta_bias + dc) : 0.0f;
-    const bool sp = a.delta_softplus != 0;
-    const IoT *x = static_cast<const IoT *>(a.x) + b * L * D;
-    const IoT *dt = static_cast<const IoT *>(a.delta) + b * L * D;
-    const IoT *Bm = static_cast<const IoT *>(a.B) + b * L * N + sub * NS;
-    for (int64_t k = 0; k < nck; ++k) {
-        if (dvalid) {
-            float *o = a.ckpt + ((b * nck + k) * D + d) * N + sub * NS;
-#pragma unroll
-            for (int i = 0; i < NP; ++i) {
-                o[2 * i] = h[i].x;
-                o[2 * i + 1] = h[i].y;
-            }
-        }
-        const int64_t t0 = k * kCk;
-        const int nst = static_cast<int>(L - t0 < kCk ? L - t0 : kCk);
-        // every load of the segment first: the owned steps' x, delta, and every
-        // step's B slice
-        float xo[kCk / G], vo[kCk / G];
-        float2 bv[kCk][NP];
-#pragma unroll
-        for (int q = 0; q < kCk / G; ++q) {
-            const int j = q * G + sub;
-            const bool ok = j < nst;
-            xo[q] = ok ? to_f32(x[(t0 + j) * D + dc]) : 0.0f;
-            vo[q] = ok ? to_f32(dt[(t0 + j) * D + dc]) : 0.0f;
-        }
-#pragma unroll
-        for (int j = 0; j < kCk; ++j) {
-            if (j < nst) load_pairs<NS>(Bm + (t0 + j) * N, bv[j]);
-            else
-#pragma unroll
-                for (int i = 0; i < NP; ++i) bv[j][i] = make_float2(0.0f, 0.0f);
-        }
-#pragma unroll
-        for (int q = 0; q < kCk / G; ++q) {
-            const float dl_o = delta_f32(vo[q], bias, sp);
-            const float dx_o = dl_o * xo[q];
-#pragma unroll
-            for (int jj = 0; jj < G; ++jj) {
-                const int j = q * G + jj;
-                const float dl = __shfl_sync(0xffffffffu, dl_o, gbase | jj);
-                const float dx = __shfl_sync(0xffffffffu, dx_o, gbase | jj);
-                if (j < nst) {
-#pragma unroll
-                    for (int i = 0; i < NP; ++i) {
-                        const float2 arg = mul2(make_float2(dl, dl), a2[i]);
-                        const float2 ab = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
-                        h[i] = fma2(ab, h[i], mul2(make_float2(dx, dx), bv[j][i]));
-                    }
-                }
-            }
-        }
     }
 }
 
@@ -493,11 +410,13 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
     for (int it = 0; it < ntiles; ++it) {
         const int k = ntiles - 1 - it;
         const int s = it % STAGES, slot = it % NOUT;
-        if (ok && (!mbar_wait_or_abort(&full[s], (it / STAGES) & 1, limit, abort_flag) ||
-                   (it >= NOUT && !mbar_wait_or_abort(&out_free[slot], ((it / NOUT) - 1) & 1,
-                                                      limit, abort_flag)))) {
-            ok = false;
-            fail();
+        if (ok) {
+            const bool got =
+                mbar_wait_or_abort(&full[s], (it / STAGES) & 1, limit, abort_flag) &&
+                (it < NOUT ||
+                 mbar_wait_or_abort(&out_free[slot], ((it / NOUT) - 1) & 1, limit, abort_flag));
+            ok = warp_agree(got);
+            if (!ok) fail();
         }
         const int64_t t_tile = int64_t(k) * TT;
         const int nsteps = static_cast<int>(L - t_tile < TT ? L - t_tile : TT);

@@ -72,13 +72,14 @@ struct OwnedStep {
     float dl, dx, gate, skg;
 };
 
-template <bool SOFTPLUS, typename IoT>
+template <bool SOFTPLUS, bool LDS, bool CKPT, typename IoT>
 __device__ __forceinline__ OwnedStep owned_step(const IoT *xs, const IoT *dts, const IoT *zs, int idx,
                                                 float bias, float dskip) {
-    const float xo = to_f32(xs[idx]);
-    const float v = to_f32(dts[idx]) + bias;
-    const float dl = SOFTPLUS ? softplus_f32(v) : v;
-    const float gate = silu_f32(to_f32(zs[idx]));
+    const float xo = LDS ? lds_f32(xs + idx) : to_f32(xs[idx]);
+    const float v = (LDS ? lds_f32(dts + idx) : to_f32(dts[idx])) + bias;
+    const float dl = SOFTPLUS ? softplus_io<IoT>(v) : v;
+    if (CKPT) return OwnedStep{dl, dl * xo, 0.0f, 0.0f};  // no output, no gate
+    const float gate = silu_f32(LDS ? lds_f32(zs + idx) : to_f32(zs[idx]));
     return OwnedStep{dl, dl * xo, gate, dskip * xo * gate};
 }
 
@@ -113,17 +114,26 @@ __device__ __forceinline__ void group_exps(const OwnedStep &o, const float2 (&a2
 // queue is long.  SOFTPLUS is a template parameter: a runtime test inside the
 // unrolled body would split it into basic blocks that the scheduler cannot
 // interleave.
-template <bool SOFTPLUS, typename IoT, int N, int G, int NS, int TT, int CC, int BCROW>
+//
+// CKPT (the backward's checkpoint pass): only the states advance; before every
+// kCk-th step of the tile the lane stores its NS states at ck + (step / kCk) *
+// ck_stride (ck null: nothing stored), and the readout, gate and output tile
+// are skipped.
+template <bool SOFTPLUS, typename IoT, int N, int G, int NS, int TT, int CC, int BCROW,
+          bool CKPT = false>
 __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float2 (&a2)[NS / 2],
                                                 float bias, float dskip,
                                                 const IoT *xs, const IoT *dts, const IoT *zs,
                                                 const float *bcs, IoT *outs, int c_local, int sub,
-                                                int gbase) {
+                                                int gbase, float *ck = nullptr,
+                                                int64_t ck_stride = 0) {
     constexpr int NG = TT / G;
     static_assert(NG >= 3, "a tile holds at least three groups");
-    OwnedStep o0 = owned_step<SOFTPLUS>(xs, dts, zs, sub * CC + c_local, bias, dskip);
-    OwnedStep o1 = owned_step<SOFTPLUS>(xs, dts, zs, (G + sub) * CC + c_local, bias, dskip);
-    OwnedStep o2 = owned_step<SOFTPLUS>(xs, dts, zs, (2 * G + sub) * CC + c_local, bias, dskip);
+    constexpr bool LDS = G == 2;  // explicit shared-space accesses (see load_bc_shared)
+    static_assert(!CKPT || (TT % kCk == 0 && kCk % G == 0), "checkpoints at group starts");
+    OwnedStep o0 = owned_step<SOFTPLUS, LDS, CKPT>(xs, dts, zs, sub * CC + c_local, bias, dskip);
+    OwnedStep o1 = owned_step<SOFTPLUS, LDS, CKPT>(xs, dts, zs, (G + sub) * CC + c_local, bias, dskip);
+    OwnedStep o2 = owned_step<SOFTPLUS, LDS, CKPT>(xs, dts, zs, (2 * G + sub) * CC + c_local, bias, dskip);
     float2 dxa[G], aba[G][NS / 2], dxb[G], abb[G][NS / 2];
     group_exps<G, NS>(o0, a2, gbase, dxa, aba);
     group_exps<G, NS>(o1, a2, gbase, dxb, abb);
@@ -132,9 +142,10 @@ __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float
         const int t0 = g * G;
         OwnedStep o3 = o2;
         if (g + 3 < NG)
-            o3 = owned_step<SOFTPLUS>(xs, dts, zs, (t0 + 3 * G + sub) * CC + c_local, bias, dskip);
+            o3 = owned_step<SOFTPLUS, LDS, CKPT>(xs, dts, zs, (t0 + 3 * G + sub) * CC + c_local, bias, dskip);
         float2 dxc[G], abc[G][NS / 2];
         float yp[G];
+        if (CKPT && (t0 % kCk) == 0 && ck) store_states<NS>(ck + (t0 / kCk) * ck_stride, h);
 #pragma unroll
         for (int j = 0; j < G; ++j) {
             if (g + 2 < NG) {
@@ -147,17 +158,24 @@ __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float
                     abc[j][i] = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
                 }
             }
-            const BCPairs<NS> bc = load_bc<NS>(bcs + (t0 + j) * BCROW, sub);
+            const BCPairs<NS> bc = LDS ? load_bc_shared<NS>(bcs + (t0 + j) * BCROW, sub)
+                                       : load_bc<NS>(bcs + (t0 + j) * BCROW, sub);
             float2 y2;
 #pragma unroll
             for (int i = 0; i < NS / 2; ++i) {
                 h[i] = fma2(aba[j][i], h[i], mul2(dxa[j], bc.b[i]));
-                y2 = i == 0 ? mul2(bc.c[i], h[i]) : fma2(bc.c[i], h[i], y2);
+                if (!CKPT) y2 = i == 0 ? mul2(bc.c[i], h[i]) : fma2(bc.c[i], h[i], y2);
             }
-            yp[j] = y2.x + y2.y;
+            yp[j] = CKPT ? 0.0f : y2.x + y2.y;
         }
-        const float y = reduce_transpose<G>(yp, sub);
-        outs[(t0 + sub) * CC + c_local] = from_f32<IoT>(fmaf(y, o0.gate, o0.skg));
+        if (!CKPT) {
+            const float y = reduce_transpose<G>(yp, sub);
+            const IoT ov = from_f32<IoT>(fmaf(y, o0.gate, o0.skg));
+            if (LDS)
+                sts_io(outs + (t0 + sub) * CC + c_local, ov);
+            else
+                outs[(t0 + sub) * CC + c_local] = ov;
+        }
 #pragma unroll
         for (int j = 0; j < G; ++j) {
             dxa[j] = dxb[j];
@@ -174,7 +192,9 @@ __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float
     }
 }
 
-template <typename IoT, int N, int G, int NW, int TT, int STAGES>
+// CKPT: the backward's checkpoint pass (see fused_tile_full): no z or C loads,
+// no output stores; args.ckpt receives the states before every kCk-th step.
+template <typename IoT, int N, int G, int NW, int TT, int STAGES, bool CKPT = false>
 __global__ void __launch_bounds__((NW + 1) * 32, 1)
     s6_scan_fused_kernel(const __grid_constant__ CUtensorMap tm_x,
                          const __grid_constant__ CUtensorMap tm_dt,
@@ -197,6 +217,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
     const int64_t ngroups = (d_inner + CC - 1) / CC;
     const int64_t ntasks = args.batch * ngroups;
     const int ntiles = static_cast<int>((seqlen + TT - 1) / TT);
+    const int64_t nck = (seqlen + kCk - 1) / kCk;  // checkpoints per sequence (CKPT)
     const int64_t my_tasks =
         static_cast<int64_t>(blockIdx.x) < ntasks ? (ntasks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const int64_t total = my_tasks * ntiles;
@@ -269,31 +290,35 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             const int s = static_cast<int>(g % STAGES);
             if ((args.debug_flags & 1u) && k == 0) return;  // test hook: withhold a first tile
             uint8_t *base = smem + s * Cfg::kStageBytes;
-            mbar_arrive_expect_tx(&full[s], Cfg::kTxBytes);
+            mbar_arrive_expect_tx(&full[s], CKPT ? Cfg::kTxBytes - Cfg::kActTile - Cfg::kBCTile
+                                                 : Cfg::kTxBytes);
             const int t0 = k * TT, bb = static_cast<int>(b);
             tma_load_3d(base, &tm_x, c0, t0, bb, &full[s]);
             tma_load_3d(base + Cfg::kActTile, &tm_dt, c0, t0, bb, &full[s]);
-            tma_load_3d(base + 2 * Cfg::kActTile, &tm_z, c0, t0, bb, &full[s]);
+            if (!CKPT) tma_load_3d(base + 2 * Cfg::kActTile, &tm_z, c0, t0, bb, &full[s]);
             tma_load_3d(base + 3 * Cfg::kActTile, &tm_B, 0, t0, bb, &full[s]);
-            tma_load_3d(base + 3 * Cfg::kActTile + Cfg::kBCTile, &tm_C, 0, t0, bb, &full[s]);
+            if (!CKPT)
+                tma_load_3d(base + 3 * Cfg::kActTile + Cfg::kBCTile, &tm_C, 0, t0, bb, &full[s]);
             armed |= 1u << s;
         };
         // store of tile g (its output buffer is complete), then release stage g
         auto retire = [&](int64_t g) -> bool {
             const int slot = static_cast<int>(g % NOUT);
-            if (!mbar_wait_or_abort(&out_full[slot], static_cast<uint32_t>(g / NOUT) & 1u, limit,
-                                    abort_flag))
+            if (!warp_agree(mbar_wait_or_abort(&out_full[slot], static_cast<uint32_t>(g / NOUT) & 1u,
+                                               limit, abort_flag)))
                 return false;
             if (lane == 0) {
-                int64_t b;
-                int c0, k;
-                tile_of(cur_store, g, b, c0, k);
-                tma_store_3d(&tm_out, smem + Cfg::kOffOut + slot * Cfg::kActTile, c0, k * TT,
-                             static_cast<int>(b));
-                bulk_commit();
+                if (!CKPT) {
+                    int64_t b;
+                    int c0, k;
+                    tile_of(cur_store, g, b, c0, k);
+                    tma_store_3d(&tm_out, smem + Cfg::kOffOut + slot * Cfg::kActTile, c0, k * TT,
+                                 static_cast<int>(b));
+                    bulk_commit();
+                }
                 issue(g + STAGES);  // the compute warps are done with stage g % STAGES
                 if (g > 0) {
-                    bulk_wait_read<1>();  // the store of tile g-1 has read its buffer
+                    if (!CKPT) bulk_wait_read<1>();  // the store of tile g-1 has read its buffer
                     mbar_arrive(&out_free[static_cast<int>((g - 1) % NOUT)]);
                 }
             }
@@ -317,8 +342,8 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             int c0, k;
             tile_of(cur_main, g, b, c0, k);
             const int s = static_cast<int>(g % STAGES);
-            if (!mbar_wait_or_abort(&full[s], static_cast<uint32_t>(g / STAGES) & 1u, limit,
-                                    abort_flag))
+            if (!warp_agree(mbar_wait_or_abort(&full[s], static_cast<uint32_t>(g / STAGES) & 1u,
+                                               limit, abort_flag)))
                 return false;
             consumed = g + 1;
             if (lane == 0) armed &= ~(1u << s);
@@ -328,8 +353,11 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             const IoT *Cs = reinterpret_cast<const IoT *>(base + 3 * Cfg::kActTile + Cfg::kBCTile);
             float *dst = bcs_all + s * Cfg::kBCe;
             // unit u = (step t, slot j, half: 0 = B, 1 = C): one slice of NS values
-            for (int u = lane; u < nsteps * 2 * G; u += 32) {
-                const int t = u / (2 * G), j = (u / 2) % G, half = u & 1;
+            // (B only for checkpoints)
+            constexpr int kHalves = CKPT ? 1 : 2;
+            for (int u = lane; u < nsteps * kHalves * G; u += 32) {
+                const int t = u / (kHalves * G), j = (u / kHalves) % G;
+                const int half = CKPT ? 0 : (u & 1);
                 stage_slice<NS>(dst + t * Cfg::kBCRow + (2 * j + half) * NS,
                                 (half ? Cs : Bs) + t * N + j * NS);
             }
@@ -393,13 +421,14 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
         const int slot = static_cast<int>(g % NOUT);
         // the output buffer was last used by tile g - NOUT, whose store must
         // have read it (the (g / NOUT - 1)-th release of this buffer)
-        if (!mbar_wait_or_abort(&bc_ready[s], static_cast<uint32_t>(g / STAGES) & 1u, limit,
-                                abort_flag) ||
-            !mbar_wait_or_abort(&full[s], static_cast<uint32_t>(g / STAGES) & 1u, limit,
-                                abort_flag) ||
-            (g >= NOUT &&
-             !mbar_wait_or_abort(&out_free[slot], static_cast<uint32_t>(g / NOUT - 1) & 1u, limit,
-                                 abort_flag))) {
+        const bool got =
+            mbar_wait_or_abort(&bc_ready[s], static_cast<uint32_t>(g / STAGES) & 1u, limit,
+                               abort_flag) &&
+            mbar_wait_or_abort(&full[s], static_cast<uint32_t>(g / STAGES) & 1u, limit, abort_flag) &&
+            (g < NOUT ||
+             mbar_wait_or_abort(&out_free[slot], static_cast<uint32_t>(g / NOUT - 1) & 1u, limit,
+                                abort_flag));
+        if (!warp_agree(got)) {
             ok = false;
             break;
         }
@@ -410,6 +439,11 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
         const IoT *zs = reinterpret_cast<const IoT *>(base + 2 * Cfg::kActTile);
         const float *bcs = bcs_all + s * Cfg::kBCe;
         IoT *outs = reinterpret_cast<IoT *>(smem + Cfg::kOffOut + slot * Cfg::kActTile);
+        // checkpoint pass: this lane's slice of the tile's first checkpoint
+        float *ck = nullptr;
+        const int64_t ck_stride = d_inner * N;
+        if (CKPT && dvalid)
+            ck = args.ckpt + ((b * nck + int64_t(k) * (TT / kCk)) * d_inner + d) * N + sub * NS;
 
         // One group of G steps starting at t0: the owner lane's scalars, the
         // exchange, G recurrence steps, the butterfly, the owner's output.
@@ -417,10 +451,9 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             const int t_own = t0 + sub;
             const int idx = t_own * CC + c_local;
             const float xo = to_f32(xs[idx]);
-            const float zo = to_f32(zs[idx]);
-            const float dl = delta_f32(to_f32(dts[idx]), bias, use_softplus);
-            const float gate = silu_f32(zo);
+            const float dl = delta_io<IoT>(to_f32(dts[idx]), bias, use_softplus);
             const float dx = dl * xo;
+            if (CKPT && (t0 % kCk) == 0 && ck) store_states<NS>(ck + (t0 / kCk) * ck_stride, h);
             float yp[G];
 #pragma unroll
             for (int j = 0; j < G; ++j) {
@@ -431,16 +464,18 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
                     yp[j] = recurrence_step<NS>(h, a2, make_float2(dlj, dxj),
                                                 bcs + (t0 + j) * Cfg::kBCRow, sub);
             }
-            const float y = reduce_transpose<G>(yp, sub);
-            if (sub < valid) outs[idx] = from_f32<IoT>((y + dskip * xo) * gate);
+            if (!CKPT) {
+                const float y = reduce_transpose<G>(yp, sub);
+                const float gate = silu_f32(to_f32(zs[idx]));
+                if (sub < valid) outs[idx] = from_f32<IoT>((y + dskip * xo) * gate);
+            }
         };
         if (nsteps == TT && use_softplus) {
-            fused_tile_full<true, IoT, N, G, NS, TT, CC, Cfg::kBCRow>(h, a2, bias, dskip, xs, dts, zs,
-                                                                     bcs, outs, c_local, sub, gbase);
+            fused_tile_full<true, IoT, N, G, NS, TT, CC, Cfg::kBCRow, CKPT>(
+                h, a2, bias, dskip, xs, dts, zs, bcs, outs, c_local, sub, gbase, ck, ck_stride);
         } else if (nsteps == TT) {
-            fused_tile_full<false, IoT, N, G, NS, TT, CC, Cfg::kBCRow>(h, a2, bias, dskip, xs, dts,
-                                                                      zs, bcs, outs, c_local, sub,
-                                                                      gbase);
+            fused_tile_full<false, IoT, N, G, NS, TT, CC, Cfg::kBCRow, CKPT>(
+                h, a2, bias, dskip, xs, dts, zs, bcs, outs, c_local, sub, gbase, ck, ck_stride);
         } else {
             for (int t0 = 0; t0 < nsteps; t0 += G) group(t0, nsteps - t0 < G ? nsteps - t0 : G);
         }

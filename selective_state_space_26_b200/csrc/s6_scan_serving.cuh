@@ -178,8 +178,8 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
         // store of tile g (its output buffer is complete), then release stage g
         auto retire = [&](int64_t g) -> bool {
             const int slot = static_cast<int>(g % NOUT);
-            if (!mbar_wait_or_abort(&out_full[slot], static_cast<uint32_t>(g / NOUT) & 1u, limit,
-                                    abort_flag))
+            if (!warp_agree(mbar_wait_or_abort(&out_full[slot], static_cast<uint32_t>(g / NOUT) & 1u,
+                                               limit, abort_flag)))
                 return false;
             const Tile t = tile_of(cur_store, g);
             const uint8_t *ob = smem + Cfg::kOffOut + slot * Cfg::kActTile;
@@ -229,8 +229,8 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
         auto widen = [&](int64_t g) -> bool {
             const Tile t = tile_of(cur_main, g);
             const int s = static_cast<int>(g % STAGES);
-            if (!mbar_wait_or_abort(&full[s], static_cast<uint32_t>(g / STAGES) & 1u, limit,
-                                    abort_flag))
+            if (!warp_agree(mbar_wait_or_abort(&full[s], static_cast<uint32_t>(g / STAGES) & 1u,
+                                               limit, abort_flag)))
                 return false;
             consumed = g + 1;
             if (lane == 0) armed &= ~(1u << s);
@@ -313,13 +313,14 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
         const int slot = static_cast<int>(g % NOUT);
         // the output buffer was last used by tile g - NOUT, whose store must
         // have read it (the (g / NOUT - 1)-th release of this buffer)
-        if (!mbar_wait_or_abort(&bc_ready[s], static_cast<uint32_t>(g / STAGES) & 1u, limit,
-                                abort_flag) ||
-            !mbar_wait_or_abort(&full[s], static_cast<uint32_t>(g / STAGES) & 1u, limit,
-                                abort_flag) ||
-            (g >= NOUT &&
-             !mbar_wait_or_abort(&out_free[slot], static_cast<uint32_t>(g / NOUT - 1) & 1u, limit,
-                                 abort_flag))) {
+        const bool got =
+            mbar_wait_or_abort(&bc_ready[s], static_cast<uint32_t>(g / STAGES) & 1u, limit,
+                               abort_flag) &&
+            mbar_wait_or_abort(&full[s], static_cast<uint32_t>(g / STAGES) & 1u, limit, abort_flag) &&
+            (g < NOUT ||
+             mbar_wait_or_abort(&out_free[slot], static_cast<uint32_t>(g / NOUT - 1) & 1u, limit,
+                                abort_flag));
+        if (!warp_agree(got)) {
             ok = false;
             break;
         }
@@ -343,7 +344,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             const int idx = t_own * CC + c_local;
             const float xo = to_f32(xs[idx]);
             const float zo = to_f32(zs[idx]);
-            const float dl = delta_f32(to_f32(dts[idx]), bias, use_softplus);
+            const float dl = delta_io<IoT>(to_f32(dts[idx]), bias, use_softplus);
             const float gate = silu_f32(zo);
             const float dx = dl * xo;
             float yp[G];

@@ -56,7 +56,7 @@ __device__ __forceinline__ void small_steps(const SmallBlock<N, U> &s, float (&h
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         if (u < nrows) {
-            const float dl = delta_f32(s.dt[u], bias, use_softplus);
+            const float dl = delta_io<IoT>(s.dt[u], bias, use_softplus);
             const float dx = dl * s.x[u];
             float y = 0.0f;
 #pragma unroll
@@ -134,8 +134,8 @@ __global__ void __launch_bounds__(128) s6_state_update_small_kernel(const Update
     const int64_t D = a.d_inner;
     const int64_t i = b * D + d;
     const float xv = to_f32(static_cast<const IoT *>(a.x)[i]);
-    const float dl = delta_f32(to_f32(static_cast<const IoT *>(a.delta)[i]),
-                               a.delta_bias ? __ldg(a.delta_bias + d) : 0.0f, a.delta_softplus != 0);
+    const float dl = delta_io<IoT>(to_f32(static_cast<const IoT *>(a.delta)[i]),
+                                   a.delta_bias ? __ldg(a.delta_bias + d) : 0.0f, a.delta_softplus != 0);
     const float dx = dl * xv;
     const IoT *Bp = static_cast<const IoT *>(a.B) + b * N;
     const IoT *Cp = static_cast<const IoT *>(a.C) + b * N;

@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(256) s6_state_update_kernel(const UpdateArgs a
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            const float dl = delta_f32(dtv[u], bias, use_softplus);
+            const float dl = delta_io<IoT>(dtv[u], bias, use_softplus);
             const float dx = dl * xv[u];
             float h[4] = {h4[u].x, h4[u].y, h4[u].z, h4[u].w};
             float y = 0.0f;
@@ -281,6 +281,7 @@ __global__ void __launch_bounds__(UpdateCfg<IoT, N, CPB, STAGES>::kThreads, 4)
         for (int r = 0; r < nr && ok; ++r)
             ok = mbar_wait_or_abort(&full[(r0 + r) % STAGES], static_cast<uint32_t>((r0 + r) / STAGES) & 1u,
                                     limit, abort_flag);
+        ok = warp_agree(ok);
         if (!ok) {
             *abort_flag = 1;
             record_status(a.status, kStTimeout);
@@ -290,7 +291,7 @@ __global__ void __launch_bounds__(UpdateCfg<IoT, N, CPB, STAGES>::kThreads, 4)
         const uint8_t *so = smem + ((r0 + (q < nr ? q : 0)) % STAGES) * Cfg::kStage;
         const IoT *xs = reinterpret_cast<const IoT *>(so + Cfg::kStateBytes);
         const float xv = to_f32(xs[c]);
-        const float dl = delta_f32(to_f32(xs[CPB + c]), bias, use_softplus);
+        const float dl = delta_io<IoT>(to_f32(xs[CPB + c]), bias, use_softplus);
         const float gate = silu_f32(to_f32(xs[2 * CPB + c]));
         const float dxo = dl * xv, skg = dskip * xv * gate;
         float yp[Q];

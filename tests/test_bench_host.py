@@ -93,29 +93,36 @@ def test_reference_arm_under_torchrun_prints_one_line():
     assert d["e2e"]["h2d_bytes_per_step"] == 0
 
 
-def test_traffic_record_follows_the_scan_library_sources(tmp_path, monkeypatch):
+def test_traffic_record_follows_the_kernel_device_sources(tmp_path, monkeypatch):
     """roofline.traffic is reported only while the recorded DRAM counters were
-    taken on the current sources of the translation unit holding the timed
-    kernels: a header it includes changes the hash, a file outside it does not."""
+    taken on the current device code of the timed kernel (its header and every
+    header that includes, directly or not) and, for the scan, on the same
+    launch shape: a header in that closure changes the hash, a file outside
+    it does not, and another launch shape drops the record."""
     csrc = tmp_path / "selective_state_space_26_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "jamba_ssm.cu").write_text('#include "a.cuh"\n#include <cuda.h>\n')
+    (csrc / "k.cuh").write_text('#include "a.cuh"\n#include <cuda.h>\n')
     (csrc / "a.cuh").write_text('#include "b.cuh"\nint a;\n')
     (csrc / "b.cuh").write_text("int b;\n")
-    (csrc / "other.cu").write_text("int other;\n")
+    (csrc / "host.cu").write_text('#include "k.cuh"\nint host;\n')
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    h0 = bench.kernel_source_hash()
-    (csrc / "other.cu").write_text("int other2;\n")
+    monkeypatch.setitem(bench.KERNEL_HEADER, "k", "k.cuh")
+    h0 = bench.kernel_source_hash("k")
+    (csrc / "host.cu").write_text('#include "k.cuh"\nint host2;\n')
     (csrc / "unrelated.cuh").write_text("int u;\n")
-    assert bench.kernel_source_hash() == h0
+    assert bench.kernel_source_hash("k") == h0
     (csrc / "b.cuh").write_text("int b2;\n")  # included indirectly
-    h1 = bench.kernel_source_hash()
+    h1 = bench.kernel_source_hash("k")
     assert h1 != h0
     prof = tmp_path / "profiles"
     prof.mkdir()
+    launch = bench.plan_launch({"variant": 2, "grid": 147, "channels_per_cta": 56})
     (prof / "dram_traffic.json").write_text(json.dumps(
-        {"k": {"w": {"bytes_per_launch": 123, "source_hash": h1}}}))
+        {"k": {"w": {"bytes_per_launch": 123, "source_hash": h1, "launch": launch}}}))
     assert bench.recorded_traffic("k", "w") == 123.0
+    assert bench.recorded_traffic("k", "w", launch) == 123.0
+    other = bench.plan_launch({"variant": 1, "grid": 64, "channels_per_cta": 128})
+    assert bench.recorded_traffic("k", "w", other) is None
     (csrc / "a.cuh").write_text('#include "b.cuh"\nint a2;\n')
     assert bench.recorded_traffic("k", "w") is None
 
