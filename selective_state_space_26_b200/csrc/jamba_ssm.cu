@@ -164,7 +164,6 @@ ScanVariant g_variants[] = {
     make_fused<float, 16, 1, 2, 32, 3, true>(1.00),          // 8:  64 channels / CTA
     make_fused<float, 8, 1, 2, 32, 3, true>(1.00),           // 9:  64 channels / CTA
     make_fused<float, 4, 1, 2, 32, 3, true>(1.00),           // 10: 64 channels / CTA
-    make_fused<__nv_bfloat16, 16, 8, 14, 64, 3>(1.40),       // 11:  56 channels / CTA
 };
 constexpr int kNumVariants = sizeof(g_variants) / sizeof(g_variants[0]);
 

@@ -75,8 +75,13 @@ struct BwdCfg {
     // per warp, one step's [channel][dB | dC] scratch (see BcScratch)
     static constexpr int kOffScr = kOffPart + kPart;
     static constexpr int kScrWords = CW * (N == 16 ? 48 : (N == 8 ? 24 : 12));
-    static constexpr int kOffBar = kOffScr + NW * kScrWords * 4;
-    static constexpr int kNumBars = 2 * STAGES + 2 * NOUT;    // full, empty, out_full, out_free
+    // per stage, B and C widened to fp32 in per-lane slots ([TT][G][2][NS], load_bc's layout)
+    static constexpr int kOffWide = kOffScr + NW * kScrWords * 4;
+    static constexpr int kWide = TT * 2 * N * 4;
+    static constexpr int kOffBar = kOffWide + STAGES * kWide;
+    static_assert(kOffWide % 16 == 0, "16-byte slot reads");
+    // full, ready, empty, out_full, out_free
+    static constexpr int kNumBars = 3 * STAGES + 2 * NOUT;
     static constexpr int kOffFlag = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffFlag + 16;
     static_assert(kAct % 128 == 0 && kBC % 128 == 0, "TMA boxes 128-byte aligned");
@@ -120,8 +125,9 @@ struct BcScratch {
 
 // One segment of kCk steps (starting at tile step s0, `nst` of them valid),
 // recomputed from h_in and walked backwards.  Owner scalars come from the
-// stage's x / delta / z / dout tiles; B / C slices from the stage's [TT][N]
-// tiles, one vector load each; the state math is on fp32 pairs.  `part` is
+// stage's x / delta / z / dout tiles; B / C slices from the stage's widened
+// fp32 slots (`wide`, [TT][G][2][NS]), 16-byte loads without conversions;
+// the state math is on fp32 pairs.  `part` is
 // the warp's [TT][2N] slab of the CTA's dB | dC partial sums and `bcs` its
 // [CW][RS] scratch for summing one step over the warp's channels.
 template <bool FULL, bool SP, typename IoT, int N, int G, int CC>
@@ -129,7 +135,7 @@ __device__ __forceinline__ void bwd_segment(
     const float2 (&h_in)[N / G / 2], float2 (&g)[N / G / 2], float2 (&dA)[N / G / 2],
     float &dD_acc, float &dbias_acc, const float2 (&a2)[N / G / 2], const float2 (&Araw)[N / G / 2],
     float bias, float dskip, const IoT *xs, const IoT *dts, const IoT *zs, const IoT *dos,
-    const IoT *Bs, const IoT *Cs, IoT *dxs, IoT *dds, IoT *dzs, float *part, float *bcs, int s0,
+    const float *wide, IoT *dxs, IoT *dds, IoT *dzs, float *part, float *bcs, int s0,
     int nst, int c_local, int sub, int gbase, int lane) {
     constexpr int NS = N / G, NP = NS / 2, NQ = kCk / G;
     using SC = BcScratch<N, G>;
@@ -158,7 +164,7 @@ __device__ __forceinline__ void bwd_segment(
             dxv[j] = __shfl_sync(0xffffffffu, dxo, gbase | jj);
             if (FULL || j < nst) {
                 float2 bv[NP];
-                load_pairs<NS>(Bs + (s0 + j) * N + sub * NS, bv);
+                load_pairs<NS>(wide + (s0 + j) * 2 * N + sub * 2 * NS, bv);
 #pragma unroll
                 for (int i = 0; i < NP; ++i) {
                     const float2 arg = mul2(make_float2(dl[j], dl[j]), a2[i]);
@@ -193,9 +199,9 @@ __device__ __forceinline__ void bwd_segment(
 #pragma unroll
             for (int i = 0; i < NP; ++i) dBp[i] = dCp[i] = make_float2(0.0f, 0.0f);
             if (FULL || j < nst) {
-                float2 bv[NP], cv[NP];
-                load_pairs<NS>(Bs + (s0 + j) * N + sub * NS, bv);
-                load_pairs<NS>(Cs + (s0 + j) * N + sub * NS, cv);
+                const BCPairs<NS> bc = load_bc<NS>(wide + (s0 + j) * 2 * N, sub);
+                const float2(&bv)[NP] = bc.b;
+                const float2(&cv)[NP] = bc.c;
                 const float2 dy2 = make_float2(dy, dy), dl2 = make_float2(dl[j], dl[j]);
                 const float2 dx2 = make_float2(dxv[j], dxv[j]);
 #pragma unroll
@@ -272,7 +278,8 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
                   NOUT = Cfg::NOUT;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
-    uint64_t *empty = full + STAGES;
+    uint64_t *ready = full + STAGES;
+    uint64_t *empty = ready + STAGES;
     uint64_t *out_full = empty + STAGES;
     uint64_t *out_free = out_full + NOUT;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffFlag);
@@ -290,6 +297,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&ready[s], 32);
             mbar_init(&empty[s], NW * 32);
         }
         for (int o = 0; o < NOUT; ++o) {
@@ -306,7 +314,71 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
     };
 
     if (warp == NW) {
-        // ===================== producer: TMA loads and stores =====================
+        // ========== producer: TMA loads and stores, B / C widening ==========
+        const int bb = static_cast<int>(b);
+        int last_i[STAGES];  // lane 0: the walked tile whose load is in flight per stage, or -1
+        for (int s = 0; s < STAGES; ++s) last_i[s] = -1;
+        // the i-th tile walked is tile ntiles - 1 - i (lane 0 only)
+        auto issue = [&](int i) -> bool {
+            const int s = i % STAGES;
+            if (i >= STAGES &&
+                !mbar_wait_or_abort(&empty[s], ((i / STAGES) & 1) ^ 1, limit, abort_flag))
+                return false;
+            if ((a.debug_flags & 1u) && i == 0) return true;  // test hook: withhold tile 0
+            uint8_t *st = smem + s * Cfg::kStage;
+            const int t0 = (ntiles - 1 - i) * TT;
+            mbar_arrive_expect_tx(&full[s], Cfg::kStage);
+            tma_load_3d(st, &maps.x, c0, t0, bb, &full[s]);
+            tma_load_3d(st + Cfg::kAct, &maps.dt, c0, t0, bb, &full[s]);
+            tma_load_3d(st + 2 * Cfg::kAct, &maps.z, c0, t0, bb, &full[s]);
+            tma_load_3d(st + 3 * Cfg::kAct, &maps.dout, c0, t0, bb, &full[s]);
+            tma_load_3d(st + 4 * Cfg::kAct, &maps.B, 0, t0, bb, &full[s]);
+            tma_load_3d(st + 4 * Cfg::kAct + Cfg::kBC, &maps.C, 0, t0, bb, &full[s]);
+            last_i[s] = i;
+            return true;
+        };
+        // walked tile i landed: B and C into the stage's fp32 slots (all lanes)
+        auto prepare = [&](int i) -> bool {
+            const int s = i % STAGES;
+            if (!warp_agree(mbar_wait_or_abort(&full[s], (i / STAGES) & 1, limit, abort_flag)))
+                return false;
+            if (lane == 0) last_i[s] = -1;
+            const uint8_t *st = smem + s * Cfg::kStage;
+            const IoT *Bs = reinterpret_cast<const IoT *>(st + 4 * Cfg::kAct);
+            const IoT *Cs = reinterpret_cast<const IoT *>(st + 4 * Cfg::kAct + Cfg::kBC);
+            float *wide = reinterpret_cast<float *>(smem + Cfg::kOffWide + s * Cfg::kWide);
+            // unit u = (step t, slot j, half: 0 = B, 1 = C): one slice of NS values
+            for (int u = lane; u < TT * 2 * G; u += 32) {
+                const int t = u / (2 * G), j = (u / 2) % G, half = u & 1;
+                stage_slice<NS>(wide + t * 2 * N + (2 * j + half) * NS,
+                                (half ? Cs : Bs) + t * N + j * NS);
+            }
+            mbar_arrive(&ready[s]);
+            return true;
+        };
+        // outputs of walked tile i are complete: store them, then refill its stage
+        auto retire = [&](int i, int &next) -> bool {
+            const int slot = i % NOUT;
+            if (!warp_agree(mbar_wait_or_abort(&out_full[slot], (i / NOUT) & 1, limit, abort_flag)))
+                return false;
+            bool ok = true;
+            if (lane == 0) {
+                uint8_t *ob = smem + Cfg::kOffOut + slot * 3 * Cfg::kAct;
+                const int t0 = (ntiles - 1 - i) * TT;
+                tma_store_3d(&maps.dx, ob, c0, t0, bb);
+                tma_store_3d(&maps.ddt, ob + Cfg::kAct, c0, t0, bb);
+                tma_store_3d(&maps.dz, ob + 2 * Cfg::kAct, c0, t0, bb);
+                bulk_commit();
+                if (next < ntiles) ok = issue(next);
+                if (i > 0) {
+                    bulk_wait_read<1>();  // the stores of tile i-1 have read their buffers
+                    mbar_arrive(&out_free[(i - 1) % NOUT]);
+                }
+            }
+            ++next;
+            return warp_agree(ok);
+        };
+        bool ok = true;
         if (lane == 0) {
             prefetch_tensormap(&maps.x);
             prefetch_tensormap(&maps.dt);
@@ -317,51 +389,17 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             prefetch_tensormap(&maps.dx);
             prefetch_tensormap(&maps.ddt);
             prefetch_tensormap(&maps.dz);
-            const int bb = static_cast<int>(b);
-            int last_i[STAGES];
-            for (int s = 0; s < STAGES; ++s) last_i[s] = -1;
-            bool ok = true;
-            // the i-th tile walked is tile ntiles - 1 - i
-            auto issue = [&](int i) -> bool {
-                const int s = i % STAGES;
-                if (i >= STAGES &&
-                    !mbar_wait_or_abort(&empty[s], ((i / STAGES) & 1) ^ 1, limit, abort_flag))
-                    return false;
-                if ((a.debug_flags & 1u) && i == 0) return true;  // test hook: withhold tile 0
-                uint8_t *st = smem + s * Cfg::kStage;
-                const int t0 = (ntiles - 1 - i) * TT;
-                mbar_arrive_expect_tx(&full[s], Cfg::kStage);
-                tma_load_3d(st, &maps.x, c0, t0, bb, &full[s]);
-                tma_load_3d(st + Cfg::kAct, &maps.dt, c0, t0, bb, &full[s]);
-                tma_load_3d(st + 2 * Cfg::kAct, &maps.z, c0, t0, bb, &full[s]);
-                tma_load_3d(st + 3 * Cfg::kAct, &maps.dout, c0, t0, bb, &full[s]);
-                tma_load_3d(st + 4 * Cfg::kAct, &maps.B, 0, t0, bb, &full[s]);
-                tma_load_3d(st + 4 * Cfg::kAct + Cfg::kBC, &maps.C, 0, t0, bb, &full[s]);
-                last_i[s] = i;
-                return true;
-            };
-            int next = 0;
-            for (; next < STAGES && next < ntiles && ok; ++next) ok = issue(next);
-            for (int i = 0; i < ntiles && ok; ++i) {
-                // outputs of walked tile i are complete: store them, then refill
-                const int slot = i % NOUT;
-                if (!mbar_wait_or_abort(&out_full[slot], (i / NOUT) & 1, limit, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t *ob = smem + Cfg::kOffOut + slot * 3 * Cfg::kAct;
-                const int t0 = (ntiles - 1 - i) * TT;
-                tma_store_3d(&maps.dx, ob, c0, t0, bb);
-                tma_store_3d(&maps.ddt, ob + Cfg::kAct, c0, t0, bb);
-                tma_store_3d(&maps.dz, ob + 2 * Cfg::kAct, c0, t0, bb);
-                bulk_commit();
-                if (next < ntiles) ok = issue(next++);
-                if (i > 0) {
-                    bulk_wait_read<1>();  // the stores of tile i-1 have read their buffers
-                    mbar_arrive(&out_free[(i - 1) % NOUT]);
-                }
-            }
-            if (!ok) fail();
+            for (int i = 0; i < STAGES && i < ntiles && ok; ++i) ok = issue(i);
+        }
+        ok = warp_agree(ok);
+        int next = STAGES;
+        if (ok && ntiles > 0) ok = prepare(0);
+        for (int i = 0; i < ntiles && ok; ++i) {
+            if (i + 1 < ntiles) ok = prepare(i + 1);
+            if (ok) ok = retire(i, next);
+        }
+        if (!ok) fail();
+        if (lane == 0) {
             // nothing in flight may outlive the CTA
             for (int s = 0; s < STAGES; ++s)
                 if (last_i[s] >= 0 && !mbar_wait_bounded(&full[s], (last_i[s] / STAGES) & 1, limit))
@@ -412,6 +450,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
         const int s = it % STAGES, slot = it % NOUT;
         if (ok) {
             const bool got =
+                mbar_wait_or_abort(&ready[s], (it / STAGES) & 1, limit, abort_flag) &&
                 mbar_wait_or_abort(&full[s], (it / STAGES) & 1, limit, abort_flag) &&
                 (it < NOUT ||
                  mbar_wait_or_abort(&out_free[slot], ((it / NOUT) - 1) & 1, limit, abort_flag));
@@ -426,8 +465,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             const IoT *dts = reinterpret_cast<const IoT *>(st + Cfg::kAct);
             const IoT *zs = reinterpret_cast<const IoT *>(st + 2 * Cfg::kAct);
             const IoT *dos = reinterpret_cast<const IoT *>(st + 3 * Cfg::kAct);
-            const IoT *Bs = reinterpret_cast<const IoT *>(st + 4 * Cfg::kAct);
-            const IoT *Cs = reinterpret_cast<const IoT *>(st + 4 * Cfg::kAct + Cfg::kBC);
+            const float *wide = reinterpret_cast<const float *>(smem + Cfg::kOffWide + s * Cfg::kWide);
             uint8_t *ob = smem + Cfg::kOffOut + slot * 3 * Cfg::kAct;
             IoT *dxs = reinterpret_cast<IoT *>(ob);
             IoT *dds = reinterpret_cast<IoT *>(ob + Cfg::kAct);
@@ -447,12 +485,12 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
                 const int rem = nsteps - sg * kCk;
                 if (rem >= kCk)
                     bwd_segment<true, SP, IoT, N, G, CC>(hcur, g, dA, dD_acc, dbias_acc, a2, Araw,
-                                                         bias, dskip, xs, dts, zs, dos, Bs, Cs, dxs,
+                                                         bias, dskip, xs, dts, zs, dos, wide, dxs,
                                                          dds, dzs, part, bcs, sg * kCk, kCk, c_local,
                                                          sub, gbase, lane);
                 else
                     bwd_segment<false, SP, IoT, N, G, CC>(hcur, g, dA, dD_acc, dbias_acc, a2, Araw,
-                                                          bias, dskip, xs, dts, zs, dos, Bs, Cs,
+                                                          bias, dskip, xs, dts, zs, dos, wide,
                                                           dxs, dds, dzs, part, bcs, sg * kCk, rem,
                                                           c_local, sub, gbase, lane);
             }

@@ -14,8 +14,12 @@
 // With a scalar decay the exp-class work is 4 operations per (token, channel)
 // -- the gate's exp and reciprocal, plus softplus and the decay once per head
 // and token -- against d_state + 4 for the diagonal scan, so this layer is not
-// bound by the MUFU pipe but by issue: a lane-step is a dozen instructions
-// (its table entry, x, its B and C slices, the packed update and readout).
+// bound by the MUFU pipe.  What bounds it is the shared-memory pipe: a 16-byte
+// vector read costs four wavefronts whatever the broadcast, and every lane
+// reads its B and C slices at every step.  So the tile is prepared once per
+// CTA into the forms that cost a lane-step the fewest wavefronts: the decay
+// (one broadcast word), Delta x (one word per channel) and the lane's B and C
+// slices side by side in the I/O type (one 16-byte vector in bf16).
 //
 // Layout: one CTA per (sequence, slice of CC channels of one head); CC divides
 // headdim.  NW compute warps with G lanes per channel, NS = N / G states per
@@ -23,10 +27,9 @@
 //  * The producer's lane 0 feeds TT-step tiles by TMA into a STAGES ring (x, z
 //    [TT x CC], the delta columns of a 16-byte box of heads [TT x 16 B], B, C
 //    [TT x N]) and stores the output tiles by TMA.
-//  * All producer lanes then prepare each landed tile for the compute warps:
-//    the [TT] table of (Delta, decay) of the CTA's head, and B and C widened to
-//    fp32 in per-lane slots (load_bc's layout), so that a compute lane-step
-//    reads one broadcast table entry, one x value and two 16-byte vectors.
+//  * All producer lanes then prepare each landed tile: the [TT] table of
+//    (Delta, decay) of the CTA's head, Delta x in fp32 [TT x CC], and the
+//    per-lane slots [TT][G][B slice | C slice].
 //  * The compute warps walk a whole tile with its loop unrolled: the G steps of
 //    a group advance the states and give G partial readouts, which the
 //    transposing butterfly turns into the owner lane's sum; the owners' skip,
@@ -62,10 +65,12 @@ struct SsdCfg {
     static constexpr int kBC = TT * N * (int)sizeof(IoT);
     static constexpr int kStage = 2 * kAct + kDt + 2 * kBC;  // x, z, delta, B, C
     static_assert(kAct % 128 == 0 && kDt % 128 == 0 && kBC % 128 == 0, "128-byte TMA boxes");
-    static constexpr int kBCRow = 2 * N;                     // widened floats per step
-    static constexpr int kOffWide = STAGES * kStage;         // [STAGES][TT][2N] fp32
-    static constexpr int kWide = TT * kBCRow * 4;
-    static constexpr int kOffTab = kOffWide + STAGES * kWide;  // [STAGES][TT] (Delta, decay)
+    // prepared per stage: Delta x [TT][CC] fp32, slots [TT][G][2 NS] IoT, (Delta, decay) [TT]
+    static constexpr int kOffDx = STAGES * kStage;
+    static constexpr int kDx = TT * CC * 4;
+    static constexpr int kOffSlot = kOffDx + STAGES * kDx;
+    static constexpr int kSlot = TT * 2 * N * (int)sizeof(IoT);
+    static constexpr int kOffTab = kOffSlot + STAGES * kSlot;
     static constexpr int NOUT = 3;
     static constexpr int kOffOut = kOffTab + STAGES * TT * 8;
     static_assert(kOffOut % 128 == 0, "TMA store sources 128-byte aligned");
@@ -73,18 +78,56 @@ struct SsdCfg {
     static constexpr int kNumBars = 2 * STAGES + 2 * NOUT;  // full, ready, out_full, out_free
     static constexpr int kOffFlag = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffFlag + 16;
-    static_assert(TT % G == 0, "whole step groups");
+    static_assert(TT % G == 0 && CC % (16 / (int)sizeof(IoT)) == 0, "whole groups and vectors");
 };
+
+// A lane's slot (its NS values of B, then its NS values of C) as fp32 pairs:
+// one 16-byte read for bf16 with NS = 4.
+template <int NS>
+__device__ __forceinline__ void load_slot(const __nv_bfloat16 *p, float2 (&b)[NS / 2],
+                                          float2 (&c)[NS / 2]) {
+    if constexpr (NS == 2) {  // B0 B1 | C0 C1: 8 bytes
+        const uint2 w = *reinterpret_cast<const uint2 *>(p);
+        b[0] = bf16x2_to_f2(w.x);
+        c[0] = bf16x2_to_f2(w.y);
+    } else if constexpr (NS == 4) {  // B0..3 | C0..3: 16 bytes
+        const uint4 w = *reinterpret_cast<const uint4 *>(p);
+        b[0] = bf16x2_to_f2(w.x);
+        b[1] = bf16x2_to_f2(w.y);
+        c[0] = bf16x2_to_f2(w.z);
+        c[1] = bf16x2_to_f2(w.w);
+    } else {  // B0..7 | C0..7: two 16-byte vectors
+        const uint4 wb = reinterpret_cast<const uint4 *>(p)[0];
+        const uint4 wc = reinterpret_cast<const uint4 *>(p)[1];
+        b[0] = bf16x2_to_f2(wb.x);
+        b[1] = bf16x2_to_f2(wb.y);
+        b[2] = bf16x2_to_f2(wb.z);
+        b[3] = bf16x2_to_f2(wb.w);
+        c[0] = bf16x2_to_f2(wc.x);
+        c[1] = bf16x2_to_f2(wc.y);
+        c[2] = bf16x2_to_f2(wc.z);
+        c[3] = bf16x2_to_f2(wc.w);
+    }
+}
+template <int NS>
+__device__ __forceinline__ void load_slot(const float *p, float2 (&b)[NS / 2], float2 (&c)[NS / 2]) {
+#pragma unroll
+    for (int i = 0; i < NS / 2; ++i) {
+        b[i] = reinterpret_cast<const float2 *>(p)[i];
+        c[i] = reinterpret_cast<const float2 *>(p + NS)[i];
+    }
+}
 
 // One tile of a compute lane: TT steps if FULL, else the first `nsteps`
 // (the states do not move past them; the rows past them are written to the
 // output buffer but clipped by the TMA store).
 template <bool FULL, typename IoT, int N, int G, int TT, int CC>
 __device__ __forceinline__ void ssd_tile(float2 (&h)[N / G / 2], const float2 *tab,
-                                         const float *wide, const IoT *xs, const IoT *zs,
-                                         IoT *outs, float dskip, int c_local, int sub,
-                                         int nsteps) {
+                                         const float *dxs, const IoT *slots, const IoT *xs,
+                                         const IoT *zs, IoT *outs, float dskip, int c_local,
+                                         int sub, int nsteps) {
     constexpr int NS = N / G, NP = NS / 2, NQ = TT / G;
+    const float *decay = reinterpret_cast<const float *>(tab) + 1;  // .y of each entry
     float yown[NQ];  // C.h of the owned steps q * G + sub
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
@@ -94,15 +137,16 @@ __device__ __forceinline__ void ssd_tile(float2 (&h)[N / G / 2], const float2 *t
             const int t = q * G + j;
             yp[j] = 0.0f;
             if (FULL || t < nsteps) {
-                const float2 dd = tab[t];
-                const float dx = dd.x * to_f32(xs[t * CC + c_local]);
-                const BCPairs<NS> bc = load_bc<NS>(wide + t * 2 * N, sub);
-                const float2 dec2 = make_float2(dd.y, dd.y), dx2 = make_float2(dx, dx);
+                const float dec = decay[2 * t];
+                const float dx = dxs[t * CC + c_local];
+                float2 bv[NP], cv[NP];
+                load_slot<NS>(slots + (t * G + sub) * 2 * NS, bv, cv);
+                const float2 dec2 = make_float2(dec, dec), dx2 = make_float2(dx, dx);
                 float2 y2;
 #pragma unroll
                 for (int i = 0; i < NP; ++i) {
-                    h[i] = fma2(dec2, h[i], mul2(dx2, bc.b[i]));
-                    y2 = i == 0 ? mul2(bc.c[i], h[i]) : fma2(bc.c[i], h[i], y2);
+                    h[i] = fma2(dec2, h[i], mul2(dx2, bv[i]));
+                    y2 = i == 0 ? mul2(cv[i], h[i]) : fma2(cv[i], h[i], y2);
                 }
                 yp[j] = y2.x + y2.y;
             }
@@ -115,6 +159,25 @@ __device__ __forceinline__ void ssd_tile(float2 (&h)[N / G / 2], const float2 *t
         const float xo = to_f32(xs[idx]);
         outs[idx] = from_f32<IoT>(fmaf(dskip, xo, yown[q]) * silu_f32(to_f32(zs[idx])));
     }
+}
+
+// One 16-byte vector of an I/O tile as floats (8 bf16 or 4 fp32).
+__device__ __forceinline__ void load_vec16(const __nv_bfloat16 *p, float (&v)[8]) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = bf16x2_to_f2(ws[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void load_vec16(const float *p, float (&v)[4]) {
+    const float4 w = *reinterpret_cast<const float4 *>(p);
+    v[0] = w.x;
+    v[1] = w.y;
+    v[2] = w.z;
+    v[3] = w.w;
 }
 
 struct SsdMaps {
@@ -182,28 +245,48 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             tma_load_3d(st + 2 * Cfg::kAct + Cfg::kDt + Cfg::kBC, &maps.C, 0, t0, bb, &full[s]);
             last_k[s] = k;
         };
-        // tile k landed: its (Delta, decay) table and widened B / C
+        // tile k landed: (Delta, decay), Delta x and the lanes' B | C slots
         auto prepare = [&](int k) -> bool {
             const int s = k % STAGES;
             if (!warp_agree(mbar_wait_or_abort(&full[s], (k / STAGES) & 1, limit, abort_flag)))
                 return false;
             if (lane == 0) last_k[s] = -1;
             const uint8_t *st = smem + s * Cfg::kStage;
+            const IoT *xs = reinterpret_cast<const IoT *>(st);
             const IoT *dts = reinterpret_cast<const IoT *>(st + 2 * Cfg::kAct);
             const IoT *Bs = reinterpret_cast<const IoT *>(st + 2 * Cfg::kAct + Cfg::kDt);
             const IoT *Cs = reinterpret_cast<const IoT *>(st + 2 * Cfg::kAct + Cfg::kDt + Cfg::kBC);
             float2 *tab = reinterpret_cast<float2 *>(smem + Cfg::kOffTab) + s * TT;
-            float *wide = reinterpret_cast<float *>(smem + Cfg::kOffWide + s * Cfg::kWide);
+            float *dxs = reinterpret_cast<float *>(smem + Cfg::kOffDx + s * Cfg::kDx);
+            IoT *slots = reinterpret_cast<IoT *>(smem + Cfg::kOffSlot + s * Cfg::kSlot);
             for (int t = lane; t < TT; t += 32) {
                 const float v = to_f32(dts[t * Cfg::kHeadsBox + (head - hbox)]) + bias;
                 const float dl = SP ? softplus_io<IoT>(v) : v;
                 tab[t] = make_float2(dl, ex2_mufu(dl * a2));
             }
-            // unit u = (step t, slot j, half: 0 = B, 1 = C): one slice of NS values
-            for (int u = lane; u < TT * 2 * G; u += 32) {
-                const int t = u / (2 * G), j = (u / 2) % G, half = u & 1;
-                stage_slice<NS>(wide + t * Cfg::kBCRow + (2 * j + half) * NS,
-                                (half ? Cs : Bs) + t * N + j * NS);
+            __syncwarp();  // each step's Delta is read by other lanes below
+            // Delta x, one 16-byte vector of x (VEC channels of one step) per unit
+            constexpr int VEC = 16 / (int)sizeof(IoT), VPR = CC / VEC;
+            for (int u = lane; u < TT * VPR; u += 32) {
+                const int t = u / VPR, cv = (u % VPR) * VEC;
+                const float dl = tab[t].x;
+                float xv[VEC];
+                load_vec16(xs + t * CC + cv, xv);
+#pragma unroll
+                for (int q = 0; q < VEC / 4; ++q)
+                    reinterpret_cast<float4 *>(dxs + t * CC + cv)[q] =
+                        make_float4(dl * xv[4 * q], dl * xv[4 * q + 1], dl * xv[4 * q + 2],
+                                    dl * xv[4 * q + 3]);
+            }
+            // slot (t, j): B[t, j NS ..] then C[t, j NS ..]
+            constexpr int W = NS * (int)sizeof(IoT) / 4;
+            for (int u = lane; u < TT * G; u += 32) {
+                const int t = u / G, j = u % G;
+                IoT *dst = slots + (t * G + j) * 2 * NS;
+                copy_words<W>(reinterpret_cast<uint32_t *>(dst),
+                              reinterpret_cast<const uint32_t *>(Bs + t * N + j * NS));
+                copy_words<W>(reinterpret_cast<uint32_t *>(dst + NS),
+                              reinterpret_cast<const uint32_t *>(Cs + t * N + j * NS));
             }
             mbar_arrive(&ready[s]);
             return true;
@@ -279,14 +362,16 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
         const IoT *xs = reinterpret_cast<const IoT *>(st);
         const IoT *zs = reinterpret_cast<const IoT *>(st + Cfg::kAct);
         const float2 *tab = reinterpret_cast<const float2 *>(smem + Cfg::kOffTab) + s * TT;
-        const float *wide = reinterpret_cast<const float *>(smem + Cfg::kOffWide + s * Cfg::kWide);
+        const float *dxs = reinterpret_cast<const float *>(smem + Cfg::kOffDx + s * Cfg::kDx);
+        const IoT *slots = reinterpret_cast<const IoT *>(smem + Cfg::kOffSlot + s * Cfg::kSlot);
         IoT *outs = reinterpret_cast<IoT *>(smem + Cfg::kOffOut + slot * Cfg::kAct);
         const int nsteps = static_cast<int>(L - int64_t(k) * TT < TT ? L - int64_t(k) * TT : TT);
         if (nsteps == TT)
-            ssd_tile<true, IoT, N, G, TT, CC>(h, tab, wide, xs, zs, outs, dskip, c_local, sub, TT);
+            ssd_tile<true, IoT, N, G, TT, CC>(h, tab, dxs, slots, xs, zs, outs, dskip, c_local,
+                                              sub, TT);
         else
-            ssd_tile<false, IoT, N, G, TT, CC>(h, tab, wide, xs, zs, outs, dskip, c_local, sub,
-                                               nsteps);
+            ssd_tile<false, IoT, N, G, TT, CC>(h, tab, dxs, slots, xs, zs, outs, dskip, c_local,
+                                               sub, nsteps);
         fence_proxy_async_smem();  // the output tile before the TMA store reads it
         mbar_arrive(&out_full[slot]);
     }
