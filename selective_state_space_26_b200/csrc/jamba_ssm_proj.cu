@@ -30,7 +30,8 @@ constexpr int kMaxDevices = 64;
 struct DeviceState {
     bool ready = false;
     bool usable = false;
-    bool dt_attr = false;  // s6_dt_proj_kernel's shared-memory limit is set
+    bool dt_attr = false;   // s6_dt_proj_kernel's shared-memory limit is set
+    bool dtp_attr = false;  // s6_dt_proj_persistent_kernel's
     bool x_attr = false;   // s6_x_proj_kernel's
     int sms = 0;
 };
@@ -177,9 +178,17 @@ JSSM_PROJ_API jamba_ssm_status jamba_ssm_dt_proj(const jamba_ssm_dt_proj_params 
         overlaps(p.delta, out_bytes, p.dt_low_lo, a_bytes) ||
         overlaps(p.delta, out_bytes, p.W_dt, w_bytes))
         return JAMBA_SSM_ERR_INVALID_ARG;
+    // dt_rank <= 256 (Jamba's included): the persistent kernel, whose CTAs keep
+    // a token block's planes resident; larger ranks: one tile per CTA.
+    const bool persistent = p.dt_rank <= int64_t(jssm::DtProjPCfg::kMaxKB) * jssm::DtProjPCfg::kBK;
+    int sms = 0;
     jamba_ssm_status st =
-        prepare_device(reinterpret_cast<const void *>(&jssm::s6_dt_proj_kernel),
-                       static_cast<int>(jssm::DtProjCfg::kSmemBytes), &DeviceState::dt_attr);
+        persistent
+            ? prepare_device(reinterpret_cast<const void *>(&jssm::s6_dt_proj_persistent_kernel),
+                             static_cast<int>(jssm::DtProjPCfg::kSmemBytes), &DeviceState::dtp_attr,
+                             &sms)
+            : prepare_device(reinterpret_cast<const void *>(&jssm::s6_dt_proj_kernel),
+                             static_cast<int>(jssm::DtProjCfg::kSmemBytes), &DeviceState::dt_attr);
     if (st != JAMBA_SSM_OK) return st;
 
     EncodeTiledFn fn = encode_fn(&st);
@@ -194,6 +203,20 @@ JSSM_PROJ_API jamba_ssm_status jamba_ssm_dt_proj(const jamba_ssm_dt_proj_params 
     int dt_rank = static_cast<int>(p.dt_rank), two = p.dt_low_lo ? 1 : 0;
     uint64_t limit = p.timeout_cycles ? p.timeout_cycles : kDefaultTimeoutCycles;
     uint32_t debug_flags = p.debug_flags;
+    if (persistent) {
+        int ntok = static_cast<int>(p.ntok), d_inner = static_cast<int>(p.d_inner);
+        const int64_t items = ((p.ntok + jssm::DtProjPCfg::kBM - 1) / jssm::DtProjPCfg::kBM) *
+                              ((p.d_inner + jssm::DtProjPCfg::kBN - 1) / jssm::DtProjPCfg::kBN);
+        const int grid = static_cast<int>(items < sms ? items : sms);
+        void *pargs[] = {&map_hi, &map_lo,  &map_w, &map_out, &ntok,
+                         &d_inner, &dt_rank, &two,  &limit,   &debug_flags};
+        cudaError_t e = cudaLaunchKernel(
+            reinterpret_cast<const void *>(&jssm::s6_dt_proj_persistent_kernel), dim3(grid),
+            dim3(jssm::DtProjPCfg::kThreads), pargs, jssm::DtProjPCfg::kSmemBytes,
+            static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e);
+        return finish_launch(stream);
+    }
     void *args[] = {&map_hi, &map_lo, &map_w, &map_out, &dt_rank, &two, &limit, &debug_flags};
     const dim3 grid(static_cast<unsigned>((p.ntok + jssm::DtProjCfg::kBM - 1) / jssm::DtProjCfg::kBM),
                     static_cast<unsigned>((p.d_inner + jssm::DtProjCfg::kBN - 1) / jssm::DtProjCfg::kBN));

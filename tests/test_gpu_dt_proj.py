@@ -30,9 +30,11 @@ def _ref(inp, rows=None, lo=True):
 
 
 # token counts and widths that leave ragged tiles on every axis: 300 tokens =
-# 2 full 128-token tiles + 44; 776 channels = 3 full 256-channel tiles + 8;
-# dt_rank 200 = 3 full 64-wide K blocks + 8 (zero-filled by TMA); 256 and 320
-# run the 2-stage ring through two and a half passes
+# 2 full 128-token tiles + 44; 776 channels = 6 full 128-channel tiles + 8;
+# dt_rank 200 = 3 full 64-wide K blocks + 8 (zero-filled by TMA).  Ranks up to
+# 256 run the persistent kernel (planes resident, W_dt through a 3-stage
+# ring); 320 runs the one-tile kernel's 2-stage ring through two and a half
+# passes
 @pytest.mark.parametrize("ntok,d_inner,dt_rank", [(300, 776, 256), (300, 776, 200),
                                                   (1, 8, 8), (128, 256, 64), (257, 512, 320)])
 def test_dt_proj_matches_oracle(ntok, d_inner, dt_rank):
@@ -92,3 +94,15 @@ def test_dt_proj_is_deterministic():
     b = jamba_ssm_dt_proj(inp.hi, inp.W_dt, dt_low_lo=inp.lo)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def test_dt_proj_persistent_walks_token_blocks():
+    """Several items per CTA, ranges that start inside a token block and cross
+    into the next (the planes are reloaded after the block's MMAs), both TMEM
+    accumulators in turn, and a ragged last token block: every output."""
+    dev = _dev()
+    inp = synth.dt_proj_inputs(2000, 4096, 256, seed=34, device=dev)
+    out = jamba_ssm_dt_proj(inp.hi, inp.W_dt, dt_low_lo=inp.lo)
+    torch.cuda.synchronize()
+    assert jamba_ssm_proj_get_status() == 0
+    assert_out(out, _ref(inp), torch.bfloat16, "dt_proj 2000 x 4096 x 256")

@@ -131,12 +131,14 @@ def test_projection_then_scan_matches_the_oracle_composition():
     assert_out(out, ref, torch.bfloat16, "composed: layer output")
 
 
-def test_dt_proj_bounded_wait_times_out_and_reports():
+@pytest.mark.parametrize("dt_rank", [256, 320])
+def test_dt_proj_bounded_wait_times_out_and_reports(dt_rank):
     """A withheld operand block makes the MMA thread's bounded wait run out:
     TIMEOUT is recorded, the CTAs drain their loads and write nothing, the
-    context stays usable and the next call is correct."""
+    context stays usable and the next call is correct.  dt_rank 256 runs the
+    persistent kernel, 320 the one-tile kernel."""
     dev = _dev()
-    inp = synth.dt_proj_inputs(300, 776, 256, seed=58, device=dev)
+    inp = synth.dt_proj_inputs(300, 776, dt_rank, seed=58, device=dev)
     assert jamba_ssm_proj_get_status() == 0
     out = torch.full((300, 776), 7.0, dtype=torch.bfloat16, device=dev)
     jamba_ssm_dt_proj(inp.hi, inp.W_dt, dt_low_lo=inp.lo, out=out, debug_flags=1,
