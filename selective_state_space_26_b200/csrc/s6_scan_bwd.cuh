@@ -72,9 +72,9 @@ struct BwdCfg {
     static constexpr int kOffOut = STAGES * kStage;           // dx, ddelta, dz per set
     static constexpr int kOffPart = kOffOut + NOUT * 3 * kAct;  // [NW][TT][2N] fp32
     static constexpr int kPart = NW * TT * 2 * N * 4;
-    // per warp, one step's [channel][dB | dC] scratch (see BcScratch)
+    // per warp, two steps' [slot][channel][dB | dC] scratch (see BcScratch)
     static constexpr int kOffScr = kOffPart + kPart;
-    static constexpr int kScrWords = CW * (N == 16 ? 48 : (N == 8 ? 24 : 12));
+    static constexpr int kScrWords = 2 * CW * (N == 16 ? 48 : (N == 8 ? 24 : 12));
     // per stage, B and C widened to fp32 in per-lane slots ([TT][G][2][NS], load_bc's layout)
     static constexpr int kOffWide = kOffScr + NW * kScrWords * 4;
     static constexpr int kWide = TT * 2 * N * 4;
@@ -113,14 +113,17 @@ __device__ __forceinline__ void load_pairs(const float *p, float2 (&v)[NS / 2]) 
 }
 
 // --------------------------------------------------------------- backward
-// Row stride (in words) of a warp's [channel][dB | dC] scratch: 2N values plus
-// padding chosen so that the lanes of one vector-store wavefront (the slices of
-// 2, 4 or 8 channels) land in distinct banks.
+// A warp's scratch for summing dB | dC over its channels, two steps at a time:
+// slot k (the step of the pair, k = step & 1) holds one row per channel of 2N
+// values.  Row stride RS (in words): 2N plus padding chosen so that the lanes
+// of one vector-store wavefront (the slices of 2, 4 or 8 channels) land in
+// distinct banks.
 template <int N, int G>
 struct BcScratch {
     static constexpr int CW = 32 / G;
     static constexpr int RS = N == 16 ? 48 : (N == 8 ? 24 : 12);
-    static constexpr int kWords = CW * RS;
+    static constexpr int kSlot = CW * RS;
+    static constexpr int kWords = 2 * kSlot;
 };
 
 // One segment of kCk steps (starting at tile step s0, `nst` of them valid),
@@ -129,7 +132,7 @@ struct BcScratch {
 // fp32 slots (`wide`, [TT][G][2][NS]), 16-byte loads without conversions;
 // the state math is on fp32 pairs.  `part` is
 // the warp's [TT][2N] slab of the CTA's dB | dC partial sums and `bcs` its
-// [CW][RS] scratch for summing one step over the warp's channels.
+// [2][CW][RS] scratch for summing two steps over the warp's channels.
 template <bool FULL, bool SP, typename IoT, int N, int G, int CC>
 __device__ __forceinline__ void bwd_segment(
     const float2 (&h_in)[N / G / 2], float2 (&g)[N / G / 2], float2 (&dA)[N / G / 2],
@@ -178,7 +181,8 @@ __device__ __forceinline__ void bwd_segment(
     }
     // ---- backward walk, groups of G steps from the last
     const int c_in_warp = lane / G;
-    float *my_row = bcs + c_in_warp * SC::RS + sub * NS;
+    float *my_row = bcs + c_in_warp * SC::RS + sub * NS;  // + (step & 1) * SC::kSlot
+    static_assert(G % 2 == 0, "steps pair up inside a group");
 #pragma unroll
     for (int q = NQ - 1; q >= 0; --q) {
         const int jo = q * G + sub;
@@ -224,20 +228,31 @@ __device__ __forceinline__ void bwd_segment(
             pa[jj] = pa2.x + pa2.y;
             gb[jj] = gb2.x + gb2.y;
             // dB / dC of this step summed over the warp's channels, through the
-            // warp's scratch: each lane stores its slices, then lane k adds
-            // slot k over the channels
-            if (FULL || j < nst) {
+            // warp's scratch, two steps at a time: each lane stores its slices
+            // (zeros for a step past the segment) in the step's slot; after the
+            // pair's second step (jj even: the walk goes down), lane l adds
+            // values 2 (l % N) and 2 (l % N) + 1 of slot l / N over the channels
+            // in order, on one fp32 pair.
+            {
+                float *row = my_row + (jj & 1) * SC::kSlot;
 #pragma unroll
                 for (int i = 0; i < NP; ++i) {
-                    reinterpret_cast<float2 *>(my_row)[i] = dBp[i];
-                    reinterpret_cast<float2 *>(my_row + N)[i] = dCp[i];
+                    reinterpret_cast<float2 *>(row)[i] = dBp[i];
+                    reinterpret_cast<float2 *>(row + N)[i] = dCp[i];
                 }
+            }
+            if ((jj & 1) == 0) {
                 __syncwarp();
-                if (lane < 2 * N) {
-                    float acc = bcs[lane];
+                const int sl = lane / N, v = 2 * (lane % N);
+                const int js = q * G + jj + sl;  // the step whose values this lane sums
+                if (lane < 2 * N && (FULL || js < nst)) {
+                    const float *src = bcs + sl * SC::kSlot + v;
+                    float2 acc = *reinterpret_cast<const float2 *>(src);
+                    const float2 one = make_float2(1.0f, 1.0f);
 #pragma unroll
-                    for (int c = 1; c < SC::CW; ++c) acc += bcs[c * SC::RS + lane];
-                    part[(s0 + j) * 2 * N + lane] = acc;
+                    for (int c = 1; c < SC::CW; ++c)
+                        acc = fma2(*reinterpret_cast<const float2 *>(src + c * SC::RS), one, acc);
+                    *reinterpret_cast<float2 *>(part + (s0 + js) * 2 * N + v) = acc;
                 }
                 __syncwarp();
             }
