@@ -339,7 +339,24 @@ def per_workload(args, dev, stream, flush_l2, sms, world):
     names.append("scan_bwd_bf16_b1_l4096_d8192_n16")
     times.append(t_b)
     meta.append((wb, "bwd"))
-    del bw
+
+    # a training step of the same layer: the forward storing the backward's
+    # checkpoints, then the backward taking them
+    inp, dout, ws = bw["inp"], bw["dout"], bw["ws"]
+    ck = torch.empty(wb.batch, (wb.seqlen + 15) // 16, wb.d_inner, wb.d_state,
+                     dtype=torch.float32, device=dev)
+    fwd_out = torch.empty_like(inp.x)
+    fwd_hf = torch.empty(wb.batch, wb.d_inner, wb.d_state, dtype=torch.float32, device=dev)
+
+    def train_step():
+        jssm.jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, D=inp.D,
+                            delta_bias=inp.delta_bias, out=fwd_out, h_final=fwd_hf, ckpt=ck)
+        jssm.jamba_ssm_scan_bwd(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, dout, D=inp.D,
+                                delta_bias=inp.delta_bias, workspace=ws, ckpt=ck)
+    names.append("train_step_bf16_b1_l4096_d8192_n16")
+    times.append(time_launches(train_step, args.pw_reps, stream, dev, flush=flush_l2))
+    meta.append((wb, "train"))
+    del bw, inp, dout, ws, ck, fwd_out, fwd_hf
 
     times = max_over_ranks(times, world, dev)
     tc_peak, tc_kind = bf16_peak()
@@ -371,6 +388,23 @@ def per_workload(args, dev, stream, flush_l2, sms, world):
                              "and the per-segment recompute add 2 d_state + 1)",
                 "timing": f"{args.pw_reps} calls (checkpoint, backward and reduction kernels) "
                           "after 1 warm-up, L2 flushed before each"}
+        elif kind == "train":
+            tok = w.batch * w.seqlen
+            ops = tok * w.d_inner * ((w.d_state + 4) + (w.d_state + 5))
+            issued = tok * w.d_inner * ((w.d_state + 3) + (2 * w.d_state + 5))
+            res[name] = {
+                "kernel_us": t * 1e6, "tokens_per_s": tok * world / t,
+                "roofline": {"bound": "alu", "achieved": ops / t / 1e12,
+                             "peak": mufu_peak / 1e12, "unit": "Top/s (exp-class, MUFU)",
+                             "frac": ops / t / mufu_peak,
+                             "algorithmic_ops": ops, "issued_ops": issued,
+                             "issued_frac": issued / t / mufu_peak},
+                "ops_basis": "algorithmic: the forward's d_state + 4 plus the backward's "
+                             "d_state + 5 exp-class ops per (token, channel); issued: the "
+                             "forward's d_state + 3 and the backward's 2 d_state + 5 (its "
+                             "recompute and walk; the checkpoints come from the forward)",
+                "timing": f"{args.pw_reps} steps (forward storing checkpoints, then backward, "
+                          "reduction) after 1 warm-up, L2 flushed before each"}
         elif kind == "ssd":
             tok, d_inner, H, N = 4096, 8192, 128, 16
             nbytes = (tok * (3 * d_inner + H + 2 * N) * 2 + (H * 2 + d_inner) * 4

@@ -64,7 +64,7 @@ extern "C" {
  * (workspace, stream) form of jamba_ssm_get_status, d_state 1 and 2 (and 4 in
  * bf16), and the status codes renumbered so that ERR_WORKSPACE is 4: a caller
  * built against an earlier version of this header must be rebuilt. */
-#define JAMBA_SSM_ABI_VERSION 3
+#define JAMBA_SSM_ABI_VERSION 4
 
 /* Bytes of the status block at the start of a workspace. */
 #define JAMBA_SSM_STATUS_BYTES 16
@@ -150,6 +150,20 @@ typedef enum {
  *                 jamba_ssm_scan_workspace_size returns, 16-byte aligned, or
  *                 NULL (the status goes to the library's per-device word).
  *                 Too small: JAMBA_SSM_ERR_WORKSPACE.
+ *
+ * Checkpoints for the backward (ABI version 4; absent -- NULL -- for a
+ * shorter struct_size).  The source pages say nothing of training kernels;
+ * this is a convenience for a training step that runs the forward and then
+ * jamba_ssm_scan_bwd on the same inputs:
+ *   ckpt          device fp32 [batch, ceil(seqlen / 16), d_inner, d_state]
+ *                 (jamba_ssm_scan_ckpt_size bytes), 16-byte aligned, or NULL.
+ *                 Non-NULL: entry [b, k] receives sequence b's state before
+ *                 step 16 k (entry [b, 0] is the initial state), and `out`
+ *                 and `h_final` are the same bits as without it.  Batched
+ *                 layout only (cu_seqlens and state_indices NULL), and the
+ *                 backward's state sizes (d_state 8 or 16 with bf16 I/O, 4, 8
+ *                 or 16 with fp32); otherwise JAMBA_SSM_ERR_UNSUPPORTED.  Must
+ *                 not overlap any input or output.
  */
 typedef struct jamba_ssm_scan_params {
     size_t struct_size;          /* = sizeof(jamba_ssm_scan_params); callers of
@@ -177,6 +191,8 @@ typedef struct jamba_ssm_scan_params {
     /* ABI version 3 */
     void *workspace;
     size_t workspace_bytes;
+    /* ABI version 4 */
+    float *ckpt;
 } jamba_ssm_scan_params;
 
 /* Bytes of workspace a scan of these sizes may use: the status block
@@ -281,6 +297,11 @@ jamba_ssm_status jamba_ssm_state_update(const jamba_ssm_state_update_params *p, 
  * overlap on the GPU.
  * debug_flags / timeout_cycles: as jamba_ssm_scan (bit 0 withholds each
  * CTA's first tile of the backward kernel).
+ * ckpt (ABI version 4; absent -- NULL -- for a shorter struct_size): the
+ *   checkpoints a forward call with the same inputs stored (see
+ *   jamba_ssm_scan_params.ckpt), or NULL.  Non-NULL: the backward uses them
+ *   and skips its own checkpoint pass; the results are the same bits either
+ *   way.  Must not overlap any output.  The workspace size is unchanged.
  */
 typedef struct jamba_ssm_scan_bwd_params {
     size_t struct_size;          /* = sizeof(jamba_ssm_scan_bwd_params)       */
@@ -305,7 +326,14 @@ typedef struct jamba_ssm_scan_bwd_params {
     size_t workspace_bytes;
     uint32_t debug_flags;
     uint64_t timeout_cycles;
+    /* ABI version 4 */
+    const float *ckpt;
 } jamba_ssm_scan_bwd_params;
+
+/* Bytes of the forward's checkpoints for these sizes (jamba_ssm_scan_params.
+ * ckpt): batch * ceil(seqlen / 16) * d_inner * d_state * 4; 0 for negative
+ * sizes. */
+size_t jamba_ssm_scan_ckpt_size(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state);
 
 /* Bytes of workspace jamba_ssm_scan_bwd needs for these sizes (0 for an
  * unsupported d_state). */

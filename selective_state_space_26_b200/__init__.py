@@ -28,7 +28,7 @@ from . import _lib
 from ._lib import JambaSSMError
 
 __all__ = ["jamba_ssm_scan", "jamba_ssm_state_update", "jamba_ssm_get_status", "scan_plan",
-           "jamba_ssm_scan_workspace_size", "jamba_ssm_scan_bwd",
+           "jamba_ssm_scan_workspace_size", "jamba_ssm_scan_ckpt_size", "jamba_ssm_scan_bwd",
            "jamba_ssm_scan_bwd_workspace_size", "jamba_ssm_ssd_scan",
            "jamba_ssm_x_proj", "jamba_ssm_dt_proj", "jamba_ssm_proj_get_status",
            "JambaSSMError"]
@@ -72,7 +72,7 @@ def _workspace(ws, device):
 
 def _scan_params(x, delta, z, B, C, A, D, delta_bias, delta_softplus, h0, out, h_final,
                  variant, debug_flags, timeout_cycles, cu_seqlens=None, state_indices=None,
-                 workspace=None):
+                 workspace=None, ckpt=None):
     if x.dtype not in _IO:
         raise TypeError(f"x must be bfloat16 or float32, got {x.dtype}")
     d_state = A.shape[-1]
@@ -103,6 +103,8 @@ def _scan_params(x, delta, z, B, C, A, D, delta_bias, delta_softplus, h0, out, h
     _check(h0, "h0", state_shape, torch.float32, dev)
     _check(h_final, "h_final", state_shape, torch.float32, dev)
     ws, ws_bytes = _workspace(workspace, dev)
+    if ckpt is not None:
+        _check(ckpt, "ckpt", (batch, (seqlen + 15) // 16, d_inner, d_state), torch.float32, dev)
     return _lib.new_scan_params(
         batch=batch, seqlen=seqlen, d_inner=d_inner, d_state=d_state, io_dtype=_IO[io],
         delta_softplus=int(bool(delta_softplus)), x=_ptr(x), delta=_ptr(delta), z=_ptr(z),
@@ -111,13 +113,13 @@ def _scan_params(x, delta, z, B, C, A, D, delta_bias, delta_softplus, h0, out, h
         debug_flags=int(debug_flags), timeout_cycles=int(timeout_cycles),
         cu_seqlens=_ptr(cu_seqlens), total_tokens=int(total),
         state_indices=_ptr(state_indices), num_slots=int(num_slots), workspace=ws,
-        workspace_bytes=ws_bytes)
+        workspace_bytes=ws_bytes, ckpt=_ptr(ckpt))
 
 
 def jamba_ssm_scan(x, delta, z, B, C, A, D=None, delta_bias=None, delta_softplus=True,
                    h0=None, out=None, h_final=None, return_final_state=True, stream=None,
                    variant: int = 0, debug_flags: int = 0, timeout_cycles: int = 0,
-                   cu_seqlens=None, state_indices=None, workspace=None):
+                   cu_seqlens=None, state_indices=None, workspace=None, ckpt=None):
     """Prefill S6 scan.  Shapes: x, delta, z [batch, seqlen, d_inner] (bf16 or
     fp32), B, C [batch, seqlen, d_state] (same dtype), A [d_inner, d_state]
     fp32, D and delta_bias [d_inner] fp32 or None, h0 [batch, d_inner, d_state]
@@ -133,7 +135,11 @@ def jamba_ssm_scan(x, delta, z, B, C, A, D=None, delta_bias=None, delta_softplus
 
     ``workspace``: an optional zero-filled device tensor of at least
     ``jamba_ssm_scan_workspace_size(...)`` bytes that holds this call's status
-    word (read with ``jamba_ssm_get_status(workspace=...)``)."""
+    word (read with ``jamba_ssm_get_status(workspace=...)``).
+
+    ``ckpt``: an optional fp32 device tensor [batch, ceil(seqlen / 16),
+    d_inner, d_state] that receives the state before every 16th step, for a
+    ``jamba_ssm_scan_bwd`` on the same inputs to take (batched layout only)."""
     if out is None:
         out = torch.empty_like(x)
     if h_final is None and return_final_state and state_indices is None:
@@ -141,11 +147,17 @@ def jamba_ssm_scan(x, delta, z, B, C, A, D=None, delta_bias=None, delta_softplus
         h_final = torch.empty(batch, x.shape[-1], A.shape[-1], dtype=torch.float32,
                               device=x.device)
     p = _scan_params(x, delta, z, B, C, A, D, delta_bias, delta_softplus, h0, out, h_final,
-                     variant, debug_flags, timeout_cycles, cu_seqlens, state_indices, workspace)
+                     variant, debug_flags, timeout_cycles, cu_seqlens, state_indices, workspace,
+                     ckpt)
     st = _lib.call_scan(p, _stream(stream, x.device))
     if st != _lib.OK:
         raise JambaSSMError(st, "jamba_ssm_scan")
     return out, h_final
+
+
+def jamba_ssm_scan_ckpt_size(batch: int, seqlen: int, d_inner: int, d_state: int) -> int:
+    """Bytes of the checkpoints jamba_ssm_scan stores when given ``ckpt``."""
+    return _lib.scan_ckpt_size(int(batch), int(seqlen), int(d_inner), int(d_state))
 
 
 def jamba_ssm_scan_bwd_workspace_size(batch: int, seqlen: int, d_inner: int,
@@ -156,7 +168,7 @@ def jamba_ssm_scan_bwd_workspace_size(batch: int, seqlen: int, d_inner: int,
 
 def jamba_ssm_scan_bwd(x, delta, z, B, C, A, dout, D=None, delta_bias=None,
                        delta_softplus=True, h0=None, dh_final=None, workspace=None,
-                       stream=None, debug_flags: int = 0, timeout_cycles: int = 0):
+                       stream=None, debug_flags: int = 0, timeout_cycles: int = 0, ckpt=None):
     """Backward pass of jamba_ssm_scan: the gradients of a loss with respect to
     every input, given dout = dL/dout [batch, seqlen, d_inner] (the dtype of x)
     and optionally dh_final = dL/dh_final [batch, d_inner, d_state] fp32.
@@ -167,7 +179,9 @@ def jamba_ssm_scan_bwd(x, delta, z, B, C, A, dout, D=None, delta_bias=None,
     ``workspace``: a device tensor of at least
     ``jamba_ssm_scan_bwd_workspace_size(...)`` bytes whose first 16 bytes are
     zero (allocated here when None; its status word is read with
-    ``jamba_ssm_get_status(workspace=...)``)."""
+    ``jamba_ssm_get_status(workspace=...)``).
+    ``ckpt``: the checkpoints a ``jamba_ssm_scan(..., ckpt=...)`` on the same
+    inputs stored; the backward then skips its own checkpoint pass."""
     if x.dtype not in _IO:
         raise TypeError(f"x must be bfloat16 or float32, got {x.dtype}")
     batch, seqlen, d_inner = x.shape
@@ -182,6 +196,8 @@ def jamba_ssm_scan_bwd(x, delta, z, B, C, A, dout, D=None, delta_bias=None,
     _check(delta_bias, "delta_bias", (d_inner,), torch.float32, dev)
     _check(h0, "h0", (batch, d_inner, d_state), torch.float32, dev)
     _check(dh_final, "dh_final", (batch, d_inner, d_state), torch.float32, dev)
+    if ckpt is not None:
+        _check(ckpt, "ckpt", (batch, (seqlen + 15) // 16, d_inner, d_state), torch.float32, dev)
     if workspace is None:
         need = jamba_ssm_scan_bwd_workspace_size(batch, seqlen, d_inner, d_state)
         workspace = torch.zeros(max(need, _lib.STATUS_BYTES), dtype=torch.uint8, device=dev)
@@ -199,7 +215,7 @@ def jamba_ssm_scan_bwd(x, delta, z, B, C, A, dout, D=None, delta_bias=None,
         dout=_ptr(dout), dh_final=_ptr(dh_final),
         **{k: _ptr(v) for k, v in g.items()},
         workspace=ws, workspace_bytes=ws_bytes, debug_flags=int(debug_flags),
-        timeout_cycles=int(timeout_cycles))
+        timeout_cycles=int(timeout_cycles), ckpt=_ptr(ckpt))
     st = _lib.call_scan_bwd(p, _stream(stream, dev))
     if st != _lib.OK:
         raise JambaSSMError(st, "jamba_ssm_scan_bwd")

@@ -23,6 +23,7 @@ BF16, F32 = 0, 1
 EXPORTS = (
     "jamba_ssm_scan",
     "jamba_ssm_scan_workspace_size",
+    "jamba_ssm_scan_ckpt_size",
     "jamba_ssm_scan_bwd",
     "jamba_ssm_scan_bwd_workspace_size",
     "jamba_ssm_scan_bwd_noalloc",
@@ -65,6 +66,8 @@ class ScanParams(ctypes.Structure):
         ("state_indices", _vp), ("num_slots", ctypes.c_int64),
         # ABI version 3
         ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+        # ABI version 4
+        ("ckpt", _fp),
     ]
 
 
@@ -101,6 +104,8 @@ class ScanBwdParams(ctypes.Structure):
         ("dA", _fp), ("dD", _fp), ("ddelta_bias", _fp), ("dh0", _fp),
         ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
         ("debug_flags", ctypes.c_uint32), ("timeout_cycles", ctypes.c_uint64),
+        # ABI version 4
+        ("ckpt", _fp),
     ]
 
 
@@ -182,6 +187,8 @@ def lib():
                 L.jamba_ssm_get_status.argtypes = [_vp, _vp]
                 L.jamba_ssm_scan_workspace_size.restype = ctypes.c_size_t
                 L.jamba_ssm_scan_workspace_size.argtypes = [ctypes.c_int64] * 4
+                L.jamba_ssm_scan_ckpt_size.restype = ctypes.c_size_t
+                L.jamba_ssm_scan_ckpt_size.argtypes = [ctypes.c_int64] * 4
                 L.jamba_ssm_scan_bwd.restype = ctypes.c_int
                 L.jamba_ssm_scan_bwd.argtypes = [ctypes.POINTER(ScanBwdParams), _vp]
                 L.jamba_ssm_ssd_scan.restype = ctypes.c_int
@@ -235,6 +242,8 @@ SCAN_PARAMS_V1_SIZE = ScanParams.cu_seqlens.offset
 STATE_UPDATE_PARAMS_V1_SIZE = StateUpdateParams.state_indices.offset
 SCAN_PARAMS_V2_SIZE = ScanParams.workspace.offset
 STATE_UPDATE_PARAMS_V2_SIZE = StateUpdateParams.workspace.offset
+SCAN_PARAMS_V3_SIZE = ScanParams.ckpt.offset
+SCAN_BWD_PARAMS_V3_SIZE = ScanBwdParams.ckpt.offset
 
 
 def new_scan_params(**kw) -> ScanParams:
@@ -287,6 +296,10 @@ def get_status(stream: int, workspace: int = 0) -> int:
 
 def scan_workspace_size(batch: int, seqlen: int, d_inner: int, d_state: int) -> int:
     return lib().jamba_ssm_scan_workspace_size(batch, seqlen, d_inner, d_state)
+
+
+def scan_ckpt_size(batch: int, seqlen: int, d_inner: int, d_state: int) -> int:
+    return lib().jamba_ssm_scan_ckpt_size(batch, seqlen, d_inner, d_state)
 
 
 def scan_bwd_workspace_size(batch: int, seqlen: int, d_inner: int, d_state: int) -> int:

@@ -115,8 +115,9 @@ struct ScanVariant {
     int smem, smem_serving;
     const void *kernel;          // batched layout
     const void *kernel_serving;  // packed layout and / or state-cache slots
-    const void *kernel_ckpt;     // the backward's checkpoint pass, or null
-    bool attr_set_ckpt[kMaxDevices];
+    const void *kernel_ckpt;      // the backward's checkpoint pass, or null
+    const void *kernel_fwd_ckpt;  // the forward storing the same checkpoints, or null
+    bool attr_set_ckpt[kMaxDevices], attr_set_fwd_ckpt[kMaxDevices];
     bool attr_set[kMaxDevices], attr_set_serving[kMaxDevices];
 };
 
@@ -139,9 +140,12 @@ ScanVariant make_fused(double step_cost) {
     v.kernel = reinterpret_cast<const void *>(&jssm::s6_scan_fused_kernel<IoT, N, G, NW, TT, S>);
     v.kernel_serving =
         reinterpret_cast<const void *>(&jssm::s6_scan_serving_kernel<IoT, N, G, NW, TT, S>);
-    if (CKPT)
+    if (CKPT) {
         v.kernel_ckpt =
-            reinterpret_cast<const void *>(&jssm::s6_scan_fused_kernel<IoT, N, G, NW, TT, S, true>);
+            reinterpret_cast<const void *>(&jssm::s6_scan_fused_kernel<IoT, N, G, NW, TT, S, 1>);
+        v.kernel_fwd_ckpt =
+            reinterpret_cast<const void *>(&jssm::s6_scan_fused_kernel<IoT, N, G, NW, TT, S, 2>);
+    }
     return v;
 }
 
@@ -152,7 +156,8 @@ ScanVariant make_fused(double step_cost) {
 // lanes give narrower CTAs, so a single sequence's 8192 channels still cover
 // the 148 SMs (56 channels per CTA -> 147 CTAs).  The variants marked `true`
 // also serve the backward's checkpoint pass (the states alone, stored every
-// kCk steps), chosen by the same cost model.
+// kCk steps) and the forward that stores those checkpoints, chosen by the same
+// cost model.
 ScanVariant g_variants[] = {
     make_fused<__nv_bfloat16, 16, 2, 8, 64, 2, true>(1.00),  // 1: 128 channels / CTA
     make_fused<__nv_bfloat16, 16, 4, 7, 64, 3, true>(1.33),  // 2:  56 channels / CTA
@@ -222,6 +227,7 @@ constexpr int64_t kMaxI32 = (int64_t(1) << 31) - 1;
 // as zero / NULL.
 constexpr size_t kScanParamsV1 = offsetof(jamba_ssm_scan_params, cu_seqlens);
 constexpr size_t kUpdateParamsV1 = offsetof(jamba_ssm_state_update_params, state_indices);
+constexpr size_t kBwdParamsV3 = offsetof(jamba_ssm_scan_bwd_params, ckpt);
 
 // A workspace, when given, holds the call's status word in its first bytes.
 jamba_ssm_status check_workspace(const void *ws, size_t bytes) {
@@ -271,6 +277,14 @@ jamba_ssm_status validate_scan(const jamba_ssm_scan_params *p) {
         return JAMBA_SSM_ERR_UNSUPPORTED;  // grid (channel blocks, sequences)
     jamba_ssm_status ws = check_workspace(p->workspace, p->workspace_bytes);
     if (ws != JAMBA_SSM_OK) return ws;
+    if (p->ckpt) {  // the backward's checkpoints: its layouts and state sizes only
+        const bool bf = p->io_dtype == JAMBA_SSM_BF16;
+        const bool n_ck = p->d_state == 16 || p->d_state == 8 || (!bf && p->d_state == 4);
+        if (p->cu_seqlens || p->state_indices || !n_ck) return JAMBA_SSM_ERR_UNSUPPORTED;
+        if (p->kernel_variant > 0 && !g_variants[p->kernel_variant - 1].kernel_fwd_ckpt)
+            return JAMBA_SSM_ERR_UNSUPPORTED;
+        if (!aligned(p->ckpt, 16)) return JAMBA_SSM_ERR_MISALIGNED;
+    }
     const int64_t tok = token_rows(p);
     const int64_t state_rows = p->state_indices ? p->num_slots : p->batch;
     const size_t state_bytes = size_t(state_rows) * p->d_inner * p->d_state * 4;
@@ -288,6 +302,14 @@ jamba_ssm_status validate_scan(const jamba_ssm_scan_params *p) {
         for (int i = 0; i < 5; ++i)
             if (overlaps(p->out, act, ins[i], insz[i])) return JAMBA_SSM_ERR_INVALID_ARG;
         if (overlaps(p->h_final, state_bytes, p->out, act)) return JAMBA_SSM_ERR_INVALID_ARG;
+        if (p->ckpt) {
+            const size_t ckb = size_t(p->batch) * size_t((p->seqlen + jssm::kCk - 1) / jssm::kCk) *
+                               p->d_inner * p->d_state * 4;
+            const void *all[] = {p->x, p->delta, p->z, p->B, p->C, p->out, p->h0, p->h_final};
+            const size_t allsz[] = {act, act, act, bc, bc, act, state_bytes, state_bytes};
+            for (int i = 0; i < 8; ++i)
+                if (overlaps(p->ckpt, ckb, all[i], allsz[i])) return JAMBA_SSM_ERR_INVALID_ARG;
+        }
     } else if (p->batch > 0) {
         if (!aligned(p->h0, 16) || !aligned(p->h_final, 16)) return JAMBA_SSM_ERR_MISALIGNED;
     }
@@ -312,7 +334,8 @@ jamba_ssm_status plan_scan(const jamba_ssm_scan_params *p, const DeviceInfo *dev
                                                                                     : plan->tasks));
         return JAMBA_SSM_OK;
     }
-    const int vi = p->kernel_variant > 0 ? p->kernel_variant - 1 : choose_variant(p, dev->sms);
+    const int vi = p->kernel_variant > 0 ? p->kernel_variant - 1
+                                         : choose_variant(p, dev->sms, p->ckpt != nullptr);
     if (vi < 0) return JAMBA_SSM_ERR_UNSUPPORTED;
     const ScanVariant &v = g_variants[vi];
     const int cc = channels_per_cta(v);
@@ -580,15 +603,19 @@ jamba_ssm_status jamba_ssm_scan(const jamba_ssm_scan_params *pin, void *stream) 
         !encode_3d(fn, &maps[4], p->C, dt, es, p->d_state, dim_t, dim_b, (int)p->d_state, v.tt))
         return JAMBA_SSM_ERR_UNSUPPORTED;
 
-    // the serving kernel for packed sequences or cache slots, else the batched one
+    // the serving kernel for packed sequences or cache slots, the batched one
+    // storing checkpoints when asked, else the batched one
     const bool serving = p->cu_seqlens != nullptr || p->state_indices != nullptr;
-    const void *kernel = serving ? v.kernel_serving : v.kernel;
+    const bool with_ckpt = p->ckpt != nullptr;
+    const void *kernel = serving ? v.kernel_serving : (with_ckpt ? v.kernel_fwd_ckpt : v.kernel);
     const int smem = serving ? v.smem_serving : v.smem;
+    args.ckpt = p->ckpt;
     int devid = 0;
     cudaGetDevice(&devid);
     {
         std::lock_guard<std::mutex> lock(g_mutex);
-        bool &set = serving ? v.attr_set_serving[devid] : v.attr_set[devid];
+        bool &set = serving ? v.attr_set_serving[devid]
+                            : (with_ckpt ? v.attr_set_fwd_ckpt[devid] : v.attr_set[devid]);
         if (!set) {
             cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  smem);
@@ -758,8 +785,16 @@ size_t jamba_ssm_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t 
     return bwd_layout(batch, seqlen, d_inner, d_state, sh.cc).total;
 }
 
-jamba_ssm_status jamba_ssm_scan_bwd(const jamba_ssm_scan_bwd_params *p, void *stream) {
-    if (!p || p->struct_size < sizeof(jamba_ssm_scan_bwd_params)) return JAMBA_SSM_ERR_INVALID_ARG;
+size_t jamba_ssm_scan_ckpt_size(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t d_state) {
+    if (batch < 0 || seqlen < 0 || d_inner < 0 || d_state < 0) return 0;
+    return size_t(batch) * size_t((seqlen + jssm::kCk - 1) / jssm::kCk) * size_t(d_inner) *
+           size_t(d_state) * 4;
+}
+
+jamba_ssm_status jamba_ssm_scan_bwd(const jamba_ssm_scan_bwd_params *pin, void *stream) {
+    jamba_ssm_scan_bwd_params prm;
+    if (!read_params(pin, kBwdParamsV3, &prm)) return JAMBA_SSM_ERR_INVALID_ARG;
+    const jamba_ssm_scan_bwd_params *p = &prm;
     if (p->batch < 0 || p->seqlen < 0 || p->d_inner < 1 || p->d_state < 1)
         return JAMBA_SSM_ERR_INVALID_ARG;
     if (p->io_dtype != JAMBA_SSM_BF16 && p->io_dtype != JAMBA_SSM_F32) return JAMBA_SSM_ERR_INVALID_ARG;
@@ -791,17 +826,19 @@ jamba_ssm_status jamba_ssm_scan_bwd(const jamba_ssm_scan_bwd_params *p, void *st
     }
     if (!aligned(p->D, 4) || !aligned(p->delta_bias, 4) || !aligned(p->dA, 4) ||
         !aligned(p->dD, 4) || !aligned(p->ddelta_bias, 4) || !aligned(p->h0, 4) ||
-        !aligned(p->dh_final, 4) || !aligned(p->dh0, 4))
+        !aligned(p->dh_final, 4) || !aligned(p->dh0, 4) || !aligned(p->ckpt, 16))
         return JAMBA_SSM_ERR_MISALIGNED;
     // no output may overlap an input, another output or the workspace
     const void *outs[] = {p->dx, p->ddelta, p->dz, p->dB, p->dC, p->dA, p->dD, p->ddelta_bias,
                           p->dh0};
     const size_t outsz[] = {act, act, act, bc, bc, an, pn, pn, st};
-    const void *ins[] = {p->x, p->delta, p->z, p->B, p->C, p->A, p->D, p->delta_bias, p->h0,
-                         p->dout, p->dh_final, p->workspace};
-    const size_t insz[] = {act, act, act, bc, bc, an, pn, pn, st, act, st, lay.total};
+    const size_t ckb = size_t(p->batch) * size_t(lay.nck) * p->d_inner * p->d_state * 4;
+    const void *ins[] = {p->x,  p->delta, p->z,        p->B,         p->C,
+                         p->A,  p->D,     p->delta_bias, p->h0,      p->dout,
+                         p->dh_final, p->workspace, p->ckpt};
+    const size_t insz[] = {act, act, act, bc, bc, an, pn, pn, st, act, st, lay.total, ckb};
     for (int i = 0; i < 9; ++i) {
-        for (int j = 0; j < 12; ++j)
+        for (int j = 0; j < 13; ++j)
             if (overlaps(outs[i], outsz[i], ins[j], insz[j])) return JAMBA_SSM_ERR_INVALID_ARG;
         for (int j = i + 1; j < 9; ++j)
             if (overlaps(outs[i], outsz[i], outs[j], outsz[j])) return JAMBA_SSM_ERR_INVALID_ARG;
@@ -850,8 +887,9 @@ jamba_ssm_status jamba_ssm_scan_bwd(const jamba_ssm_scan_bwd_params *p, void *st
     a.h0 = p->h0;
     a.dh_final = p->dh_final;
     a.delta_softplus = p->delta_softplus != 0;
+    // the forward's checkpoints when the caller has them, else this call's own
     float *ckpt = reinterpret_cast<float *>(ws + lay.off_ckpt);
-    a.ckpt = ckpt;
+    a.ckpt = p->ckpt ? p->ckpt : ckpt;
     a.part_bc = reinterpret_cast<float *>(ws + lay.off_bc);
     a.part_par = reinterpret_cast<float *>(ws + lay.off_par);
     a.dh0 = p->dh0;
@@ -861,9 +899,10 @@ jamba_ssm_status jamba_ssm_scan_bwd(const jamba_ssm_scan_bwd_params *p, void *st
 
     const CUtensorMapDataType dt = p->io_dtype == JAMBA_SSM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    // 1. checkpoints: the forward kernel in its checkpoint mode, the variant
-    //    the forward's cost model picks for this shape
-    {
+    // 1. checkpoints (unless the caller passed the forward's): the forward
+    //    kernel in its checkpoint mode, the variant the forward's cost model
+    //    picks for this shape
+    if (!p->ckpt) {
         jamba_ssm_scan_params fp{};
         fp.struct_size = sizeof(fp);
         fp.batch = p->batch;
@@ -1081,12 +1120,12 @@ __global__ void s6_noalloc_status_kernel(const int *word) {
 
 extern "C" jamba_ssm_status jamba_ssm_scan_bwd_noalloc(const jamba_ssm_scan_bwd_params *pin,
                                                        void *stream) {
-    if (!pin || pin->struct_size < sizeof(jamba_ssm_scan_bwd_params)) return JAMBA_SSM_ERR_INVALID_ARG;
-    if (pin->workspace || pin->workspace_bytes) return JAMBA_SSM_ERR_INVALID_ARG;
-    const size_t need =
-        jamba_ssm_scan_bwd_workspace_size(pin->batch, pin->seqlen, pin->d_inner, pin->d_state);
+    jamba_ssm_scan_bwd_params q;  // an ABI version 3 caller's struct reads with ckpt NULL
+    if (!read_params(pin, kBwdParamsV3, &q)) return JAMBA_SSM_ERR_INVALID_ARG;
+    if (q.workspace || q.workspace_bytes) return JAMBA_SSM_ERR_INVALID_ARG;
+    const size_t need = jamba_ssm_scan_bwd_workspace_size(q.batch, q.seqlen, q.d_inner, q.d_state);
     if (need == 0)  // sizes the backward does not take
-        return (pin->batch < 0 || pin->seqlen < 0 || pin->d_inner < 1 || pin->d_state < 1)
+        return (q.batch < 0 || q.seqlen < 0 || q.d_inner < 1 || q.d_state < 1)
                    ? JAMBA_SSM_ERR_INVALID_ARG
                    : JAMBA_SSM_ERR_UNSUPPORTED;
     if (need > JAMBA_SSM_BWD_NOALLOC_SCRATCH_BYTES) return JAMBA_SSM_ERR_WORKSPACE;
@@ -1111,7 +1150,7 @@ extern "C" jamba_ssm_status jamba_ssm_scan_bwd_noalloc(const jamba_ssm_scan_bwd_
     // start at zero (every other part is written before it is read)
     e = cudaMemsetAsync(scratch, 0, JAMBA_SSM_STATUS_BYTES, s);
     if (e != cudaSuccess) return cuda_fail(e);
-    jamba_ssm_scan_bwd_params q = *pin;
+    q.struct_size = sizeof(q);
     q.workspace = scratch;
     q.workspace_bytes = JAMBA_SSM_BWD_NOALLOC_SCRATCH_BYTES;
     st = jamba_ssm_scan_bwd(&q, stream);

@@ -72,13 +72,13 @@ struct OwnedStep {
     float dl, dx, gate, skg;
 };
 
-template <bool SOFTPLUS, bool LDS, bool CKPT, typename IoT>
+template <bool SOFTPLUS, bool LDS, bool NO_OUT, typename IoT>
 __device__ __forceinline__ OwnedStep owned_step(const IoT *xs, const IoT *dts, const IoT *zs, int idx,
                                                 float bias, float dskip) {
     const float xo = LDS ? lds_f32(xs + idx) : to_f32(xs[idx]);
     const float v = (LDS ? lds_f32(dts + idx) : to_f32(dts[idx])) + bias;
     const float dl = SOFTPLUS ? softplus_io<IoT>(v) : v;
-    if (CKPT) return OwnedStep{dl, dl * xo, 0.0f, 0.0f};  // no output, no gate
+    if (NO_OUT) return OwnedStep{dl, dl * xo, 0.0f, 0.0f};  // no output, no gate
     const float gate = silu_f32(LDS ? lds_f32(zs + idx) : to_f32(zs[idx]));
     return OwnedStep{dl, dl * xo, gate, dskip * xo * gate};
 }
@@ -115,12 +115,13 @@ __device__ __forceinline__ void group_exps(const OwnedStep &o, const float2 (&a2
 // unrolled body would split it into basic blocks that the scheduler cannot
 // interleave.
 //
-// CKPT (the backward's checkpoint pass): only the states advance; before every
-// kCk-th step of the tile the lane stores its NS states at ck + (step / kCk) *
-// ck_stride (ck null: nothing stored), and the readout, gate and output tile
-// are skipped.
+// MODE 0: the forward.  MODE 1 (the backward's checkpoint pass): only the
+// states advance; before every kCk-th step of the tile the lane stores its NS
+// states at ck + (step / kCk) * ck_stride (ck null: nothing stored), and the
+// readout, gate and output tile are skipped.  MODE 2: the forward, storing the
+// same checkpoints as it goes (for a backward that follows).
 template <bool SOFTPLUS, typename IoT, int N, int G, int NS, int TT, int CC, int BCROW,
-          bool CKPT = false>
+          int MODE = 0>
 __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float2 (&a2)[NS / 2],
                                                 float bias, float dskip,
                                                 const IoT *xs, const IoT *dts, const IoT *zs,
@@ -130,10 +131,11 @@ __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float
     constexpr int NG = TT / G;
     static_assert(NG >= 3, "a tile holds at least three groups");
     constexpr bool LDS = G == 2;  // explicit shared-space accesses (see load_bc_shared)
-    static_assert(!CKPT || (TT % kCk == 0 && kCk % G == 0), "checkpoints at group starts");
-    OwnedStep o0 = owned_step<SOFTPLUS, LDS, CKPT>(xs, dts, zs, sub * CC + c_local, bias, dskip);
-    OwnedStep o1 = owned_step<SOFTPLUS, LDS, CKPT>(xs, dts, zs, (G + sub) * CC + c_local, bias, dskip);
-    OwnedStep o2 = owned_step<SOFTPLUS, LDS, CKPT>(xs, dts, zs, (2 * G + sub) * CC + c_local, bias, dskip);
+    constexpr bool kStoreCk = MODE != 0, kNoOut = MODE == 1;
+    static_assert(!kStoreCk || (TT % kCk == 0 && kCk % G == 0), "checkpoints at group starts");
+    OwnedStep o0 = owned_step<SOFTPLUS, LDS, kNoOut>(xs, dts, zs, sub * CC + c_local, bias, dskip);
+    OwnedStep o1 = owned_step<SOFTPLUS, LDS, kNoOut>(xs, dts, zs, (G + sub) * CC + c_local, bias, dskip);
+    OwnedStep o2 = owned_step<SOFTPLUS, LDS, kNoOut>(xs, dts, zs, (2 * G + sub) * CC + c_local, bias, dskip);
     float2 dxa[G], aba[G][NS / 2], dxb[G], abb[G][NS / 2];
     group_exps<G, NS>(o0, a2, gbase, dxa, aba);
     group_exps<G, NS>(o1, a2, gbase, dxb, abb);
@@ -142,10 +144,10 @@ __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float
         const int t0 = g * G;
         OwnedStep o3 = o2;
         if (g + 3 < NG)
-            o3 = owned_step<SOFTPLUS, LDS, CKPT>(xs, dts, zs, (t0 + 3 * G + sub) * CC + c_local, bias, dskip);
+            o3 = owned_step<SOFTPLUS, LDS, kNoOut>(xs, dts, zs, (t0 + 3 * G + sub) * CC + c_local, bias, dskip);
         float2 dxc[G], abc[G][NS / 2];
         float yp[G];
-        if (CKPT && (t0 % kCk) == 0 && ck) store_states<NS>(ck + (t0 / kCk) * ck_stride, h);
+        if (kStoreCk && (t0 % kCk) == 0 && ck) store_states<NS>(ck + (t0 / kCk) * ck_stride, h);
 #pragma unroll
         for (int j = 0; j < G; ++j) {
             if (g + 2 < NG) {
@@ -164,11 +166,11 @@ __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float
 #pragma unroll
             for (int i = 0; i < NS / 2; ++i) {
                 h[i] = fma2(aba[j][i], h[i], mul2(dxa[j], bc.b[i]));
-                if (!CKPT) y2 = i == 0 ? mul2(bc.c[i], h[i]) : fma2(bc.c[i], h[i], y2);
+                if (!kNoOut) y2 = i == 0 ? mul2(bc.c[i], h[i]) : fma2(bc.c[i], h[i], y2);
             }
-            yp[j] = CKPT ? 0.0f : y2.x + y2.y;
+            yp[j] = kNoOut ? 0.0f : y2.x + y2.y;
         }
-        if (!CKPT) {
+        if (!kNoOut) {
             const float y = reduce_transpose<G>(yp, sub);
             const IoT ov = from_f32<IoT>(fmaf(y, o0.gate, o0.skg));
             if (LDS)
@@ -192,9 +194,10 @@ __device__ __forceinline__ void fused_tile_full(float2 (&h)[NS / 2], const float
     }
 }
 
-// CKPT: the backward's checkpoint pass (see fused_tile_full): no z or C loads,
-// no output stores; args.ckpt receives the states before every kCk-th step.
-template <typename IoT, int N, int G, int NW, int TT, int STAGES, bool CKPT = false>
+// MODE (see fused_tile_full): 0 the forward; 1 the backward's checkpoint pass
+// (no z or C loads, no output stores); 2 the forward storing checkpoints.  In
+// modes 1 and 2 args.ckpt receives the states before every kCk-th step.
+template <typename IoT, int N, int G, int NW, int TT, int STAGES, int MODE = 0>
 __global__ void __launch_bounds__((NW + 1) * 32, 1)
     s6_scan_fused_kernel(const __grid_constant__ CUtensorMap tm_x,
                          const __grid_constant__ CUtensorMap tm_dt,
@@ -217,7 +220,8 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
     const int64_t ngroups = (d_inner + CC - 1) / CC;
     const int64_t ntasks = args.batch * ngroups;
     const int ntiles = static_cast<int>((seqlen + TT - 1) / TT);
-    const int64_t nck = (seqlen + kCk - 1) / kCk;  // checkpoints per sequence (CKPT)
+    constexpr bool kStoreCk = MODE != 0, kNoOut = MODE == 1;
+    const int64_t nck = (seqlen + kCk - 1) / kCk;  // checkpoints per sequence (modes 1, 2)
     const int64_t my_tasks =
         static_cast<int64_t>(blockIdx.x) < ntasks ? (ntasks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const int64_t total = my_tasks * ntiles;
@@ -290,14 +294,14 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             const int s = static_cast<int>(g % STAGES);
             if ((args.debug_flags & 1u) && k == 0) return;  // test hook: withhold a first tile
             uint8_t *base = smem + s * Cfg::kStageBytes;
-            mbar_arrive_expect_tx(&full[s], CKPT ? Cfg::kTxBytes - Cfg::kActTile - Cfg::kBCTile
+            mbar_arrive_expect_tx(&full[s], kNoOut ? Cfg::kTxBytes - Cfg::kActTile - Cfg::kBCTile
                                                  : Cfg::kTxBytes);
             const int t0 = k * TT, bb = static_cast<int>(b);
             tma_load_3d(base, &tm_x, c0, t0, bb, &full[s]);
             tma_load_3d(base + Cfg::kActTile, &tm_dt, c0, t0, bb, &full[s]);
-            if (!CKPT) tma_load_3d(base + 2 * Cfg::kActTile, &tm_z, c0, t0, bb, &full[s]);
+            if (!kNoOut) tma_load_3d(base + 2 * Cfg::kActTile, &tm_z, c0, t0, bb, &full[s]);
             tma_load_3d(base + 3 * Cfg::kActTile, &tm_B, 0, t0, bb, &full[s]);
-            if (!CKPT)
+            if (!kNoOut)
                 tma_load_3d(base + 3 * Cfg::kActTile + Cfg::kBCTile, &tm_C, 0, t0, bb, &full[s]);
             armed |= 1u << s;
         };
@@ -308,7 +312,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
                                                limit, abort_flag)))
                 return false;
             if (lane == 0) {
-                if (!CKPT) {
+                if (!kNoOut) {
                     int64_t b;
                     int c0, k;
                     tile_of(cur_store, g, b, c0, k);
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
                 }
                 issue(g + STAGES);  // the compute warps are done with stage g % STAGES
                 if (g > 0) {
-                    if (!CKPT) bulk_wait_read<1>();  // the store of tile g-1 has read its buffer
+                    if (!kNoOut) bulk_wait_read<1>();  // the store of tile g-1 has read its buffer
                     mbar_arrive(&out_free[static_cast<int>((g - 1) % NOUT)]);
                 }
             }
@@ -354,10 +358,10 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             float *dst = bcs_all + s * Cfg::kBCe;
             // unit u = (step t, slot j, half: 0 = B, 1 = C): one slice of NS values
             // (B only for checkpoints)
-            constexpr int kHalves = CKPT ? 1 : 2;
+            constexpr int kHalves = kNoOut ? 1 : 2;
             for (int u = lane; u < nsteps * kHalves * G; u += 32) {
                 const int t = u / (kHalves * G), j = (u / kHalves) % G;
-                const int half = CKPT ? 0 : (u & 1);
+                const int half = kNoOut ? 0 : (u & 1);
                 stage_slice<NS>(dst + t * Cfg::kBCRow + (2 * j + half) * NS,
                                 (half ? Cs : Bs) + t * N + j * NS);
             }
@@ -442,7 +446,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
         // checkpoint pass: this lane's slice of the tile's first checkpoint
         float *ck = nullptr;
         const int64_t ck_stride = d_inner * N;
-        if (CKPT && dvalid)
+        if (kStoreCk && dvalid)
             ck = args.ckpt + ((b * nck + int64_t(k) * (TT / kCk)) * d_inner + d) * N + sub * NS;
 
         // One group of G steps starting at t0: the owner lane's scalars, the
@@ -453,7 +457,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
             const float xo = to_f32(xs[idx]);
             const float dl = delta_io<IoT>(to_f32(dts[idx]), bias, use_softplus);
             const float dx = dl * xo;
-            if (CKPT && (t0 % kCk) == 0 && ck) store_states<NS>(ck + (t0 / kCk) * ck_stride, h);
+            if (kStoreCk && (t0 % kCk) == 0 && ck) store_states<NS>(ck + (t0 / kCk) * ck_stride, h);
             float yp[G];
 #pragma unroll
             for (int j = 0; j < G; ++j) {
@@ -464,17 +468,17 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1)
                     yp[j] = recurrence_step<NS>(h, a2, make_float2(dlj, dxj),
                                                 bcs + (t0 + j) * Cfg::kBCRow, sub);
             }
-            if (!CKPT) {
+            if (!kNoOut) {
                 const float y = reduce_transpose<G>(yp, sub);
                 const float gate = silu_f32(to_f32(zs[idx]));
                 if (sub < valid) outs[idx] = from_f32<IoT>((y + dskip * xo) * gate);
             }
         };
         if (nsteps == TT && use_softplus) {
-            fused_tile_full<true, IoT, N, G, NS, TT, CC, Cfg::kBCRow, CKPT>(
+            fused_tile_full<true, IoT, N, G, NS, TT, CC, Cfg::kBCRow, MODE>(
                 h, a2, bias, dskip, xs, dts, zs, bcs, outs, c_local, sub, gbase, ck, ck_stride);
         } else if (nsteps == TT) {
-            fused_tile_full<false, IoT, N, G, NS, TT, CC, Cfg::kBCRow, CKPT>(
+            fused_tile_full<false, IoT, N, G, NS, TT, CC, Cfg::kBCRow, MODE>(
                 h, a2, bias, dskip, xs, dts, zs, bcs, outs, c_local, sub, gbase, ck, ck_stride);
         } else {
             for (int t0 = 0; t0 < nsteps; t0 += G) group(t0, nsteps - t0 < G ? nsteps - t0 : G);

@@ -89,7 +89,7 @@ def test_struct_layout_matches_header(tmp_path):
 
 
 def test_status_strings_and_version(L):
-    assert L.jamba_ssm_abi_version() == 3
+    assert L.jamba_ssm_abi_version() == 4
     for s in range(8):
         assert _lib.status_string(s) != "unknown status"
     assert _lib.status_string(99) == "unknown status"
@@ -396,3 +396,73 @@ def test_proj_abi_from_plain_c(P, tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert "passed" in r.stdout
+
+
+# ---------------------------------------------------------------- ABI version 4
+_CK = 0xB0000000  # fake, 16-byte aligned, clear of every buffer of _valid_scan
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ckpt=_CK + 8), _lib.ERR_MISALIGNED),
+    (dict(ckpt=_CK, cu_seqlens=0x3000, total_tokens=100), _lib.ERR_UNSUPPORTED),
+    (dict(ckpt=_CK, state_indices=0x3000, num_slots=4), _lib.ERR_UNSUPPORTED),
+    (dict(ckpt=_CK, d_state=4), _lib.ERR_UNSUPPORTED),      # bf16 d_state 4: no backward
+    (dict(ckpt=_CK, kernel_variant=3), _lib.ERR_UNSUPPORTED),  # a variant without that kernel
+    (dict(ckpt=0x90000000), _lib.ERR_INVALID_ARG),          # on top of out
+    (dict(ckpt=0x10000000 - 0x100), _lib.ERR_INVALID_ARG),  # runs into x
+])
+def test_scan_checkpoint_argument_errors(L, kw, expect):
+    assert _scan(_valid_scan(**kw)) == expect
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_scan_with_checkpoints_reaches_the_device_query(L):
+    assert _scan(_valid_scan(ckpt=_CK)) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
+    # fp32 I/O also takes d_state 4
+    assert _scan(_valid_scan(ckpt=_CK, io_dtype=_lib.F32, d_state=4)) in (
+        _lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_version_3_struct_size_is_accepted(L):
+    """A version-3 caller's struct ends before ckpt: whatever lies past it is
+    ignored, for the scan and for the backward (and its no-allocation form)."""
+    p = _valid_scan(ckpt=_CK + 8)  # misaligned if it were read
+    p.struct_size = _lib.SCAN_PARAMS_V3_SIZE
+    assert _scan(p) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
+    b = _valid_bwd(ckpt=_CK + 8)
+    b.struct_size = _lib.SCAN_BWD_PARAMS_V3_SIZE
+    assert _lib.call_scan_bwd(b, 0) in (_lib.ERR_NO_DEVICE, _lib.ERR_CUDA)
+    b.struct_size = _lib.SCAN_BWD_PARAMS_V3_SIZE - 8
+    assert _lib.call_scan_bwd(b, 0) == _lib.ERR_INVALID_ARG
+    n = _valid_bwd(ckpt=_CK + 8, workspace=None, workspace_bytes=0)
+    n.struct_size = _lib.SCAN_BWD_PARAMS_V3_SIZE
+    assert L.jamba_ssm_scan_bwd_noalloc(ctypes.byref(n), None) in (_lib.ERR_NO_DEVICE,
+                                                                     _lib.ERR_CUDA)
+
+
+def _valid_bwd(**kw):
+    base = dict(batch=1, seqlen=100, d_inner=256, d_state=16, io_dtype=_lib.BF16,
+                delta_softplus=1, x=0x10000000, delta=0x11000000, z=0x12000000,
+                B=0x13000000, C=0x14000000, A=0x15000000, dout=0x16000000, dx=0x17000000,
+                ddelta=0x18000000, dz=0x19000000, dB=0x1A000000, dC=0x1B000000,
+                workspace=0x40000000, workspace_bytes=1 << 26)
+    base.update(kw)
+    return _lib.new_scan_bwd_params(**base)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ckpt=_CK + 8), _lib.ERR_MISALIGNED),
+    (dict(ckpt=0x17000000), _lib.ERR_INVALID_ARG),  # an output (dx) on top of it
+])
+def test_backward_checkpoint_argument_errors(L, kw, expect):
+    assert _lib.call_scan_bwd(_valid_bwd(**kw), 0) == expect
+
+
+def test_checkpoint_size(L):
+    # ceil(100 / 16) = 7 checkpoints per sequence
+    assert _lib.scan_ckpt_size(2, 100, 256, 16) == 2 * 7 * 256 * 16 * 4
+    assert _lib.scan_ckpt_size(1, 0, 256, 16) == 0
+    assert _lib.scan_ckpt_size(1, 16, 8, 8) == 8 * 8 * 4
+    assert _lib.scan_ckpt_size(-1, 16, 8, 8) == 0
+

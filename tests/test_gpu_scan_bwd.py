@@ -8,6 +8,7 @@ the parameters and of the initial state -- dA, dD, ddelta_bias, dh0 -- under
 the rule for the fp32 state (rel-L2 <= 1e-4 with bf16 inputs, <= 1e-5 with fp32
 inputs): the inputs are identical on both sides, so only fp32 rounding inside
 the kernels differs, as for the forward's final state."""
+import numpy as np
 import pytest
 import torch
 
@@ -158,3 +159,81 @@ def test_backward_bounded_wait_times_out_and_reports():
     _compare(_run(inp, dout, dh, workspace=ws), _oracle(inp, dout, dh), torch.bfloat16,
              "after a timeout")
     assert jamba_ssm_get_status(workspace=ws) == _lib.OK
+
+
+# ------------------------------------------ checkpoints stored by the forward
+def _ckpt(inp):
+    b, L, d = inp.x.shape
+    return torch.full((b, (L + 15) // 16, d, inp.A.shape[-1]), float("nan"),
+                      dtype=torch.float32, device=inp.x.device)
+
+
+@pytest.mark.parametrize("dtype,n", [(torch.bfloat16, 16), (torch.bfloat16, 8),
+                                     (torch.float32, 16), (torch.float32, 4)])
+def test_forward_checkpoints_are_the_oracle_states_and_change_nothing(dtype, n):
+    """jamba_ssm_scan with ckpt: out and h_final are the same bits as without;
+    entry [b, k] is the state before step 16 k, which the oracle gives as the
+    final state of the first 16 k steps (entry 0 is h0)."""
+    d = 200 if dtype == torch.bfloat16 else 196
+    inp, _, _ = _case(2, 203, d, n, dtype, seed=67)
+    kw = dict(D=inp.D, delta_bias=inp.delta_bias, delta_softplus=inp.delta_softplus, h0=inp.h0)
+    out0, hf0 = jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, **kw)
+    ck = _ckpt(inp)
+    out1, hf1 = jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, ckpt=ck, **kw)
+    torch.cuda.synchronize()
+    assert jamba_ssm_get_status() == _lib.OK
+    assert torch.equal(out0, out1) and torch.equal(hf0, hf1)
+    assert not torch.isnan(ck).any(), "a checkpoint was not written"
+    refs = [inp.h0.cpu().double().numpy()]
+    for k in range(1, ck.shape[1]):
+        t = 16 * k
+        sl = lambda v: v[:, :t].contiguous()  # noqa: E731
+        _, hk = oracle.scan(sl(inp.x), sl(inp.delta), sl(inp.z), sl(inp.B), sl(inp.C), inp.A,
+                            D=inp.D, delta_bias=inp.delta_bias,
+                            delta_softplus=inp.delta_softplus, h0=inp.h0)
+        refs.append(hk)
+    ref = np.stack(refs, axis=1)
+    assert_state(ck, ref, dtype, f"checkpoints {dtype} N={n}")
+
+
+@pytest.mark.parametrize("dtype,n", [(torch.bfloat16, 16), (torch.float32, 8)])
+def test_backward_takes_the_forward_checkpoints(dtype, n):
+    """jamba_ssm_scan_bwd given the forward's checkpoints skips its own pass and
+    returns the same bits."""
+    d = 200 if dtype == torch.bfloat16 else 196
+    inp, dout, dh = _case(2, 203, d, n, dtype, seed=68)
+    ck = _ckpt(inp)
+    jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, D=inp.D,
+                   delta_bias=inp.delta_bias, delta_softplus=inp.delta_softplus, h0=inp.h0,
+                   ckpt=ck)
+    a = _run(inp, dout, dh)
+    b = _run(inp, dout, dh, ckpt=ck)
+    assert jamba_ssm_get_status() == _lib.OK
+    for k in IO_GRADS + F32_GRADS:
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_training_step_at_the_headline_size():
+    """Forward with checkpoints then backward with them, at Jamba's layer (one
+    sequence of 4096 tokens, d_inner 8192, d_state 16): the same gradients, bit
+    for bit, as the backward that makes its own checkpoints."""
+    dev = _dev()
+    w = synth.WORKLOADS["s6_prefill_bf16_b1_l4096_d8192_n16"]
+    inp = synth.workload_inputs(w, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(69)
+    dout = torch.randn(inp.x.shape, generator=g, device=dev).to(w.dtype)
+    ck = _ckpt(inp)
+    out, hf = jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, D=inp.D,
+                             delta_bias=inp.delta_bias, ckpt=ck)
+    out0, hf0 = jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, D=inp.D,
+                               delta_bias=inp.delta_bias)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out0) and torch.equal(hf, hf0)
+    kw = dict(D=inp.D, delta_bias=inp.delta_bias)
+    a = jamba_ssm_scan_bwd(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, dout, **kw)
+    b = jamba_ssm_scan_bwd(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, dout, ckpt=ck, **kw)
+    torch.cuda.synchronize()
+    assert jamba_ssm_get_status() == _lib.OK
+    for k in IO_GRADS + F32_GRADS:
+        assert torch.equal(a[k], b[k]), k
