@@ -15,7 +15,7 @@ import torch
 import oracle
 from selective_state_space_26_b200 import (_lib, jamba_ssm_get_status, jamba_ssm_scan,
                                            jamba_ssm_scan_bwd, jamba_ssm_scan_bwd_workspace_size,
-                                           synth)
+                                           scan_plan, synth)
 from tests.parity import assert_out, assert_state
 
 pytestmark = pytest.mark.gpu
@@ -237,3 +237,49 @@ def test_training_step_at_the_headline_size():
     assert jamba_ssm_get_status() == _lib.OK
     for k in IO_GRADS + F32_GRADS:
         assert torch.equal(a[k], b[k]), k
+
+
+@pytest.mark.parametrize("variant", [1, 2, 5, 7, 8, 9, 10])
+def test_forward_checkpoints_on_every_variant_that_stores_them(variant):
+    """Each launch shape with a checkpoint-storing forward, forced: the output is
+    the same bits as that variant's plain forward, and the checkpoints are the
+    oracle's states (the 2-lane variants are the library's choice at batch >= 2
+    and are not reached by the shapes above)."""
+    info = _lib.variant_info(variant)
+    dtype = torch.bfloat16 if info["io_dtype"] == _lib.BF16 else torch.float32
+    n = info["d_state"]
+    inp, _, _ = _case(2, 150, 256, n, dtype, seed=70 + variant)
+    kw = dict(D=inp.D, delta_bias=inp.delta_bias, delta_softplus=inp.delta_softplus, h0=inp.h0,
+              variant=variant)
+    out0, hf0 = jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, **kw)
+    ck = _ckpt(inp)
+    out1, hf1 = jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, ckpt=ck, **kw)
+    torch.cuda.synchronize()
+    assert jamba_ssm_get_status() == _lib.OK
+    assert torch.equal(out0, out1) and torch.equal(hf0, hf1)
+    refs = [inp.h0.cpu().double().numpy()]
+    for k in range(1, ck.shape[1]):
+        sl = lambda v: v[:, :16 * k].contiguous()  # noqa: E731
+        refs.append(oracle.scan(sl(inp.x), sl(inp.delta), sl(inp.z), sl(inp.B), sl(inp.C),
+                                inp.A, D=inp.D, delta_bias=inp.delta_bias,
+                                delta_softplus=inp.delta_softplus, h0=inp.h0)[1])
+    assert_state(ck, np.stack(refs, axis=1), dtype, f"checkpoints, variant {variant}")
+
+
+def test_backward_many_sequences_takes_the_two_lane_checkpoint_pass():
+    """32 sequences of 1024 channels: the cost model picks the 2-lane variant
+    for the backward's checkpoint pass (and for a forward storing checkpoints),
+    with two tasks per persistent CTA; the gradients match the oracle and the
+    forward's checkpoints give the same bits."""
+    inp, dout, dh = _case(32, 70, 1024, 16, torch.bfloat16, seed=79)
+    plan = scan_plan(inp.x, inp.A)
+    assert plan["lanes_per_channel"] == 2, plan
+    got = _run(inp, dout, dh)
+    _compare(got, _oracle(inp, dout, dh), torch.bfloat16, "bwd, 16 sequences")
+    ck = _ckpt(inp)
+    jamba_ssm_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, D=inp.D,
+                   delta_bias=inp.delta_bias, delta_softplus=inp.delta_softplus, h0=inp.h0,
+                   ckpt=ck)
+    again = _run(inp, dout, dh, ckpt=ck)
+    for k in IO_GRADS + F32_GRADS:
+        assert torch.equal(got[k], again[k]), k
