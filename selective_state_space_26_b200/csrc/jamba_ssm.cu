@@ -140,7 +140,7 @@ ScanVariant make_fused(double step_cost) {
     v.kernel = reinterpret_cast<const void *>(&jssm::s6_scan_fused_kernel<IoT, N, G, NW, TT, S>);
     v.kernel_serving =
         reinterpret_cast<const void *>(&jssm::s6_scan_serving_kernel<IoT, N, G, NW, TT, S>);
-    if (CKPT) {
+    if constexpr (CKPT) {
         v.kernel_ckpt =
             reinterpret_cast<const void *>(&jssm::s6_scan_fused_kernel<IoT, N, G, NW, TT, S, 1>);
         v.kernel_fwd_ckpt =
