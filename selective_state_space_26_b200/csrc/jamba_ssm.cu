@@ -16,6 +16,7 @@
 #include "s6_scan_serving.cuh"
 #include "s6_scan_small.cuh"
 #include "s6_ssd.cuh"
+#include "s6_ssd_chunk.cuh"
 #include "s6_state_update.cuh"
 
 using jssm::ScanArgs;
@@ -96,14 +97,15 @@ EncodeTiledFn encode_fn(jamba_ssm_status *st) {
 
 // 3-D map over [dim2][dim1][dim0] (dim0 innermost), box {box0, box1, 1}.
 bool encode_3d(EncodeTiledFn fn, CUtensorMap *map, const void *ptr, CUtensorMapDataType dt,
-               int elem_bytes, int64_t dim0, int64_t dim1, int64_t dim2, int box0, int box1) {
+               int elem_bytes, int64_t dim0, int64_t dim1, int64_t dim2, int box0, int box1,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
     cuuint64_t dims[3] = {(cuuint64_t)dim0, (cuuint64_t)dim1, (cuuint64_t)dim2};
     cuuint64_t strides[2] = {(cuuint64_t)(dim0 * elem_bytes), (cuuint64_t)(dim0 * dim1 * elem_bytes)};
     cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)box1, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, dt, 3, const_cast<void *>(ptr), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -432,6 +434,16 @@ SsdKernel g_ssd[2][2][2] = {
      {make_ssd<__nv_bfloat16, 8, false>(), make_ssd<__nv_bfloat16, 8, true>()}},
     {{make_ssd<float, 16, false>(), make_ssd<float, 16, true>()},
      {make_ssd<float, 8, false>(), make_ssd<float, 8, true>()}},
+};
+
+// The chunked tensor-core form (bf16, d_state 16, headdim 64), softplus off / on.
+struct SsdChunkKernel {
+    const void *k;
+    bool attr[kMaxDevices];
+};
+SsdChunkKernel g_ssd_chunk[2] = {
+    {reinterpret_cast<const void *>(&jssm::s6_ssd_chunk_kernel<false>), {}},
+    {reinterpret_cast<const void *>(&jssm::s6_ssd_chunk_kernel<true>), {}},
 };
 
 }  // namespace
@@ -1033,10 +1045,59 @@ jamba_ssm_status jamba_ssm_ssd_scan(const jamba_ssm_ssd_params *p, void *stream)
                               : cudaMemsetAsync(p->h_final, 0, st, s);
         return e == cudaSuccess ? finish_launch(s, p->workspace) : cuda_fail(e);
     }
-    SsdKernel &K = g_ssd[p->io_dtype == JAMBA_SSM_BF16 ? 0 : 1][p->d_state == 16 ? 0 : 1]
-                        [p->delta_softplus ? 1 : 0];
     EncodeTiledFn fn = encode_fn(&stt);
     if (!fn) return stt;
+    int devid = 0;
+    cudaGetDevice(&devid);
+    const uint64_t timeout = p->timeout_cycles ? p->timeout_cycles : (uint64_t(1) << 31);
+    if (p->io_dtype == JAMBA_SSM_BF16 && p->d_state == 16 && p->headdim == jssm::SsdChunkCfg::P &&
+        !(p->debug_flags & 2u)) {
+        // chunked form on the tensor cores: one CTA per (sequence, head)
+        using CC = jssm::SsdChunkCfg;
+        const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        jssm::SsdChunkMaps m;
+        if (!encode_3d(fn, &m.x, p->x, bf, 2, D, p->seqlen, p->batch, CC::P, CC::Q,
+                       CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_3d(fn, &m.z, p->z, bf, 2, D, p->seqlen, p->batch, CC::P, CC::Q,
+                       CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_3d(fn, &m.dt, p->delta, bf, 2, p->nheads, p->seqlen, p->batch, CC::kHeadsBox,
+                       CC::Q) ||
+            !encode_3d(fn, &m.B, p->B, bf, 2, CC::N, p->seqlen, p->batch, CC::N, CC::Q,
+                       CU_TENSOR_MAP_SWIZZLE_32B) ||
+            !encode_3d(fn, &m.C, p->C, bf, 2, CC::N, p->seqlen, p->batch, CC::N, CC::Q,
+                       CU_TENSOR_MAP_SWIZZLE_32B))
+            return JAMBA_SSM_ERR_UNSUPPORTED;
+        SsdChunkKernel &K = g_ssd_chunk[p->delta_softplus ? 1 : 0];
+        {
+            std::lock_guard<std::mutex> lock(g_mutex);
+            if (!K.attr[devid]) {
+                cudaError_t e = cudaFuncSetAttribute(K.k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     static_cast<int>(CC::kSmemBytes));
+                if (e != cudaSuccess) return cuda_fail(e);
+                K.attr[devid] = true;
+            }
+        }
+        jssm::SsdChunkArgs a{};
+        a.seqlen = p->seqlen;
+        a.nheads = p->nheads;
+        a.A = p->A;
+        a.D = p->D;
+        a.delta_bias = p->delta_bias;
+        a.h0 = p->h0;
+        a.h_final = p->h_final;
+        a.out = static_cast<__nv_bfloat16 *>(p->out);
+        a.status = static_cast<int *>(p->workspace);
+        a.debug_flags = p->debug_flags;
+        a.timeout_cycles = timeout;
+        const dim3 grid(static_cast<unsigned>(p->nheads), static_cast<unsigned>(p->batch));
+        void *kargs[] = {&m, &a};
+        cudaError_t e = cudaLaunchKernel(K.k, grid, dim3(CC::kThreads), kargs,
+                                         static_cast<size_t>(CC::kSmemBytes), s);
+        if (e != cudaSuccess) return cuda_fail(e);
+        return finish_launch(s, p->workspace);
+    }
+    SsdKernel &K = g_ssd[p->io_dtype == JAMBA_SSM_BF16 ? 0 : 1][p->d_state == 16 ? 0 : 1]
+                        [p->delta_softplus ? 1 : 0];
     const CUtensorMapDataType dt =
         p->io_dtype == JAMBA_SSM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     jssm::SsdMaps m;
@@ -1047,8 +1108,6 @@ jamba_ssm_status jamba_ssm_ssd_scan(const jamba_ssm_ssd_params *p, void *stream)
         !encode_3d(fn, &m.B, p->B, dt, es, p->d_state, p->seqlen, p->batch, (int)p->d_state, kSsdTT) ||
         !encode_3d(fn, &m.C, p->C, dt, es, p->d_state, p->seqlen, p->batch, (int)p->d_state, kSsdTT))
         return JAMBA_SSM_ERR_UNSUPPORTED;
-    int devid = 0;
-    cudaGetDevice(&devid);
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         if (!K.attr[devid]) {
@@ -1070,7 +1129,7 @@ jamba_ssm_status jamba_ssm_ssd_scan(const jamba_ssm_ssd_params *p, void *stream)
     a.delta_softplus = p->delta_softplus != 0;
     a.status = static_cast<int *>(p->workspace);
     a.debug_flags = p->debug_flags;
-    a.timeout_cycles = p->timeout_cycles ? p->timeout_cycles : (uint64_t(1) << 31);
+    a.timeout_cycles = timeout;
     const dim3 grid(static_cast<unsigned>(D / kSsdCC), static_cast<unsigned>(p->batch));
     void *kargs[] = {&m, &a};
     cudaError_t e = cudaLaunchKernel(K.k, grid, dim3(K.threads), kargs,

@@ -10,7 +10,7 @@ import torch
 import oracle
 from selective_state_space_26_b200 import (_lib, jamba_ssm_get_status, jamba_ssm_scan,
                                            jamba_ssm_ssd_scan, synth)
-from tests.parity import assert_out, assert_state, compare_out
+from tests.parity import BF16_REL_L2, assert_out, assert_state, compare_out, rel_l2
 
 pytestmark = pytest.mark.gpu
 THREADS = max(1, min(32, os.cpu_count() or 1))
@@ -27,6 +27,8 @@ def _gpu(inp, **kw):
                                  delta_bias=inp.delta_bias, delta_softplus=inp.delta_softplus,
                                  h0=inp.h0, **kw)
     torch.cuda.synchronize()
+    if not kw.get("debug_flags", 0) & 1:  # no wait ran out
+        assert jamba_ssm_get_status() == _lib.OK
     return out, hf
 
 
@@ -124,3 +126,83 @@ def test_ssd_deterministic_and_timeout():
     assert jamba_ssm_get_status() == _lib.OK
     c = _gpu(inp)
     assert torch.equal(c[0], a[0])
+
+
+# ---------------------------------------------------------------- chunked form
+# bf16 I/O with d_state 16 and headdim 64 runs the chunked tensor-core kernel
+# (128-token chunks); bit 1 of debug_flags forces the per-step kernel.
+
+@pytest.mark.parametrize("batch,seqlen,h0_std", [(1, 1, 0.0), (2, 127, 0.5), (1, 128, 0.3),
+                                                 (3, 129, 0.0), (2, 515, 0.4)])
+def test_ssd_chunked_lengths_against_oracle(batch, seqlen, h0_std):
+    """One token, a chunk short by one, exactly one chunk, one past it, and
+    several chunks with a ragged tail; several sequences (one CTA per sequence
+    and head), with and without an initial state."""
+    dev = _dev()
+    inp = synth.ssd_inputs(batch, seqlen, 8, 64, 16, torch.bfloat16, seed=80 + seqlen, device=dev,
+                           h0_std=h0_std)
+    out, hf = _gpu(inp)
+    ref, ref_h = _oracle(inp)
+    assert_out(out, ref, torch.bfloat16, f"chunked L={seqlen}")
+    assert_state(hf, ref_h, torch.bfloat16, f"chunked L={seqlen}")
+
+
+def test_ssd_chunked_and_per_step_kernels_agree():
+    """The two kernels compute one map: each within the bf16 rule of the
+    oracle and of each other, softplus on and off, 16 heads."""
+    dev = _dev()
+    for sp in (True, False):
+        inp = synth.ssd_inputs(2, 300, 16, 64, 16, torch.bfloat16, seed=88, device=dev, h0_std=0.3)
+        if not sp:  # Delta = delta + bias itself: keep it positive
+            inp.delta.copy_((inp.delta.float().abs() * 0.05).to(torch.bfloat16))
+            inp.delta_bias.fill_(0.01)
+            inp.delta_softplus = False
+        out_c, hf_c = _gpu(inp)
+        out_s, hf_s = _gpu(inp, debug_flags=2)
+        ref, ref_h = _oracle(inp)
+        assert_out(out_c, ref, torch.bfloat16, f"chunked softplus={sp}")
+        assert_out(out_s, ref, torch.bfloat16, f"per-step softplus={sp}")
+        assert_state(hf_c, ref_h, torch.bfloat16, f"chunked softplus={sp}")
+        # two bf16 results: the max-excess rule needs an exact reference, so
+        # between the kernels only the rel-L2 part applies
+        assert rel_l2(out_c, out_s) <= BF16_REL_L2
+        assert_state(hf_c, hf_s, torch.bfloat16, "chunked vs per-step")
+
+
+def test_ssd_chunked_strong_decay_and_split():
+    """Steps large enough that e^{s_t - s_j} underflows inside a chunk (A down
+    to -16, Delta near 1), and the sequence cut at a point that is not a chunk
+    boundary and resumed from its final state: the concatenation is the whole
+    scan up to fp32 rounding order."""
+    dev = _dev()
+    inp = synth.ssd_inputs(1, 400, 8, 64, 16, torch.bfloat16, seed=89, device=dev, h0_std=0.2)
+    inp.A.copy_(-torch.linspace(0.5, 16.0, 8, device=dev))
+    inp.delta_bias.fill_(0.5)
+    out, hf = _gpu(inp)
+    ref, ref_h = _oracle(inp)
+    assert_out(out, ref, torch.bfloat16, "strong decay")
+    assert_state(hf, ref_h, torch.bfloat16, "strong decay")
+    cut = 200
+    part = lambda t, sl: t[:, sl].contiguous()  # noqa: E731
+    a = synth.SsdInputs(*(part(getattr(inp, k), slice(0, cut)) for k in ("x", "delta", "z", "B", "C")),
+                        inp.A, inp.D, inp.delta_bias, inp.h0, True)
+    o1, h1 = _gpu(a)
+    b = synth.SsdInputs(*(part(getattr(inp, k), slice(cut, None)) for k in ("x", "delta", "z", "B", "C")),
+                        inp.A, inp.D, inp.delta_bias, h1, True)
+    o2, h2 = _gpu(b)
+    assert_out(torch.cat([o1, o2], 1), ref, torch.bfloat16, "split at 200")
+    assert_state(h2, ref_h, torch.bfloat16, "split at 200")
+
+
+def test_ssd_chunked_deterministic_and_timeout():
+    dev = _dev()
+    inp = synth.ssd_inputs(2, 300, 8, 64, 16, torch.bfloat16, seed=90, device=dev)
+    a = _gpu(inp)
+    b = _gpu(inp)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    assert jamba_ssm_get_status() == _lib.OK
+    _gpu(inp, debug_flags=1, timeout_cycles=2_000_000)
+    assert jamba_ssm_get_status() == _lib.ERR_TIMEOUT
+    assert jamba_ssm_get_status() == _lib.OK
+    c = _gpu(inp)
+    assert torch.equal(c[0], a[0]) and torch.equal(c[1], a[1])
