@@ -1060,8 +1060,6 @@ jamba_ssm_status jamba_ssm_ssd_scan(const jamba_ssm_ssd_params *p, void *stream)
                        CU_TENSOR_MAP_SWIZZLE_128B) ||
             !encode_3d(fn, &m.z, p->z, bf, 2, D, p->seqlen, p->batch, CC::P, CC::Q,
                        CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !encode_3d(fn, &m.dt, p->delta, bf, 2, p->nheads, p->seqlen, p->batch, CC::kHeadsBox,
-                       CC::Q) ||
             !encode_3d(fn, &m.B, p->B, bf, 2, CC::N, p->seqlen, p->batch, CC::N, CC::Q,
                        CU_TENSOR_MAP_SWIZZLE_32B) ||
             !encode_3d(fn, &m.C, p->C, bf, 2, CC::N, p->seqlen, p->batch, CC::N, CC::Q,
@@ -1080,6 +1078,7 @@ jamba_ssm_status jamba_ssm_ssd_scan(const jamba_ssm_ssd_params *p, void *stream)
         jssm::SsdChunkArgs a{};
         a.seqlen = p->seqlen;
         a.nheads = p->nheads;
+        a.delta = static_cast<const __nv_bfloat16 *>(p->delta);
         a.A = p->A;
         a.D = p->D;
         a.delta_bias = p->delta_bias;

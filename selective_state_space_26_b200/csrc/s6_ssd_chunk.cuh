@@ -47,18 +47,24 @@
 //         chunk h = e^{s_127} h + DS (DS read from TMEM lanes 0-15), then h as
 //         hi / lo planes into the buffer the next chunk's YI reads; h_final.
 //   1     producer: lane 0 feeds a 3-stage ring by TMA (x, z [128 x 64], C, B
-//         [128 x 16], the delta box [128 x 8 heads]); all lanes then compute the
-//         chunk's Delta_t (softplus, bias; zero past the sequence's end) and
-//         sigma_t = s_t log2(e) (a compensated warp prefix sum).
+//         [128 x 16]); all lanes then compute the chunk's Delta_t (from plain
+//         loads of delta, one chunk ahead; softplus, bias; zero past the
+//         sequence's end) and sigma_t = s_t log2(e) (a compensated warp prefix
+//         sum), as soon as the chunk lands.
 //   2     allocates TMEM (CB 128 columns, Y and YI two buffers of 64 each, DS
 //         64) and one lane issues the MMAs, in the order
-//         [Y_c, DS_c] -> [CB_{c+1}] -> [YI_c, once h_{c-1} is there].
+//         [Y_c] -> [CB_{c+1}] -> [DS_c] -> [YI_c, once h_{c-1} is there], so
+//         that the M buffer and CB are handed back to the math warps early.
 //   3-10  math warps, two groups of four (one per TMEM lane quarter), each
 //         thread one token row: build M_c (the group's half of the 16-column
-//         blocks, blocks above the diagonal are zeros) and W_c (the group's 8
-//         rows), then the epilogue of chunk c - 1: Y + e^{s_t} YI + D x, times
-//         silu(z), rounded to bf16 and stored to global memory (64 bytes per
-//         thread and chunk half).
+//         blocks, blocks above the diagonal are zeros; the exponent as
+//         (sigma_t - sigma_j0) + delta_j, the first term once per block and
+//         delta_j = sigma_j0 - sigma_j, j0 the block's first token, from the
+//         producer's table); the warps of lane quarters 0 and 1, whose share of
+//         M is the smallest, also write W_c into the stage (one token each);
+//         then the epilogue of chunk c - 1: Y + e^{s_t} YI + D x, times silu(z),
+//         rounded to bf16 and stored to global memory (64 bytes per thread and
+//         chunk half).
 // Every wait is bounded and watches the CTA's abort flag; a wait that runs out
 // records JAMBA_SSM_ERR_TIMEOUT.  Before the CTA frees TMEM the producer waits
 // (bounded) for the loads it issued and the MMA lane for the MMAs it issued.
@@ -77,22 +83,21 @@ struct SsdChunkCfg {
     static constexpr int P = 64;   // channels per head: the MMAs' N
     static constexpr int N = 16;   // d_state
     static constexpr int STAGES = 3;
-    static constexpr int kHeadsBox = 8;  // delta columns per 16-byte TMA row
     // one ring stage
     static constexpr uint32_t kX = 0;              // x [128][64] bf16, 128-byte swizzle
     static constexpr uint32_t kZ = 16384;          // z, the same
     static constexpr uint32_t kC = 32768;          // C [128][16] bf16, 32-byte swizzle
     static constexpr uint32_t kB = 36864;          // B, the same
-    static constexpr uint32_t kDt = 40960;         // delta [128][8 heads] bf16
-    static constexpr uint32_t kDel = 43008;        // Delta_t fp32 [128]
+    static constexpr uint32_t kDel = 40960;        // Delta_t fp32 [128]
     static constexpr uint32_t kSig = kDel + 512;   // sigma_t as hi [128] and lo [128] fp32
-    static constexpr uint32_t kStage = 45056;
-    static constexpr uint32_t kLoadBytes = 2 * 16384 + 2 * 4096 + 2048;
+    static constexpr uint32_t kDlt = kSig + 1024;  // delta_t = sigma_{16 floor(t/16)} - sigma_t fp32 [128]
     // W: per plane two K atoms (tokens 0-63, 64-127) of 16 rows x 128 bytes
-    static constexpr uint32_t kOffW = STAGES * kStage;
+    static constexpr uint32_t kW = 43008;
     static constexpr uint32_t kWPlane = 4096;
+    static constexpr uint32_t kStage = kW + 2 * kWPlane;  // 50 KB
+    static constexpr uint32_t kLoadBytes = 2 * 16384 + 2 * 4096;
     // M: per plane two K atoms of 128 rows x 128 bytes
-    static constexpr uint32_t kOffM = kOffW + 2 * kWPlane;
+    static constexpr uint32_t kOffM = STAGES * kStage;
     static constexpr uint32_t kMPlane = 32768;
     // h_in operand: two buffers x (hi, lo) of 16 rows x 128 bytes
     static constexpr uint32_t kOffH = kOffM + 2 * kMPlane;
@@ -105,13 +110,14 @@ struct SsdChunkCfg {
     static constexpr int kThreads = 352;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColCB = 0, kColY = 128, kColYI = 256, kColDS = 384;
-    static_assert(kStage % 1024 == 0 && kOffW % 1024 == 0 && kOffM % 1024 == 0 &&
+    static_assert(kStage % 1024 == 0 && kW % 1024 == 0 && kOffM % 1024 == 0 &&
                       kOffH % 1024 == 0,
                   "swizzled operands keep their 1 KB alignment");
-    static_assert(kSig + 1024 <= kStage, "the stage holds its tables");
+    static_assert(kDlt + 512 <= kW, "the stage holds its tables");
     // W's descriptor reads 128 rows (16 KB) from each K atom's start: they must
-    // stay inside the buffers that follow it.
-    static_assert(kOffW + kWPlane + kWPlane / 2 + 16384 + 128 <= kOffH, "W's don't-care rows");
+    // stay inside the buffers that follow it (the next stage, or M).
+    static_assert((STAGES - 1) * kStage + kW + kWPlane + kWPlane / 2 + 16384 + 128 <= kOffH,
+                  "W's don't-care rows");
     static_assert(kSmemBytes <= 232448, "fits the opt-in shared memory of one CTA");
     // kind::f16, fp32 accumulator, A and B bf16, M = 128: N = 128 with both
     // operands K-major (C . B^T); N = 64 with B MN-major (bit 16) for the rest.
@@ -122,11 +128,12 @@ struct SsdChunkCfg {
 };
 
 struct SsdChunkMaps {
-    CUtensorMap x, z, dt, B, C;
+    CUtensorMap x, z, B, C;
 };
 
 struct SsdChunkArgs {
     int64_t seqlen, nheads;
+    const __nv_bfloat16 *delta;  // [batch, seqlen, nheads]
     const float *A, *D, *delta_bias, *h0;
     float *h_final;
     __nv_bfloat16 *out;
@@ -205,7 +212,6 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
         fence_mbarrier_init();
         prefetch_tensormap(&maps.x);
         prefetch_tensormap(&maps.z);
-        prefetch_tensormap(&maps.dt);
         prefetch_tensormap(&maps.B);
         prefetch_tensormap(&maps.C);
     }
@@ -223,7 +229,6 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
     if (warp == 1) {
         // ================= producer: TMA ring and the chunk tables =================
         const int bb = static_cast<int>(b);
-        const int hbox = head & ~(C::kHeadsBox - 1);
         const float a2 = __ldg(a.A + head) * kLog2e;
         const float bias = a.delta_bias ? __ldg(a.delta_bias + head) : 0.0f;
         int last[S];  // lane 0: the chunk whose loads are in flight in each stage, or -1
@@ -239,18 +244,32 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
             tma_load_3d(st + C::kZ, &maps.z, head * C::P, t0, bb, &loaded[s]);
             tma_load_3d(st + C::kC, &maps.C, 0, t0, bb, &loaded[s]);
             tma_load_3d(st + C::kB, &maps.B, 0, t0, bb, &loaded[s]);
-            tma_load_3d(st + C::kDt, &maps.dt, hbox, t0, bb, &loaded[s]);
             last[s] = k;
         };
         // chunk k landed: Delta_t and sigma_t = log2(e) A sum_{tau <= t} Delta_tau
+        const __nv_bfloat16 *dseq = a.delta + b * L * a.nheads + head;  // + t * nheads
+        // this lane's 4 tokens of delta for chunk k (plain loads, one chunk ahead)
+        auto fetch = [&](int k, __nv_bfloat16 (&raw)[4]) {
+            const int64_t rem = L - int64_t(k) * C::Q;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = lane * 4 + i;
+                raw[i] = k < nc && t < rem ? dseq[(int64_t(k) * C::Q + t) * a.nheads]
+                                           : __float2bfloat16_rn(0.0f);
+            }
+        };
+        __nv_bfloat16 raw[4];
         auto prepare = [&](int k) -> bool {
             const int s = k % S;
+            const int64_t rem = L - int64_t(k) * C::Q;  // tokens left in the sequence
+            float rv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rv[i] = to_f32(raw[i]);
+            fetch(k + 1, raw);
             if (!warp_agree(mbar_wait_or_abort(&loaded[s], (k / S) & 1, limit, abort_flag)))
                 return false;
             if (lane == 0) last[s] = -1;
-            const uint8_t *st = smem + s * C::kStage;
-            const __nv_bfloat16 *dts = reinterpret_cast<const __nv_bfloat16 *>(st + C::kDt);
-            const int64_t rem = L - int64_t(k) * C::Q;  // tokens left in the sequence
+            uint8_t *st = smem + s * C::kStage;
             // Delta_t, and the prefix sums of Delta as hi + lo pairs (TwoSum at
             // every addition: within the lane, then a warp scan of the lanes'
             // totals)
@@ -258,7 +277,7 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int t = lane * 4 + i;
-                const float v = to_f32(dts[t * C::kHeadsBox + (head - hbox)]) + bias;
+                const float v = rv[i] + bias;
                 dl[i] = t < rem ? (SP ? softplus_io<__nv_bfloat16>(v) : v) : 0.0f;
                 if (i == 0) {
                     ch[0] = dl[0];
@@ -282,8 +301,6 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
             float eh = __shfl_up_sync(0xffffffffu, ih, 1);  // exclusive prefix
             float el = __shfl_up_sync(0xffffffffu, il, 1);
             if (lane == 0) eh = el = 0.0f;
-            float *del = reinterpret_cast<float *>(smem + s * C::kStage + C::kDel);
-            float *sgh = reinterpret_cast<float *>(smem + s * C::kStage + C::kSig);
             float sh[4], sl[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -294,9 +311,17 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                 sh[i] = a2 * h;
                 sl[i] = fmaf(a2, h, -sh[i]) + a2 * l;
             }
-            reinterpret_cast<float4 *>(del)[lane] = make_float4(dl[0], dl[1], dl[2], dl[3]);
-            reinterpret_cast<float4 *>(sgh)[lane] = make_float4(sh[0], sh[1], sh[2], sh[3]);
-            reinterpret_cast<float4 *>(sgh + C::Q)[lane] = make_float4(sl[0], sl[1], sl[2], sl[3]);
+            // within each 16-token block, sigma relative to the block's first
+            // token (held by lane 4 (lane / 4), component 0)
+            const float bh = __shfl_sync(0xffffffffu, sh[0], lane & ~3);
+            const float bl = __shfl_sync(0xffffffffu, sl[0], lane & ~3);
+            float dt4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dt4[i] = (bh - sh[i]) + (bl - sl[i]);
+            reinterpret_cast<float4 *>(st + C::kDel)[lane] = make_float4(dl[0], dl[1], dl[2], dl[3]);
+            reinterpret_cast<float4 *>(st + C::kSig)[lane] = make_float4(sh[0], sh[1], sh[2], sh[3]);
+            reinterpret_cast<float4 *>(st + C::kSig + 512)[lane] = make_float4(sl[0], sl[1], sl[2], sl[3]);
+            reinterpret_cast<float4 *>(st + C::kDlt)[lane] = make_float4(dt4[0], dt4[1], dt4[2], dt4[3]);
             mbar_arrive(&full[s]);
             return true;
         };
@@ -309,13 +334,17 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
             __syncwarp();
             return true;
         };
+        // Each chunk's tables are prepared as soon as its loads land, so that
+        // they are never what the MMA lane waits for.
         if (lane == 0)
             for (int k = 0; k < S; ++k) issue(k);
         __syncwarp();
-        bool ok = nc == 0 || prepare(0);
+        fetch(0, raw);
+        bool ok = true;
+        for (int k = 0; ok && k < S && k < nc; ++k) ok = prepare(k);
         for (int k = 0; ok && k < nc; ++k) {
-            if (k + 1 < nc) ok = prepare(k + 1);
-            if (ok) ok = retire(k);
+            ok = retire(k);  // the stage of chunk k takes chunk k + S
+            if (ok && k + S < nc) ok = prepare(k + S);
         }
         if (!ok) fail();
         if (lane == 0)
@@ -345,11 +374,11 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                 const int s = c % S, yb = c & 1;
                 if (!wait(m_full, c & 1)) break;
                 if (c >= 2 && !wait(&y_empty[yb], ((c >> 1) - 1) & 1)) break;
-                if (c >= 1 && !wait(ds_empty, (c - 1) & 1)) break;
                 tc_fence_after();
                 const uint32_t xs = stage_u32(s) + C::kX;
                 const uint32_t mh = sbase + C::kOffM, ml = mh + C::kMPlane;
-                const uint32_t wh = sbase + C::kOffW, wl = wh + C::kWPlane;
+                const uint32_t wh = stage_u32(s) + C::kW, wl = wh + C::kWPlane;
+                // Y_c = M_c X_c; the M buffer is released as soon as these complete
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {  // K = 128 tokens in steps of 16
                     const uint64_t bx = umma_desc_sw128_mn(xs + kk * 2048u);
@@ -358,13 +387,9 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                               kk > 0 ? 1u : 0u);
                     umma_bf16(tmem + C::kColY + 64u * yb, umma_desc_sw128(ml + ka), bx, C::kIdescX,
                               1u);
-                    const uint32_t kw = (kk >> 2) * C::kWPlane / 2 + (kk & 3) * 32u;
-                    umma_bf16(tmem + C::kColDS, umma_desc_sw128(wh + kw), bx, C::kIdescX,
-                              kk > 0 ? 1u : 0u);
-                    umma_bf16(tmem + C::kColDS, umma_desc_sw128(wl + kw), bx, C::kIdescX, 1u);
                 }
                 tc_commit(m_free);
-                tc_commit(ds_full);
+                // CB_{c+1}, so that the math warps can build M_{c+1} meanwhile
                 if (c + 1 < nc) {
                     const int s1 = (c + 1) % S;
                     if (!wait(&loaded[s1], ((c + 1) / S) & 1) || !wait(&full[s1], ((c + 1) / S) & 1))
@@ -372,6 +397,18 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                     tc_fence_after();
                     mma_cb(c + 1);
                 }
+                // DS_c = W_c X_c, once the state warp has read DS_{c-1}
+                if (c >= 1 && !wait(ds_empty, (c - 1) & 1)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t bx = umma_desc_sw128_mn(xs + kk * 2048u);
+                    const uint32_t kw = (kk >> 2) * C::kWPlane / 2 + (kk & 3) * 32u;
+                    umma_bf16(tmem + C::kColDS, umma_desc_sw128(wh + kw), bx, C::kIdescX,
+                              kk > 0 ? 1u : 0u);
+                    umma_bf16(tmem + C::kColDS, umma_desc_sw128(wl + kw), bx, C::kIdescX, 1u);
+                }
+                tc_commit(ds_full);
                 if (!wait(&h_ready[yb], (c >> 1) & 1)) break;  // h_{c-1} in buffer c % 2
                 tc_fence_after();
                 const uint32_t hb = sbase + C::kOffH + uint32_t(yb) * 2 * C::kHPlane;
@@ -420,7 +457,7 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
         };
         put_h(0);
         bool ok = true;
-        for (int c = 0; c < nc; ++c) {
+        for (int c = 0; ok && c < nc; ++c) {
             const int s = c % S;
             const bool got = mbar_wait_or_abort(ds_full, c & 1, limit, abort_flag) &&
                              mbar_wait_or_abort(&full[s], (c / S) & 1, limit, abort_flag);
@@ -435,6 +472,8 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                 tmem_ld16_async(tmem + C::kColDS + 16u * i,
                                 *reinterpret_cast<uint32_t(*)[16]>(r + 16 * i));
             tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(r + 16 * i));
             tc_fence_before();
             mbar_arrive(ds_empty);
             const float *sgs = reinterpret_cast<const float *>(smem + s * C::kStage + C::kSig);
@@ -467,7 +506,6 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
         const int r = q * 32 + lane;     // this thread's token row of the chunk
         const uint32_t lane_off = uint32_t(q * 32) << 16;
         const uint32_t mh = sbase + C::kOffM, ml = mh + C::kMPlane;
-        const uint32_t wh = sbase + C::kOffW, wl = wh + C::kWPlane;
         bool ok = true;
         for (int it = 0; it <= nc; ++it) {
             if (it < nc) {
@@ -485,8 +523,19 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                 const float *del = reinterpret_cast<const float *>(smem + s * C::kStage + C::kDel);
                 const float *sgh = reinterpret_cast<const float *>(smem + s * C::kStage + C::kSig);
                 const float *sgl = sgh + C::Q;
+                const float *dlt = reinterpret_cast<const float *>(smem + s * C::kStage + C::kDlt);
                 const float shr = sgh[r], slr = sgl[r];
                 const uint32_t rowm = uint32_t(r) * 128u;
+                // CB of this group's active 16-column blocks, all requested at once
+                uint32_t v[4][16];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (16 * (wg + 2 * i) <= q * 32 + 31)
+                        tmem_ld16_async(tmem + lane_off + C::kColCB + uint32_t(16 * (wg + 2 * i)), v[i]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (16 * (wg + 2 * i) <= q * 32 + 31) tmem_regs_ready(v[i]);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int jb = wg + 2 * i;  // this group's 16-column blocks
@@ -496,22 +545,31 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
 #pragma unroll
                         for (int u = 0; u < 8; ++u) hi[u] = lo[u] = 0u;
                     } else {
-                        uint32_t v[16];
-                        tmem_ld16_async(tmem + lane_off + C::kColCB + uint32_t(j0), v);
-                        tmem_wait_ld();
+                        // sigma_r - sigma_j = (sigma_r - sigma_j0) + delta_j: the first
+                        // term once per block (from the hi + lo pairs), the second
+                        // from the table
+                        const float base = (shr - sgh[j0]) + (slr - sgl[j0]);
+                        const float2 base2 = make_float2(base, base), one2 = make_float2(1.0f, 1.0f);
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
+                        for (int u = 0; u < 8; u += 2) {
                             const int j = j0 + 2 * u;
-                            const float2 hj = *reinterpret_cast<const float2 *>(sgh + j);
-                            const float2 lj = *reinterpret_cast<const float2 *>(sgl + j);
-                            const float2 dj = *reinterpret_cast<const float2 *>(del + j);
-                            const float e0 = ex2_mufu((shr - hj.x) + (slr - lj.x));
-                            const float e1 = ex2_mufu((shr - hj.y) + (slr - lj.y));
-                            float m0 = __uint_as_float(v[2 * u]) * dj.x * e0;
-                            float m1 = __uint_as_float(v[2 * u + 1]) * dj.y * e1;
-                            if (j > r) m0 = 0.0f;
-                            if (j + 1 > r) m1 = 0.0f;
-                            split_bf16x2(m0, m1, hi[u], lo[u]);
+                            const float4 d4 = *reinterpret_cast<const float4 *>(del + j);
+                            const float4 t4 = *reinterpret_cast<const float4 *>(dlt + j);
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const float2 dj = hh ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+                                const float2 tj = hh ? make_float2(t4.z, t4.w) : make_float2(t4.x, t4.y);
+                                const float2 arg = fma2(base2, one2, tj);
+                                const float2 e2 = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
+                                const int uu = u + hh, jj = j + 2 * hh;
+                                float2 m = mul2(mul2(make_float2(__uint_as_float(v[i][2 * uu]),
+                                                                 __uint_as_float(v[i][2 * uu + 1])),
+                                                     dj),
+                                                e2);
+                                if (jj > r) m.x = 0.0f;
+                                if (jj + 1 > r) m.y = 0.0f;
+                                split_bf16x2(m.x, m.y, hi[uu], lo[uu]);
+                            }
                         }
                     }
                     // row r of the K-major 128-byte-swizzled M planes: K atom j0 / 64,
@@ -524,28 +582,33 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                     st_shared_v4(ml + atom + o0, make_uint4(lo[0], lo[1], lo[2], lo[3]));
                     st_shared_v4(ml + atom + o1, make_uint4(lo[4], lo[5], lo[6], lo[7]));
                 }
-                {
-                    // W[n][r] for this group's rows n = 8 wg .. 8 wg + 7
-                    const float w =
-                        del[r] * ex2_mufu((sgh[C::Q - 1] - shr) + (sgl[C::Q - 1] - slr));
-                    const uint32_t brow = stage_u32(s) + C::kB + uint32_t(r) * 32u +
-                                          (uint32_t(wg ^ ((r >> 2) & 1)) << 4);
-                    const uint4 bv = ld_shared_v4(brow);
-                    const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-                    const uint32_t col = uint32_t(r >> 6) * (C::kWPlane / 2) + uint32_t(r & 7) * 2u;
+                if (q < 2) {
+                    // W of the chunk into the stage, by the warps of the first two
+                    // lane quarters (their share of M is the smallest): token
+                    // j = 32 (2 q + wg) + lane, w_j = Delta_j e^{s_127 - s_j},
+                    // W[n][j] = w_j B_j[n]
+                    const int j = 32 * (2 * q + wg) + lane;
+                    const float w = del[j] * ex2_mufu((sgh[C::Q - 1] - sgh[j]) + (sgl[C::Q - 1] - sgl[j]));
+                    const uint32_t brow = stage_u32(s) + C::kB + uint32_t(j) * 32u;
+                    const uint32_t sw = uint32_t((j >> 2) & 1);
+                    const uint4 b0 = ld_shared_v4(brow + (sw << 4));         // n 0-7
+                    const uint4 b1 = ld_shared_v4(brow + ((sw ^ 1u) << 4));  // n 8-15
+                    const uint32_t bwd[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                    const uint32_t wh = stage_u32(s) + C::kW, wl = wh + C::kWPlane;
+                    const uint32_t col = uint32_t(j >> 6) * (C::kWPlane / 2) + uint32_t(j & 7) * 2u;
+                    const uint32_t chk = uint32_t((j & 63) >> 3);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float2 bf = bf16x2_to_f2(bw[u]);
-                        uint32_t hi2, lo2;
-                        split_bf16x2(w * bf.x, w * bf.y, hi2, lo2);
+                    for (int u = 0; u < 8; ++u) {
+                        const float2 bf = bf16x2_to_f2(bwd[u]);
+                        uint32_t h2, l2;
+                        split_bf16x2(w * bf.x, w * bf.y, h2, l2);
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
-                            const int nn = 8 * wg + 2 * u + e;  // row of W
-                            const uint32_t off = col + uint32_t(nn >> 3) * 1024u +
-                                                 uint32_t(nn & 7) * 128u +
-                                                 ((uint32_t((r & 63) >> 3) ^ uint32_t(nn & 7)) << 4);
-                            st_shared_u16(wh + off, uint16_t(e ? hi2 >> 16 : hi2 & 0xFFFFu));
-                            st_shared_u16(wl + off, uint16_t(e ? lo2 >> 16 : lo2 & 0xFFFFu));
+                            const int nn = 2 * u + e;  // row of W
+                            const uint32_t off = col + uint32_t(nn >> 3) * 1024u + uint32_t(nn & 7) * 128u +
+                                                 ((chk ^ uint32_t(nn & 7)) << 4);
+                            st_shared_u16(wh + off, uint16_t(e ? h2 >> 16 : h2 & 0xFFFFu));
+                            st_shared_u16(wl + off, uint16_t(e ? l2 >> 16 : l2 & 0xFFFFu));
                         }
                     }
                 }
@@ -566,38 +629,52 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                 const int64_t t = int64_t(e) * C::Q + r;
                 const uint32_t xrow = stage_u32(s) + C::kX + uint32_t(r) * 128u;
                 const uint32_t zrow = stage_u32(s) + C::kZ + uint32_t(r) * 128u;
+                // this group's 32 columns: x and z from shared memory, Y and YI
+                // from TMEM, all requested before the first wait
+                uint4 xv[4], zv[4];
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const uint32_t off = ((uint32_t(4 * wg + g) ^ uint32_t(r & 7)) << 4);
+                    xv[g] = ld_shared_v4(xrow + off);
+                    zv[g] = ld_shared_v4(zrow + off);
+                }
+                uint32_t yv[32], yi[32];
+                const uint32_t ty = tmem + lane_off + C::kColY + 64u * yb + 32u * wg;
+                const uint32_t tyi = tmem + lane_off + C::kColYI + 64u * yb + 32u * wg;
+                tmem_ld16_async(ty, *reinterpret_cast<uint32_t(*)[16]>(yv));
+                tmem_ld16_async(ty + 16, *reinterpret_cast<uint32_t(*)[16]>(yv + 16));
+                tmem_ld16_async(tyi, *reinterpret_cast<uint32_t(*)[16]>(yi));
+                tmem_ld16_async(tyi + 16, *reinterpret_cast<uint32_t(*)[16]>(yi + 16));
+                tmem_wait_ld();
+                tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(yv));
+                tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(yv + 16));
+                tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(yi));
+                tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(yi + 16));
+                const float2 coef2 = make_float2(coef, coef), one2 = make_float2(1.0f, 1.0f);
+                const float2 nl2 = make_float2(-kLog2e, -kLog2e);
                 uint4 o[4];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int p0 = 32 * wg + 16 * hh;
-                    uint32_t yv[16], yi[16];
-                    tmem_ld16_async(tmem + lane_off + C::kColY + 64u * yb + uint32_t(p0), yv);
-                    tmem_ld16_async(tmem + lane_off + C::kColYI + 64u * yb + uint32_t(p0), yi);
-                    tmem_wait_ld();
+                for (int g = 0; g < 4; ++g) {
+                    const uint32_t xw[4] = {xv[g].x, xv[g].y, xv[g].z, xv[g].w};
+                    const uint32_t zw[4] = {zv[g].x, zv[g].y, zv[g].z, zv[g].w};
+                    uint32_t ow[4];
 #pragma unroll
-                    for (int g = 0; g < 2; ++g) {
-                        const uint32_t ch = uint32_t(p0 / 8 + g);
-                        const uint32_t off = (ch ^ uint32_t(r & 7)) << 4;
-                        const uint4 xv = ld_shared_v4(xrow + off);
-                        const uint4 zv = ld_shared_v4(zrow + off);
-                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                        const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
-                        uint32_t ow[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int k = 8 * g + 2 * u;  // column p0 + k
-                            const float2 xf = bf16x2_to_f2(xw[u]);
-                            const float2 zf = bf16x2_to_f2(zw[u]);
-                            const float2 dd = *reinterpret_cast<const float2 *>(dsk + p0 + k);
-                            const float y0 = fmaf(dd.x, xf.x,
-                                                  fmaf(coef, __uint_as_float(yi[k]), __uint_as_float(yv[k])));
-                            const float y1 =
-                                fmaf(dd.y, xf.y,
-                                     fmaf(coef, __uint_as_float(yi[k + 1]), __uint_as_float(yv[k + 1])));
-                            ow[u] = pack_bf16x2(y0 * silu_f32(zf.x), y1 * silu_f32(zf.y));
-                        }
-                        o[2 * hh + g] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    for (int u = 0; u < 4; ++u) {
+                        const int k = 8 * g + 2 * u;  // column 32 wg + k
+                        const float2 xf = bf16x2_to_f2(xw[u]);
+                        const float2 zf = bf16x2_to_f2(zw[u]);
+                        const float2 dd = *reinterpret_cast<const float2 *>(dsk + 32 * wg + k);
+                        // y = Y + e^{s_t} YI + D x;  out = y z / (1 + e^{-z})
+                        float2 y = fma2(coef2, make_float2(__uint_as_float(yi[k]), __uint_as_float(yi[k + 1])),
+                                        make_float2(__uint_as_float(yv[k]), __uint_as_float(yv[k + 1])));
+                        y = fma2(dd, xf, y);
+                        const float2 nz = mul2(zf, nl2);
+                        const float2 den = fma2(make_float2(ex2_mufu(nz.x), ex2_mufu(nz.y)), one2, one2);
+                        const float2 g2 = mul2(zf, make_float2(rcp_mufu(den.x), rcp_mufu(den.y)));
+                        const float2 ov = mul2(y, g2);
+                        ow[u] = pack_bf16x2(ov.x, ov.y);
                     }
+                    o[g] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }
                 tc_fence_before();
                 mbar_arrive(&y_empty[yb]);  // Y and YI of this buffer may be overwritten
