@@ -327,9 +327,14 @@ def per_workload(args, dev, stream, flush_l2, sms, world):
                                                         ssd.A, D=ssd.D, delta_bias=ssd.delta_bias,
                                                         out=ssd_out, h_final=ssd_hf),
                         max(args.pw_reps, 10), stream, dev, flush=flush_l2)
+    # the per-step kernel on the same inputs (bit 1 of debug_flags), for comparison
+    t_s1 = time_launches(lambda: jssm.jamba_ssm_ssd_scan(ssd.x, ssd.delta, ssd.z, ssd.B, ssd.C,
+                                                         ssd.A, D=ssd.D, delta_bias=ssd.delta_bias,
+                                                         out=ssd_out, h_final=ssd_hf, debug_flags=2),
+                         max(args.pw_reps, 10), stream, dev, flush=flush_l2)
     names.append("ssd_bf16_b1_l4096_h128_p64_n16")
     times.append(t_s)
-    meta.append((None, "ssd"))
+    meta.append((t_s1, "ssd"))
     del ssd, ssd_out, ssd_hf
 
     # the backward pass of the headline layer (training): all three kernels
@@ -410,10 +415,12 @@ def per_workload(args, dev, stream, flush_l2, sms, world):
             nbytes = (tok * (3 * d_inner + H + 2 * N) * 2 + (H * 2 + d_inner) * 4
                       + d_inner * N * 4)
             res[name] = {
+                "kernel": "s6_ssd_chunk_kernel (128-token chunks on the tensor cores)",
                 "kernel_us": t * 1e6, "tokens_per_s": tok * world / t,
                 "roofline": {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": hbm_gbs,
                              "unit": "GB/s", "frac": nbytes / t / 1e9 / hbm_gbs,
                              "algorithmic_bytes": nbytes},
+                "per_step_kernel_us": w * 1e6,
                 "timing": f"{max(args.pw_reps, 10)} launches after 1 warm-up, L2 flushed before each"}
         elif kind == "decode":
             nbytes = decode_bytes(w.batch, w.d_inner, w.d_state, 2)

@@ -526,30 +526,26 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                 const float *dlt = reinterpret_cast<const float *>(smem + s * C::kStage + C::kDlt);
                 const float shr = sgh[r], slr = sgl[r];
                 const uint32_t rowm = uint32_t(r) * 128u;
-                // CB of this group's active 16-column blocks, all requested at once
-                uint32_t v[4][16];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    if (16 * (wg + 2 * i) <= q * 32 + 31)
-                        tmem_ld16_async(tmem + lane_off + C::kColCB + uint32_t(16 * (wg + 2 * i)), v[i]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    if (16 * (wg + 2 * i) <= q * 32 + 31) tmem_regs_ready(v[i]);
-#pragma unroll
+                // this group's 16-column blocks, one at a time (a rolled loop keeps
+                // the warps' code small)
+#pragma unroll 1
                 for (int i = 0; i < 4; ++i) {
-                    const int jb = wg + 2 * i;  // this group's 16-column blocks
+                    const int jb = wg + 2 * i;
                     const int j0 = 16 * jb;
                     uint32_t hi[8], lo[8];
                     if (j0 > q * 32 + 31) {  // above the diagonal for every row of the warp
 #pragma unroll
                         for (int u = 0; u < 8; ++u) hi[u] = lo[u] = 0u;
                     } else {
+                        uint32_t v[16];
+                        tmem_ld16_async(tmem + lane_off + C::kColCB + uint32_t(j0), v);
                         // sigma_r - sigma_j = (sigma_r - sigma_j0) + delta_j: the first
                         // term once per block (from the hi + lo pairs), the second
                         // from the table
                         const float base = (shr - sgh[j0]) + (slr - sgl[j0]);
                         const float2 base2 = make_float2(base, base), one2 = make_float2(1.0f, 1.0f);
+                        tmem_wait_ld();
+                        tmem_regs_ready(v);
 #pragma unroll
                         for (int u = 0; u < 8; u += 2) {
                             const int j = j0 + 2 * u;
@@ -562,8 +558,8 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                                 const float2 arg = fma2(base2, one2, tj);
                                 const float2 e2 = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
                                 const int uu = u + hh, jj = j + 2 * hh;
-                                float2 m = mul2(mul2(make_float2(__uint_as_float(v[i][2 * uu]),
-                                                                 __uint_as_float(v[i][2 * uu + 1])),
+                                float2 m = mul2(mul2(make_float2(__uint_as_float(v[2 * uu]),
+                                                                 __uint_as_float(v[2 * uu + 1])),
                                                      dj),
                                                 e2);
                                 if (jj > r) m.x = 0.0f;
@@ -629,62 +625,63 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                 const int64_t t = int64_t(e) * C::Q + r;
                 const uint32_t xrow = stage_u32(s) + C::kX + uint32_t(r) * 128u;
                 const uint32_t zrow = stage_u32(s) + C::kZ + uint32_t(r) * 128u;
-                // this group's 32 columns: x and z from shared memory, Y and YI
-                // from TMEM, all requested before the first wait
-                uint4 xv[4], zv[4];
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const uint32_t off = ((uint32_t(4 * wg + g) ^ uint32_t(r & 7)) << 4);
-                    xv[g] = ld_shared_v4(xrow + off);
-                    zv[g] = ld_shared_v4(zrow + off);
-                }
-                uint32_t yv[32], yi[32];
-                const uint32_t ty = tmem + lane_off + C::kColY + 64u * yb + 32u * wg;
-                const uint32_t tyi = tmem + lane_off + C::kColYI + 64u * yb + 32u * wg;
-                tmem_ld16_async(ty, *reinterpret_cast<uint32_t(*)[16]>(yv));
-                tmem_ld16_async(ty + 16, *reinterpret_cast<uint32_t(*)[16]>(yv + 16));
-                tmem_ld16_async(tyi, *reinterpret_cast<uint32_t(*)[16]>(yi));
-                tmem_ld16_async(tyi + 16, *reinterpret_cast<uint32_t(*)[16]>(yi + 16));
-                tmem_wait_ld();
-                tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(yv));
-                tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(yv + 16));
-                tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(yi));
-                tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(yi + 16));
                 const float2 coef2 = make_float2(coef, coef), one2 = make_float2(1.0f, 1.0f);
                 const float2 nl2 = make_float2(-kLog2e, -kLog2e);
-                uint4 o[4];
+                uint4 *dst = reinterpret_cast<uint4 *>(a.out + (b * L + t) * Dm + int64_t(head) * C::P +
+                                                       32 * wg);
+                // this group's 32 columns in two rolled halves of 16 (small code):
+                // Y and YI from TMEM, x and z from shared memory, the 32 bytes of
+                // output straight to global memory
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int p0 = 32 * wg + 16 * hh;
+                    uint32_t yv[16], yi[16];
+                    tmem_ld16_async(tmem + lane_off + C::kColY + 64u * yb + uint32_t(p0), yv);
+                    tmem_ld16_async(tmem + lane_off + C::kColYI + 64u * yb + uint32_t(p0), yi);
+                    uint4 xv[2], zv[2];
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const uint32_t xw[4] = {xv[g].x, xv[g].y, xv[g].z, xv[g].w};
-                    const uint32_t zw[4] = {zv[g].x, zv[g].y, zv[g].z, zv[g].w};
-                    uint32_t ow[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int k = 8 * g + 2 * u;  // column 32 wg + k
-                        const float2 xf = bf16x2_to_f2(xw[u]);
-                        const float2 zf = bf16x2_to_f2(zw[u]);
-                        const float2 dd = *reinterpret_cast<const float2 *>(dsk + 32 * wg + k);
-                        // y = Y + e^{s_t} YI + D x;  out = y z / (1 + e^{-z})
-                        float2 y = fma2(coef2, make_float2(__uint_as_float(yi[k]), __uint_as_float(yi[k + 1])),
-                                        make_float2(__uint_as_float(yv[k]), __uint_as_float(yv[k + 1])));
-                        y = fma2(dd, xf, y);
-                        const float2 nz = mul2(zf, nl2);
-                        const float2 den = fma2(make_float2(ex2_mufu(nz.x), ex2_mufu(nz.y)), one2, one2);
-                        const float2 g2 = mul2(zf, make_float2(rcp_mufu(den.x), rcp_mufu(den.y)));
-                        const float2 ov = mul2(y, g2);
-                        ow[u] = pack_bf16x2(ov.x, ov.y);
+                    for (int g = 0; g < 2; ++g) {
+                        const uint32_t off = ((uint32_t(p0 / 8 + g) ^ uint32_t(r & 7)) << 4);
+                        xv[g] = ld_shared_v4(xrow + off);
+                        zv[g] = ld_shared_v4(zrow + off);
                     }
-                    o[g] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    tmem_wait_ld();
+                    tmem_regs_ready(yv);
+                    tmem_regs_ready(yi);
+                    uint4 o[2];
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        const uint32_t xw[4] = {xv[g].x, xv[g].y, xv[g].z, xv[g].w};
+                        const uint32_t zw[4] = {zv[g].x, zv[g].y, zv[g].z, zv[g].w};
+                        uint32_t ow[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int k = 8 * g + 2 * u;  // column p0 + k
+                            const float2 xf = bf16x2_to_f2(xw[u]);
+                            const float2 zf = bf16x2_to_f2(zw[u]);
+                            const float2 dd = *reinterpret_cast<const float2 *>(dsk + p0 + k);
+                            // y = Y + e^{s_t} YI + D x;  out = y z / (1 + e^{-z})
+                            float2 y = fma2(coef2,
+                                            make_float2(__uint_as_float(yi[k]), __uint_as_float(yi[k + 1])),
+                                            make_float2(__uint_as_float(yv[k]), __uint_as_float(yv[k + 1])));
+                            y = fma2(dd, xf, y);
+                            const float2 nz = mul2(zf, nl2);
+                            const float2 den =
+                                fma2(make_float2(ex2_mufu(nz.x), ex2_mufu(nz.y)), one2, one2);
+                            const float2 g2 = mul2(zf, make_float2(rcp_mufu(den.x), rcp_mufu(den.y)));
+                            const float2 ov = mul2(y, g2);
+                            ow[u] = pack_bf16x2(ov.x, ov.y);
+                        }
+                        o[g] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    }
+                    if (t < L) {
+                        dst[2 * hh] = o[0];
+                        dst[2 * hh + 1] = o[1];
+                    }
                 }
                 tc_fence_before();
                 mbar_arrive(&y_empty[yb]);  // Y and YI of this buffer may be overwritten
                 mbar_arrive(&empty[s]);     // and the stage refilled
-                if (t < L) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(a.out + (b * L + t) * Dm +
-                                                           int64_t(head) * C::P + 32 * wg);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) dst[u] = o[u];
-                }
             }
         }
         if (!ok) fail();
