@@ -257,17 +257,34 @@ __global__ void __launch_bounds__(XProjCfg::kThreads, 1)
                                4u * static_cast<uint32_t>((rank * rows_per_owner +
                                                            row % rows_per_owner) * C::kRowWords);
         const uint32_t dst = ks > 1 ? map_to_rank(local, owner) : local;
+        // 16 columns at a time; the next group's TMEM load is in flight while
+        // this group is sent
+        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+        uint32_t va[16], vb[16];
+        auto send = [&](int c, const uint32_t (&v)[16]) {
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+                float f[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)  // an empty K slice never wrote the accumulator
+                    f[e] = nkb == 0 ? 0.0f : __uint_as_float(v[j + e]);
+                st_cluster_v4(dst + 4u * (c + j), f[0], f[1], f[2], f[3]);
+            }
+        };
+        tmem_ld16_async(trow, va);
+        tmem_wait_ld();
+        tmem_regs_ready(va);
+        static_assert(C::kCols % 32 == 0, "pairs of 16-column groups");
 #pragma unroll 1
         for (int c = 0; c < C::kCols; c += 32) {
-            float v[32];  // kCols is a multiple of 32
-            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
-            if (nkb == 0) {  // this K slice was empty: the accumulator was never written
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-            }
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                st_cluster_v4(dst + 4u * (c + j), v[j], v[j + 1], v[j + 2], v[j + 3]);
+            tmem_ld16_async(trow + (uint32_t)(c + 16), vb);
+            send(c, va);
+            tmem_wait_ld();
+            tmem_regs_ready(vb);
+            if (c + 32 < C::kCols) tmem_ld16_async(trow + (uint32_t)(c + 32), va);
+            send(c + 16, vb);
+            tmem_wait_ld();
+            tmem_regs_ready(va);
         }
     }
     tc_fence_before();
@@ -276,13 +293,13 @@ __global__ void __launch_bounds__(XProjCfg::kThreads, 1)
     bool cluster_aborted = false;
     for (int r = 0; r < ks; ++r) cluster_aborted |= abort_all[r] != 0;
 
-    if (warp >= 2 && !cluster_aborted) {
-        // Owner epilogue: warp w takes rows (w - 2), (w - 2) + 4, ... of this
+    if (!cluster_aborted) {
+        // Owner epilogue, all six warps: warp w takes rows w, w + 6, ... of this
         // CTA's share; lane j holds columns j + 32 k (k = 0..7: dt_low; k = 8:
         // B for j < 16, C for j >= 16).
         const bool is_b = lane < 16;
         const float *w8 = is_b ? args.w_B : args.w_C;
-        for (int r = warp - 2; r < rows_per_owner; r += 4) {
+        for (int r = warp; r < rows_per_owner; r += C::kThreads / 32) {
             const int m = m0 + static_cast<int>(rank) * rows_per_owner + r;
             float v[9];
 #pragma unroll
