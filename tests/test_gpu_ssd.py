@@ -206,3 +206,22 @@ def test_ssd_chunked_deterministic_and_timeout():
     assert jamba_ssm_get_status() == _lib.OK
     c = _gpu(inp)
     assert torch.equal(c[0], a[0]) and torch.equal(c[1], a[1])
+
+
+def test_ssd_chunked_degenerate_decays():
+    """A = 0 on some heads (no decay: the state only accumulates, sigma stays
+    at 0), and softplus off with Delta exactly 0 on whole stretches of tokens
+    (the state and the decay sums do not move there), over exactly two chunks."""
+    dev = _dev()
+    inp = synth.ssd_inputs(1, 256, 8, 64, 16, torch.bfloat16, seed=91, device=dev, h0_std=0.3)
+    inp.A[::2] = 0.0
+    d = (inp.delta.float().abs() * 0.02).to(torch.bfloat16)
+    d[:, 40:90] = 0.0
+    d[:, 200:230] = 0.0
+    inp.delta.copy_(d)
+    inp.delta_bias.zero_()
+    inp.delta_softplus = False
+    out, hf = _gpu(inp)
+    ref, ref_h = _oracle(inp)
+    assert_out(out, ref, torch.bfloat16, "degenerate decays")
+    assert_state(hf, ref_h, torch.bfloat16, "degenerate decays")
