@@ -90,7 +90,8 @@ struct SsdChunkCfg {
     static constexpr uint32_t kB = 36864;          // B, the same
     static constexpr uint32_t kDel = 40960;        // Delta_t fp32 [128]
     static constexpr uint32_t kSig = kDel + 512;   // sigma_t as hi [128] and lo [128] fp32
-    static constexpr uint32_t kDlt = kSig + 1024;  // delta_t = sigma_{16 floor(t/16)} - sigma_t fp32 [128]
+    // delta_t = sigma_{16 floor(t/16)} - sigma_t (+ log2 Delta_t with softplus) fp32 [128]
+    static constexpr uint32_t kDlt = kSig + 1024;
     // W: per plane two K atoms (tokens 0-63, 64-127) of 16 rows x 128 bytes
     static constexpr uint32_t kW = 43008;
     static constexpr uint32_t kWPlane = 4096;
@@ -141,6 +142,13 @@ struct SsdChunkArgs {
     uint32_t debug_flags;
     uint64_t timeout_cycles;
 };
+
+// log2(x) on the special-function unit (flush-to-zero; log2(0) = -inf).
+__device__ __forceinline__ float lg2_mufu(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // s + e = a + b exactly, s = fl(a + b) (Knuth's TwoSum, six additions).
 __device__ __forceinline__ void two_sum(float a, float b, float &s, float &e) {
@@ -317,7 +325,12 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
             const float bl = __shfl_sync(0xffffffffu, sl[0], lane & ~3);
             float dt4[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dt4[i] = (bh - sh[i]) + (bl - sl[i]);
+            for (int i = 0; i < 4; ++i) {
+                dt4[i] = (bh - sh[i]) + (bl - sl[i]);
+                // with softplus, Delta >= 0: log2(Delta) joins the exponent, so that
+                // M's Delta factor costs no multiply (Delta = 0 gives -inf, e^-inf = 0)
+                if (SP) dt4[i] += lg2_mufu(dl[i]);
+            }
             reinterpret_cast<float4 *>(st + C::kDel)[lane] = make_float4(dl[0], dl[1], dl[2], dl[3]);
             reinterpret_cast<float4 *>(st + C::kSig)[lane] = make_float4(sh[0], sh[1], sh[2], sh[3]);
             reinterpret_cast<float4 *>(st + C::kSig + 512)[lane] = make_float4(sl[0], sl[1], sl[2], sl[3]);
@@ -549,7 +562,8 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
 #pragma unroll
                         for (int u = 0; u < 8; u += 2) {
                             const int j = j0 + 2 * u;
-                            const float4 d4 = *reinterpret_cast<const float4 *>(del + j);
+                            const float4 d4 = SP ? make_float4(1.0f, 1.0f, 1.0f, 1.0f)
+                                                 : *reinterpret_cast<const float4 *>(del + j);
                             const float4 t4 = *reinterpret_cast<const float4 *>(dlt + j);
 #pragma unroll
                             for (int hh = 0; hh < 2; ++hh) {
@@ -558,10 +572,9 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                                 const float2 arg = fma2(base2, one2, tj);
                                 const float2 e2 = make_float2(ex2_mufu(arg.x), ex2_mufu(arg.y));
                                 const int uu = u + hh, jj = j + 2 * hh;
-                                float2 m = mul2(mul2(make_float2(__uint_as_float(v[2 * uu]),
-                                                                 __uint_as_float(v[2 * uu + 1])),
-                                                     dj),
-                                                e2);
+                                const float2 cb = make_float2(__uint_as_float(v[2 * uu]),
+                                                              __uint_as_float(v[2 * uu + 1]));
+                                float2 m = mul2(SP ? cb : mul2(cb, dj), e2);
                                 if (jj > r) m.x = 0.0f;
                                 if (jj + 1 > r) m.y = 0.0f;
                                 split_bf16x2(m.x, m.y, hi[uu], lo[uu]);
