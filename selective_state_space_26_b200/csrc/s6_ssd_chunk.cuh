@@ -88,9 +88,10 @@ struct SsdChunkCfg {
     static constexpr uint32_t kZ = 16384;          // z, the same
     static constexpr uint32_t kC = 32768;          // C [128][16] bf16, 32-byte swizzle
     static constexpr uint32_t kB = 36864;          // B, the same
-    static constexpr uint32_t kDel = 40960;        // Delta_t fp32 [128]
+    static constexpr uint32_t kDel = 40960;        // Delta_t (softplus: e^{s_j1 - s_t} Delta_t) fp32 [128]
     static constexpr uint32_t kSig = kDel + 512;   // sigma_t as hi [128] and lo [128] fp32
-    // delta_t = sigma_{16 floor(t/16)} - sigma_t (+ log2 Delta_t with softplus) fp32 [128]
+    // delta_t = sigma_ref - sigma_t, ref the first token of t's 16-token block
+    // (with softplus: its last, + log2 Delta_t) fp32 [128]
     static constexpr uint32_t kDlt = kSig + 1024;
     // W: per plane two K atoms (tokens 0-63, 64-127) of 16 rows x 128 bytes
     static constexpr uint32_t kW = 43008;
@@ -319,19 +320,28 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                 sh[i] = a2 * h;
                 sl[i] = fmaf(a2, h, -sh[i]) + a2 * l;
             }
-            // within each 16-token block, sigma relative to the block's first
-            // token (held by lane 4 (lane / 4), component 0)
-            const float bh = __shfl_sync(0xffffffffu, sh[0], lane & ~3);
-            const float bl = __shfl_sync(0xffffffffu, sl[0], lane & ~3);
-            float dt4[4];
+            // within each 16-token block, sigma relative to a reference token of
+            // the block: its first (lane 4 (lane / 4), component 0) without
+            // softplus; its last (lane 4 (lane / 4) + 3, component 3) with it
+            const int ref_lane = SP ? (lane | 3) : (lane & ~3);
+            const float bh = __shfl_sync(0xffffffffu, SP ? sh[3] : sh[0], ref_lane);
+            const float bl = __shfl_sync(0xffffffffu, SP ? sl[3] : sl[0], ref_lane);
+            float dt4[4], tab[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 dt4[i] = (bh - sh[i]) + (bl - sl[i]);
-                // with softplus, Delta >= 0: log2(Delta) joins the exponent, so that
-                // M's Delta factor costs no multiply (Delta = 0 gives -inf, e^-inf = 0)
-                if (SP) dt4[i] += lg2_mufu(dl[i]);
+                tab[i] = dl[i];
+                if (SP) {
+                    // with softplus, Delta >= 0: log2(Delta) joins the exponent, so
+                    // that M's Delta factor costs no multiply (Delta = 0 gives
+                    // -inf, e^-inf = 0); and the Delta table holds
+                    // e^{s_j1 - s_j} Delta_j instead (j1 the block's last token:
+                    // at most Delta_j, so it never overflows)
+                    dt4[i] += lg2_mufu(dl[i]);
+                    tab[i] = ex2_mufu(dt4[i]);
+                }
             }
-            reinterpret_cast<float4 *>(st + C::kDel)[lane] = make_float4(dl[0], dl[1], dl[2], dl[3]);
+            reinterpret_cast<float4 *>(st + C::kDel)[lane] = make_float4(tab[0], tab[1], tab[2], tab[3]);
             reinterpret_cast<float4 *>(st + C::kSig)[lane] = make_float4(sh[0], sh[1], sh[2], sh[3]);
             reinterpret_cast<float4 *>(st + C::kSig + 512)[lane] = make_float4(sl[0], sl[1], sl[2], sl[3]);
             reinterpret_cast<float4 *>(st + C::kDlt)[lane] = make_float4(dt4[0], dt4[1], dt4[2], dt4[3]);
@@ -552,13 +562,36 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                     } else {
                         uint32_t v[16];
                         tmem_ld16_async(tmem + lane_off + C::kColCB + uint32_t(j0), v);
-                        // sigma_r - sigma_j = (sigma_r - sigma_j0) + delta_j: the first
-                        // term once per block (from the hi + lo pairs), the second
-                        // from the table
-                        const float base = (shr - sgh[j0]) + (slr - sgl[j0]);
+                        // sigma_r - sigma_j = (sigma_r - sigma_ref) + delta_j: the first
+                        // term once per block (from the hi + lo pairs; ref the block's
+                        // first token, or with softplus its last), the second from
+                        // the table
+                        const int jr = SP ? j0 + 15 : j0;
+                        const float base = (shr - sgh[jr]) + (slr - sgl[jr]);
                         const float2 base2 = make_float2(base, base), one2 = make_float2(1.0f, 1.0f);
                         tmem_wait_ld();
                         tmem_regs_ready(v);
+                        if (SP && j0 + 15 <= q * 32) {
+                            // the block is below the diagonal for every row of the
+                            // warp: e^{s_r - s_j} Delta_j = e^{s_r - s_j1} (e^{s_j1 - s_j}
+                            // Delta_j), one exp for the block and the table's factor,
+                            // both at most 1 (resp. Delta_j)
+                            const float ub = ex2_mufu(base);
+                            const float2 u2 = make_float2(ub, ub);
+#pragma unroll
+                            for (int u = 0; u < 8; u += 2) {
+                                const float4 w4 = *reinterpret_cast<const float4 *>(del + j0 + 2 * u);
+#pragma unroll
+                                for (int hh = 0; hh < 2; ++hh) {
+                                    const int uu = u + hh;
+                                    const float2 wj = hh ? make_float2(w4.z, w4.w) : make_float2(w4.x, w4.y);
+                                    const float2 cb = make_float2(__uint_as_float(v[2 * uu]),
+                                                                  __uint_as_float(v[2 * uu + 1]));
+                                    const float2 m = mul2(mul2(cb, wj), u2);
+                                    split_bf16x2(m.x, m.y, hi[uu], lo[uu]);
+                                }
+                            }
+                        } else
 #pragma unroll
                         for (int u = 0; u < 8; u += 2) {
                             const int j = j0 + 2 * u;
@@ -597,7 +630,9 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                     // j = 32 (2 q + wg) + lane, w_j = Delta_j e^{s_127 - s_j},
                     // W[n][j] = w_j B_j[n]
                     const int j = 32 * (2 * q + wg) + lane;
-                    const float w = del[j] * ex2_mufu((sgh[C::Q - 1] - sgh[j]) + (sgl[C::Q - 1] - sgl[j]));
+                    // SP: del holds e^{s_j1 - s_j} Delta_j, j1 = j | 15
+                    const int jw = SP ? (j | 15) : j;
+                    const float w = del[j] * ex2_mufu((sgh[C::Q - 1] - sgh[jw]) + (sgl[C::Q - 1] - sgl[jw]));
                     const uint32_t brow = stage_u32(s) + C::kB + uint32_t(j) * 32u;
                     const uint32_t sw = uint32_t((j >> 2) & 1);
                     const uint4 b0 = ld_shared_v4(brow + (sw << 4));         // n 0-7
