@@ -58,9 +58,12 @@
 //   3-10  math warps, two groups of four (one per TMEM lane quarter), each
 //         thread one token row: build M_c (the group's half of the 16-column
 //         blocks, blocks above the diagonal are zeros; the exponent as
-//         (sigma_t - sigma_j0) + delta_j, the first term once per block and
-//         delta_j = sigma_j0 - sigma_j, j0 the block's first token, from the
-//         producer's table); the warps of lane quarters 0 and 1, whose share of
+//         (sigma_t - sigma_ref) + delta_j, the first term once per block and
+//         delta_j = sigma_ref - sigma_j from the producer's table, ref the
+//         block's first token, or with softplus its last, j1; with softplus a
+//         block below the diagonal for all the warp's rows takes one exp,
+//         e^{s_t - s_j1}, times the table's e^{s_j1 - s_j} Delta_j, both at
+//         most 1 or Delta_j); the warps of lane quarters 0 and 1, whose share of
 //         M is the smallest, also write W_c into the stage (one token each);
 //         then the epilogue of chunk c - 1: Y + e^{s_t} YI + D x, times silu(z),
 //         rounded to bf16 and stored to global memory (64 bytes per thread and
