@@ -225,3 +225,15 @@ def test_ssd_chunked_degenerate_decays():
     ref, ref_h = _oracle(inp)
     assert_out(out, ref, torch.bfloat16, "degenerate decays")
     assert_state(hf, ref_h, torch.bfloat16, "degenerate decays")
+
+
+def test_ssd_chunked_more_ctas_than_sms():
+    """4 sequences x 48 heads: 192 CTAs of one (sequence, head) each, more than
+    the SMs, so the chunked kernel runs in two waves; sequences of 300 steps
+    from different initial states."""
+    dev = _dev()
+    inp = synth.ssd_inputs(4, 300, 48, 64, 16, torch.bfloat16, seed=92, device=dev, h0_std=0.4)
+    out, hf = _gpu(inp)
+    ref, ref_h = _oracle(inp)
+    assert_out(out, ref, torch.bfloat16, "two waves")
+    assert_state(hf, ref_h, torch.bfloat16, "two waves")
