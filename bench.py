@@ -254,11 +254,13 @@ def replica_seq_offset(rank, batch):
     return rank * batch
 
 
-# ------------------------------------------------------------- the other configs
+# ----------------------------------------------------------- the other workloads
 def per_workload(args, dev, stream, flush_l2, sms, world):
-    """The other BASELINE configurations, each timed on its own with CUDA
-    events (the max over ranks) against its own bound, plus the two projection
-    kernels that feed the scan: {name: {kernel_us, tokens_per_s, roofline}}."""
+    """The other workloads (the 256K-token sequence, the batch of 16 x 16K,
+    decode of 256 requests), each timed on its own with CUDA events (the max
+    over ranks) against its own bound, plus the projection kernels that feed
+    the scan, the scalar-identity variant, the backward and a training step:
+    {name: {kernel_us, tokens_per_s, roofline}}."""
     import selective_state_space_26_b200 as jssm
     from selective_state_space_26_b200 import synth
 
