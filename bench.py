@@ -506,18 +506,27 @@ def profile_one(args):
 
 
 # ------------------------------------------------------------- our arm
-def time_e2e(e2e_step, tokens, world, k_e2e, h2d, d2h, dev, stream, method=""):
+def time_e2e(e2e_step, tokens, world, k_e2e, h2d, d2h, dev, stream, method="", begin=None,
+             end=None):
     """Whole-step time through the public API with host<->device copies of
-    every step's inputs and results inside the timed region (max over ranks)."""
+    every step's inputs and results inside the timed region (max over ranks).
+    `begin` (after the start event) makes the step's other streams wait for
+    it; `end` (before the stop event) makes `stream` wait for them."""
     for _ in range(3):
         e2e_step()
+    if end:
+        end()
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    if begin:
+        begin()
     for _ in range(k_e2e):
         e2e_step()
+    if end:
+        end()
     b.record(stream)
     torch.cuda.synchronize(dev)
     (t_e2e,) = max_over_ranks([a.elapsed_time(b)], world, dev)
@@ -634,8 +643,13 @@ def run_ours(args, rank, world, local_rank):
         sizes = [t.numel() * t.element_size() for t in parts]
         offs = [sum(sizes[:i]) for i in range(len(sizes))]
         assert all(o % 16 == 0 for o in offs)
-        hflat = [torch.empty(sum(sizes), dtype=torch.uint8).pin_memory() for _ in range(nch)]
-        dflat = [torch.empty(sum(sizes), dtype=torch.uint8, device=dev) for _ in range(nch)]
+        # two sets of buffers, used by alternate steps: step k + 1's copies in
+        # run while step k's last chunks are scanned and copied back
+        NSET = 2
+        hflat = [[torch.empty(sum(sizes), dtype=torch.uint8).pin_memory() for _ in range(nch)]
+                 for _ in range(NSET)]
+        dflat = [[torch.empty(sum(sizes), dtype=torch.uint8, device=dev) for _ in range(nch)]
+                 for _ in range(NSET)]
 
         def views(flat):
             out = {}
@@ -643,46 +657,64 @@ def run_ours(args, rank, world, local_rank):
                 t = getattr(inp, k)
                 out[k] = flat[o:o + n].view(t.dtype).view(t.shape[0], lc, t.shape[2])
             return out
-        host = [views(hflat[c]) for c in range(nch)]
-        dbuf = [views(dflat[c]) for c in range(nch)]
-        for c in range(nch):
-            for k in keys:
-                host[c][k].copy_(getattr(inp, k)[:, c * lc:(c + 1) * lc])
-        dout = [torch.empty_like(dbuf[c]["x"]) for c in range(nch)]
-        h_out = [torch.empty(dout[c].shape, dtype=out.dtype).pin_memory() for c in range(nch)]
-        h_hf = torch.empty(hf.shape, dtype=hf.dtype).pin_memory()
-        h_dec = torch.empty(dec_out.shape, dtype=dec_out.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in hflat)
-        d2h = sum(t.numel() * t.element_size() for t in h_out + [h_hf, h_dec])
+        host = [[views(hflat[q][c]) for c in range(nch)] for q in range(NSET)]
+        dbuf = [[views(dflat[q][c]) for c in range(nch)] for q in range(NSET)]
+        for q in range(NSET):
+            for c in range(nch):
+                for k in keys:
+                    host[q][c][k].copy_(getattr(inp, k)[:, c * lc:(c + 1) * lc])
+        dout = [[torch.empty_like(dbuf[q][c]["x"]) for c in range(nch)] for q in range(NSET)]
+        h_out = [[torch.empty(dout[q][c].shape, dtype=out.dtype).pin_memory() for c in range(nch)]
+                 for q in range(NSET)]
+        hfs = [hf] + [torch.empty_like(hf) for _ in range(NSET - 1)]  # each set's running state
+        h_hf = [torch.empty(hf.shape, dtype=hf.dtype).pin_memory() for _ in range(NSET)]
+        decs = [dec_out] + [torch.empty_like(dec_out) for _ in range(NSET - 1)]
+        h_dec = [torch.empty(dec_out.shape, dtype=dec_out.dtype).pin_memory() for _ in range(NSET)]
+        h2d = sum(t.numel() * t.element_size() for t in hflat[0])
+        d2h = sum(t.numel() * t.element_size() for t in h_out[0] + [h_hf[0], h_dec[0]])
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         ev_in = [torch.cuda.Event() for _ in range(nch)]
         ev_sc = [torch.cuda.Event() for _ in range(nch + 1)]
+        ev_done = [None] * NSET  # a set's last use: its results are on the host
+        ctr_e = [0]
 
         def e2e_step():
-            s_in.wait_stream(stream)  # the previous step has finished with the buffers
-            s_out.wait_stream(stream)
+            q = ctr_e[0] % NSET
+            ctr_e[0] += 1
+            if ev_done[q] is not None:  # the step two before has finished with this set
+                s_in.wait_event(ev_done[q])
             with torch.cuda.stream(s_in):
                 for c in range(nch):
-                    dflat[c].copy_(hflat[c], non_blocking=True)
+                    dflat[q][c].copy_(hflat[q][c], non_blocking=True)
                     ev_in[c].record(s_in)
             for c in range(nch):
                 stream.wait_event(ev_in[c])
-                jssm.jamba_ssm_scan(dbuf[c]["x"], dbuf[c]["delta"], dbuf[c]["z"], dbuf[c]["B"],
-                                    dbuf[c]["C"], inp.A, D=inp.D, delta_bias=inp.delta_bias,
-                                    h0=None if c == 0 else hf, out=dout[c], h_final=hf)
+                jssm.jamba_ssm_scan(dbuf[q][c]["x"], dbuf[q][c]["delta"], dbuf[q][c]["z"],
+                                    dbuf[q][c]["B"], dbuf[q][c]["C"], inp.A, D=inp.D,
+                                    delta_bias=inp.delta_bias, h0=None if c == 0 else hfs[q],
+                                    out=dout[q][c], h_final=hfs[q])
                 ev_sc[c].record(stream)
                 s_out.wait_event(ev_sc[c])
                 with torch.cuda.stream(s_out):
-                    h_out[c].copy_(dout[c], non_blocking=True)
-            jssm.jamba_ssm_state_update(hf, nxt.x, nxt.delta, nxt.z, nxt.B, nxt.C, inp.A,
-                                        D=inp.D, delta_bias=inp.delta_bias, out=dec_out)
+                    h_out[q][c].copy_(dout[q][c], non_blocking=True)
+            jssm.jamba_ssm_state_update(hfs[q], nxt.x, nxt.delta, nxt.z, nxt.B, nxt.C, inp.A,
+                                        D=inp.D, delta_bias=inp.delta_bias, out=decs[q])
             ev_sc[nch].record(stream)
             s_out.wait_event(ev_sc[nch])
             with torch.cuda.stream(s_out):
-                h_hf.copy_(hf, non_blocking=True)
-                h_dec.copy_(dec_out, non_blocking=True)
-            stream.wait_stream(s_out)  # the step ends when its results are on the host
+                h_hf[q].copy_(hfs[q], non_blocking=True)
+                h_dec[q].copy_(decs[q], non_blocking=True)
+                ev_done[q] = torch.cuda.Event()
+                ev_done[q].record(s_out)
+
+        def e2e_begin():  # no copy of the timed steps starts before the start event
+            s_in.wait_stream(stream)
+            s_out.wait_stream(stream)
+
+        def e2e_end():  # the timed region ends when every step's results are on the host
+            stream.wait_stream(s_out)
     else:
+        e2e_begin = e2e_end = None
         h_steps = [{k: getattr(s, k).cpu().pin_memory() for k in ("x", "delta", "z", "B", "C")}
                    for s in steps_in[:8]]
         dbuf = {k: torch.empty_like(getattr(steps_in[0], k)) for k in h_steps[0]}
@@ -702,11 +734,13 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_e2e:
         method = ("inputs in pinned host memory; the sequence streamed through jamba_ssm_scan "
                   f"in {nch} chunks (h0 resume) with H2D, scans and D2H on three streams; each "
-                  "chunk's five inputs packed in one pinned buffer, one copy per chunk"
+                  "chunk's five inputs packed in one pinned buffer, one copy per chunk; two "
+                  "buffer sets, so that a step's copies in overlap the previous step's last "
+                  "scans and copies out"
                   if w.kind == "prefill" else
                   "inputs in pinned host memory; H2D, jamba_ssm_state_update, D2H")
         e2e = time_e2e(e2e_step, tokens, world, max(3, min(args.steps, 20)), h2d, d2h, dev,
-                       stream, method)
+                       stream, method, begin=e2e_begin, end=e2e_end)
 
     # ---- roofline of the dominant kernel
     hbm_gbs, sm_mhz_peak, peak_kind = peaks()
