@@ -466,3 +466,51 @@ def test_checkpoint_size(L):
     assert _lib.scan_ckpt_size(1, 16, 8, 8) == 8 * 8 * 4
     assert _lib.scan_ckpt_size(-1, 16, 8, 8) == 0
 
+
+
+def _valid_ssd(**kw):
+    base = dict(batch=2, seqlen=100, nheads=8, headdim=64, d_state=16, io_dtype=_lib.BF16,
+                delta_softplus=1, x=0x10000000, delta=0x20000000, z=0x30000000,
+                B=0x40000000, C=0x50000000, A=0x60000000, D=0x70000000,
+                delta_bias=0x80000000, h0=None, out=0x90000000, h_final=0xA0000000)
+    base.update(kw)
+    return _lib.new_ssd_params(**base)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(batch=-1), _lib.ERR_INVALID_ARG),
+    (dict(seqlen=-5), _lib.ERR_INVALID_ARG),
+    (dict(nheads=0), _lib.ERR_INVALID_ARG),
+    (dict(headdim=0), _lib.ERR_INVALID_ARG),
+    (dict(d_state=0), _lib.ERR_INVALID_ARG),
+    (dict(io_dtype=7), _lib.ERR_INVALID_ARG),
+    (dict(d_state=4), _lib.ERR_UNSUPPORTED),
+    (dict(d_state=32), _lib.ERR_UNSUPPORTED),
+    (dict(headdim=48), _lib.ERR_UNSUPPORTED),   # heads of whole 32-channel slices
+    (dict(nheads=4), _lib.ERR_UNSUPPORTED),     # bf16 delta rows of 16-byte multiples
+    (dict(batch=70000), _lib.ERR_UNSUPPORTED),  # grid y
+    (dict(x=None), _lib.ERR_INVALID_ARG),
+    (dict(delta=None), _lib.ERR_INVALID_ARG),
+    (dict(A=None), _lib.ERR_INVALID_ARG),
+    (dict(out=None), _lib.ERR_INVALID_ARG),
+    (dict(x=0x10000002), _lib.ERR_MISALIGNED),
+    (dict(B=0x40000008), _lib.ERR_MISALIGNED),
+    (dict(h0=0xB0000004), _lib.ERR_MISALIGNED),
+    (dict(A=0x60000002), _lib.ERR_MISALIGNED),
+    (dict(out=0x10000000 + 64), _lib.ERR_INVALID_ARG),        # out overlaps x
+    (dict(out=0x20000000), _lib.ERR_INVALID_ARG),             # out overlaps delta
+    (dict(h_final=0x90000000 + 1024), _lib.ERR_INVALID_ARG),  # h_final inside out
+    (dict(h0=0xA0000000 + 16), _lib.ERR_INVALID_ARG),         # h0 partially overlaps h_final
+    (dict(workspace=0xC0000008, workspace_bytes=64), _lib.ERR_MISALIGNED),
+    (dict(workspace=0xC0000000, workspace_bytes=8), _lib.ERR_WORKSPACE),
+])
+def test_ssd_argument_errors(L, kw, expect):
+    """jamba_ssm_ssd_scan's checks, all taken before any device is touched."""
+    assert _lib.call_ssd(_valid_ssd(**kw), 0) == expect
+
+
+def test_ssd_struct_size_and_null(L):
+    p = _valid_ssd()
+    p.struct_size = 8
+    assert _lib.call_ssd(p, 0) == _lib.ERR_INVALID_ARG
+    assert L.jamba_ssm_ssd_scan(None, None) == _lib.ERR_INVALID_ARG
