@@ -71,7 +71,8 @@ def bf16_peak():
 # and every csrc header that header includes, directly or not.
 KERNEL_HEADER = {"s6_scan_fused_kernel": "s6_scan_fused.cuh",
                  "s6_state_update_kernel": "s6_state_update.cuh",
-                 "s6_ssd_kernel": "s6_ssd.cuh"}
+                 "s6_ssd_kernel": "s6_ssd.cuh",
+                 "s6_ssd_chunk_kernel": "s6_ssd_chunk.cuh"}
 
 
 def kernel_source_hash(kernel: str):
@@ -421,7 +422,8 @@ def per_workload(args, dev, stream, flush_l2, sms, world):
                 "kernel_us": t * 1e6, "tokens_per_s": tok * world / t,
                 "roofline": {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": hbm_gbs,
                              "unit": "GB/s", "frac": nbytes / t / 1e9 / hbm_gbs,
-                             "algorithmic_bytes": nbytes},
+                             "algorithmic_bytes": nbytes,
+                             "traffic": recorded_traffic("s6_ssd_chunk_kernel", name)},
                 "per_step_kernel_us": w * 1e6,
                 "timing": f"{max(args.pw_reps, 10)} launches after 1 warm-up, L2 flushed before each"}
         elif kind == "decode":
