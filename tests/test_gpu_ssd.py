@@ -237,3 +237,25 @@ def test_ssd_chunked_more_ctas_than_sms():
     ref, ref_h = _oracle(inp)
     assert_out(out, ref, torch.bfloat16, "two waves")
     assert_state(hf, ref_h, torch.bfloat16, "two waves")
+
+
+def test_ssd_chunked_in_place_state_and_optional_inputs():
+    """The chunked kernel with the state updated in place (h_final is h0), no
+    skip term (D absent) and no bias; then the same call without a final state
+    at all (the output alone)."""
+    dev = _dev()
+    inp = synth.ssd_inputs(2, 260, 8, 64, 16, torch.bfloat16, seed=93, device=dev, h0_std=0.4)
+    ref, ref_h = oracle.ssd_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, 8, D=None,
+                                 delta_bias=None, h0=inp.h0, threads=THREADS)
+    h = inp.h0.clone()
+    out, hf = jamba_ssm_ssd_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, h0=h, h_final=h)
+    torch.cuda.synchronize()
+    assert jamba_ssm_get_status() == _lib.OK
+    assert hf.data_ptr() == h.data_ptr()
+    assert_out(out, ref, torch.bfloat16, "in place")
+    assert_state(h, ref_h, torch.bfloat16, "in place")
+    out2, hf2 = jamba_ssm_ssd_scan(inp.x, inp.delta, inp.z, inp.B, inp.C, inp.A, h0=inp.h0,
+                                   return_final_state=False)
+    torch.cuda.synchronize()
+    assert jamba_ssm_get_status() == _lib.OK
+    assert hf2 is None and torch.equal(out2, out)
