@@ -395,10 +395,11 @@ jamba_ssm_status jamba_ssm_scan_bwd_noalloc(const jamba_ssm_scan_bwd_params *p, 
  *   workspace   optional status block, as for jamba_ssm_scan.
  * debug_flags / timeout_cycles: as jamba_ssm_scan; bit 1 of debug_flags runs
  *               the per-step kernel where the chunked one would be used.
- * Kernels: bf16 I/O with d_state 16 and headdim 64 runs the chunked form on
- * the tensor cores (128-token chunks: per chunk and head the products
- * C B^T, M x and W x of the unrolled recurrence, the state passed from chunk
- * to chunk in fp32); every other shape runs the per-step recurrence.
+ * Kernels: bf16 I/O with d_state 16 and headdim a multiple of 64 runs the
+ * chunked form on the tensor cores (128-token chunks: per chunk and 64-channel
+ * slice of a head the products C B^T, M x and W x of the unrolled recurrence,
+ * the state passed from chunk to chunk in fp32); every other shape runs the
+ * per-step recurrence.
  */
 typedef struct jamba_ssm_ssd_params {
     size_t struct_size;          /* = sizeof(jamba_ssm_ssd_params)            */

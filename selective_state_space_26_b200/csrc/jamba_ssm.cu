@@ -1050,9 +1050,10 @@ jamba_ssm_status jamba_ssm_ssd_scan(const jamba_ssm_ssd_params *p, void *stream)
     int devid = 0;
     cudaGetDevice(&devid);
     const uint64_t timeout = p->timeout_cycles ? p->timeout_cycles : (uint64_t(1) << 31);
-    if (p->io_dtype == JAMBA_SSM_BF16 && p->d_state == 16 && p->headdim == jssm::SsdChunkCfg::P &&
+    if (p->io_dtype == JAMBA_SSM_BF16 && p->d_state == 16 && p->headdim % jssm::SsdChunkCfg::P == 0 &&
         !(p->debug_flags & 2u)) {
-        // chunked form on the tensor cores: one CTA per (sequence, head)
+        // chunked form on the tensor cores: one CTA per (sequence, 64-channel
+        // slice of a head)
         using CC = jssm::SsdChunkCfg;
         const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
         jssm::SsdChunkMaps m;
@@ -1078,6 +1079,7 @@ jamba_ssm_status jamba_ssm_ssd_scan(const jamba_ssm_ssd_params *p, void *stream)
         jssm::SsdChunkArgs a{};
         a.seqlen = p->seqlen;
         a.nheads = p->nheads;
+        a.headdim = p->headdim;
         a.delta = static_cast<const __nv_bfloat16 *>(p->delta);
         a.A = p->A;
         a.D = p->D;
@@ -1088,7 +1090,7 @@ jamba_ssm_status jamba_ssm_ssd_scan(const jamba_ssm_ssd_params *p, void *stream)
         a.status = static_cast<int *>(p->workspace);
         a.debug_flags = p->debug_flags;
         a.timeout_cycles = timeout;
-        const dim3 grid(static_cast<unsigned>(p->nheads), static_cast<unsigned>(p->batch));
+        const dim3 grid(static_cast<unsigned>(D / CC::P), static_cast<unsigned>(p->batch));
         void *kargs[] = {&m, &a};
         cudaError_t e = cudaLaunchKernel(K.k, grid, dim3(CC::kThreads), kargs,
                                          static_cast<size_t>(CC::kSmemBytes), s);

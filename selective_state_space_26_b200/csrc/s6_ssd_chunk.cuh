@@ -42,7 +42,9 @@
 // into the same accumulator, which keeps them to ~2^-17 relative (a single bf16
 // rounding, 2^-9, would exceed the layer's bf16 parity bound).
 //
-// One CTA per (sequence, head) walks the sequence's chunks in order.  Warps:
+// One CTA per (sequence, 64-channel slice of a head) walks the sequence's chunks
+// in order; a head wider than 64 channels takes several CTAs, each repeating the
+// head's per-token work (Delta, sigma, M, W).  Warps:
 //   0     the state warp: lanes n < 16 keep h[n][0..63] in fp32 registers; per
 //         chunk h = e^{s_127} h + DS (DS read from TMEM lanes 0-15), then h as
 //         hi / lo planes into the buffer the next chunk's YI reads; h_final.
@@ -137,7 +139,7 @@ struct SsdChunkMaps {
 };
 
 struct SsdChunkArgs {
-    int64_t seqlen, nheads;
+    int64_t seqlen, nheads, headdim;  // headdim a multiple of 64
     const __nv_bfloat16 *delta;  // [batch, seqlen, nheads]
     const float *A, *D, *delta_bias, *h0;
     float *h_final;
@@ -161,8 +163,8 @@ __device__ __forceinline__ void two_sum(float a, float b, float &s, float &e) {
     e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
 }
 
-// grid (nheads, batch), 352 threads; SP: softplus on.  headdim 64, d_state 16,
-// bf16 I/O, nheads a multiple of 8.
+// grid (nheads * headdim / 64, batch), 352 threads; SP: softplus on.  headdim a
+// multiple of 64, d_state 16, bf16 I/O, nheads a multiple of 8.
 template <bool SP>
 __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
     s6_ssd_chunk_kernel(const __grid_constant__ SsdChunkMaps maps, const SsdChunkArgs a) {
@@ -192,9 +194,13 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
     float *dsk = reinterpret_cast<float *>(smem + C::kOffD);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int head = blockIdx.x;
+    // this CTA's 64 channels: slice blockIdx.x % (headdim / 64) of head
+    // blockIdx.x / (headdim / 64); channel d = head * headdim + p, so the slice
+    // starts at channel blockIdx.x * 64
+    const int head = static_cast<int>(blockIdx.x / (a.headdim / C::P));
+    const int64_t c0 = int64_t(blockIdx.x) * C::P;
     const int64_t b = blockIdx.y;
-    const int64_t L = a.seqlen, Dm = a.nheads * C::P;
+    const int64_t L = a.seqlen, Dm = a.nheads * a.headdim;
     const int nc = static_cast<int>((L + C::Q - 1) / C::Q);
     const uint64_t limit = a.timeout_cycles;
     auto fail = [&]() {
@@ -228,7 +234,7 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
         prefetch_tensormap(&maps.C);
     }
     if (threadIdx.x < C::P)
-        dsk[threadIdx.x] = a.D ? __ldg(a.D + int64_t(head) * C::P + threadIdx.x) : 0.0f;
+        dsk[threadIdx.x] = a.D ? __ldg(a.D + c0 + threadIdx.x) : 0.0f;
     if (warp == 2) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
@@ -252,8 +258,8 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
             uint8_t *st = smem + s * C::kStage;
             const int t0 = k * C::Q;
             mbar_arrive_expect_tx(&loaded[s], C::kLoadBytes);
-            tma_load_3d(st + C::kX, &maps.x, head * C::P, t0, bb, &loaded[s]);
-            tma_load_3d(st + C::kZ, &maps.z, head * C::P, t0, bb, &loaded[s]);
+            tma_load_3d(st + C::kX, &maps.x, static_cast<int>(c0), t0, bb, &loaded[s]);
+            tma_load_3d(st + C::kZ, &maps.z, static_cast<int>(c0), t0, bb, &loaded[s]);
             tma_load_3d(st + C::kC, &maps.C, 0, t0, bb, &loaded[s]);
             tma_load_3d(st + C::kB, &maps.B, 0, t0, bb, &loaded[s]);
             last[s] = k;
@@ -457,7 +463,7 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
         // TMEM loads and arrivals.
         const int n = lane & 15;
         const bool own = lane < 16;
-        const int64_t hrow = (b * Dm + int64_t(head) * C::P) * C::N + n;  // + p * N
+        const int64_t hrow = (b * Dm + c0) * C::N + n;  // + p * N
         float h[64];
 #pragma unroll
         for (int p = 0; p < 64; ++p) h[p] = own && a.h0 ? __ldg(a.h0 + hrow + p * C::N) : 0.0f;
@@ -678,7 +684,7 @@ __global__ void __launch_bounds__(SsdChunkCfg::kThreads, 1)
                 const uint32_t zrow = stage_u32(s) + C::kZ + uint32_t(r) * 128u;
                 const float2 coef2 = make_float2(coef, coef), one2 = make_float2(1.0f, 1.0f);
                 const float2 nl2 = make_float2(-kLog2e, -kLog2e);
-                uint4 *dst = reinterpret_cast<uint4 *>(a.out + (b * L + t) * Dm + int64_t(head) * C::P +
+                uint4 *dst = reinterpret_cast<uint4 *>(a.out + (b * L + t) * Dm + c0 +
                                                        32 * wg);
                 // this group's 32 columns in two rolled halves of 16 (small code):
                 // Y and YI from TMEM, x and z from shared memory, the 32 bytes of

@@ -259,3 +259,18 @@ def test_ssd_chunked_in_place_state_and_optional_inputs():
     torch.cuda.synchronize()
     assert jamba_ssm_get_status() == _lib.OK
     assert hf2 is None and torch.equal(out2, out)
+
+
+@pytest.mark.parametrize("headdim", [128, 192])
+def test_ssd_chunked_wider_heads(headdim):
+    """Heads of 128 and 192 channels run the chunked kernel as 2 or 3 CTAs per
+    head, each a 64-channel slice repeating the head's per-token work."""
+    dev = _dev()
+    inp = synth.ssd_inputs(2, 300, 8, headdim, 16, torch.bfloat16, seed=94 + headdim, device=dev,
+                           h0_std=0.3)
+    out, hf = _gpu(inp)
+    ref, ref_h = _oracle(inp)
+    assert_out(out, ref, torch.bfloat16, f"headdim {headdim}")
+    assert_state(hf, ref_h, torch.bfloat16, f"headdim {headdim}")
+    out_s, _ = _gpu(inp, debug_flags=2)
+    assert rel_l2(out, out_s) <= BF16_REL_L2
